@@ -1,0 +1,463 @@
+#!/usr/bin/env python
+"""Benchmark: SmolVLA action-chunk generation on B200 through libsvla.
+
+One step = one pass of the whole hot path over one batch: prefix prefill into
+the per-layer K/V cache, then the 10-step Euler denoise of the 50 x 32 chunk.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Default workload: smolvla_b1 (B = 1, 177 prefix tokens, chunk 50, 10 steps),
+on which the headline metric "ms per 50-action chunk (b=1)" is quoted; a
+secondary line-item measures chunks/s at b = 32 (smolvla_b32). For N > 1 (one
+process per GPU under torchrun) every rank runs its own replica of the same
+workload (independent queries, no collective on the path): weak scaling.
+
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "ms per 50-action chunk (b=1)"
+L2_BYTES = 126 * 1024 * 1024
+
+# DRAM bytes (read + write) per launch of the GEMM kernel from the ncu capture
+# summarised in profiles/; None until a capture of the current kernel exists.
+NCU_TRAFFIC_PER_LAUNCH = None
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work of one chunk
+# ---------------------------------------------------------------------------
+def gemm_list(s, B, L, H, n_steps):
+    """Every GEMM launch of one chunk as (M, N, K, out_bytes_per_elem, rmw)."""
+    hd = s.head_dim
+    qp, kvp = s.p_heads * hd, s.p_kv_heads * hd
+    qe, kve = s.e_heads * hd, s.e_kv_heads * hd
+    Mp, Me = B * L, B * H
+    g = []
+    for l in range(s.p_layers):
+        g.append((Mp, qp + 2 * kvp, s.p_width, 2, False))
+        if l == s.p_layers - 1:
+            break
+        g += [(Mp, s.p_width, qp, 4, True), (Mp, 2 * s.p_ffn, s.p_width, 1, False),
+              (Mp, s.p_width, s.p_ffn, 4, True)]
+    for l in range(1, s.e_layers, 2):
+        g += [(Mp, kve, kvp, 2, False)] * 2
+    step = [(Me, s.e_width, s.e_width, 2, False), (Me, s.e_width, s.e_width, 4, False)]
+    for l in range(s.e_layers):
+        step.append((Me, qe + 2 * kve, s.e_width, 2, False) if l % 2 == 0 else (Me, qe, s.e_width, 2, False))
+        step += [(Me, s.e_width, qe, 4, True), (Me, 2 * s.e_ffn, s.e_width, 1, False),
+                 (Me, s.e_width, s.e_ffn, 4, True)]
+    return g + step * n_steps
+
+
+def gemm_bytes(M, N, K, ob, rmw):
+    return 2 * (M * K + N * K) + M * N * ob * (2 if rmw else 1)
+
+
+def chunk_work(s, B, L, H, n_steps):
+    """(algorithmic HBM bytes, GEMM FLOPs, attention FLOPs) of one chunk."""
+    flops = sum(2 * M * N * K for M, N, K, _, _ in gemm_list(s, B, L, H, n_steps))
+    wbytes = sum(2 * int(np.prod(shp)) for _, shp in synth.manifest(s))
+    hd = s.head_dim
+    kvw = s.p_kv_heads * hd
+    kv_bytes = 2 * s.p_layers * B * L * kvw * 2
+    n_odd = s.e_layers // 2
+    kvx_bytes = n_odd * 2 * B * L * s.e_kv_width * 2
+    # weights once for prefill + once per denoise step (the expert's 196 MB do not fit in L2),
+    # K/V written once, odd-layer cache read once by the hoist, projected K'/V' read every step
+    pre_w = sum(2 * int(np.prod(shp)) for n, shp in synth.manifest(s) if n.startswith("p"))
+    exp_w = wbytes - pre_w
+    hbm = pre_w + kv_bytes + (kv_bytes // 2) + kvx_bytes + n_steps * (exp_w + kvx_bytes)
+    att = 0
+    for _ in range(s.p_layers - 1):
+        att += 4 * B * s.p_heads * L * L * hd
+    att_step = 0
+    for l in range(s.e_layers):
+        att_step += 4 * B * s.e_heads * H * (H if l % 2 == 0 else L) * hd
+    att += n_steps * att_step
+    return hbm, flops, att
+
+
+def launches_per_chunk(s, n_steps):
+    """Kernels libsvla launches for one prefill + denoise (the CUDA graphs' kernel nodes)."""
+    pre = 1 + 2 * s.p_layers + 5 * (s.p_layers - 1)
+    hoist = 2 * (s.e_layers // 2)
+    step = 1 + 2 + 7 * s.e_layers + 1
+    return pre + hoist + n_steps * step
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ---------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((d.get("num_threads", 1) for d in info), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_chunk_timer(wl_name):
+    """Returns a callable running the oracle on one chunk of query 0 (ms)."""
+    import oracle
+    wl = synth.WORKLOADS[wl_name]
+    s = wl.model
+    W = oracle.load_weights(synth.gen_weights(s, wl.seed))
+    inp = synth.gen_inputs(wl, B=1)
+    emb = synth.bf16_bits_to_f32(inp["embeds"][0]).astype(np.float64)
+    valid = inp["valid"][0]
+    noise = inp["noise"][0].astype(np.float64)
+
+    def run():
+        t0 = time.perf_counter()
+        oracle.sample(W, s, emb, valid, noise, wl.n_steps)
+        return (time.perf_counter() - t0) * 1e3
+    return run
+
+
+def reference_arm(args, rank):
+    """The oracle as it stands, timed on this machine's host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS["smolvla_b1"]
+    run = oracle_chunk_timer(wl.name)
+    for _ in range(max(args.warmup, 0)):
+        run()
+    times = [run() for _ in range(args.steps)]
+    ms = float(np.mean(times))
+    cores = _blas_threads()
+    sample = "one full chunk of smolvla_b1 per step (prefill + 10 Euler steps, query 0)"
+    line = {"impl": "reference", "metric": METRIC, "value": ms, "unit": "ms", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": 1, "prefix_len": wl.L, "chunk": wl.H,
+                       "euler_steps": wl.n_steps, "parallelism": "host oracle"},
+            "cpu_baseline": {"value": ms, "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": ms, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def gpu_setup(wl_name, dev, B=None):
+    import torch
+    from vision_language_action_b200.runtime import SmolVLA
+    wl = synth.WORKLOADS[wl_name]
+    s = wl.model
+    B = wl.B if B is None else B
+    blob = synth.pack_blob(s, synth.gen_weights(s, wl.seed))
+    m = SmolVLA(s, blob, max_batch=B, max_prefix=wl.L, max_chunk=wl.H, device=dev)
+    del blob
+    inp = synth.gen_inputs(wl, B=B)
+    host = {
+        "embeds": torch.from_numpy(inp["embeds"].view(np.int16)).view(torch.bfloat16).pin_memory(),
+        "valid": torch.from_numpy(inp["valid"]).pin_memory(),
+        "noise": torch.from_numpy(inp["noise"]).pin_memory(),
+    }
+    d = {k: v.to(f"cuda:{dev}") for k, v in host.items()}
+    d["kv"] = m.new_kv_cache(B, wl.L)
+    d["actions"] = torch.empty_like(d["noise"])
+    return m, wl, host, d
+
+
+def time_steps(fn, steps, warmup, barrier):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    return e0.elapsed_time(e1)
+
+
+def gemm_roofline(s, B, L, H, n_steps, dev, hbm_peak):
+    """Live CUDA-event timing of the GEMM kernel over one chunk's GEMM launches
+    (same shapes and tile/split plans as the schedule; distinct weight buffers
+    per launch, so nothing is served from L2 that the path would not)."""
+    import ctypes
+    import torch
+    from vision_language_action_b200 import _abi
+    lib = _abi.load()
+    launches = gemm_list(s, B, L, H, 1)   # prefill + hoist + one denoise step
+    n_pre = len(gemm_list(s, B, L, H, 0))
+    acts = {}
+    ws_bytes = max(lib.svla_op_gemm_workspace_bytes(M, N, K, 0) for M, N, K, _, _ in launches)
+    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    plans = []
+    for i, (M, N, K, ob, rmw) in enumerate(launches):
+        W = torch.randn(N, K, device=dev).to(torch.bfloat16)
+        key = (M, K)
+        if key not in acts:
+            acts[key] = torch.randn(M, K, device=dev).to(torch.bfloat16)
+        C = torch.empty(M, N, device=dev, dtype=torch.float32 if ob == 4 else torch.bfloat16)
+        epi = _abi.EPI_ADD_F32 if rmw else (_abi.EPI_F32 if ob == 4 else _abi.EPI_BF16)
+        plans.append((epi, acts[key], W, C, M, N, K, gemm_bytes(M, N, K, ob, rmw)))
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+
+    def launch(p):
+        epi, A, W, C, M, N, K, _ = p
+        _abi.check(lib.svla_op_gemm(epi, P(A), K, P(W), K, M, N, K, P(C), N, None, 0, P(ws), ws_bytes, None, stream))
+
+    for p in plans:
+        launch(p)
+    torch.cuda.synchronize()
+    reps = 5
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in plans]
+    dur = np.zeros(len(plans))
+    for _ in range(reps):
+        for p, (a, b) in zip(plans, ev):
+            a.record()
+            launch(p)
+            b.record()
+        torch.cuda.synchronize()
+        dur += np.array([a.elapsed_time(b) for a, b in ev])
+    dur /= reps
+    # one chunk = prefill GEMMs + hoist + n_steps x step GEMMs
+    t_pre = dur[:n_pre].sum()
+    t_step = dur[n_pre:].sum()
+    b_pre = sum(p[7] for p in plans[:n_pre])
+    b_step = sum(p[7] for p in plans[n_pre:])
+    t_chunk = t_pre + n_steps * t_step
+    bytes_chunk = b_pre + n_steps * b_step
+    n_launch = n_pre + n_steps * (len(plans) - n_pre)
+    achieved = bytes_chunk / (t_chunk * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "gemm_tc_kernel", "achieved": round(achieved, 1), "peak": hbm_peak,
+            "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+            "traffic": NCU_TRAFFIC_PER_LAUNCH,
+            "launches_per_chunk": n_launch, "avg_launch_us": round(1e3 * t_chunk / n_launch, 2),
+            "algorithmic_bytes_per_launch": int(bytes_chunk / n_launch),
+            "gemm_ms_per_chunk": round(float(t_chunk), 4)}
+
+
+def ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    dev = local_rank
+    torch.cuda.set_device(dev)
+    barrier = (lambda: dist.barrier()) if world > 1 else (lambda: None)
+    hbm_peak, tf_peak, tf_sus, peak_kind = _peaks()
+
+    m, wl, host, d = gpu_setup("smolvla_b1", dev)
+    s = wl.model
+
+    def step():
+        m.prefill(d["embeds"], d["valid"], d["kv"])
+        m.denoise(d["kv"], d["valid"], d["noise"], wl.n_steps, actions=d["actions"])
+
+    clocks = Clocks(dev)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    clocks.start()
+    ms_total = time_steps(step, args.steps, args.warmup, barrier)
+    clk = clocks.stop()
+    st = m.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the timed region")
+    if world > 1:
+        t = torch.tensor([ms_total], device=f"cuda:{dev}")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    chunks_per_step = wl.B * world
+    value = ms_total / (args.steps * chunks_per_step)
+
+    # end to end through the public API with host buffers: H2D inputs, both calls, D2H actions
+    out_host = torch.empty_like(host["noise"]).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        d["embeds"].copy_(host["embeds"], non_blocking=True)
+        d["valid"].copy_(host["valid"], non_blocking=True)
+        d["noise"].copy_(host["noise"], non_blocking=True)
+        m.prefill(d["embeds"], d["valid"], d["kv"])
+        m.denoise(d["kv"], d["valid"], d["noise"], wl.n_steps, actions=d["actions"])
+        out_host.copy_(d["actions"], non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    ms_e2e = time_steps(e2e_step, args.steps, args.warmup, barrier)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=f"cuda:{dev}")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    hbm_bytes, gflops, aflops = chunk_work(s, wl.B, wl.L, wl.H, wl.n_steps)
+    chunk_s = value * 1e-3 * world  # per-rank chunk latency in s
+    roof = gemm_roofline(s, wl.B, wl.L, wl.H, wl.n_steps, f"cuda:{dev}", hbm_peak)
+    m.close()
+    del d
+    torch.cuda.empty_cache()
+
+    secondary = None
+    if not args.no_secondary:
+        m3, wl3, host3, d3 = gpu_setup("smolvla_b32", dev)
+
+        def step3():
+            m3.prefill(d3["embeds"], d3["valid"], d3["kv"])
+            m3.denoise(d3["kv"], d3["valid"], d3["noise"], wl3.n_steps, actions=d3["actions"])
+
+        def den3():
+            m3.denoise(d3["kv"], d3["valid"], d3["noise"], wl3.n_steps, actions=d3["actions"])
+
+        steps3 = max(3, args.steps // 2)
+        ms3 = time_steps(step3, steps3, args.warmup, barrier) / steps3
+        msd = time_steps(den3, steps3, args.warmup, barrier) / steps3
+        _, g3, a3 = chunk_work(wl3.model, wl3.B, wl3.L, wl3.H, wl3.n_steps)
+        _, g3p, a3p = chunk_work(wl3.model, wl3.B, wl3.L, wl3.H, 0)
+        den_flops = (g3 - g3p) + (a3 - a3p)
+        den_tf = den_flops / (msd * 1e-3) / 1e12
+        secondary = {"metric": "chunks/s (b=32)", "value": round(wl3.B * world / (ms3 * 1e-3), 2),
+                     "unit": "chunks/s", "ms_per_step": round(ms3, 4), "denoise_ms": round(msd, 4),
+                     "denoise_roofline": {"bound": "tensor", "achieved": round(den_tf, 1), "peak": tf_sus,
+                                          "unit": "TFLOP/s", "frac": round(den_tf / tf_sus, 4),
+                                          "peak_kind": f"{peak_kind} sustained bf16"},
+                     "config": {"workload": wl3.name, "batch": wl3.B, "prefix_len": wl3.L, "chunk": wl3.H,
+                                "euler_steps": wl3.n_steps}}
+        m3.close()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        run = oracle_chunk_timer("smolvla_b1")
+        run()
+        times = [run() for _ in range(3)]
+        cpu = {"value": round(float(np.mean(times)), 2), "unit": "ms", "cores": _blas_threads(), "kind": "oracle",
+               "sample": "3 full chunks of smolvla_b1 (prefill + 10 Euler steps, query 0), float64 numpy"}
+
+    if rank == 0:
+        achieved_chunk = hbm_bytes / chunk_s / 1e9
+        line = {
+            "metric": METRIC, "value": round(value, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.B, "prefix_len": wl.L, "chunk": wl.H,
+                       "euler_steps": wl.n_steps, "global_batch": wl.B * world,
+                       "parallelism": f"replicas x{world}",
+                       "l2_policy": "no flush: every step streams 514 MB of weights (> 126 MB L2)"},
+            "roofline": roof,
+            "chunk_roofline": {"bound": "hbm", "achieved": round(achieved_chunk, 1), "peak": hbm_peak,
+                               "unit": "GB/s", "frac": round(achieved_chunk / hbm_peak, 4),
+                               "algorithmic_bytes": int(hbm_bytes), "peak_kind": peak_kind},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(ms_e2e / (args.steps * chunks_per_step), 4), "unit": "ms",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "gpu_launches": launches_per_chunk(s, wl.n_steps) * args.steps,
+            "clocks": clk,
+            "secondary": secondary,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        reference_arm(args, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,208 @@
+/*
+ * svla.h — C ABI of libsvla: SmolVLA action-chunk generation on NVIDIA B200
+ * (sm_100a).
+ *
+ * What the library computes ("noeira docs, SmolVLA" §Architecture; "Paper vs
+ * hardware 11: SmolVLA" §claims):
+ *   1. prefill: the SmolLM2 prefix LM (RMSNorm, GQA attention with RoPE,
+ *      SwiGLU) runs once over the prefix embeddings and writes every layer's
+ *      keys and values into a K/V cache;
+ *   2. denoise: the action expert runs n_steps times; even layers do causal
+ *      self-attention over the chunk, odd layers cross-attend to the cached
+ *      K/V; a sinusoidal time embedding enters through the action-time MLP;
+ *      each step applies x <- x + dt * v, dt = -1/n_steps, from Gaussian
+ *      noise at t = 1 toward t = 0 (flow matching: x_t = t*eps + (1-t)*a).
+ *
+ * Conventions for every function below.
+ *   - Pointers named "device" must point to memory of the handle's device
+ *     (cudaMalloc'd, or a torch CUDA tensor's data_ptr). The library never
+ *     frees caller memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). All device work is enqueued on it asynchronously; a call
+ *     returns once the work is enqueued.
+ *   - bf16 is IEEE bfloat16 stored as uint16; matrices are row-major.
+ *   - Return value: SVLA_OK (0) or a negative svla_status. Argument and shape
+ *     errors are detected on the host before anything is enqueued. Errors
+ *     found on the device (a query with no valid prefix token, a bounded wait
+ *     that ran out) are sticky in a per-device status word, reported by
+ *     svla_device_status().
+ *   - A handle may be used from one host thread at a time. Calls that use the
+ *     same handle on different streams must not overlap in time on the GPU
+ *     (they share the handle's workspace).
+ */
+#ifndef SVLA_H_
+#define SVLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SVLA_API __attribute__((visibility("default")))
+#else
+#define SVLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int svla_status;
+#define SVLA_OK                 0
+#define SVLA_ERR_ARG           -1   /* null pointer, negative size, bad enum      */
+#define SVLA_ERR_SHAPE         -2   /* size outside the handle's limits / layout  */
+#define SVLA_ERR_BLOB_SIZE     -3   /* weight blob is not exactly the manifest    */
+#define SVLA_ERR_EMPTY_PREFIX  -4   /* a query has no valid prefix token          */
+#define SVLA_ERR_CUDA          -5   /* a CUDA runtime call failed                 */
+#define SVLA_ERR_OOM           -6   /* device allocation failed                   */
+#define SVLA_ERR_TIMEOUT       -7   /* a device-side bounded wait ran out         */
+#define SVLA_ERR_UNSUPPORTED   -8   /* no sm_100 device                           */
+
+typedef struct svla_handle svla_handle;
+
+/* Model shape and handle limits. The SmolVLA instance is
+ * {16, 960, 15, 5, 64, 2560, 16, 720, 15, 5, 2048, 32, 1e4, 1e-5, 4e-3, 4.0, ...}.
+ * Constraints: head_dim in {32, 64}; p_heads % p_kv_heads == 0 and
+ * e_heads % e_kv_heads == 0; p_layers == e_layers (expert layer l reads prefix
+ * layer l's cache on odd l); every width a multiple of 64 except e_width,
+ * action_dim (multiples of 8, action_dim <= 64) and p_ffn, e_ffn (multiples of 64). */
+typedef struct svla_config {
+  int p_layers, p_width, p_heads, p_kv_heads, head_dim, p_ffn;
+  int e_layers, e_width, e_heads, e_kv_heads, e_ffn, action_dim;
+  float rope_base, rms_eps, t_min_period, t_max_period;
+  int max_batch, max_prefix, max_chunk;
+} svla_config;
+
+/* Create a handle on `device` from a flat weight blob.
+ *   blob: bf16, host or device memory, the weights in manifest order —
+ *     per prefix layer l: in_norm[D], wq[nq*hd, D], wk[nkv*hd, D], wv[nkv*hd, D],
+ *       wo[D, nq*hd], post_norm[D], wg[F, D], wu[F, D], wd[D, F];
+ *     per expert layer l: in_norm[E], wq[eq*hd, E], wk[ekv*hd, X], wv[ekv*hd, X]
+ *       (X = E on even l, X = nkv*hd on odd l: the cross projection of the
+ *       cached prefix K/V), wo[E, eq*hd], post_norm[E], wg[Fe, E], wu[Fe, E], wd[E, Fe];
+ *     then final_norm[E], w_in[E, A], b_in[E], w_t1[E, 2E], b_t1[E], w_t2[E, E],
+ *       b_t2[E], w_out[A, E], b_out[A].
+ *     Matrices are [out, in] as nn.Linear stores them ("noeira docs, SmolVLA"
+ *     §Weights). The blob is copied; the caller may free it on return.
+ *   blob_bytes must equal the manifest total, else SVLA_ERR_BLOB_SIZE.
+ * Allocates the weights, a workspace sized by max_batch/max_prefix/max_chunk
+ * and small tables; *out receives the handle (NULL on error). */
+SVLA_API svla_status svla_create(const svla_config* cfg, const void* blob, size_t blob_bytes,
+                        int device, svla_handle** out);
+
+/* Free everything the handle owns (synchronises its device first). NULL is ok. */
+SVLA_API svla_status svla_destroy(svla_handle* h);
+
+/* Exact byte size of a K/V cache for B queries of L prefix tokens:
+ * K block then V block, each [p_layers][B][L][p_kv_heads*head_dim] bf16
+ * (token-major; K after RoPE). 0 on bad arguments. */
+SVLA_API size_t svla_kv_cache_bytes(const svla_handle* h, int B, int L);
+
+/* Bytes of the blob the handle expects (the manifest total). */
+SVLA_API size_t svla_blob_bytes(const svla_config* cfg);
+
+/* Prefix prefill ("noeira docs, SmolVLA" §Architecture: the VLM runs once over
+ * the prefix and caches its keys and values).
+ *   prefix_embeds: device bf16 [B, L, p_width].
+ *   pad_mask:      device uint8 [B, L], 1 = real token, 0 = padding (anywhere).
+ *                  Positions are cumsum(valid) - 1; a query with no valid token
+ *                  sets SVLA_ERR_EMPTY_PREFIX in the device status.
+ *   kv_cache:      device, svla_kv_cache_bytes(h, B, L) bytes, written in full
+ *                  except that pad slots hold values readers must mask.
+ * 1 <= B <= max_batch, 1 <= L <= max_prefix. */
+SVLA_API svla_status svla_prefill(svla_handle* h, const void* prefix_embeds, const uint8_t* pad_mask,
+                         int B, int L, void* kv_cache, void* stream);
+
+/* Euler flow-matching denoise of the action chunk ("noeira docs, SmolVLA"
+ * §Architecture: from Gaussian noise at t = 1, each of the steps predicts a
+ * velocity and moves toward t = 0).
+ *   kv_cache, pad_mask: as written / read by svla_prefill (same B, L).
+ *   noise:   device float32 [B, H, action_dim], x at t = 1.
+ *   actions: device float32 [B, H, action_dim], receives x after n_steps (may
+ *            alias noise).
+ *   trace:   NULL, or device float32 [n_steps][2][B][H][action_dim]: per step k
+ *            the velocity v_k at (x_k, t_k) and the state x_{k+1}.
+ * 1 <= H <= max_chunk, 1 <= n_steps <= 1000. The whole loop (the hoisted cross
+ * K/V projection and every step) is replayed from one CUDA graph per shape and
+ * buffer set. */
+SVLA_API svla_status svla_denoise(svla_handle* h, const void* kv_cache, const uint8_t* pad_mask,
+                         int B, int L, const float* noise, int H, int n_steps,
+                         float* actions, float* trace, void* stream);
+
+/* Draw the noise, prefill, denoise, on one stream.
+ * Noise: Philox4x32-10 keyed by seed (key = {seed low 32, seed high 32}),
+ * counter {block, query, 0, 0}; element e of a query's [H, A] noise is lane
+ * e % 4 of block e / 4; Box–Muller on the pairs (r0, r1) and (r2, r3) with
+ * u1 = ((r >> 8) + 1) / 2^24, u2 = (r >> 8) / 2^24.
+ *   kv_cache: device buffer as for svla_prefill (written).
+ *   noise_out: NULL or device float32 [B, H, A] receiving the drawn noise. */
+SVLA_API svla_status svla_sample(svla_handle* h, const void* prefix_embeds, const uint8_t* pad_mask,
+                        int B, int L, uint64_t seed, int H, int n_steps,
+                        void* kv_cache, float* noise_out, float* actions, void* stream);
+
+/* Synchronise `stream`, then return and clear the device status word of the
+ * handle's device (SVLA_OK, SVLA_ERR_EMPTY_PREFIX, SVLA_ERR_TIMEOUT) — or
+ * SVLA_ERR_CUDA if the synchronisation itself failed. */
+SVLA_API svla_status svla_device_status(svla_handle* h, void* stream);
+
+/* Text of the last error set on this handle (or, for h == NULL, by the last
+ * failing call of this thread). Never NULL. */
+SVLA_API const char* svla_last_error(const svla_handle* h);
+SVLA_API const char* svla_status_string(svla_status s);
+
+/* ---------------------------------------------------------------------------
+ * Kernel-level entry points (no handle). They expose single kernels of the
+ * path so each can be checked on its own; they use the same code as the path.
+ * ------------------------------------------------------------------------- */
+
+/* Epilogues of svla_op_gemm. */
+#define SVLA_EPI_F32        0   /* C(f32)  = acc (+ bias)                     */
+#define SVLA_EPI_BF16       1   /* C(bf16) = acc (+ bias)                     */
+#define SVLA_EPI_ADD_F32    2   /* C(f32) += acc (+ bias)    (residual add)   */
+#define SVLA_EPI_SILU_BF16  3   /* C(bf16) = silu(acc + bias)                 */
+
+/* C[M, N] = A[M, K] · W[N, K]^T on the tcgen05 tensor cores, bf16 inputs,
+ * fp32 accumulation (the projections of every layer: "noeira docs, SmolVLA"
+ * §Architecture, nn.Linear [out, in] weights).
+ *   A: device bf16, row stride lda >= K elements; W: device bf16, row stride
+ *   ldw >= K; C: device, row stride ldc >= N (f32 or bf16 per epilogue);
+ *   bias: NULL or device float32 [N].
+ *   Strides must be multiples of 8 elements and pointers 16-byte aligned (TMA).
+ *   splits: K-split count (0 = choose); with splits > 1 partial tiles go to
+ *   `workspace` (device, >= svla_op_gemm_workspace_bytes(M, N, K, splits)
+ *   bytes, its counter area zeroed once before first use and left zeroed by
+ *   every call) and the last CTA of each tile sums them in fixed order, so the
+ *   result is bitwise deterministic.
+ *   status: device int, set (first error wins) to SVLA_ERR_TIMEOUT if a
+ *   bounded wait ran out; may be NULL. */
+SVLA_API svla_status svla_op_gemm(int epilogue, const void* A, int lda, const void* W, int ldw,
+                         int M, int N, int K, void* C, int ldc, const float* bias,
+                         int splits, void* workspace, size_t workspace_bytes,
+                         int* status, void* stream);
+SVLA_API size_t svla_op_gemm_workspace_bytes(int M, int N, int K, int splits);
+/* The K-split count svla_op_gemm picks for splits = 0. */
+SVLA_API int svla_op_gemm_splits(int M, int N, int K);
+
+/* GQA attention (readings 1, 4–7): out = softmax(q k^T / sqrt(hd) + mask) v.
+ *   q: device bf16 [B, Lq, n_q*hd] (row stride ldq), k/v: device bf16
+ *   [B, Lk, n_kv*hd] (row stride ldkv); out: device bf16 [B, Lq, n_q*hd]
+ *   (row stride ldo). key_valid: NULL (all valid) or device uint8 [B, Lk].
+ *   causal: key j visible to row i only if j <= i. Query head h reads kv head
+ *   h / (n_q / n_kv). hd in {32, 64}. Every row needs >= 1 visible key. */
+SVLA_API svla_status svla_op_attention(const void* q, int ldq, const void* k, const void* v, int ldkv,
+                              const uint8_t* key_valid, int B, int n_q, int n_kv, int hd,
+                              int Lq, int Lk, int causal, void* out, int ldo, void* stream);
+
+/* RMSNorm (reading 8): y(bf16)[M, D] = x(f32)[M, D] / sqrt(mean(x^2) + eps) * g(bf16)[D]. */
+SVLA_API svla_status svla_op_rmsnorm(const float* x, const void* g, int M, int D, float eps,
+                            void* y, void* stream);
+
+/* Set the limit, in nanoseconds, of every device-side bounded wait of later
+ * launches (default 1e9). A limit of 0 makes any wait that is not already
+ * satisfied give up at once and report SVLA_ERR_TIMEOUT; it exists to test
+ * that path. Process-wide. */
+SVLA_API void svla_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SVLA_H_ */

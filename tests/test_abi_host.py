@@ -1,0 +1,110 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any CUDA work."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+from vision_language_action_b200 import _abi
+from vision_language_action_b200.runtime import config_from_shape
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "svla.h")).read()
+    return sorted(set(re.findall(r"SVLA_API\s+[\w\s\*]+?\b(svla_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _abi.load()
+    declared = _declared_symbols()
+    assert len(declared) >= 16
+    for name in declared:
+        assert hasattr(lib, name), name
+        assert name in _abi.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings():
+    lib = _abi.load()
+    for code, name in _abi.STATUS.items():
+        assert lib.svla_status_string(code).decode() == name
+
+
+@pytest.mark.parametrize("shape", ["tiny", "smolvla"])
+def test_blob_bytes_matches_manifest(shape):
+    lib = _abi.load()
+    s = synth.SHAPES[shape]
+    cfg = config_from_shape(s, 1, 8, 8)
+    n = sum(int(np.prod(shp)) for _, shp in synth.manifest(s))
+    assert lib.svla_blob_bytes(ctypes.byref(cfg)) == 2 * n
+
+
+def test_create_rejects_wrong_blob_size_before_touching_the_gpu():
+    lib = _abi.load()
+    s = synth.SHAPES["tiny"]
+    cfg = config_from_shape(s, 1, 24, 8)
+    n = lib.svla_blob_bytes(ctypes.byref(cfg))
+    blob = np.zeros(n // 2 + 4, np.uint16)
+    h = ctypes.c_void_p()
+    for nbytes in (n - 2, n + 2, 0):
+        st = lib.svla_create(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), nbytes, 0, ctypes.byref(h))
+        assert st == _abi.SVLA_ERR_BLOB_SIZE
+        assert h.value is None
+        assert b"manifest" in lib.svla_last_error(None)
+
+
+def test_create_rejects_bad_config():
+    lib = _abi.load()
+    s = synth.SHAPES["tiny"]
+    blob = np.zeros(16, np.uint16)
+    h = ctypes.c_void_p()
+    for bad in (dict(head_dim=48), dict(p_kv_heads=3), dict(action_dim=100), dict(e_layers=3),
+                dict(p_ffn=100), dict(rms_eps=0.0)):
+        cfg = config_from_shape(s.replace(**bad), 1, 24, 8)
+        st = lib.svla_create(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, ctypes.byref(h))
+        assert st == _abi.SVLA_ERR_SHAPE, bad
+    cfg = config_from_shape(s, 0, 24, 8)
+    assert lib.svla_create(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0,
+                           ctypes.byref(h)) == _abi.SVLA_ERR_SHAPE
+    assert lib.svla_create(None, None, 0, 0, ctypes.byref(h)) == _abi.SVLA_ERR_ARG
+
+
+def test_null_handle_calls_fail_cleanly():
+    lib = _abi.load()
+    assert lib.svla_prefill(None, None, None, 1, 1, None, None) == _abi.SVLA_ERR_ARG
+    assert lib.svla_denoise(None, None, None, 1, 1, None, 1, 1, None, None, None) == _abi.SVLA_ERR_ARG
+    assert lib.svla_device_status(None, None) == _abi.SVLA_ERR_ARG
+    assert lib.svla_kv_cache_bytes(None, 1, 1) == 0
+    assert lib.svla_destroy(None) == _abi.SVLA_OK
+
+
+def test_op_argument_checks():
+    lib = _abi.load()
+    p = ctypes.c_void_p(16)
+    # unknown epilogue, bad strides, misaligned pointers: rejected before any launch
+    assert lib.svla_op_gemm(9, p, 64, p, 64, 4, 4, 64, p, 4, None, 0, None, 0, None, None) == _abi.SVLA_ERR_ARG
+    assert lib.svla_op_gemm(0, p, 60, p, 64, 4, 4, 64, p, 4, None, 0, None, 0, None, None) == _abi.SVLA_ERR_SHAPE
+    assert lib.svla_op_gemm(0, ctypes.c_void_p(18), 64, p, 64, 4, 4, 64, p, 4, None, 0, None, 0, None,
+                            None) == _abi.SVLA_ERR_ARG
+    assert lib.svla_op_attention(p, 64, p, p, 64, None, 1, 3, 2, 64, 1, 1, 0, p, 64, None) == _abi.SVLA_ERR_SHAPE
+    assert lib.svla_op_attention(p, 64, p, p, 64, None, 1, 1, 1, 48, 1, 1, 0, p, 64, None) == _abi.SVLA_ERR_SHAPE
+    assert lib.svla_op_rmsnorm(ctypes.c_void_p(16), p, 1, 6, 1e-5, p, None) == _abi.SVLA_ERR_SHAPE
+
+
+def test_gemm_plan_workspace_rules():
+    lib = _abi.load()
+    # large M: one split, no workspace
+    assert lib.svla_op_gemm_splits(12800, 4096, 720) == 1
+    assert lib.svla_op_gemm_workspace_bytes(12800, 4096, 720, 0) == 0
+    # batch-1 shapes split K to cover the SMs, never more splits than K blocks
+    for (M, N, K) in [(50, 720, 2048), (50, 4096, 720), (50, 1600, 720), (1, 320, 64), (177, 960, 960)]:
+        sp = lib.svla_op_gemm_splits(M, N, K)
+        assert 1 <= sp <= (K + 63) // 64
+        ws = lib.svla_op_gemm_workspace_bytes(M, N, K, 0)
+        assert (ws > 0) == (sp > 1)
+    assert lib.svla_op_gemm_splits(50, 720, 2048) > 1
+    assert lib.svla_op_gemm_workspace_bytes(50, 720, 2048, 1) == 0

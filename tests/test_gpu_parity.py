@@ -1,0 +1,191 @@
+"""End-to-end parity of the CUDA path (through the C ABI) with the CPU oracle on
+the five synthetic workloads, plus determinism, batch/padding invariance, the
+empty-prefix error and svla_sample's noise.
+
+Gates (bf16 storage, fp32 accumulation): per-layer K/V relative L2 <= 5e-3 over
+valid positions; final chunk max|diff| <= 2e-2 and relative L2 <= 1e-2. The
+per-step trace (velocity and state of every Euler step) is held to the same
+chunk gates. Large batches are checked on a seeded subset of queries: queries
+are independent, so the oracle runs them one by one.
+"""
+import gc
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import synth  # noqa: E402
+from tests import helpers as H  # noqa: E402
+from vision_language_action_b200 import _abi  # noqa: E402
+from vision_language_action_b200.runtime import SmolVLA  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+DEV = "cuda:0"
+
+
+class Run:
+    """GPU run of a workload: handle, device inputs, K/V, chunk and trace."""
+
+    def __init__(self, wl_name, random_affine=False, B=None):
+        wl = synth.WORKLOADS[wl_name]
+        s, _, blob = H.weights(wl_name, random_affine)
+        inp = H.inputs(wl_name)
+        self.wl, self.s = wl, s
+        self.B = wl.B if B is None else B
+        self.m = SmolVLA(s, blob, max_batch=self.B, max_prefix=wl.L, max_chunk=wl.H)
+        self.valid = torch.from_numpy(inp["valid"][:self.B]).to(DEV)
+        self.noise = torch.from_numpy(inp["noise"][:self.B]).to(DEV)
+        if wl.prefix_kind == "kv_given":
+            kv = np.stack([inp["k"][:, :self.B], inp["v"][:, :self.B]])
+            self.kv = torch.from_numpy(kv.reshape(2, s.p_layers, self.B, wl.L, -1).view(np.int16)).to(DEV)
+            self.kv = self.kv.view(torch.bfloat16)
+        else:
+            self.embeds = torch.from_numpy(inp["embeds"][:self.B].view(np.int16)).to(DEV).view(torch.bfloat16)
+            self.kv = self.m.prefill(self.embeds, self.valid)
+        self.actions, self.trace = self.m.denoise(self.kv, self.valid, self.noise, wl.n_steps, trace=True)
+        assert self.m.device_status() == _abi.SVLA_OK
+        torch.cuda.synchronize()
+
+    def kv_np(self):
+        L, s = self.wl.L, self.s
+        kv = self.kv.float().cpu().numpy().reshape(2, s.p_layers, self.B, L, s.p_kv_heads, s.head_dim)
+        return kv[0], kv[1]
+
+    def close(self):
+        self.m.close()
+
+
+def check_query(run: Run, b: int, random_affine=False):
+    wl, s = run.wl, run.s
+    K, V, vs, xs, x = H.oracle_query(wl.name, b, random_affine)
+    valid = H.inputs(wl.name)["valid"][b].astype(bool)
+    if wl.prefix_kind != "kv_given":
+        Kg, Vg = run.kv_np()
+        for l in range(s.p_layers):
+            rk = H.rel_l2(Kg[l, b][valid], K[l][valid])
+            rv = H.rel_l2(Vg[l, b][valid], V[l][valid])
+            assert rk <= H.KV_REL_L2 and rv <= H.KV_REL_L2, (wl.name, b, l, rk, rv)
+    tr = run.trace.cpu().numpy()
+    for k in range(wl.n_steps):
+        assert H.max_abs(tr[k, 1, b], xs[k]) <= H.CHUNK_MAX_ABS, (wl.name, b, "step", k)
+        assert H.rel_l2(tr[k, 0, b], vs[k]) <= H.CHUNK_REL_L2, (wl.name, b, "velocity", k)
+    got = run.actions[b].cpu().numpy()
+    assert np.array_equal(got, tr[-1, 1, b])
+    assert H.max_abs(got, x) <= H.CHUNK_MAX_ABS, (wl.name, b, H.max_abs(got, x))
+    assert H.rel_l2(got, x) <= H.CHUNK_REL_L2, (wl.name, b, H.rel_l2(got, x))
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    r = Run("tiny")
+    yield r
+    r.close()
+
+
+def test_tiny_parity(tiny):
+    check_query(tiny, 0)
+
+
+def test_tiny_random_affine_parity():
+    r = Run("tiny", random_affine=True)
+    try:
+        check_query(r, 0, random_affine=True)
+    finally:
+        r.close()
+
+
+def test_smolvla_b1_parity():
+    r = Run("smolvla_b1")
+    try:
+        check_query(r, 0)
+        # run-to-run bitwise determinism of prefill and denoise
+        kv2 = r.m.prefill(r.embeds, r.valid)
+        a2, t2 = r.m.denoise(kv2, r.valid, r.noise, r.wl.n_steps, trace=True)
+        torch.cuda.synchronize()
+        assert torch.equal(kv2, r.kv)
+        assert torch.equal(a2, r.actions) and torch.equal(t2, r.trace)
+    finally:
+        r.close()
+        gc.collect()
+
+
+def test_smolvla_b32_parity_and_batch_invariance():
+    r = Run("smolvla_b32")
+    try:
+        for b in (0, 13, 31):
+            check_query(r, b)
+        # query 13 alone gives the same chunk as inside the batch (within tolerance)
+        e1 = r.embeds[13:14].contiguous()
+        v1 = r.valid[13:14].contiguous()
+        n1 = r.noise[13:14].contiguous()
+        kv1 = r.m.prefill(e1, v1)
+        a1, _ = r.m.denoise(kv1, v1, n1, r.wl.n_steps)
+        torch.cuda.synchronize()
+        assert H.max_abs(a1[0].cpu().numpy(), r.actions[13].cpu().numpy()) <= 5e-3
+        # padding invariance: the same query with its pads removed
+        keep = torch.nonzero(r.valid[13]).flatten()
+        ec = r.embeds[13:14, keep].contiguous()
+        vc = torch.ones(1, keep.numel(), dtype=torch.uint8, device=DEV)
+        kvc = r.m.prefill(ec, vc)
+        ac, _ = r.m.denoise(kvc, vc, n1, r.wl.n_steps)
+        torch.cuda.synchronize()
+        assert H.max_abs(ac[0].cpu().numpy(), r.actions[13].cpu().numpy()) <= 5e-3
+    finally:
+        r.close()
+        gc.collect()
+
+
+def test_long_prefix_b8_parity():
+    r = Run("long_prefix_b8")
+    try:
+        for b in (0, 7):
+            check_query(r, b)
+    finally:
+        r.close()
+        gc.collect()
+
+
+def test_denoise_b256_parity():
+    r = Run("denoise_b256")
+    try:
+        for b in (0, 101, 255):
+            check_query(r, b)
+    finally:
+        r.close()
+        gc.collect()
+
+
+def test_empty_prefix_sets_device_status(tiny):
+    v0 = tiny.valid.clone()
+    v0[0] = 0
+    tiny.m.prefill(tiny.embeds, v0)
+    assert tiny.m.device_status() == _abi.SVLA_ERR_EMPTY_PREFIX
+    assert tiny.m.device_status() == _abi.SVLA_OK  # cleared on read
+
+
+def test_host_shape_errors(tiny):
+    with pytest.raises(_abi.SvlaError) as e:
+        tiny.m.denoise(tiny.kv, tiny.valid, tiny.noise, 0)
+    assert e.value.status == _abi.SVLA_ERR_SHAPE
+    big = torch.zeros(1, tiny.wl.L + 1, dtype=torch.uint8, device=DEV)
+    with pytest.raises(_abi.SvlaError) as e:
+        tiny.m.prefill(tiny.embeds, big)
+    assert e.value.status == _abi.SVLA_ERR_SHAPE
+
+
+def test_sample_noise_matches_philox_and_denoise(tiny):
+    import oracle
+    seed = 0x1234_5678_9ABC
+    actions, kv, noise = tiny.m.sample(tiny.embeds, tiny.valid, seed, tiny.wl.H, tiny.wl.n_steps,
+                                       return_noise=True)
+    torch.cuda.synchronize()
+    want = oracle.gaussian_noise(seed, 1, tiny.wl.H, tiny.s.action_dim)
+    assert H.max_abs(noise.cpu().numpy(), want) <= 2e-5
+    a2, _ = tiny.m.denoise(kv, tiny.valid, noise, tiny.wl.n_steps)
+    torch.cuda.synchronize()
+    assert torch.equal(a2, actions)

@@ -1,0 +1,417 @@
+// tcgen05 / TMEM / TMA GEMM for sm_100a:  C[M, N] = A[M, K] · W[N, K]^T
+//
+// Every projection of the SmolLM2 prefix layers and of the action expert is
+// this contraction on nn.Linear [out, in] weights ("noeira docs, SmolVLA"
+// §Architecture, §Weights). bf16 operands, fp32 accumulation in tensor memory.
+//
+// CTA = one 128 x BN output tile and one slice of K (split-K over gridDim.z).
+//   warp 0      : TMA producer (one lane): A and W tiles, 128-byte swizzle,
+//                 into a STAGES-deep shared-memory ring (no multicast).
+//   warp 1      : allocates BN TMEM columns; one lane issues tcgen05.mma
+//                 (M = 128, N = BN, K = 16 per instruction) and commits each
+//                 stage back to the producer, then the accumulator to the
+//                 epilogue.
+//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4).. (its rows) with
+//                 tcgen05.ld, applies the fused epilogue and stores.
+// Split-K: every CTA of a tile writes its fp32 partial tile to the workspace,
+// the last to arrive (atomic counter) sums the partials in split order and
+// runs the epilogue, then re-arms the counter, so the result does not depend
+// on arrival order.
+// Every mbarrier wait is bounded; on time-out the CTA records
+// SVLA_ERR_TIMEOUT, drains its in-flight copies and MMAs (with a fixed
+// limit), frees its tensor memory and returns.
+#pragma once
+
+#include "common.cuh"
+
+namespace svla {
+
+enum GemmEpi : int {
+  GE_F32 = 0,        // out f32 = acc + bias
+  GE_BF16 = 1,       // out bf16 = acc + bias
+  GE_ADD_F32 = 2,    // out f32 += acc + bias
+  GE_SILU_BF16 = 3,  // out bf16 = silu(acc + bias)
+  GE_SWIGLU = 4,     // W rows interleaved in 32-row groups [gate 32 | up 32]; out bf16 = silu(g) * u
+  GE_QKV_ROPE64 = 5, // columns [q | k | v] of 64-wide heads; RoPE on q and k; q -> q_out, k -> k_out, v -> v_out
+  GE_QKV_ROPE32 = 6, // the same with 32-wide heads
+};
+
+struct GemmArgs {
+  int M, N, K;
+  void* out;             // main output (GE_F32/BF16/ADD/SILU/SWIGLU)
+  int ldo;               // elements
+  const float* bias;     // [N] or null
+  // GE_QKV_ROPE
+  bf16* q_out;
+  int ldq;
+  bf16* k_out;
+  bf16* v_out;
+  int ldkv;
+  int q_cols, kv_cols;
+  const int* pos;        // per-row position, or null: row % pos_mod
+  int pos_mod;
+  const float2* rope_cs; // [pos][head_dim/2] (cos, sin)
+  // split-K
+  float* partials;       // [tiles][splits][128][BN]
+  int* counters;         // [tiles], zero between launches
+  int* status;
+  unsigned long long wait_ns;
+};
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BK = 64;
+constexpr int GEMM_THREADS = 192;
+constexpr unsigned long long GEMM_DRAIN_NS = 2000000000ull;  // fixed limit for the drain path
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int STAGES = BN <= 64 ? 8 : (BN <= 128 ? 6 : 4);
+  static constexpr uint32_t A_BYTES = GEMM_BM * GEMM_BK * 2;
+  static constexpr uint32_t B_BYTES = BN * GEMM_BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
+  // ring + barriers/flags area + alignment slack
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 256 + 1024;
+};
+
+// ---------------------------------------------------------------------------
+// epilogue helpers (one thread = one output row, 16 consecutive columns)
+// ---------------------------------------------------------------------------
+SVLA_DEV void store16_f32(float* dst, const float (&v)[16], int ncols) {
+  if (ncols >= 16) {
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  } else {
+    for (int i = 0; i < ncols; ++i) dst[i] = v[i];
+  }
+}
+
+SVLA_DEV void add16_f32(float* dst, const float (&v)[16], int ncols) {
+  if (ncols >= 16) {
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float4 o = d4[i];
+      o.x += v[4 * i];
+      o.y += v[4 * i + 1];
+      o.z += v[4 * i + 2];
+      o.w += v[4 * i + 3];
+      d4[i] = o;
+    }
+  } else {
+    for (int i = 0; i < ncols; ++i) dst[i] += v[i];
+  }
+}
+
+SVLA_DEV void store16_bf16(bf16* dst, const float (&v)[16], int ncols) {
+  if (ncols >= 16) {
+    uint4 a, b;
+    a.x = pack_bf16x2(v[0], v[1]);
+    a.y = pack_bf16x2(v[2], v[3]);
+    a.z = pack_bf16x2(v[4], v[5]);
+    a.w = pack_bf16x2(v[6], v[7]);
+    b.x = pack_bf16x2(v[8], v[9]);
+    b.y = pack_bf16x2(v[10], v[11]);
+    b.z = pack_bf16x2(v[12], v[13]);
+    b.w = pack_bf16x2(v[14], v[15]);
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    d[0] = a;
+    d[1] = b;
+  } else {
+    for (int i = 0; i < ncols; ++i) dst[i] = __float2bfloat16_rn(v[i]);
+  }
+}
+
+SVLA_DEV void add_bias16(float (&v)[16], const float* bias, int col, int N) {
+  if (bias) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (col + i < N) v[i] += __ldg(bias + col + i);
+  }
+}
+
+// Fetches 16 accumulator columns [c, c+16) of this thread's row: from TMEM,
+// or (split-K reducer) the sum of the partial tiles in split order.
+template <int BN>
+struct AccSource {
+  uint32_t taddr_row;
+  const float* part_row;  // partials of split 0, this row; next split at +split_stride
+  size_t split_stride;
+  int splits;
+  SVLA_DEV void get(int c, float (&v)[16]) const {
+    if (splits == 1) {
+      tmem_ld16(taddr_row + (uint32_t)c, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      for (int z = 0; z < splits; ++z) {
+        const float4* p = reinterpret_cast<const float4*>(part_row + z * split_stride + c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float4 t = __ldcg(p + i);
+          v[4 * i] += t.x;
+          v[4 * i + 1] += t.y;
+          v[4 * i + 2] += t.z;
+          v[4 * i + 3] += t.w;
+        }
+      }
+    }
+  }
+};
+
+template <int BN, int EPI>
+SVLA_DEV void run_epilogue(const GemmArgs& a, const AccSource<BN>& src, int m, int n0, bool row_ok) {
+  // tcgen05.ld is warp-collective: every lane walks the same columns; only
+  // rows inside M store.
+  if constexpr (EPI == GE_SWIGLU) {
+    // tile columns [64j, 64j+32) gate, [64j+32, 64j+64) up, features n0/2 + 32j + ..
+    bf16* out = reinterpret_cast<bf16*>(a.out);
+    const int F = a.N / 2;
+#pragma unroll 1
+    for (int j = 0; j < BN / 64; ++j) {
+#pragma unroll 1
+      for (int c = 0; c < 32; c += 16) {
+        float g[16], u[16];
+        src.get(64 * j + c, g);
+        src.get(64 * j + 32 + c, u);
+        const int f = n0 / 2 + 32 * j + c;
+        if (row_ok && f < F) {
+          float h[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) h[i] = silu_f(g[i]) * u[i];
+          store16_bf16(out + (size_t)m * a.ldo + f, h, F - f);
+        }
+      }
+    }
+  } else if constexpr (EPI == GE_QKV_ROPE64 || EPI == GE_QKV_ROPE32) {
+    constexpr int HD = EPI == GE_QKV_ROPE64 ? 64 : 32;
+    constexpr int HALF = HD / 2;
+    int p = 0;
+    if (row_ok) {
+      p = a.pos ? __ldg(a.pos + m) : (m % a.pos_mod);
+      if (p < 0) p = 0;  // leading pad slots (unspecified output)
+    }
+#pragma unroll 1
+    for (int hb = 0; hb < BN; hb += HD) {
+      const int col = n0 + hb;
+      float x[HD];
+#pragma unroll
+      for (int c = 0; c < HD; c += 16) src.get(hb + c, *reinterpret_cast<float(*)[16]>(x + c));
+      if (!row_ok || col >= a.N) continue;
+      bf16* dst;
+      bool rot = true;
+      if (col < a.q_cols) {
+        dst = a.q_out + (size_t)m * a.ldq + col;
+      } else if (col < a.q_cols + a.kv_cols) {
+        dst = a.k_out + (size_t)m * a.ldkv + (col - a.q_cols);
+      } else {
+        dst = a.v_out + (size_t)m * a.ldkv + (col - a.q_cols - a.kv_cols);
+        rot = false;
+      }
+      if (rot) {
+        // rotate-half RoPE: pairs (i, i + HD/2), angle pos * base^(-2i/HD)
+        const float2* cs = a.rope_cs + (size_t)p * HALF;
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) {
+          const float2 t = __ldg(cs + i);
+          const float x1 = x[i], x2 = x[i + HALF];
+          x[i] = x1 * t.x - x2 * t.y;
+          x[i + HALF] = x2 * t.x + x1 * t.y;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < HD; c += 16) store16_bf16(dst + c, *reinterpret_cast<float(*)[16]>(x + c), 16);
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      src.get(c, v);
+      const int col = n0 + c;
+      if (!row_ok || col >= a.N) continue;
+      const int ncols = a.N - col;
+      add_bias16(v, a.bias, col, a.N);
+      if constexpr (EPI == GE_F32) {
+        store16_f32(reinterpret_cast<float*>(a.out) + (size_t)m * a.ldo + col, v, ncols);
+      } else if constexpr (EPI == GE_ADD_F32) {
+        add16_f32(reinterpret_cast<float*>(a.out) + (size_t)m * a.ldo + col, v, ncols);
+      } else if constexpr (EPI == GE_BF16) {
+        store16_bf16(reinterpret_cast<bf16*>(a.out) + (size_t)m * a.ldo + col, v, ncols);
+      } else if constexpr (EPI == GE_SILU_BF16) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = silu_f(v[i]);
+        store16_bf16(reinterpret_cast<bf16*>(a.out) + (size_t)m * a.ldo + col, v, ncols);
+      }
+    }
+  }
+}
+
+// named barrier over the 4 epilogue warps (ids 2..5)
+SVLA_DEV void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                   const GemmArgs args) {
+  using C = GemmCfg<BN>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+  // bars[0..S) full, [S..2S) empty, [2S] accumulator ready
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(bars + 2 * STAGES + 1);
+  // misc[0] tmem base, misc[1] abort flag, misc[2] k-blocks issued, misc[3] k-blocks consumed,
+  // misc[4] "this CTA reduces"
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_blk = blockIdx.x, m_blk = blockIdx.y, split = blockIdx.z, splits = gridDim.z;
+  const int KB = (args.K + GEMM_BK - 1) / GEMM_BK;
+  const int kb0 = (int)(((long long)split * KB) / splits);
+  const int kb1 = (int)(((long long)(split + 1) * KB) / splits);
+  const int nkb = kb1 - kb0;
+
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+  const uint32_t acc_bar = smem_u32(bars + 2 * STAGES);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(acc_bar, 1);
+    misc[1] = 0;
+    misc[2] = 0;
+    misc[3] = 0;
+    misc[4] = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)&misc[0]), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = misc[0];
+  const unsigned long long lim = args.wait_ns;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < nkb; ++i) {
+        if (misc[1]) break;
+        const int s = i % STAGES;
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+        if (i >= STAGES && !mbar_wait(empty_bar(s), ph ^ 1u, lim)) {
+          misc[1] = 1;
+          set_status(args.status, SVLA_ERR_TIMEOUT);
+          break;
+        }
+        const uint32_t sa = smem_u32(ring + s * C::STAGE_BYTES);
+        mbar_arrive_expect_tx(full_bar(s), C::STAGE_BYTES);
+        tma_load_2d(sa, &tmA, full_bar(s), (kb0 + i) * GEMM_BK, m_blk * GEMM_BM);
+        tma_load_2d(sa + C::A_BYTES, &tmW, full_bar(s), (kb0 + i) * GEMM_BK, n_blk * BN);
+        misc[2] = i + 1;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, BN);
+      for (int i = 0; i < nkb; ++i) {
+        if (misc[1]) break;
+        const int s = i % STAGES;
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+        if (!mbar_wait(full_bar(s), ph, lim)) {
+          misc[1] = 1;
+          set_status(args.status, SVLA_ERR_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(ring + s * C::STAGE_BYTES);
+        const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+        for (int k = 0; k < GEMM_BK / 16; ++k) {
+          tc_mma_bf16(tmem_base, smem_desc_sw128(sa + 32 * k), smem_desc_sw128(sb + 32 * k), IDESC,
+                      (i > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit(empty_bar(s));
+        misc[3] = i + 1;
+      }
+      tc_commit(acc_bar);  // always: lets waiters know every issued MMA finished
+    }
+  } else {
+    // ---------------- epilogue warps ----------------
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int m = m_blk * GEMM_BM + row;
+    const bool row_ok = m < args.M;
+    const int n0 = n_blk * BN;
+    bool ok = mbar_wait(acc_bar, 0, lim);
+    if (!ok) {
+      misc[1] = 1;
+      set_status(args.status, SVLA_ERR_TIMEOUT);
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    const bool aborted = misc[1] != 0;
+    if (ok && !aborted) {
+      AccSource<BN> src;
+      src.taddr_row = tmem_base + ((uint32_t)(quad * 32) << 16);
+      src.splits = 1;
+      src.part_row = nullptr;
+      src.split_stride = 0;
+      if (splits == 1) {
+        run_epilogue<BN, EPI>(args, src, m, n0, row_ok);
+      } else {
+        const int tile = m_blk * gridDim.x + n_blk;
+        float* tile_part = args.partials + (size_t)tile * splits * GEMM_BM * BN;
+        // 1) this split's partial rows
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          float v[16];
+          tmem_ld16(src.taddr_row + (uint32_t)c, v);
+          if (row_ok) store16_f32(tile_part + ((size_t)split * GEMM_BM + row) * BN + c, v, 16);
+        }
+        __threadfence();
+        epi_bar();
+        if (threadIdx.x == 64) {
+          const int old = atomicAdd(args.counters + tile, 1);
+          misc[4] = (old == splits - 1) ? 1u : 0u;
+        }
+        epi_bar();
+        if (misc[4]) {
+          __threadfence();
+          src.splits = splits;
+          src.part_row = tile_part + (size_t)row * BN;
+          src.split_stride = (size_t)GEMM_BM * BN;
+          run_epilogue<BN, EPI>(args, src, m, n0, row_ok);
+          if (threadIdx.x == 64) args.counters[tile] = 0;  // re-arm for the next launch
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (misc[1]) {
+    // time-out path: let every issued TMA copy land and every MMA finish
+    if (threadIdx.x == 0) {
+      const int issued = (int)misc[2], consumed = (int)misc[3];
+      for (int i = consumed; i < issued; ++i)
+        mbar_wait(full_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u, GEMM_DRAIN_NS);
+    }
+    if (threadIdx.x == 32) mbar_wait(acc_bar, 0, GEMM_DRAIN_NS);
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace svla

@@ -1,0 +1,781 @@
+// libsvla: the C ABI of include/svla.h — handle, weight layout, workspace,
+// and the prefill / denoise schedules, each replayed from a CUDA graph.
+//
+// Path ("noeira docs, SmolVLA" §Architecture):
+//   prefill:  positions -> 16 x [RMSNorm, QKV GEMM (+RoPE, K/V cache write),
+//             attention, O GEMM (+residual), RMSNorm, gate/up GEMM (+SwiGLU),
+//             down GEMM (+residual)]; the last layer stops after its K/V write.
+//   denoise:  hoisted cross K/V projection of the odd layers' caches, then per
+//             Euler step: action/time prologue, time-MLP GEMMs, 16 expert
+//             layers, final norm + action_out + x <- x + dt v.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <list>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "attention.cuh"
+#include "gemm_host.cuh"
+#include "small_kernels.cuh"
+
+using namespace svla;
+
+namespace {
+
+std::atomic<unsigned long long> g_wait_ns{1000000000ull};
+thread_local std::string t_last_error = "no error";
+
+const char* status_str(svla_status s) {
+  switch (s) {
+    case SVLA_OK: return "SVLA_OK";
+    case SVLA_ERR_ARG: return "SVLA_ERR_ARG";
+    case SVLA_ERR_SHAPE: return "SVLA_ERR_SHAPE";
+    case SVLA_ERR_BLOB_SIZE: return "SVLA_ERR_BLOB_SIZE";
+    case SVLA_ERR_EMPTY_PREFIX: return "SVLA_ERR_EMPTY_PREFIX";
+    case SVLA_ERR_CUDA: return "SVLA_ERR_CUDA";
+    case SVLA_ERR_OOM: return "SVLA_ERR_OOM";
+    case SVLA_ERR_TIMEOUT: return "SVLA_ERR_TIMEOUT";
+    case SVLA_ERR_UNSUPPORTED: return "SVLA_ERR_UNSUPPORTED";
+  }
+  return "unknown svla_status";
+}
+
+// per-device one-time kernel attribute setup
+std::mutex g_attr_mu;
+bool g_attr_done[64] = {};
+
+cudaError_t ensure_attrs(int dev) {
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (g_attr_done[dev]) return cudaSuccess;
+  cudaError_t e = gemm_set_attrs();
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(step_end_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)AttnCfg<64>::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attention_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)AttnCfg<32>::SMEM);
+  if (e == cudaSuccess && !encode_fn()) e = cudaErrorNotSupported;  // resolve outside any capture
+  if (e == cudaSuccess) g_attr_done[dev] = true;
+  return e;
+}
+
+bool device_is_sm100(int dev) {
+  cudaDeviceProp p;
+  if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return false;
+  return p.major == 10;
+}
+
+// ---- manifest -------------------------------------------------------------
+struct Entry {
+  size_t off, n;
+};
+
+struct Layout {
+  std::vector<Entry> p, e;  // 9 entries per layer
+  Entry final_norm, w_in, b_in, w_t1, b_t1, w_t2, b_t2, w_out, b_out;
+  size_t total = 0;
+};
+
+Layout make_layout(const svla_config& c) {
+  Layout L;
+  size_t off = 0;
+  auto add = [&](size_t n) {
+    Entry e{off, n};
+    off += n;
+    return e;
+  };
+  const size_t D = c.p_width, hd = c.head_dim, E = c.e_width;
+  for (int l = 0; l < c.p_layers; ++l) {
+    L.p.push_back(add(D));
+    L.p.push_back(add((size_t)c.p_heads * hd * D));
+    L.p.push_back(add((size_t)c.p_kv_heads * hd * D));
+    L.p.push_back(add((size_t)c.p_kv_heads * hd * D));
+    L.p.push_back(add(D * c.p_heads * hd));
+    L.p.push_back(add(D));
+    L.p.push_back(add((size_t)c.p_ffn * D));
+    L.p.push_back(add((size_t)c.p_ffn * D));
+    L.p.push_back(add(D * c.p_ffn));
+  }
+  for (int l = 0; l < c.e_layers; ++l) {
+    const size_t kv_in = (l % 2 == 0) ? E : (size_t)c.p_kv_heads * hd;
+    L.e.push_back(add(E));
+    L.e.push_back(add((size_t)c.e_heads * hd * E));
+    L.e.push_back(add((size_t)c.e_kv_heads * hd * kv_in));
+    L.e.push_back(add((size_t)c.e_kv_heads * hd * kv_in));
+    L.e.push_back(add(E * c.e_heads * hd));
+    L.e.push_back(add(E));
+    L.e.push_back(add((size_t)c.e_ffn * E));
+    L.e.push_back(add((size_t)c.e_ffn * E));
+    L.e.push_back(add(E * c.e_ffn));
+  }
+  const size_t A = c.action_dim;
+  L.final_norm = add(E);
+  L.w_in = add(E * A);
+  L.b_in = add(E);
+  L.w_t1 = add(E * 2 * E);
+  L.b_t1 = add(E);
+  L.w_t2 = add(E * E);
+  L.b_t2 = add(E);
+  L.w_out = add(A * E);
+  L.b_out = add(A);
+  L.total = off;
+  return L;
+}
+
+const char* check_config(const svla_config& c) {
+  if (c.p_layers < 1 || c.e_layers < 1 || c.p_layers != c.e_layers) return "p_layers must equal e_layers (>= 1)";
+  if (c.head_dim != 32 && c.head_dim != 64) return "head_dim must be 32 or 64";
+  if (c.p_heads < 1 || c.p_kv_heads < 1 || c.p_heads % c.p_kv_heads) return "p_heads % p_kv_heads != 0";
+  if (c.e_heads < 1 || c.e_kv_heads < 1 || c.e_heads % c.e_kv_heads) return "e_heads % e_kv_heads != 0";
+  if (c.p_width < 64 || c.p_width % 64 || c.p_width > 2048) return "p_width must be a multiple of 64, <= 2048";
+  if (c.e_width < 16 || c.e_width % 16 || c.e_width > 2048) return "e_width must be a multiple of 16, <= 2048";
+  if (c.p_ffn < 64 || c.p_ffn % 64 || c.e_ffn < 64 || c.e_ffn % 64) return "ffn widths must be multiples of 64";
+  if (c.action_dim < 8 || c.action_dim % 8 || c.action_dim > 64) return "action_dim must be a multiple of 8, <= 64";
+  if (c.max_batch < 1 || c.max_prefix < 1 || c.max_chunk < 1) return "max sizes must be >= 1";
+  if (!(c.rms_eps > 0.f) || !(c.rope_base > 1.f) || !(c.t_min_period > 0.f) || !(c.t_max_period > 0.f))
+    return "rope_base, rms_eps and the time periods must be positive";
+  return nullptr;
+}
+
+__global__ void interleave_gu_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, int F, int K) {
+  // dst row r: group g = r / 64; rows [0,32) of a group are gate rows 32g.., [32,64) up rows 32g..
+  const int r = blockIdx.x;
+  const int g = r / 64, w = r % 64;
+  const int sr = (w < 32) ? (32 * g + w) : (F + 32 * g + (w - 32));
+  for (int k = threadIdx.x; k < K; k += blockDim.x) dst[(size_t)r * K + k] = src[(size_t)sr * K + k];
+}
+
+__global__ void bf16_to_f32_kernel(const uint16_t* __restrict__ src, float* __restrict__ dst, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = __uint_as_float(((uint32_t)src[i]) << 16);
+}
+
+struct GraphEntry {
+  std::vector<uint64_t> key;
+  cudaGraphExec_t exec = nullptr;
+};
+
+}  // namespace
+
+struct svla_handle {
+  svla_config cfg;
+  int device = 0;
+  Layout lay;
+  uint16_t* w = nullptr;  // device weights (manifest order, gate/up rows interleaved)
+  float* b_t2_f32 = nullptr;
+  float2* rope_cs = nullptr;
+  int rope_max_pos = 0;
+  double* inv_period = nullptr;
+  int* status = nullptr;
+  // prefill workspace
+  float* p_x = nullptr;
+  bf16 *p_y = nullptr, *p_q = nullptr, *p_o = nullptr, *p_h = nullptr;
+  int* p_pos = nullptr;
+  float* p_part = nullptr;
+  int* p_cnt = nullptr;
+  // denoise workspace
+  float* e_r = nullptr;
+  bf16 *e_y = nullptr, *e_q = nullptr, *e_k = nullptr, *e_v = nullptr, *e_o = nullptr, *e_h = nullptr;
+  bf16 *e_a = nullptr, *e_h1 = nullptr, *kvx = nullptr;
+  float* e_c = nullptr;
+  float* e_part = nullptr;
+  int* e_cnt = nullptr;
+  float* noise_buf = nullptr;
+  cudaStream_t cap = nullptr;  // capture stream
+  std::list<GraphEntry> graphs;
+  std::vector<void*> allocs;
+  std::string last_error = "no error";
+
+  const bf16* W(size_t off) const { return reinterpret_cast<const bf16*>(w + off); }
+};
+
+namespace {
+
+constexpr size_t PART_BYTES = (size_t)NUM_SMS_B200 * GEMM_BM * 256 * sizeof(float);
+constexpr int CNT_INTS = 4096;
+
+svla_status fail(svla_handle* h, svla_status s, const std::string& msg) {
+  const std::string m = std::string(status_str(s)) + ": " + msg;
+  if (h) h->last_error = m;
+  t_last_error = m;
+  return s;
+}
+
+svla_status cuda_fail(svla_handle* h, cudaError_t e, const char* what) {
+  return fail(h, e == cudaErrorMemoryAllocation ? SVLA_ERR_OOM : SVLA_ERR_CUDA,
+              std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+template <typename T>
+cudaError_t halloc(svla_handle* h, T** p, size_t count) {
+  void* q = nullptr;
+  cudaError_t e = cudaMalloc(&q, count * sizeof(T) + 256);
+  if (e == cudaSuccess) {
+    h->allocs.push_back(q);
+    *p = reinterpret_cast<T*>(q);
+  }
+  return e;
+}
+
+void free_all(svla_handle* h) {
+  for (auto& g : h->graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  h->graphs.clear();
+  for (void* p : h->allocs) cudaFree(p);
+  h->allocs.clear();
+  if (h->cap) cudaStreamDestroy(h->cap);
+  h->cap = nullptr;
+}
+
+// one GEMM of the schedule
+cudaError_t gemm(svla_handle* h, int epi, const bf16* A, int lda, const bf16* W, int ldw, int M, int N, int K,
+                 GemmArgs args, float* part, int* cnt, cudaStream_t s) {
+  GemmPlan p = plan_gemm(M, N, K, 0);
+  args.status = h->status;
+  args.wait_ns = g_wait_ns.load();
+  return run_gemm(epi, A, lda, W, ldw, M, N, K, args, p, part, cnt, s);
+}
+
+GemmArgs out_args(void* out, int ldo, const float* bias = nullptr) {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.out = out;
+  a.ldo = ldo;
+  a.bias = bias;
+  return a;
+}
+
+cudaError_t rmsnorm(const void* x, bool x_bf16, float* x_copy, const bf16* g, int M, int D, float eps, bf16* y,
+                    cudaStream_t s) {
+  const int blocks = (M + 7) / 8;
+  if (x_bf16)
+    rmsnorm_kernel<true><<<blocks, 256, 0, s>>>(x, x_copy, g, M, D, eps, y);
+  else
+    rmsnorm_kernel<false><<<blocks, 256, 0, s>>>(x, nullptr, g, M, D, eps, y);
+  return cudaGetLastError();
+}
+
+cudaError_t attention(const bf16* q, int ldq, const bf16* k, const bf16* v, int ldkv, const uint8_t* valid, int B,
+                      int nq, int nkv, int hd, int Lq, int Lk, int causal, bf16* out, int ldo, cudaStream_t s) {
+  AttnArgs a;
+  a.q = q;
+  a.ldq = ldq;
+  a.k = k;
+  a.v = v;
+  a.ldkv = ldkv;
+  a.key_valid = valid;
+  a.out = out;
+  a.ldo = ldo;
+  a.n_q = nq;
+  a.n_kv = nkv;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.causal = causal;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)hd));
+  dim3 grid((Lq + ATT_BQ - 1) / ATT_BQ, nq, B);
+  if (hd == 64)
+    attention_kernel<64><<<grid, ATT_THREADS, AttnCfg<64>::SMEM, s>>>(a);
+  else
+    attention_kernel<32><<<grid, ATT_THREADS, AttnCfg<32>::SMEM, s>>>(a);
+  return cudaGetLastError();
+}
+
+#define SVLA_TRY(expr)                        \
+  do {                                        \
+    cudaError_t e_ = (expr);                  \
+    if (e_ != cudaSuccess) return e_;         \
+  } while (0)
+
+// ---- prefill schedule -------------------------------------------------------
+cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pad, int B, int L, void* kv,
+                           cudaStream_t s) {
+  const svla_config& c = h->cfg;
+  const int M = B * L, D = c.p_width, hd = c.head_dim;
+  const int qw = c.p_heads * hd, kvw = c.p_kv_heads * hd;
+  bf16* cache = reinterpret_cast<bf16*>(kv);
+  const size_t layer_elems = (size_t)B * L * kvw;
+  positions_kernel<<<(B + 7) / 8, 256, 0, s>>>(pad, B, L, h->p_pos, h->status);
+  SVLA_TRY(cudaGetLastError());
+  for (int l = 0; l < c.p_layers; ++l) {
+    const Entry* e = &h->lay.p[9 * l];
+    bf16* Kl = cache + (size_t)l * layer_elems;
+    bf16* Vl = cache + (size_t)(c.p_layers + l) * layer_elems;
+    if (l == 0)
+      SVLA_TRY(rmsnorm(embeds, true, h->p_x, h->W(e[0].off), M, D, c.rms_eps, h->p_y, s));
+    else
+      SVLA_TRY(rmsnorm(h->p_x, false, nullptr, h->W(e[0].off), M, D, c.rms_eps, h->p_y, s));
+    GemmArgs qa = out_args(nullptr, 0);
+    qa.q_out = h->p_q;
+    qa.ldq = qw;
+    qa.k_out = Kl;
+    qa.v_out = Vl;
+    qa.ldkv = kvw;
+    qa.q_cols = qw;
+    qa.kv_cols = kvw;
+    qa.pos = h->p_pos;
+    qa.pos_mod = 1;
+    qa.rope_cs = h->rope_cs;
+    SVLA_TRY(gemm(h, hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32, h->p_y, D, h->W(e[1].off), D, M, qw + 2 * kvw, D, qa,
+                  h->p_part, h->p_cnt, s));
+    if (l == c.p_layers - 1) break;  // nothing reads the last layer's attention / MLP output
+    SVLA_TRY(attention(h->p_q, qw, Kl, Vl, kvw, pad, B, c.p_heads, c.p_kv_heads, hd, L, L, 0, h->p_o, qw, s));
+    SVLA_TRY(gemm(h, GE_ADD_F32, h->p_o, qw, h->W(e[4].off), qw, M, D, qw, out_args(h->p_x, D), h->p_part, h->p_cnt, s));
+    SVLA_TRY(rmsnorm(h->p_x, false, nullptr, h->W(e[5].off), M, D, c.rms_eps, h->p_y, s));
+    SVLA_TRY(gemm(h, GE_SWIGLU, h->p_y, D, h->W(e[6].off), D, M, 2 * c.p_ffn, D, out_args(h->p_h, c.p_ffn), h->p_part,
+                  h->p_cnt, s));
+    SVLA_TRY(gemm(h, GE_ADD_F32, h->p_h, c.p_ffn, h->W(e[8].off), c.p_ffn, M, D, c.p_ffn, out_args(h->p_x, D),
+                  h->p_part, h->p_cnt, s));
+  }
+  return cudaSuccess;
+}
+
+// ---- denoise schedule -------------------------------------------------------
+cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise, int H,
+                           int n_steps, float* actions, float* trace, cudaStream_t s) {
+  const svla_config& c = h->cfg;
+  const int M = B * H, E = c.e_width, hd = c.head_dim, A = c.action_dim;
+  const int qw = c.e_heads * hd, kvw = c.e_kv_heads * hd, pkvw = c.p_kv_heads * hd;
+  const int Mp = B * L;
+  const bf16* cache = reinterpret_cast<const bf16*>(kv);
+  const size_t layer_elems = (size_t)Mp * pkvw;
+  if (actions != noise) SVLA_TRY(cudaMemcpyAsync(actions, noise, (size_t)M * A * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  // hoisted cross K/V projection (once per query, not per step)
+  for (int l = 1; l < c.e_layers; l += 2) {
+    const Entry* e = &h->lay.e[9 * l];
+    bf16* kx = h->kvx + (size_t)(l / 2) * 2 * Mp * kvw;
+    bf16* vx = kx + (size_t)Mp * kvw;
+    SVLA_TRY(gemm(h, GE_BF16, cache + (size_t)l * layer_elems, pkvw, h->W(e[2].off), pkvw, Mp, kvw, pkvw,
+                  out_args(kx, kvw), h->e_part, h->e_cnt, s));
+    SVLA_TRY(gemm(h, GE_BF16, cache + (size_t)(c.p_layers + l) * layer_elems, pkvw, h->W(e[3].off), pkvw, Mp, kvw,
+                  pkvw, out_args(vx, kvw), h->e_part, h->e_cnt, s));
+  }
+  const Layout& Lh = h->lay;
+  const int se_smem = (E * A + SE_WARPS * E) * (int)sizeof(float);
+  int se_blocks = (M + SE_WARPS - 1) / SE_WARPS;
+  if (se_blocks > 2 * NUM_SMS_B200) se_blocks = 2 * NUM_SMS_B200;
+  for (int k = 0; k < n_steps; ++k) {
+    StepBeginArgs sb;
+    sb.x = actions;
+    sb.M = M;
+    sb.A = A;
+    sb.De = E;
+    sb.w_in = h->W(Lh.w_in.off);
+    sb.b_in = h->W(Lh.b_in.off);
+    sb.w_t1 = h->W(Lh.w_t1.off);
+    sb.b_t1 = h->W(Lh.b_t1.off);
+    sb.inv_period = h->inv_period;
+    sb.step = k;
+    sb.n_steps = n_steps;
+    sb.a_out = h->e_a;
+    sb.c_out = h->e_c;
+    sb.nA = (M + 7) / 8;
+    step_begin_kernel<<<sb.nA + (E + 7) / 8, 256, 0, s>>>(sb);
+    SVLA_TRY(cudaGetLastError());
+    // time MLP: h1 = silu(W_t1[:, :E] a + c), r = W_t2 h1 + b_t2
+    SVLA_TRY(gemm(h, GE_SILU_BF16, h->e_a, E, h->W(Lh.w_t1.off), 2 * E, M, E, E, out_args(h->e_h1, E, h->e_c),
+                  h->e_part, h->e_cnt, s));
+    SVLA_TRY(gemm(h, GE_F32, h->e_h1, E, h->W(Lh.w_t2.off), E, M, E, E, out_args(h->e_r, E, h->b_t2_f32), h->e_part,
+                  h->e_cnt, s));
+    for (int l = 0; l < c.e_layers; ++l) {
+      const Entry* e = &Lh.e[9 * l];
+      SVLA_TRY(rmsnorm(h->e_r, false, nullptr, h->W(e[0].off), M, E, c.rms_eps, h->e_y, s));
+      if (l % 2 == 0) {
+        GemmArgs qa = out_args(nullptr, 0);
+        qa.q_out = h->e_q;
+        qa.ldq = qw;
+        qa.k_out = h->e_k;
+        qa.v_out = h->e_v;
+        qa.ldkv = kvw;
+        qa.q_cols = qw;
+        qa.kv_cols = kvw;
+        qa.pos = nullptr;
+        qa.pos_mod = H;  // chunk positions 0..H-1 (reading 4)
+        qa.rope_cs = h->rope_cs;
+        SVLA_TRY(gemm(h, hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32, h->e_y, E, h->W(e[1].off), E, M, qw + 2 * kvw, E,
+                      qa, h->e_part, h->e_cnt, s));
+        SVLA_TRY(attention(h->e_q, qw, h->e_k, h->e_v, kvw, nullptr, B, c.e_heads, c.e_kv_heads, hd, H, H, 1, h->e_o,
+                           qw, s));
+      } else {
+        SVLA_TRY(gemm(h, GE_BF16, h->e_y, E, h->W(e[1].off), E, M, qw, E, out_args(h->e_q, qw), h->e_part, h->e_cnt,
+                      s));
+        const bf16* kx = h->kvx + (size_t)(l / 2) * 2 * Mp * kvw;
+        SVLA_TRY(attention(h->e_q, qw, kx, kx + (size_t)Mp * kvw, kvw, pad, B, c.e_heads, c.e_kv_heads, hd, H, L, 0,
+                           h->e_o, qw, s));
+      }
+      SVLA_TRY(gemm(h, GE_ADD_F32, h->e_o, qw, h->W(e[4].off), qw, M, E, qw, out_args(h->e_r, E), h->e_part,
+                    h->e_cnt, s));
+      SVLA_TRY(rmsnorm(h->e_r, false, nullptr, h->W(e[5].off), M, E, c.rms_eps, h->e_y, s));
+      SVLA_TRY(gemm(h, GE_SWIGLU, h->e_y, E, h->W(e[6].off), E, M, 2 * c.e_ffn, E, out_args(h->e_h, c.e_ffn),
+                    h->e_part, h->e_cnt, s));
+      SVLA_TRY(gemm(h, GE_ADD_F32, h->e_h, c.e_ffn, h->W(e[8].off), c.e_ffn, M, E, c.e_ffn, out_args(h->e_r, E),
+                    h->e_part, h->e_cnt, s));
+    }
+    StepEndArgs se;
+    se.r = h->e_r;
+    se.M = M;
+    se.A = A;
+    se.De = E;
+    se.final_norm = h->W(Lh.final_norm.off);
+    se.w_out = h->W(Lh.w_out.off);
+    se.b_out = h->W(Lh.b_out.off);
+    se.eps = c.rms_eps;
+    se.dt = -1.0f / (float)n_steps;
+    se.x = actions;
+    se.trace_v = trace ? trace + (size_t)(2 * k) * M * A : nullptr;
+    se.trace_x = trace ? trace + (size_t)(2 * k + 1) * M * A : nullptr;
+    step_end_kernel<<<se_blocks, 256, se_smem, s>>>(se);
+    SVLA_TRY(cudaGetLastError());
+  }
+  return cudaSuccess;
+}
+
+// Capture `rec` on the handle's capture stream (cached by key) and launch on `s`.
+template <typename Rec>
+svla_status run_graph(svla_handle* h, const std::vector<uint64_t>& key, Rec rec, cudaStream_t s, const char* what) {
+  cudaGraphExec_t exec = nullptr;
+  for (auto it = h->graphs.begin(); it != h->graphs.end(); ++it) {
+    if (it->key == key) {
+      exec = it->exec;
+      h->graphs.splice(h->graphs.begin(), h->graphs, it);
+      break;
+    }
+  }
+  if (!exec) {
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaStreamBeginCapture");
+    cudaError_t er = rec(h->cap);
+    e = cudaStreamEndCapture(h->cap, &g);
+    if (er != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      return cuda_fail(h, er, what);
+    }
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaStreamEndCapture");
+    e = cudaGraphInstantiate(&exec, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaGraphInstantiate");
+    h->graphs.push_front(GraphEntry{key, exec});
+    while (h->graphs.size() > 16) {
+      cudaGraphExecDestroy(h->graphs.back().exec);
+      h->graphs.pop_back();
+    }
+  }
+  cudaError_t e = cudaGraphLaunch(exec, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaGraphLaunch");
+  return SVLA_OK;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    int cur;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+const char* svla_status_string(svla_status s) { return status_str(s); }
+
+const char* svla_last_error(const svla_handle* h) {
+  return h ? h->last_error.c_str() : t_last_error.c_str();
+}
+
+void svla_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns); }
+
+size_t svla_blob_bytes(const svla_config* cfg) {
+  if (!cfg || check_config(*cfg)) return 0;
+  return make_layout(*cfg).total * 2;
+}
+
+svla_status svla_create(const svla_config* cfg, const void* blob, size_t blob_bytes, int device, svla_handle** out) {
+  if (out) *out = nullptr;
+  if (!cfg || !blob || !out) return fail(nullptr, SVLA_ERR_ARG, "null argument");
+  if (const char* why = check_config(*cfg)) return fail(nullptr, SVLA_ERR_SHAPE, why);
+  Layout lay = make_layout(*cfg);
+  if (blob_bytes != lay.total * 2)
+    return fail(nullptr, SVLA_ERR_BLOB_SIZE,
+                "blob has " + std::to_string(blob_bytes) + " bytes, manifest needs " + std::to_string(lay.total * 2));
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev)
+    return fail(nullptr, SVLA_ERR_UNSUPPORTED, "no such CUDA device");
+  if (!device_is_sm100(device)) return fail(nullptr, SVLA_ERR_UNSUPPORTED, "device is not sm_100 (B200)");
+  DeviceGuard dg(device);
+  if (cudaError_t e = ensure_attrs(device); e != cudaSuccess) return cuda_fail(nullptr, e, "kernel attributes");
+
+  svla_handle* h = new svla_handle();
+  h->cfg = *cfg;
+  h->device = device;
+  h->lay = lay;
+  const svla_config& c = *cfg;
+  auto bail = [&](cudaError_t e, const char* what) {
+    svla_status st = cuda_fail(nullptr, e, what);
+    cudaDeviceSynchronize();
+    free_all(h);
+    delete h;
+    return st;
+  };
+  cudaError_t e;
+  if ((e = halloc(h, &h->w, lay.total)) != cudaSuccess) return bail(e, "weights");
+  if ((e = cudaMemcpy(h->w, blob, blob_bytes, cudaMemcpyDefault)) != cudaSuccess) return bail(e, "weight copy");
+  // gate/up rows -> interleaved 32-row groups [gate | up], in place via a scratch copy
+  {
+    size_t max_gu = std::max((size_t)2 * c.p_ffn * c.p_width, (size_t)2 * c.e_ffn * c.e_width);
+    uint16_t* tmp = nullptr;
+    if ((e = cudaMalloc(&tmp, max_gu * 2)) != cudaSuccess) return bail(e, "scratch");
+    for (int l = 0; l < c.p_layers + c.e_layers && e == cudaSuccess; ++l) {
+      const bool pre = l < c.p_layers;
+      const Entry& g = pre ? lay.p[9 * l + 6] : lay.e[9 * (l - c.p_layers) + 6];
+      const int F = pre ? c.p_ffn : c.e_ffn, K = pre ? c.p_width : c.e_width;
+      e = cudaMemcpy(tmp, h->w + g.off, (size_t)2 * F * K * 2, cudaMemcpyDeviceToDevice);
+      if (e == cudaSuccess) {
+        interleave_gu_kernel<<<2 * F, 256>>>(tmp, h->w + g.off, F, K);
+        e = cudaGetLastError();
+      }
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    cudaFree(tmp);
+    if (e != cudaSuccess) return bail(e, "gate/up layout");
+  }
+  if ((e = halloc(h, &h->b_t2_f32, c.e_width)) != cudaSuccess) return bail(e, "bias");
+  bf16_to_f32_kernel<<<(c.e_width + 255) / 256, 256>>>(h->w + lay.b_t2.off, h->b_t2_f32, c.e_width);
+  // RoPE table (reading 3), computed in double on the host
+  {
+    h->rope_max_pos = std::max(c.max_prefix, c.max_chunk);
+    const int half = c.head_dim / 2;
+    std::vector<float2> cs((size_t)h->rope_max_pos * half);
+    for (int p = 0; p < h->rope_max_pos; ++p)
+      for (int i = 0; i < half; ++i) {
+        const double ang = (double)p * std::pow((double)c.rope_base, -2.0 * i / c.head_dim);
+        cs[(size_t)p * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+      }
+    if ((e = halloc(h, &h->rope_cs, cs.size())) != cudaSuccess) return bail(e, "rope");
+    if ((e = cudaMemcpy(h->rope_cs, cs.data(), cs.size() * sizeof(float2), cudaMemcpyHostToDevice)) != cudaSuccess)
+      return bail(e, "rope copy");
+    // sinusoid periods (reading 12)
+    const int th = c.e_width / 2;
+    std::vector<double> ip(th);
+    for (int i = 0; i < th; ++i) {
+      const double frac = th > 1 ? (double)i / (th - 1) : 0.0;
+      ip[i] = 1.0 / ((double)c.t_min_period * std::pow((double)c.t_max_period / c.t_min_period, frac));
+    }
+    if ((e = halloc(h, &h->inv_period, th)) != cudaSuccess) return bail(e, "periods");
+    if ((e = cudaMemcpy(h->inv_period, ip.data(), th * sizeof(double), cudaMemcpyHostToDevice)) != cudaSuccess)
+      return bail(e, "periods copy");
+  }
+  if ((e = halloc(h, &h->status, 1)) != cudaSuccess) return bail(e, "status");
+  cudaMemset(h->status, 0, sizeof(int));
+  // workspaces
+  const size_t Mp = (size_t)c.max_batch * c.max_prefix, Me = (size_t)c.max_batch * c.max_chunk;
+  const size_t pq = (size_t)c.p_heads * c.head_dim, eq = (size_t)c.e_heads * c.head_dim;
+  const size_t ekv = (size_t)c.e_kv_heads * c.head_dim;
+  if ((e = halloc(h, &h->p_x, Mp * c.p_width)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->p_y, Mp * c.p_width)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->p_q, Mp * pq)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->p_o, Mp * pq)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->p_h, Mp * c.p_ffn)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->p_pos, Mp)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_r, Me * c.e_width)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_y, Me * c.e_width)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_q, Me * eq)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_k, Me * ekv)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_v, Me * ekv)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_o, Me * eq)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_h, Me * c.e_ffn)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_a, Me * c.e_width)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_h1, Me * c.e_width)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_c, (size_t)c.e_width)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->kvx, (size_t)((c.e_layers + 1) / 2) * 2 * Mp * ekv)) != cudaSuccess)
+    return bail(e, "workspace");
+  if ((e = halloc(h, &h->noise_buf, Me * c.action_dim)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, reinterpret_cast<uint8_t**>(&h->p_part), PART_BYTES)) != cudaSuccess) return bail(e, "split-K");
+  if ((e = halloc(h, reinterpret_cast<uint8_t**>(&h->e_part), PART_BYTES)) != cudaSuccess) return bail(e, "split-K");
+  if ((e = halloc(h, &h->p_cnt, CNT_INTS)) != cudaSuccess) return bail(e, "split-K");
+  if ((e = halloc(h, &h->e_cnt, CNT_INTS)) != cudaSuccess) return bail(e, "split-K");
+  cudaMemset(h->p_cnt, 0, CNT_INTS * sizeof(int));
+  cudaMemset(h->e_cnt, 0, CNT_INTS * sizeof(int));
+  if ((e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking)) != cudaSuccess) return bail(e, "stream");
+  if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(e, "create");
+  *out = h;
+  return SVLA_OK;
+}
+
+svla_status svla_destroy(svla_handle* h) {
+  if (!h) return SVLA_OK;
+  DeviceGuard dg(h->device);
+  cudaDeviceSynchronize();
+  free_all(h);
+  delete h;
+  return SVLA_OK;
+}
+
+size_t svla_kv_cache_bytes(const svla_handle* h, int B, int L) {
+  if (!h || B < 1 || L < 1) return 0;
+  return (size_t)2 * h->cfg.p_layers * B * L * h->cfg.p_kv_heads * h->cfg.head_dim * 2;
+}
+
+svla_status svla_prefill(svla_handle* h, const void* embeds, const uint8_t* pad, int B, int L, void* kv,
+                         void* stream) {
+  if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
+  if (!embeds || !pad || !kv) return fail(h, SVLA_ERR_ARG, "null pointer");
+  if (B < 1 || L < 1 || B > h->cfg.max_batch || L > h->cfg.max_prefix)
+    return fail(h, SVLA_ERR_SHAPE, "B or L outside [1, max_batch] x [1, max_prefix]");
+  DeviceGuard dg(h->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  std::vector<uint64_t> key = {1, (uint64_t)B, (uint64_t)L, (uint64_t)(uintptr_t)embeds, (uint64_t)(uintptr_t)pad,
+                               (uint64_t)(uintptr_t)kv, g_wait_ns.load()};
+  return run_graph(h, key, [&](cudaStream_t cs) { return record_prefill(h, embeds, pad, B, L, kv, cs); }, s,
+                   "prefill");
+}
+
+svla_status svla_denoise(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise, int H,
+                         int n_steps, float* actions, float* trace, void* stream) {
+  if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
+  if (!kv || !pad || !noise || !actions) return fail(h, SVLA_ERR_ARG, "null pointer");
+  if (B < 1 || L < 1 || B > h->cfg.max_batch || L > h->cfg.max_prefix)
+    return fail(h, SVLA_ERR_SHAPE, "B or L outside [1, max_batch] x [1, max_prefix]");
+  if (H < 1 || H > h->cfg.max_chunk) return fail(h, SVLA_ERR_SHAPE, "H outside [1, max_chunk]");
+  if (n_steps < 1 || n_steps > 1000) return fail(h, SVLA_ERR_SHAPE, "n_steps outside [1, 1000]");
+  DeviceGuard dg(h->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  std::vector<uint64_t> key = {2, (uint64_t)B, (uint64_t)L, (uint64_t)H, (uint64_t)n_steps,
+                               (uint64_t)(uintptr_t)kv, (uint64_t)(uintptr_t)pad, (uint64_t)(uintptr_t)noise,
+                               (uint64_t)(uintptr_t)actions, (uint64_t)(uintptr_t)trace, g_wait_ns.load()};
+  return run_graph(
+      h, key, [&](cudaStream_t cs) { return record_denoise(h, kv, pad, B, L, noise, H, n_steps, actions, trace, cs); },
+      s, "denoise");
+}
+
+svla_status svla_sample(svla_handle* h, const void* embeds, const uint8_t* pad, int B, int L, uint64_t seed, int H,
+                        int n_steps, void* kv, float* noise_out, float* actions, void* stream) {
+  if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
+  if (!embeds || !pad || !kv || !actions) return fail(h, SVLA_ERR_ARG, "null pointer");
+  if (B < 1 || L < 1 || B > h->cfg.max_batch || L > h->cfg.max_prefix)
+    return fail(h, SVLA_ERR_SHAPE, "B or L outside [1, max_batch] x [1, max_prefix]");
+  if (H < 1 || H > h->cfg.max_chunk) return fail(h, SVLA_ERR_SHAPE, "H outside [1, max_chunk]");
+  if (n_steps < 1 || n_steps > 1000) return fail(h, SVLA_ERR_SHAPE, "n_steps outside [1, 1000]");
+  DeviceGuard dg(h->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* noise = noise_out ? noise_out : h->noise_buf;
+  const int n_el = H * h->cfg.action_dim;
+  const long long threads = (long long)B * ((n_el + 3) / 4);
+  philox_noise_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>((unsigned long long)seed, B, n_el, noise);
+  if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return cuda_fail(h, e, "noise");
+  svla_status st = svla_prefill(h, embeds, pad, B, L, kv, stream);
+  if (st != SVLA_OK) return st;
+  return svla_denoise(h, kv, pad, B, L, noise, H, n_steps, actions, nullptr, stream);
+}
+
+svla_status svla_device_status(svla_handle* h, void* stream) {
+  if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
+  DeviceGuard dg(h->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(h, e, "device status");
+  if (v != 0) return fail(h, v, "device-side error");
+  return SVLA_OK;
+}
+
+// ---- kernel-level entry points ---------------------------------------------
+static int epi_code(int epi) {
+  switch (epi) {
+    case SVLA_EPI_F32: return GE_F32;
+    case SVLA_EPI_BF16: return GE_BF16;
+    case SVLA_EPI_ADD_F32: return GE_ADD_F32;
+    case SVLA_EPI_SILU_BF16: return GE_SILU_BF16;
+  }
+  return -1;
+}
+
+int svla_op_gemm_splits(int M, int N, int K) {
+  if (M < 1 || N < 1 || K < 1) return 0;
+  return plan_gemm(M, N, K, 0).splits;
+}
+
+static size_t cnt_bytes(const GemmPlan& p) { return (((size_t)p.m_tiles * p.n_tiles * sizeof(int)) + 255) / 256 * 256; }
+
+size_t svla_op_gemm_workspace_bytes(int M, int N, int K, int splits) {
+  if (M < 1 || N < 1 || K < 1 || splits < 0) return 0;
+  GemmPlan p = plan_gemm(M, N, K, splits);
+  if (p.splits <= 1) return 0;
+  return cnt_bytes(p) + gemm_partials_bytes(p);
+}
+
+svla_status svla_op_gemm(int epilogue, const void* A, int lda, const void* W, int ldw, int M, int N, int K, void* C,
+                         int ldc, const float* bias, int splits, void* workspace, size_t workspace_bytes, int* status,
+                         void* stream) {
+  const int epi = epi_code(epilogue);
+  if (epi < 0) return fail(nullptr, SVLA_ERR_ARG, "unknown epilogue");
+  if (!A || !W || !C) return fail(nullptr, SVLA_ERR_ARG, "null pointer");
+  if (M < 1 || N < 1 || K < 1 || splits < 0 || lda < K || ldw < K || ldc < N || lda % 8 || ldw % 8 ||
+      (epi != GE_F32 && epi != GE_ADD_F32 ? ldc % 8 : ldc % 4))
+    return fail(nullptr, SVLA_ERR_SHAPE, "bad sizes or strides");
+  if (((uintptr_t)A | (uintptr_t)W | (uintptr_t)C) & 15) return fail(nullptr, SVLA_ERR_ARG, "pointers must be 16-byte aligned");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!device_is_sm100(dev)) return fail(nullptr, SVLA_ERR_UNSUPPORTED, "device is not sm_100 (B200)");
+  if (cudaError_t e = ensure_attrs(dev); e != cudaSuccess) return cuda_fail(nullptr, e, "kernel attributes");
+  GemmPlan p = plan_gemm(M, N, K, splits);
+  float* part = nullptr;
+  int* cnt = nullptr;
+  if (p.splits > 1) {
+    const size_t need = cnt_bytes(p) + gemm_partials_bytes(p);
+    if (!workspace || workspace_bytes < need) return fail(nullptr, SVLA_ERR_ARG, "workspace missing or too small");
+    cnt = reinterpret_cast<int*>(workspace);
+    part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + cnt_bytes(p));
+  }
+  GemmArgs a = out_args(C, ldc, bias);
+  a.status = status;
+  a.wait_ns = g_wait_ns.load();
+  cudaError_t e = run_gemm(epi, A, lda, W, ldw, M, N, K, a, p, part, cnt, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(nullptr, e, "gemm launch");
+  return SVLA_OK;
+}
+
+svla_status svla_op_attention(const void* q, int ldq, const void* k, const void* v, int ldkv, const uint8_t* key_valid,
+                              int B, int n_q, int n_kv, int hd, int Lq, int Lk, int causal, void* out, int ldo,
+                              void* stream) {
+  if (!q || !k || !v || !out) return fail(nullptr, SVLA_ERR_ARG, "null pointer");
+  if (hd != 32 && hd != 64) return fail(nullptr, SVLA_ERR_SHAPE, "hd must be 32 or 64");
+  if (B < 1 || n_q < 1 || n_kv < 1 || n_q % n_kv || Lq < 1 || Lk < 1 || ldq < n_q * hd || ldkv < n_kv * hd ||
+      ldo < n_q * hd || ldq % 8 || ldkv % 8 || ldo % 2)
+    return fail(nullptr, SVLA_ERR_SHAPE, "bad sizes or strides");
+  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v) & 15) return fail(nullptr, SVLA_ERR_ARG, "pointers must be 16-byte aligned");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (cudaError_t e = ensure_attrs(dev); e != cudaSuccess) return cuda_fail(nullptr, e, "kernel attributes");
+  cudaError_t e = attention(reinterpret_cast<const bf16*>(q), ldq, reinterpret_cast<const bf16*>(k),
+                            reinterpret_cast<const bf16*>(v), ldkv, key_valid, B, n_q, n_kv, hd, Lq, Lk, causal,
+                            reinterpret_cast<bf16*>(out), ldo, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(nullptr, e, "attention launch");
+  return SVLA_OK;
+}
+
+svla_status svla_op_rmsnorm(const float* x, const void* g, int M, int D, float eps, void* y, void* stream) {
+  if (!x || !g || !y) return fail(nullptr, SVLA_ERR_ARG, "null pointer");
+  if (M < 1 || D < 4 || D % 4 || D > 2048 || !(eps > 0.f)) return fail(nullptr, SVLA_ERR_SHAPE, "bad sizes");
+  cudaError_t e = rmsnorm(x, false, nullptr, reinterpret_cast<const bf16*>(g), M, D, eps, reinterpret_cast<bf16*>(y),
+                          reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(nullptr, e, "rmsnorm launch");
+  return SVLA_OK;
+}
+
+}  // extern "C"

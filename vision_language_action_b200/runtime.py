@@ -1,0 +1,130 @@
+"""Python face of libsvla: argument marshalling over the C ABI, nothing else.
+
+Every step of the path runs in the library's CUDA kernels; torch is used only
+to own device memory and to name the current CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import torch
+
+from . import _abi
+
+__all__ = ["SmolVLA", "config_from_shape"]
+
+
+def config_from_shape(shape, max_batch: int, max_prefix: int, max_chunk: int) -> _abi.SvlaConfig:
+    """Build an svla_config from any object with the model-shape attributes."""
+    c = _abi.SvlaConfig()
+    for name, _ in _abi.SvlaConfig._fields_:
+        if name in ("max_batch", "max_prefix", "max_chunk"):
+            continue
+        setattr(c, name, getattr(shape, name))
+    c.max_batch, c.max_prefix, c.max_chunk = max_batch, max_prefix, max_chunk
+    return c
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors passed to libsvla must be contiguous CUDA tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class SmolVLA:
+    """One svla_handle: weights on one GPU plus the workspace for the limits given.
+
+    ``blob`` is the flat bf16 weight blob in manifest order, as a numpy uint16
+    array, a torch uint16/bfloat16 tensor (host or CUDA), or raw bytes.
+    """
+
+    def __init__(self, shape, blob, max_batch: int, max_prefix: int, max_chunk: int,
+                 device: int = 0):
+        self.lib = _abi.load()
+        self.cfg = config_from_shape(shape, max_batch, max_prefix, max_chunk)
+        self.action_dim = shape.action_dim
+        self.device = device
+        if isinstance(blob, torch.Tensor):
+            t = blob.contiguous()
+            ptr, nbytes = t.data_ptr(), t.numel() * t.element_size()
+            self._blob_keep = t
+        else:
+            import numpy as np
+            arr = np.ascontiguousarray(blob)
+            ptr, nbytes = arr.ctypes.data, arr.nbytes
+            self._blob_keep = arr
+        h = ctypes.c_void_p()
+        st = self.lib.svla_create(ctypes.byref(self.cfg), ctypes.c_void_p(ptr), nbytes, device,
+                                  ctypes.byref(h))
+        self._blob_keep = None
+        _abi.check(st, None)
+        self.h = h
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            self.lib.svla_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------------
+    def kv_cache_bytes(self, B: int, L: int) -> int:
+        return int(self.lib.svla_kv_cache_bytes(self.h, B, L))
+
+    def new_kv_cache(self, B: int, L: int) -> torch.Tensor:
+        """A K/V cache buffer: bf16, [2, p_layers, B, L, p_kv_heads * head_dim]."""
+        c = self.cfg
+        return torch.empty((2, c.p_layers, B, L, c.p_kv_heads * c.head_dim), dtype=torch.bfloat16,
+                           device=f"cuda:{self.device}")
+
+    def prefill(self, embeds: torch.Tensor, pad_mask: torch.Tensor,
+                kv_cache: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        B, L = pad_mask.shape
+        if kv_cache is None:
+            kv_cache = self.new_kv_cache(B, L)
+        st = self.lib.svla_prefill(self.h, _ptr(embeds), _ptr(pad_mask), B, L, _ptr(kv_cache), _stream(stream))
+        _abi.check(st, self.h)
+        return kv_cache
+
+    def denoise(self, kv_cache: torch.Tensor, pad_mask: torch.Tensor, noise: torch.Tensor, n_steps: int,
+                actions: Optional[torch.Tensor] = None, trace: bool = False,
+                stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+        B, H, A = noise.shape
+        L = pad_mask.shape[1]
+        if actions is None:
+            actions = torch.empty_like(noise)
+        tr = None
+        if trace:
+            tr = torch.empty((n_steps, 2, B, H, A), dtype=torch.float32, device=noise.device)
+        st = self.lib.svla_denoise(self.h, _ptr(kv_cache), _ptr(pad_mask), B, L, _ptr(noise), H, n_steps,
+                                   _ptr(actions), _ptr(tr), _stream(stream))
+        _abi.check(st, self.h)
+        return actions, tr
+
+    def sample(self, embeds: torch.Tensor, pad_mask: torch.Tensor, seed: int, H: int, n_steps: int,
+               kv_cache: Optional[torch.Tensor] = None, return_noise: bool = False, stream=None):
+        B, L = pad_mask.shape
+        if kv_cache is None:
+            kv_cache = self.new_kv_cache(B, L)
+        actions = torch.empty((B, H, self.action_dim), dtype=torch.float32, device=embeds.device)
+        noise = torch.empty_like(actions) if return_noise else None
+        st = self.lib.svla_sample(self.h, _ptr(embeds), _ptr(pad_mask), B, L, seed, H, n_steps,
+                                  _ptr(kv_cache), _ptr(noise), _ptr(actions), _stream(stream))
+        _abi.check(st, self.h)
+        return (actions, kv_cache, noise) if return_noise else (actions, kv_cache)
+
+    def device_status(self, stream=None) -> int:
+        """Synchronise the stream; return (and clear) the device-side status."""
+        return int(self.lib.svla_device_status(self.h, _stream(stream)))
