@@ -132,33 +132,57 @@ SVLA_DEV void add_bias16(float (&v)[16], const float* bias, int col, int N) {
 }
 
 // Fetches 16 accumulator columns [c, c+16) of this thread's row: from TMEM,
-// or (split-K reducer) the sum of the partial tiles in split order.
+// or (split-K reducer) from the reduced tile staged in shared memory.
 template <int BN>
 struct AccSource {
   uint32_t taddr_row;
-  const float* part_row;  // partials of split 0, this row; next split at +split_stride
-  size_t split_stride;
-  int splits;
+  const float* smem_row;  // null: read TMEM
   SVLA_DEV void get(int c, float (&v)[16]) const {
-    if (splits == 1) {
+    if (smem_row == nullptr) {
       tmem_ld16(taddr_row + (uint32_t)c, v);
     } else {
+      const float4* p = reinterpret_cast<const float4*>(smem_row + c);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = 0.f;
-      for (int z = 0; z < splits; ++z) {
-        const float4* p = reinterpret_cast<const float4*>(part_row + z * split_stride + c);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float4 t = __ldcg(p + i);
-          v[4 * i] += t.x;
-          v[4 * i + 1] += t.y;
-          v[4 * i + 2] += t.z;
-          v[4 * i + 3] += t.w;
-        }
+      for (int i = 0; i < 4; ++i) {
+        const float4 t = p[i];
+        v[4 * i] = t.x;
+        v[4 * i + 1] = t.y;
+        v[4 * i + 2] = t.z;
+        v[4 * i + 3] = t.w;
       }
     }
   }
 };
+
+// Split-K reduction by the last CTA of a tile: the 128 epilogue threads sum
+// the partial tiles [split][128][BN] in split order (coalesced float4 loads,
+// all splits in flight) into a shared-memory tile [128][BN + 4].
+template <int BN>
+SVLA_DEV void reduce_partials(const float* tile_part, int splits, int rows, float* red, int t) {
+  constexpr int V4 = BN / 4;
+  const int nvec = rows * V4;
+  const size_t sstride = (size_t)GEMM_BM * BN / 4;
+  const float4* part = reinterpret_cast<const float4*>(tile_part);
+  for (int idx = t; idx < nvec; idx += 128) {
+    const int r = idx / V4, c4 = idx % V4;
+    const float4* p = part + (size_t)r * V4 + c4;
+    float4 acc = __ldcg(p);
+    int z = 1;
+    for (; z + 3 < splits; z += 4) {
+      const float4 a = __ldcg(p + z * sstride), b = __ldcg(p + (z + 1) * sstride);
+      const float4 c = __ldcg(p + (z + 2) * sstride), d = __ldcg(p + (z + 3) * sstride);
+      acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
+      acc.x += b.x; acc.y += b.y; acc.z += b.z; acc.w += b.w;
+      acc.x += c.x; acc.y += c.y; acc.z += c.z; acc.w += c.w;
+      acc.x += d.x; acc.y += d.y; acc.z += d.z; acc.w += d.w;
+    }
+    for (; z < splits; ++z) {
+      const float4 a = __ldcg(p + z * sstride);
+      acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
+    }
+    *reinterpret_cast<float4*>(red + r * (BN + 4) + 4 * c4) = acc;
+  }
+}
 
 template <int BN, int EPI>
 SVLA_DEV void run_epilogue(const GemmArgs& a, const AccSource<BN>& src, int m, int n0, bool row_ok) {
@@ -362,9 +386,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (ok && !aborted) {
       AccSource<BN> src;
       src.taddr_row = tmem_base + ((uint32_t)(quad * 32) << 16);
-      src.splits = 1;
-      src.part_row = nullptr;
-      src.split_stride = 0;
+      src.smem_row = nullptr;
       if (splits == 1) {
         run_epilogue<BN, EPI>(args, src, m, n0, row_ok);
       } else {
@@ -385,10 +407,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         epi_bar();
         if (misc[4]) {
+          // 2) last CTA: sum all splits in split order into shared memory (the
+          //    operand ring is idle now), then run the epilogue from there
           __threadfence();
-          src.splits = splits;
-          src.part_row = tile_part + (size_t)row * BN;
-          src.split_stride = (size_t)GEMM_BM * BN;
+          float* red = reinterpret_cast<float*>(ring);
+          const int rows = min(GEMM_BM, args.M - m_blk * GEMM_BM);
+          reduce_partials<BN>(tile_part, splits, rows, red, threadIdx.x - 64);
+          epi_bar();
+          src.smem_row = red + row * (BN + 4);
           run_epilogue<BN, EPI>(args, src, m, n0, row_ok);
           if (threadIdx.x == 64) args.counters[tile] = 0;  // re-arm for the next launch
         }

@@ -66,9 +66,9 @@ cudaError_t ensure_attrs(int dev) {
 }
 
 bool device_is_sm100(int dev) {
-  cudaDeviceProp p;
-  if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return false;
-  return p.major == 10;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  return major == 10;
 }
 
 // ---- manifest -------------------------------------------------------------
