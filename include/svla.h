@@ -196,6 +196,31 @@ SVLA_API svla_status svla_op_attention(const void* q, int ldq, const void* k, co
 SVLA_API svla_status svla_op_rmsnorm(const float* x, const void* g, int M, int D, float eps,
                             void* y, void* stream);
 
+/* svla_op_gemm without a workspace argument, for callers that cannot allocate
+ * GPU memory themselves: code that must not call cudaMalloc once it is running
+ * (a robot control loop that forbids allocation after start-up because its
+ * latency is unpredictable), a host that owns all device memory through its
+ * own pool, or a plain-C caller with no allocator of its own. This entry point
+ * has no counterpart in the paper; it exists only for these callers.
+ *   Same arguments and results as svla_op_gemm, minus the workspace. The
+ *   split-K scratch is a fixed device array of SVLA_NOALLOC_SCRATCH_BYTES
+ *   (8 MiB) in the library, present on every GPU that loads it until the
+ *   process exits. A GEMM whose plan needs more scratch than that
+ *   (svla_op_gemm_workspace_bytes(M, N, K, splits) > 8 MiB) is rejected with
+ *   SVLA_ERR_SHAPE and a message naming both sizes; nothing is launched.
+ *   The first call on a device resolves the array's device address and zeroes
+ *   it synchronously, so make that first call before any stream capture. Each
+ *   later call clears the counter part of the scratch on `stream` before its
+ *   launch. The function never calls cudaMalloc, cudaFree or any allocating
+ *   library routine.
+ *   All calls on a device share the one scratch array: calls whose kernels
+ *   overlap on the GPU (different streams, or several host threads) race and
+ *   may give wrong results; issue them in one stream order. */
+#define SVLA_NOALLOC_SCRATCH_BYTES (8u << 20)
+SVLA_API svla_status svla_op_gemm_noalloc(int epilogue, const void* A, int lda, const void* W, int ldw,
+                                          int M, int N, int K, void* C, int ldc, const float* bias,
+                                          int splits, int* status, void* stream);
+
 /* Set the limit, in nanoseconds, of every device-side bounded wait of later
  * launches (default 1e9). A limit of 0 makes any wait that is not already
  * satisfied give up at once and report SVLA_ERR_TIMEOUT; it exists to test

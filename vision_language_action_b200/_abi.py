@@ -47,6 +47,7 @@ SIGNATURES = {
     "svla_last_error": (ctypes.c_char_p, [_P]),
     "svla_status_string": (ctypes.c_char_p, [_I]),
     "svla_op_gemm": (_I, [_I, _P, _I, _P, _I, _I, _I, _I, _P, _I, _P, _I, _P, _S, _P, _P]),
+    "svla_op_gemm_noalloc": (_I, [_I, _P, _I, _P, _I, _I, _I, _I, _P, _I, _P, _I, _P, _P]),
     "svla_op_gemm_workspace_bytes": (_S, [_I, _I, _I, _I]),
     "svla_op_gemm_splits": (_I, [_I, _I, _I]),
     "svla_op_attention": (_I, [_P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P]),

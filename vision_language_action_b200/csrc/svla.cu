@@ -485,6 +485,10 @@ struct DeviceGuard {
 
 }  // namespace
 
+// Library-internal (hidden): lets another translation unit of libsvla report
+// an error through svla_last_error(NULL).
+svla_status svla_internal_fail(svla_status s, const char* msg) { return fail(nullptr, s, msg); }
+
 // ============================================================================
 // C ABI
 // ============================================================================
