@@ -250,56 +250,64 @@ def time_steps(fn, steps, warmup, barrier):
 
 
 def gemm_roofline(s, B, L, H, n_steps, dev, hbm_peak):
-    """Live CUDA-event timing of the GEMM kernel over one chunk's GEMM launches
-    (same shapes and tile/split plans as the schedule; distinct weight buffers
-    per launch, so nothing is served from L2 that the path would not)."""
+    """Live CUDA-event timing of the GEMM kernel over one chunk's GEMM launches.
+
+    The launches of the prefill (+ hoisted cross K/V projection) and of one
+    denoise step are captured, with the same shapes and tile/split plans as the
+    path and distinct weight buffers per launch (nothing is served from L2 that
+    the path would not), into two CUDA graphs that are replayed back to back
+    (PDL-chained like the path) and timed with events on the launch stream.
+    achieved = algorithmic bytes of a chunk's GEMMs / their time per chunk."""
     import ctypes
     import torch
     from vision_language_action_b200 import _abi
     lib = _abi.load()
-    launches = gemm_list(s, B, L, H, 1)   # prefill + hoist + one denoise step
-    n_pre = len(gemm_list(s, B, L, H, 0))
-    acts = {}
-    ws_bytes = max(lib.svla_op_gemm_workspace_bytes(M, N, K, 0) for M, N, K, _, _ in launches)
-    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    plans = []
-    for i, (M, N, K, ob, rmw) in enumerate(launches):
-        W = torch.randn(N, K, device=dev).to(torch.bfloat16)
-        key = (M, K)
-        if key not in acts:
-            acts[key] = torch.randn(M, K, device=dev).to(torch.bfloat16)
-        C = torch.empty(M, N, device=dev, dtype=torch.float32 if ob == 4 else torch.bfloat16)
-        epi = _abi.EPI_ADD_F32 if rmw else (_abi.EPI_F32 if ob == 4 else _abi.EPI_BF16)
-        plans.append((epi, acts[key], W, C, M, N, K, gemm_bytes(M, N, K, ob, rmw)))
-    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    pre = gemm_list(s, B, L, H, 0)
+    step = gemm_list(s, B, L, H, 1)[len(pre):]
+
+    def build(launches):
+        acts, plans = {}, []
+        for (M, N, K, ob, rmw) in launches:
+            W = torch.randn(N, K, device=dev).to(torch.bfloat16)
+            if (M, K) not in acts:
+                acts[(M, K)] = torch.randn(M, K, device=dev).to(torch.bfloat16)
+            C = torch.zeros(M, N, device=dev, dtype=torch.float32 if ob == 4 else torch.bfloat16)
+            epi = _abi.EPI_ADD_F32 if rmw else (_abi.EPI_F32 if ob == 4 else _abi.EPI_BF16)
+            plans.append((epi, acts[(M, K)], W, C, M, N, K))
+        return plans
+
     P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
 
-    def launch(p):
-        epi, A, W, C, M, N, K, _ = p
-        _abi.check(lib.svla_op_gemm(epi, P(A), K, P(W), K, M, N, K, P(C), N, None, 0, P(ws), ws_bytes, None, stream))
+    def run(plans):
+        st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        for epi, A, W, C, M, N, K in plans:
+            _abi.check(lib.svla_op_gemm(epi, P(A), K, P(W), K, M, N, K, P(C), N, None, 0, None, 0, None, st))
 
-    for p in plans:
-        launch(p)
-    torch.cuda.synchronize()
-    reps = 5
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in plans]
-    dur = np.zeros(len(plans))
-    for _ in range(reps):
-        for p, (a, b) in zip(plans, ev):
-            a.record()
-            launch(p)
-            b.record()
-        torch.cuda.synchronize()
-        dur += np.array([a.elapsed_time(b) for a, b in ev])
-    dur /= reps
-    # one chunk = prefill GEMMs + hoist + n_steps x step GEMMs
-    t_pre = dur[:n_pre].sum()
-    t_step = dur[n_pre:].sum()
-    b_pre = sum(p[7] for p in plans[:n_pre])
-    b_step = sum(p[7] for p in plans[n_pre:])
+    def graph_time(plans, reps=10):
+        cs = torch.cuda.Stream()
+        with torch.cuda.stream(cs):
+            run(plans)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cs):
+                run(plans)
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(cs)
+            for _ in range(reps):
+                g.replay()
+            e1.record(cs)
+            torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    t_pre = graph_time(build(pre))
+    t_step = graph_time(build(step))
+    b_pre = sum(gemm_bytes(*x) for x in pre)
+    b_step = sum(gemm_bytes(*x) for x in step)
     t_chunk = t_pre + n_steps * t_step
     bytes_chunk = b_pre + n_steps * b_step
-    n_launch = n_pre + n_steps * (len(plans) - n_pre)
+    n_launch = len(pre) + n_steps * len(step)
     achieved = bytes_chunk / (t_chunk * 1e-3) / 1e9
     return {"bound": "hbm", "kernel": "gemm_tc_kernel", "achieved": round(achieved, 1), "peak": hbm_peak,
             "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),

@@ -100,11 +100,13 @@ def test_gemm_plan_workspace_rules():
     # large M: one split, no workspace
     assert lib.svla_op_gemm_splits(12800, 4096, 720) == 1
     assert lib.svla_op_gemm_workspace_bytes(12800, 4096, 720, 0) == 0
-    # batch-1 shapes split K to cover the SMs, never more splits than K blocks
+    # batch-1 shapes split K over a cluster of at most 8 CTAs to cover the SMs,
+    # never more splits than K blocks; cluster reductions need no workspace
     for (M, N, K) in [(50, 720, 2048), (50, 4096, 720), (50, 1600, 720), (1, 320, 64), (177, 960, 960)]:
         sp = lib.svla_op_gemm_splits(M, N, K)
-        assert 1 <= sp <= (K + 63) // 64
-        ws = lib.svla_op_gemm_workspace_bytes(M, N, K, 0)
-        assert (ws > 0) == (sp > 1)
+        assert 1 <= sp <= min(8, (K + 63) // 64)
+        assert lib.svla_op_gemm_workspace_bytes(M, N, K, 0) == 0
     assert lib.svla_op_gemm_splits(50, 720, 2048) > 1
     assert lib.svla_op_gemm_workspace_bytes(50, 720, 2048, 1) == 0
+    # more than 8 forced splits reduce through a global workspace
+    assert lib.svla_op_gemm_workspace_bytes(50, 720, 2048, 16) > 0

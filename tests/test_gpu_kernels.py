@@ -86,37 +86,44 @@ def test_gemm_epilogues(M, N, K):
     assert ((Cs.double() - silu).abs() <= 2 ** -7 * silu.abs() + 1e-3).all()
 
 
-def test_gemm_split_k_is_deterministic():
+@pytest.mark.parametrize("splits", [2, 5, 8, 16])
+def test_gemm_split_k_is_deterministic(splits):
+    """<= 8 splits reduce across a thread-block cluster, more through the global
+    workspace; both sum the splits in a fixed order."""
     g = torch.Generator(device="cpu").manual_seed(11)
     A = torch.randn(50, 2048, generator=g).to(torch.bfloat16).to(DEV)
     W = (0.05 * torch.randn(720, 2048, generator=g)).to(torch.bfloat16).to(DEV)
     outs = []
     for _ in range(3):
         C = torch.empty(50, 720, device=DEV)
-        gemm(_abi.EPI_F32, A, W, C, None, 16)
+        gemm(_abi.EPI_F32, A, W, C, None, splits)
         outs.append(C)
     torch.cuda.synchronize()
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    ref = A.double() @ W.double().T
+    assert ((outs[0].double() - ref).abs() <= 1e-5 * (A.double().abs() @ W.double().abs().T) + 1e-6).all()
 
 
-def test_gemm_timeout_path_reports_and_recovers():
+@pytest.mark.parametrize("M,splits", [(256, 1), (50, 4), (50, 12)])
+def test_gemm_timeout_path_reports_and_recovers(M, splits):
     """A wait limit of 0 makes the first unsatisfied wait give up: the kernel
-    records SVLA_ERR_TIMEOUT, drains and returns; the context stays usable."""
+    records SVLA_ERR_TIMEOUT, drains its copies, still meets every cluster
+    barrier, frees its tensor memory and returns; the context stays usable."""
     lib = _abi.load()
     g = torch.Generator(device="cpu").manual_seed(5)
-    A = torch.randn(256, 960, generator=g).to(torch.bfloat16).to(DEV)
+    A = torch.randn(M, 960, generator=g).to(torch.bfloat16).to(DEV)
     W = (0.05 * torch.randn(960, 960, generator=g)).to(torch.bfloat16).to(DEV)
-    C = torch.zeros(256, 960, device=DEV)
+    C = torch.zeros(M, 960, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     try:
         lib.svla_set_wait_limit_ns(0)
-        gemm(_abi.EPI_F32, A, W, C, None, 1, status)
+        gemm(_abi.EPI_F32, A, W, C, None, splits, status)
         torch.cuda.synchronize()
     finally:
         lib.svla_set_wait_limit_ns(1_000_000_000)
     assert status.item() == _abi.SVLA_ERR_TIMEOUT
     status.zero_()
-    gemm(_abi.EPI_F32, A, W, C, None, 1, status)
+    gemm(_abi.EPI_F32, A, W, C, None, splits, status)
     torch.cuda.synchronize()
     assert status.item() == 0
     ref = A.double() @ W.double().T

@@ -31,33 +31,34 @@ def S():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def with_workspace(epi, A, W, C, bias):
+def with_workspace(epi, A, W, C, bias, splits):
     lib = _abi.load()
     M, K = A.shape
     N = W.shape[0]
-    nbytes = lib.svla_op_gemm_workspace_bytes(M, N, K, 0)
+    nbytes = lib.svla_op_gemm_workspace_bytes(M, N, K, splits)
     ws = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=DEV)
-    _abi.check(lib.svla_op_gemm(epi, P(A), K, P(W), K, M, N, K, P(C), C.stride(0), P(bias), 0, P(ws), nbytes,
+    _abi.check(lib.svla_op_gemm(epi, P(A), K, P(W), K, M, N, K, P(C), C.stride(0), P(bias), splits, P(ws), nbytes,
                                 None, S()))
     torch.cuda.synchronize()
 
 
-def without_workspace(epi, A, W, C, bias, status):
+def without_workspace(epi, A, W, C, bias, splits, status):
     lib = _abi.load()
     M, K = A.shape
     N = W.shape[0]
-    _abi.check(lib.svla_op_gemm_noalloc(epi, P(A), K, P(W), K, M, N, K, P(C), C.stride(0), P(bias), 0, P(status),
-                                        S()))
+    _abi.check(lib.svla_op_gemm_noalloc(epi, P(A), K, P(W), K, M, N, K, P(C), C.stride(0), P(bias), splits,
+                                        P(status), S()))
     torch.cuda.synchronize()
 
 
-# batch-1 and prefix shapes of the path: all split K, so all use the scratch
-@pytest.mark.parametrize("M,N,K", [(50, 720, 2048), (50, 4096, 720), (177, 1600, 960), (50, 960, 720)])
+# batch-1 shapes of the path with more K splits than one cluster holds: the
+# partial tiles go through the scratch (global-memory reduction)
+@pytest.mark.parametrize("M,N,K,splits", [(50, 720, 2048, 16), (50, 960, 720, 12), (64, 320, 2048, 16),
+                                          (50, 1600, 720, 9)])
 @pytest.mark.parametrize("epi", [_abi.EPI_F32, _abi.EPI_ADD_F32, _abi.EPI_BF16])
-def test_noalloc_matches_workspace_entry_point_twice(M, N, K, epi):
+def test_noalloc_matches_workspace_entry_point_twice(M, N, K, splits, epi):
     lib = _abi.load()
-    assert lib.svla_op_gemm_splits(M, N, K) > 1
-    assert 0 < lib.svla_op_gemm_workspace_bytes(M, N, K, 0) <= 8 << 20
+    assert 0 < lib.svla_op_gemm_workspace_bytes(M, N, K, splits) <= 8 << 20
     g = torch.Generator(device="cpu").manual_seed(M + N + K + epi)
     A = torch.randn(M, K, generator=g).to(torch.bfloat16).to(DEV)
     W = (0.05 * torch.randn(N, K, generator=g)).to(torch.bfloat16).to(DEV)
@@ -65,13 +66,13 @@ def test_noalloc_matches_workspace_entry_point_twice(M, N, K, epi):
     dt = torch.bfloat16 if epi == _abi.EPI_BF16 else torch.float32
     R0 = torch.randn(M, N, generator=g).to(DEV).to(dt)
     ref = R0.clone()
-    with_workspace(epi, A, W, ref, bias)
+    with_workspace(epi, A, W, ref, bias, splits)
     scale = (A.double().abs() @ W.double().abs().T) + bias.double().abs() + R0.double().abs()
     tol = 1e-5 * scale + 1e-6 if epi != _abi.EPI_BF16 else 2 ** -8 * scale + 1e-4
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     for _ in range(2):   # two calls in a row share (and must re-arm) the static scratch
         out = R0.clone()
-        without_workspace(epi, A, W, out, bias, status)
+        without_workspace(epi, A, W, out, bias, splits, status)
         assert status.item() == 0
         assert ((out.double() - ref.double()).abs() <= tol).all()
 

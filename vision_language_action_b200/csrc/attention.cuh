@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a
   bf16* sV = sK + 2 * C::TILE;        // [2][64][LDS]
   uint8_t* sF = reinterpret_cast<uint8_t*>(sV + 2 * C::TILE);  // [2][64] key flags
 
+  griddep_launch_dependents();
+  griddep_wait();
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g_kv = h / (a.n_q / a.n_kv);
   const int q0 = qb * ATT_BQ;

@@ -44,6 +44,41 @@ SVLA_DEV uint32_t smem_u32(const void* p) {
 }
 
 // ------------------------------------------------------------------------
+// programmatic dependent launch: the next kernel in the stream may start
+// early; griddep_wait() blocks until every prerequisite grid has completed and
+// its memory is visible. Kernels touch no activation buffer (read or write)
+// before griddep_wait(); only immutable weights may be fetched earlier.
+// ------------------------------------------------------------------------
+SVLA_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+SVLA_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ------------------------------------------------------------------------
+// thread-block clusters / distributed shared memory
+// ------------------------------------------------------------------------
+SVLA_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// all threads of all CTAs of the cluster; release my shared-memory writes, acquire the peers'
+SVLA_DEV void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+SVLA_DEV uint32_t dsmem_addr(uint32_t local_saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_saddr), "r"(rank));
+  return r;
+}
+SVLA_DEV float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// ------------------------------------------------------------------------
 // mbarrier
 // ------------------------------------------------------------------------
 SVLA_DEV void mbar_init(uint32_t bar, uint32_t count) {

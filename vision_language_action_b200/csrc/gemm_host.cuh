@@ -41,75 +41,109 @@ inline bool make_tmap_bf16(CUtensorMap* m, const void* ptr, int rows, int cols, 
 
 struct GemmPlan {
   int bn = 64;
+  int stages = 4;
   int splits = 1;
+  int red = GEMM_RED_NONE;
   int m_tiles = 1, n_tiles = 1;
 };
 
 constexpr int NUM_SMS_B200 = 148;
 
-inline GemmPlan plan_gemm(int M, int N, int K, int forced_splits) {
+// Tile, stage and split-K plan of one GEMM.
+//  * enough 128 x 256 / 128 x 128 tiles to fill the 148 SMs: no split;
+//  * otherwise (the batch-1 and prefix shapes) 128 x 64 or 128 x 32 tiles with
+//    K split over a thread-block cluster of up to 8 CTAs, so that about one
+//    wave of CTAs streams the weights; 4 stages keep the CTA small enough for
+//    two per SM (the next kernel's CTA prefetches its weights beside it).
+// forced_splits > 0 fixes the split count; more than 8 splits (or 256-wide
+// tiles) use the global-workspace reduction. min_bn: the epilogue's smallest
+// tile width (64 for 64-wide heads and for SwiGLU's gate/up groups).
+inline GemmPlan plan_gemm(int M, int N, int K, int forced_splits, int min_bn = 32) {
   GemmPlan p;
   const int KB = (K + GEMM_BK - 1) / GEMM_BK;
   p.m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
   auto tiles = [&](int bn) { return p.m_tiles * ((N + bn - 1) / bn); };
-  if (tiles(256) >= NUM_SMS_B200)
+  auto clamp_splits = [&](int sp) {
+    if (sp > KB) sp = KB;
+    if (sp > GEMM_MAX_CLUSTER) sp = GEMM_MAX_CLUSTER;
+    return sp < 1 ? 1 : sp;
+  };
+  if (tiles(256) >= NUM_SMS_B200) {
     p.bn = 256;
-  else if (tiles(128) >= 100)
+    p.stages = 4;
+  } else if (tiles(128) >= 100) {
     p.bn = 128;
-  else
-    p.bn = 64;
-  p.n_tiles = (N + p.bn - 1) / p.bn;
-  const int t = p.m_tiles * p.n_tiles;
-  if (forced_splits > 0) {
-    p.splits = forced_splits;
-  } else if (t < 120) {
-    p.splits = NUM_SMS_B200 / t;
-    if (p.splits < 1) p.splits = 1;
+    p.stages = 6;
+  } else {
+    const int t64 = tiles(64), t32 = tiles(32);
+    const int s64 = clamp_splits(NUM_SMS_B200 / t64), s32 = clamp_splits(NUM_SMS_B200 / t32);
+    const int c64 = t64 * s64, c32 = t32 * s32;
+    p.bn = (c64 >= 120 || c64 >= c32 || min_bn > 32) ? 64 : 32;
+    p.stages = 4;
+    p.splits = p.bn == 64 ? s64 : s32;
   }
-  if (p.splits > KB) p.splits = KB;
-  if (p.splits < 1) p.splits = 1;
+  if (forced_splits > 0) p.splits = forced_splits > KB ? KB : forced_splits;
+  p.n_tiles = (N + p.bn - 1) / p.bn;
+  if (p.splits > 1) p.red = (p.splits <= GEMM_MAX_CLUSTER && p.bn <= 128) ? GEMM_RED_CLUSTER : GEMM_RED_GLOBAL;
   return p;
 }
 
+inline int gemm_min_bn(int epi) { return (epi == GE_SWIGLU || epi == GE_QKV_ROPE64) ? 64 : 32; }
+
 inline size_t gemm_partials_bytes(const GemmPlan& p) {
-  if (p.splits <= 1) return 0;
+  if (p.red != GEMM_RED_GLOBAL) return 0;
   return (size_t)p.m_tiles * p.n_tiles * p.splits * GEMM_BM * p.bn * sizeof(float);
 }
 
-// Launch one GEMM. A [M, K] (lda), W [N, K] (ldw), both bf16, rows 16-byte aligned.
-// `args` carries the epilogue fields; M/N/K, partials/counters, status and the
-// wait limit are filled in here. Returns a cudaError_t (cudaErrorInvalidValue
-// if a tensor map could not be encoded or the plan needs a workspace that was
-// not given).
-template <int BN, int EPI>
+// One instance: launched with programmatic stream serialization (PDL) and, for
+// the cluster reduction, a (1, 1, splits) cluster.
+template <int BN, int ST, int EPI>
 inline cudaError_t launch_gemm_inst(const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& args, dim3 grid,
-                                    cudaStream_t s) {
-  gemm_tc_kernel<BN, EPI><<<grid, GEMM_THREADS, GemmCfg<BN>::SMEM, s>>>(ta, tw, args);
-  return cudaGetLastError();
+                                    int cluster_z, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = GemmCfg<BN, ST>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  int n = 0;
+  at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_z > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = 1;
+    at[n].val.clusterDim.y = 1;
+    at[n].val.clusterDim.z = (unsigned)cluster_z;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, EPI, ST>, ta, tw, args);
 }
 
-template <int BN>
+template <int BN, int ST>
 inline cudaError_t dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& a, dim3 g,
-                                cudaStream_t s) {
+                                int cz, cudaStream_t s) {
   switch (epi) {
-    case GE_F32: return launch_gemm_inst<BN, GE_F32>(ta, tw, a, g, s);
-    case GE_BF16: return launch_gemm_inst<BN, GE_BF16>(ta, tw, a, g, s);
-    case GE_ADD_F32: return launch_gemm_inst<BN, GE_ADD_F32>(ta, tw, a, g, s);
-    case GE_SILU_BF16: return launch_gemm_inst<BN, GE_SILU_BF16>(ta, tw, a, g, s);
-    case GE_SWIGLU: return launch_gemm_inst<BN, GE_SWIGLU>(ta, tw, a, g, s);
-    case GE_QKV_ROPE64: return launch_gemm_inst<BN, GE_QKV_ROPE64>(ta, tw, a, g, s);
-    case GE_QKV_ROPE32: return launch_gemm_inst<BN, GE_QKV_ROPE32>(ta, tw, a, g, s);
+    case GE_F32: return launch_gemm_inst<BN, ST, GE_F32>(ta, tw, a, g, cz, s);
+    case GE_BF16: return launch_gemm_inst<BN, ST, GE_BF16>(ta, tw, a, g, cz, s);
+    case GE_ADD_F32: return launch_gemm_inst<BN, ST, GE_ADD_F32>(ta, tw, a, g, cz, s);
+    case GE_SILU_BF16: return launch_gemm_inst<BN, ST, GE_SILU_BF16>(ta, tw, a, g, cz, s);
+    case GE_SWIGLU: return launch_gemm_inst<BN, ST, GE_SWIGLU>(ta, tw, a, g, cz, s);
+    case GE_QKV_ROPE64: return launch_gemm_inst<BN, ST, GE_QKV_ROPE64>(ta, tw, a, g, cz, s);
+    case GE_QKV_ROPE32: return launch_gemm_inst<BN, ST, GE_QKV_ROPE32>(ta, tw, a, g, cz, s);
   }
   return cudaErrorInvalidValue;
 }
 
-template <int BN>
-inline cudaError_t set_attrs_bn() {
+template <int BN, int ST>
+inline cudaError_t set_attrs_inst() {
   cudaError_t e = cudaSuccess;
-  const int smem = (int)GemmCfg<BN>::SMEM;
-#define SVLA_SET(EPI)                                                                                     \
-  if (e == cudaSuccess)                                                                                   \
-    e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = (int)GemmCfg<BN, ST>::SMEM;
+#define SVLA_SET(EPI)                                                                                         \
+  if (e == cudaSuccess)                                                                                       \
+    e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   SVLA_SET(GE_F32)
   SVLA_SET(GE_BF16)
   SVLA_SET(GE_ADD_F32)
@@ -122,30 +156,32 @@ inline cudaError_t set_attrs_bn() {
 }
 
 inline cudaError_t gemm_set_attrs() {
-  cudaError_t e = set_attrs_bn<64>();
-  if (e == cudaSuccess) e = set_attrs_bn<128>();
-  if (e == cudaSuccess) e = set_attrs_bn<256>();
+  cudaError_t e = set_attrs_inst<32, 4>();
+  if (e == cudaSuccess) e = set_attrs_inst<64, 4>();
+  if (e == cudaSuccess) e = set_attrs_inst<128, 6>();
+  if (e == cudaSuccess) e = set_attrs_inst<256, 4>();
   return e;
 }
 
-// Full launch: plan, encode maps, dispatch.
+// Full launch: encode the maps and dispatch the plan's instance.
 inline cudaError_t run_gemm(int epi, const void* A, int lda, const void* W, int ldw, int M, int N, int K,
                             GemmArgs args, const GemmPlan& p, float* partials, int* counters, cudaStream_t s) {
   CUtensorMap ta, tw;
   if (!make_tmap_bf16(&ta, A, M, K, lda, GEMM_BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&tw, W, N, K, ldw, p.bn)) return cudaErrorInvalidValue;
-  if (p.splits > 1 && (!partials || !counters)) return cudaErrorInvalidValue;
+  if (p.red == GEMM_RED_GLOBAL && (!partials || !counters)) return cudaErrorInvalidValue;
   args.M = M;
   args.N = N;
   args.K = K;
   args.partials = partials;
   args.counters = counters;
+  args.red_mode = p.red;
   dim3 grid(p.n_tiles, p.m_tiles, p.splits);
-  switch (p.bn) {
-    case 64: return dispatch_epi<64>(epi, ta, tw, args, grid, s);
-    case 128: return dispatch_epi<128>(epi, ta, tw, args, grid, s);
-    case 256: return dispatch_epi<256>(epi, ta, tw, args, grid, s);
-  }
+  const int cz = p.red == GEMM_RED_CLUSTER ? p.splits : 1;
+  if (p.bn == 32 && p.stages == 4) return dispatch_epi<32, 4>(epi, ta, tw, args, grid, cz, s);
+  if (p.bn == 64 && p.stages == 4) return dispatch_epi<64, 4>(epi, ta, tw, args, grid, cz, s);
+  if (p.bn == 128 && p.stages == 6) return dispatch_epi<128, 6>(epi, ta, tw, args, grid, cz, s);
+  if (p.bn == 256 && p.stages == 4) return dispatch_epi<256, 4>(epi, ta, tw, args, grid, cz, s);
   return cudaErrorInvalidValue;
 }
 

@@ -52,26 +52,43 @@ struct GemmArgs {
   int pos_mod;
   const float2* rope_cs; // [pos][head_dim/2] (cos, sin)
   // split-K
-  float* partials;       // [tiles][splits][128][BN]
+  float* partials;       // [tiles][splits][128][BN]   (red_mode GEMM_RED_GLOBAL)
   int* counters;         // [tiles], zero between launches
+  int red_mode;          // how split-K partial tiles are summed (GemmRed)
   int* status;
   unsigned long long wait_ns;
 };
+
+// Split-K reduction of the partial tiles:
+//   GEMM_RED_NONE    one split, the epilogue reads TMEM;
+//   GEMM_RED_CLUSTER the splits of a tile form one thread-block cluster; each
+//                    CTA stages its partial tile in its shared memory, then
+//                    CTA r sums rows r, r + S, .. over the peers' tiles in
+//                    split order (distributed shared memory) and runs their
+//                    epilogue: no global scratch, deterministic;
+//   GEMM_RED_GLOBAL  partial tiles in a global workspace, the last CTA of the
+//                    tile to arrive sums them in split order (any split count).
+enum GemmRed : int { GEMM_RED_NONE = 0, GEMM_RED_CLUSTER = 1, GEMM_RED_GLOBAL = 2 };
+constexpr int GEMM_MAX_CLUSTER = 8;
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;
 constexpr int GEMM_THREADS = 192;
 constexpr unsigned long long GEMM_DRAIN_NS = 2000000000ull;  // fixed limit for the drain path
 
-template <int BN>
+template <int BN, int STAGES_>
 struct GemmCfg {
-  static constexpr int STAGES = BN <= 64 ? 8 : (BN <= 128 ? 6 : 4);
+  static constexpr int STAGES = STAGES_;
   static constexpr uint32_t A_BYTES = GEMM_BM * GEMM_BK * 2;
   static constexpr uint32_t B_BYTES = BN * GEMM_BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
   // ring + barriers/flags area + alignment slack
   static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 256 + 1024;
+  // two CTAs per SM when they fit, so a dependent GEMM can start next to this one
+  static constexpr int MIN_BLOCKS = SMEM <= 113 * 1024 ? 2 : 1;
+  static constexpr size_t RED_TILE = (size_t)GEMM_BM * (BN + 4) * sizeof(float);
+  static constexpr bool CLUSTER_OK = 2 * RED_TILE <= (size_t)STAGES * STAGE_BYTES;
 };
 
 // ---------------------------------------------------------------------------
@@ -274,12 +291,11 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, const AccSource<BN>& src, int m, i
 // named barrier over the 4 epilogue warps (ids 2..5)
 SVLA_DEV void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int BN, int EPI>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+template <int BN, int EPI, int STAGES>
+__global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES>::MIN_BLOCKS)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                    const GemmArgs args) {
-  using C = GemmCfg<BN>;
-  constexpr int STAGES = C::STAGES;
+  using C = GemmCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
@@ -301,6 +317,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
   const uint32_t acc_bar = smem_u32(bars + 2 * STAGES);
 
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
@@ -327,11 +344,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int i = 0; i < nkb; ++i) {
+      // the weights do not depend on earlier kernels: start streaming the first
+      // stages' W tiles before waiting for the producer of A
+      const int pre = nkb < STAGES ? nkb : STAGES;
+      for (int i = 0; i < pre; ++i) {
+        const uint32_t sa = smem_u32(ring + i * C::STAGE_BYTES);
+        mbar_arrive_expect_tx(full_bar(i), C::STAGE_BYTES);
+        tma_load_2d(sa + C::A_BYTES, &tmW, full_bar(i), (kb0 + i) * GEMM_BK, n_blk * BN);
+      }
+      griddep_wait();
+      for (int i = 0; i < pre; ++i) {
+        const uint32_t sa = smem_u32(ring + i * C::STAGE_BYTES);
+        tma_load_2d(sa, &tmA, full_bar(i), (kb0 + i) * GEMM_BK, m_blk * GEMM_BM);
+      }
+      misc[2] = pre;
+      for (int i = pre; i < nkb; ++i) {
         if (misc[1]) break;
         const int s = i % STAGES;
         const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-        if (i >= STAGES && !mbar_wait(empty_bar(s), ph ^ 1u, lim)) {
+        if (!mbar_wait(empty_bar(s), ph ^ 1u, lim)) {
           misc[1] = 1;
           set_status(args.status, SVLA_ERR_TIMEOUT);
           break;
@@ -370,6 +401,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
   } else {
     // ---------------- epilogue warps ----------------
+    griddep_wait();  // outputs, residuals, biases and positions come from earlier kernels
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const int m = m_blk * GEMM_BM + row;
@@ -389,6 +421,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       src.smem_row = nullptr;
       if (splits == 1) {
         run_epilogue<BN, EPI>(args, src, m, n0, row_ok);
+      } else if (C::CLUSTER_OK && args.red_mode == GEMM_RED_CLUSTER) {
+        // stage this split's partial tile in shared memory (the operand ring is idle)
+        float* red = reinterpret_cast<float*>(ring);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          float v[16];
+          tmem_ld16(src.taddr_row + (uint32_t)c, v);
+          float4* d = reinterpret_cast<float4*>(red + row * (BN + 4) + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
       } else {
         const int tile = m_blk * gridDim.x + n_blk;
         float* tile_part = args.partials + (size_t)tile * splits * GEMM_BM * BN;
@@ -433,6 +476,52 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     if (threadIdx.x == 32) mbar_wait(acc_bar, 0, GEMM_DRAIN_NS);
     __syncthreads();
+  }
+  if constexpr (C::CLUSTER_OK) {
+    if (args.red_mode == GEMM_RED_CLUSTER && splits > 1) {
+      // Every thread of every CTA of the cluster reaches both barriers exactly
+      // once, whatever happened before (no early exit exists in this kernel).
+      cluster_sync();
+      if (warp >= 2) {
+        const int t = threadIdx.x - 64;
+        const uint32_t rank = cluster_ctarank();
+        const int rows = min(GEMM_BM, args.M - m_blk * GEMM_BM);
+        float* red = reinterpret_cast<float*>(ring);
+        float* fin = red + GEMM_BM * (BN + 4);
+        const uint32_t red_s = smem_u32(red);
+        constexpr int V4 = BN / 4;
+        const int my_rows = (rows - (int)rank + splits - 1) / splits;
+        for (int item = t; item < my_rows * V4; item += 128) {
+          const int r = (int)rank + splits * (item / V4), c4 = item % V4;
+          const uint32_t off = (uint32_t)((r * (BN + 4) + 4 * c4) * 4);
+          float4 part[GEMM_MAX_CLUSTER];
+#pragma unroll
+          for (int p = 0; p < GEMM_MAX_CLUSTER; ++p)
+            if (p < splits) part[p] = ld_dsmem_f4(dsmem_addr(red_s + off, (uint32_t)p));
+          float4 acc = part[0];
+#pragma unroll
+          for (int p = 1; p < GEMM_MAX_CLUSTER; ++p) {
+            if (p < splits) {
+              acc.x += part[p].x;
+              acc.y += part[p].y;
+              acc.z += part[p].z;
+              acc.w += part[p].w;
+            }
+          }
+          *reinterpret_cast<float4*>(fin + r * (BN + 4) + 4 * c4) = acc;
+        }
+        epi_bar();
+        const int row = (warp & 3) * 32 + lane;
+        const int m = m_blk * GEMM_BM + row;
+        if (misc[1] == 0 && row < rows && row % splits == (int)rank) {
+          AccSource<BN> src;
+          src.taddr_row = 0;
+          src.smem_row = fin + row * (BN + 4);
+          run_epilogue<BN, EPI>(args, src, m, n_blk * BN, true);
+        }
+      }
+      cluster_sync();  // peers have finished reading this CTA's partial tile
+    }
   }
   if (warp == 1) {
     tc_fence_after();

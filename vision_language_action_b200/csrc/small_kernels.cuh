@@ -16,10 +16,19 @@ template <bool X_BF16>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const void* __restrict__ x, float* __restrict__ x_out,
                                                       const bf16* __restrict__ gain, int M, int D, float eps,
                                                       bf16* __restrict__ y) {
+  griddep_launch_dependents();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= M) return;
   const int D4 = D / 4;
+  // gains are weights: fetch them before waiting for the producer of x
+  uint2 gg[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int c = lane + 32 * i;
+    if (c < D4) gg[i] = __ldg(reinterpret_cast<const uint2*>(gain) + c);
+  }
+  griddep_wait();
+  if (warp >= M) return;
   float acc = 0.f;
   // at most 16 float4 per lane are kept in registers (D <= 2048)
   float4 v[16];
@@ -47,9 +56,8 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const void* __restrict__ x
   for (int i = 0; i < 16; ++i) {
     const int c = lane + 32 * i;
     if (c < D4) {
-      const uint2 gg = __ldg(reinterpret_cast<const uint2*>(gain) + c);
-      const float g0 = __uint_as_float(gg.x << 16), g1 = __uint_as_float(gg.x & 0xffff0000u);
-      const float g2 = __uint_as_float(gg.y << 16), g3 = __uint_as_float(gg.y & 0xffff0000u);
+      const float g0 = __uint_as_float(gg[i].x << 16), g1 = __uint_as_float(gg[i].x & 0xffff0000u);
+      const float g2 = __uint_as_float(gg[i].y << 16), g3 = __uint_as_float(gg[i].y & 0xffff0000u);
       uint2 o;
       o.x = pack_bf16x2(v[i].x * r * g0, v[i].y * r * g1);
       o.y = pack_bf16x2(v[i].z * r * g2, v[i].w * r * g3);
@@ -65,6 +73,8 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const void* __restrict__ x
 // ---------------------------------------------------------------------------
 __global__ void positions_kernel(const uint8_t* __restrict__ valid, int B, int L, int* __restrict__ pos,
                                  int* status) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= B) return;
@@ -106,22 +116,41 @@ struct StepBeginArgs {
 __global__ void __launch_bounds__(256) step_begin_kernel(const StepBeginArgs p) {
   __shared__ float xs[8][64];
   __shared__ float es[2048];
+  griddep_launch_dependents();
   if ((int)blockIdx.x < p.nA) {
     const int m0 = blockIdx.x * 8;
+    const int A8 = p.A / 8;
+    auto load_w = [&](int o, uint4 (&w)[8]) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (c < A8) w[c] = __ldg(reinterpret_cast<const uint4*>(p.w_in + (size_t)o * p.A) + c);
+    };
+    // this thread's first W_in row (weights) is fetched before the dependency wait
+    uint4 w[8];
+    if ((int)threadIdx.x < p.De) load_w(threadIdx.x, w);
+    griddep_wait();
     for (int i = threadIdx.x; i < 8 * p.A; i += blockDim.x) {
       const int r = i / p.A, c = i % p.A;
       xs[r][c] = (m0 + r < p.M) ? p.x[(size_t)(m0 + r) * p.A + c] : 0.f;
     }
     __syncthreads();
     for (int o = threadIdx.x; o < p.De; o += blockDim.x) {
-      float w[64];
-      const uint16_t* wr = reinterpret_cast<const uint16_t*>(p.w_in) + (size_t)o * p.A;
-      for (int c = 0; c < p.A; ++c) w[c] = bf2f(wr[c]);
+      if (o != (int)threadIdx.x) load_w(o, w);
       const float bias = bf2f(reinterpret_cast<const uint16_t*>(p.b_in)[o]);
       for (int r = 0; r < 8; ++r) {
         if (m0 + r >= p.M) break;
         float acc = 0.f;
-        for (int c = 0; c < p.A; ++c) acc = fmaf(xs[r][c], w[c], acc);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (c < A8) {
+            const uint32_t u[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              acc = fmaf(xs[r][8 * c + 2 * k], __uint_as_float(u[k] << 16), acc);
+              acc = fmaf(xs[r][8 * c + 2 * k + 1], __uint_as_float(u[k] & 0xffff0000u), acc);
+            }
+          }
+        }
         p.a_out[(size_t)(m0 + r) * p.De + o] = __float2bfloat16_rn(acc + bias);
       }
     }
@@ -137,21 +166,22 @@ __global__ void __launch_bounds__(256) step_begin_kernel(const StepBeginArgs p) 
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int o = ((int)blockIdx.x - p.nA) * 8 + warp;
+    float acc = 0.f;
     if (o < p.De) {
       const uint16_t* wr = reinterpret_cast<const uint16_t*>(p.w_t1) + (size_t)o * 2 * p.De + p.De;
-      float acc = 0.f;
       for (int i = lane; i < p.De; i += 32) acc = fmaf(bf2f(wr[i]), es[i], acc);
 #pragma unroll
       for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-      if (lane == 0) p.c_out[o] = acc + bf2f(reinterpret_cast<const uint16_t*>(p.b_t1)[o]);
     }
+    griddep_wait();  // c_out is read by the previous step's GEMM
+    if (o < p.De && lane == 0) p.c_out[o] = acc + bf2f(reinterpret_cast<const uint16_t*>(p.b_t1)[o]);
   }
 }
 
 // ---------------------------------------------------------------------------
 // Step epilogue (readings 8, 13): v = RMSNorm(r; final_norm) W_out^T + b_out
 // in fp32, then x <- x + dt v (dt = -1/n); optional trace of v_k and x_{k+1}.
-// One warp per chunk row; W_out is staged transposed in shared memory.
+// One warp per chunk row; W_out is staged in shared memory once per block.
 // ---------------------------------------------------------------------------
 struct StepEndArgs {
   const float* r;          // [M, De] expert output (residual stream)
@@ -168,41 +198,91 @@ struct StepEndArgs {
 
 constexpr int SE_WARPS = 8;
 
+// Sum 32 per-lane partial vectors across the warp: afterwards lane o holds the
+// total of component o (recursive halving, 31 shuffles, fixed order).
+SVLA_DEV float warp_transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float send = upper ? v[i] : v[i + s];
+      const float keep = upper ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
+}
+
 __global__ void __launch_bounds__(256) step_end_kernel(const StepEndArgs p) {
-  extern __shared__ float se_smem[];
-  float* wt = se_smem;                    // [De][A] transposed W_out
-  float* ys = se_smem + p.De * p.A;       // [SE_WARPS][De]
-  for (int i = threadIdx.x; i < p.De * p.A; i += blockDim.x) {
-    const int o = i / p.De, j = i % p.De;
-    wt[j * p.A + o] = bf2f(reinterpret_cast<const uint16_t*>(p.w_out)[i]);
+  extern __shared__ __align__(16) uint16_t se_w[];  // W_out [A][De] bf16, staged once per block
+  griddep_launch_dependents();
+  {
+    const int n16 = p.A * p.De / 8;  // 16-byte chunks (A * De is a multiple of 8)
+    const uint4* src = reinterpret_cast<const uint4*>(p.w_out);
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) reinterpret_cast<uint4*>(se_w)[i] = __ldg(src + i);
   }
   __syncthreads();
+  griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* y = ys + warp * p.De;
+  const int D4 = p.De / 4;
   for (int m = blockIdx.x * SE_WARPS + warp; m < p.M; m += gridDim.x * SE_WARPS) {
-    const float* rr = p.r + (size_t)m * p.De;
+    const float4* rr = reinterpret_cast<const float4*>(p.r + (size_t)m * p.De);
+    float4 y[16];
     float acc = 0.f;
-    for (int j = lane; j < p.De; j += 32) {
-      const float v = rr[j];
-      y[j] = v;
-      acc += v * v;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = lane + 32 * i;
+      if (c < D4) {
+        y[i] = rr[c];
+        acc += y[i].x * y[i].x + y[i].y * y[i].y + y[i].z * y[i].z + y[i].w * y[i].w;
+      }
     }
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
     const float inv = rsqrtf(acc / (float)p.De + p.eps);
-    for (int j = lane; j < p.De; j += 32)
-      y[j] = y[j] * inv * bf2f(reinterpret_cast<const uint16_t*>(p.final_norm)[j]);
-    __syncwarp();
-    for (int o = lane; o < p.A; o += 32) {
-      float v = 0.f;
-      for (int j = 0; j < p.De; ++j) v = fmaf(y[j], wt[j * p.A + o], v);
-      v += bf2f(reinterpret_cast<const uint16_t*>(p.b_out)[o]);
-      const float xn = p.x[(size_t)m * p.A + o] + p.dt * v;
-      p.x[(size_t)m * p.A + o] = xn;
-      if (p.trace_v) p.trace_v[(size_t)m * p.A + o] = v;
-      if (p.trace_x) p.trace_x[(size_t)m * p.A + o] = xn;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = lane + 32 * i;
+      if (c < D4) {
+        const uint2 g = __ldg(reinterpret_cast<const uint2*>(p.final_norm) + c);
+        y[i].x *= inv * __uint_as_float(g.x << 16);
+        y[i].y *= inv * __uint_as_float(g.x & 0xffff0000u);
+        y[i].z *= inv * __uint_as_float(g.y << 16);
+        y[i].w *= inv * __uint_as_float(g.y & 0xffff0000u);
+      }
     }
-    __syncwarp();
+    for (int o0 = 0; o0 < p.A; o0 += 32) {
+      float part[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float s = 0.f;
+        if (o0 + j < p.A) {
+          const uint2* wr = reinterpret_cast<const uint2*>(se_w + (size_t)(o0 + j) * p.De);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c = lane + 32 * i;
+            if (c < D4) {
+              const uint2 w = wr[c];
+              s = fmaf(y[i].x, __uint_as_float(w.x << 16), s);
+              s = fmaf(y[i].y, __uint_as_float(w.x & 0xffff0000u), s);
+              s = fmaf(y[i].z, __uint_as_float(w.y << 16), s);
+              s = fmaf(y[i].w, __uint_as_float(w.y & 0xffff0000u), s);
+            }
+          }
+        }
+        part[j] = s;
+      }
+      const float v = warp_transpose_sum32(part, lane);
+      const int o = o0 + lane;
+      if (o < p.A) {
+        const float vv = v + bf2f(reinterpret_cast<const uint16_t*>(p.b_out)[o]);
+        const float xn = p.x[(size_t)m * p.A + o] + p.dt * vv;
+        p.x[(size_t)m * p.A + o] = xn;
+        if (p.trace_v) p.trace_v[(size_t)m * p.A + o] = vv;
+        if (p.trace_x) p.trace_x[(size_t)m * p.A + o] = xn;
+      }
+    }
   }
 }
 
@@ -226,6 +306,8 @@ SVLA_DEV void philox4x32_10(uint32_t (&c)[4], uint32_t k0, uint32_t k1) {
 }
 
 __global__ void philox_noise_kernel(unsigned long long seed, int B, int n_el, float* __restrict__ out) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int n_blk = (n_el + 3) / 4;
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gid >= (long long)B * n_blk) return;

@@ -13,6 +13,7 @@
 #include <cstring>
 #include <atomic>
 #include <list>
+#include <utility>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -137,6 +138,7 @@ const char* check_config(const svla_config& c) {
   if (c.e_width < 16 || c.e_width % 16 || c.e_width > 2048) return "e_width must be a multiple of 16, <= 2048";
   if (c.p_ffn < 64 || c.p_ffn % 64 || c.e_ffn < 64 || c.e_ffn % 64) return "ffn widths must be multiples of 64";
   if (c.action_dim < 8 || c.action_dim % 8 || c.action_dim > 64) return "action_dim must be a multiple of 8, <= 64";
+  if ((size_t)c.action_dim * c.e_width * 2 > 200 * 1024) return "action_dim * e_width * 2 must be <= 200 KiB";
   if (c.max_batch < 1 || c.max_prefix < 1 || c.max_chunk < 1) return "max sizes must be >= 1";
   if (!(c.rms_eps > 0.f) || !(c.rope_base > 1.f) || !(c.t_min_period > 0.f) || !(c.t_max_period > 0.f))
     return "rope_base, rms_eps and the time periods must be positive";
@@ -233,10 +235,28 @@ void free_all(svla_handle* h) {
   h->cap = nullptr;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while its
+// predecessor drains; it touches activations only after griddep_wait().
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // one GEMM of the schedule
 cudaError_t gemm(svla_handle* h, int epi, const bf16* A, int lda, const bf16* W, int ldw, int M, int N, int K,
                  GemmArgs args, float* part, int* cnt, cudaStream_t s) {
-  GemmPlan p = plan_gemm(M, N, K, 0);
+  GemmPlan p = plan_gemm(M, N, K, 0, gemm_min_bn(epi));
   args.status = h->status;
   args.wait_ns = g_wait_ns.load();
   return run_gemm(epi, A, lda, W, ldw, M, N, K, args, p, part, cnt, s);
@@ -254,11 +274,8 @@ GemmArgs out_args(void* out, int ldo, const float* bias = nullptr) {
 cudaError_t rmsnorm(const void* x, bool x_bf16, float* x_copy, const bf16* g, int M, int D, float eps, bf16* y,
                     cudaStream_t s) {
   const int blocks = (M + 7) / 8;
-  if (x_bf16)
-    rmsnorm_kernel<true><<<blocks, 256, 0, s>>>(x, x_copy, g, M, D, eps, y);
-  else
-    rmsnorm_kernel<false><<<blocks, 256, 0, s>>>(x, nullptr, g, M, D, eps, y);
-  return cudaGetLastError();
+  if (x_bf16) return launch_pdl(rmsnorm_kernel<true>, dim3(blocks), dim3(256), 0, s, x, x_copy, g, M, D, eps, y);
+  return launch_pdl(rmsnorm_kernel<false>, dim3(blocks), dim3(256), 0, s, x, (float*)nullptr, g, M, D, eps, y);
 }
 
 cudaError_t attention(const bf16* q, int ldq, const bf16* k, const bf16* v, int ldkv, const uint8_t* valid, int B,
@@ -279,11 +296,8 @@ cudaError_t attention(const bf16* q, int ldq, const bf16* k, const bf16* v, int 
   a.causal = causal;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)hd));
   dim3 grid((Lq + ATT_BQ - 1) / ATT_BQ, nq, B);
-  if (hd == 64)
-    attention_kernel<64><<<grid, ATT_THREADS, AttnCfg<64>::SMEM, s>>>(a);
-  else
-    attention_kernel<32><<<grid, ATT_THREADS, AttnCfg<32>::SMEM, s>>>(a);
-  return cudaGetLastError();
+  if (hd == 64) return launch_pdl(attention_kernel<64>, grid, dim3(ATT_THREADS), AttnCfg<64>::SMEM, s, a);
+  return launch_pdl(attention_kernel<32>, grid, dim3(ATT_THREADS), AttnCfg<32>::SMEM, s, a);
 }
 
 #define SVLA_TRY(expr)                        \
@@ -300,8 +314,7 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
   const int qw = c.p_heads * hd, kvw = c.p_kv_heads * hd;
   bf16* cache = reinterpret_cast<bf16*>(kv);
   const size_t layer_elems = (size_t)B * L * kvw;
-  positions_kernel<<<(B + 7) / 8, 256, 0, s>>>(pad, B, L, h->p_pos, h->status);
-  SVLA_TRY(cudaGetLastError());
+  SVLA_TRY(launch_pdl(positions_kernel, dim3((B + 7) / 8), dim3(256), 0, s, pad, B, L, h->p_pos, h->status));
   for (int l = 0; l < c.p_layers; ++l) {
     const Entry* e = &h->lay.p[9 * l];
     bf16* Kl = cache + (size_t)l * layer_elems;
@@ -356,7 +369,6 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
                   pkvw, out_args(vx, kvw), h->e_part, h->e_cnt, s));
   }
   const Layout& Lh = h->lay;
-  const int se_smem = (E * A + SE_WARPS * E) * (int)sizeof(float);
   int se_blocks = (M + SE_WARPS - 1) / SE_WARPS;
   if (se_blocks > 2 * NUM_SMS_B200) se_blocks = 2 * NUM_SMS_B200;
   for (int k = 0; k < n_steps; ++k) {
@@ -375,8 +387,7 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
     sb.a_out = h->e_a;
     sb.c_out = h->e_c;
     sb.nA = (M + 7) / 8;
-    step_begin_kernel<<<sb.nA + (E + 7) / 8, 256, 0, s>>>(sb);
-    SVLA_TRY(cudaGetLastError());
+    SVLA_TRY(launch_pdl(step_begin_kernel, dim3(sb.nA + (E + 7) / 8), dim3(256), 0, s, sb));
     // time MLP: h1 = silu(W_t1[:, :E] a + c), r = W_t2 h1 + b_t2
     SVLA_TRY(gemm(h, GE_SILU_BF16, h->e_a, E, h->W(Lh.w_t1.off), 2 * E, M, E, E, out_args(h->e_h1, E, h->e_c),
                   h->e_part, h->e_cnt, s));
@@ -429,8 +440,7 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
     se.x = actions;
     se.trace_v = trace ? trace + (size_t)(2 * k) * M * A : nullptr;
     se.trace_x = trace ? trace + (size_t)(2 * k + 1) * M * A : nullptr;
-    step_end_kernel<<<se_blocks, 256, se_smem, s>>>(se);
-    SVLA_TRY(cudaGetLastError());
+    SVLA_TRY(launch_pdl(step_end_kernel, dim3(se_blocks), dim3(256), (size_t)A * E * 2, s, se));
   }
   return cudaSuccess;
 }
@@ -678,8 +688,10 @@ svla_status svla_sample(svla_handle* h, const void* embeds, const uint8_t* pad, 
   float* noise = noise_out ? noise_out : h->noise_buf;
   const int n_el = H * h->cfg.action_dim;
   const long long threads = (long long)B * ((n_el + 3) / 4);
-  philox_noise_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>((unsigned long long)seed, B, n_el, noise);
-  if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return cuda_fail(h, e, "noise");
+  if (cudaError_t e = launch_pdl(philox_noise_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, s,
+                                 (unsigned long long)seed, B, n_el, noise);
+      e != cudaSuccess)
+    return cuda_fail(h, e, "noise");
   svla_status st = svla_prefill(h, embeds, pad, B, L, kv, stream);
   if (st != SVLA_OK) return st;
   return svla_denoise(h, kv, pad, B, L, noise, H, n_steps, actions, nullptr, stream);
@@ -719,7 +731,7 @@ static size_t cnt_bytes(const GemmPlan& p) { return (((size_t)p.m_tiles * p.n_ti
 size_t svla_op_gemm_workspace_bytes(int M, int N, int K, int splits) {
   if (M < 1 || N < 1 || K < 1 || splits < 0) return 0;
   GemmPlan p = plan_gemm(M, N, K, splits);
-  if (p.splits <= 1) return 0;
+  if (p.red != GEMM_RED_GLOBAL) return 0;
   return cnt_bytes(p) + gemm_partials_bytes(p);
 }
 
@@ -740,7 +752,7 @@ svla_status svla_op_gemm(int epilogue, const void* A, int lda, const void* W, in
   GemmPlan p = plan_gemm(M, N, K, splits);
   float* part = nullptr;
   int* cnt = nullptr;
-  if (p.splits > 1) {
+  if (p.red == GEMM_RED_GLOBAL) {
     const size_t need = cnt_bytes(p) + gemm_partials_bytes(p);
     if (!workspace || workspace_bytes < need) return fail(nullptr, SVLA_ERR_ARG, "workspace missing or too small");
     cnt = reinterpret_cast<int*>(workspace);
