@@ -103,9 +103,9 @@ def chunk_work(s, B, L, H, n_steps):
 
 def launches_per_chunk(s, n_steps):
     """Kernels libsvla launches for one prefill + denoise (the CUDA graphs' kernel nodes)."""
-    pre = 1 + 2 * s.p_layers + 5 * (s.p_layers - 1)
+    pre = 2 + s.p_layers + 4 * (s.p_layers - 1)   # positions, residual init, QKV per layer, attn/O/GU/D
     hoist = 2 * (s.e_layers // 2)
-    step = 1 + 2 + 7 * s.e_layers + 1
+    step = 1 + 2 + 5 * s.e_layers + 1              # step begin, time MLP, 5 per layer, step end
     return pre + hoist + n_steps * step
 
 

@@ -122,15 +122,24 @@ SVLA_DEV bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait until the phase with `parity` has completed, for at most limit_ns.
+// Wait until the phase with `parity` has completed, for at most about limit_ns.
 // Returns false if the limit ran out (limit 0: give up unless already done).
+// The fast path is try_wait alone (it suspends the thread until the phase
+// completes or a hardware time slice ends); the clock is read only after 64
+// unsuccessful tries, so a wait that succeeds costs no timer reads.
 SVLA_DEV bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_test(bar, parity)) return true;
   if (limit_ns == 0) return false;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
+    if ((i & 63u) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0)
+        t0 = now;
+      else if (now - t0 > limit_ns)
+        return false;
+    }
   }
 }
 

@@ -4,7 +4,7 @@
 
 #include <mutex>
 
-#include "gemm_tc.cuh"
+#include "gemm_persistent.cuh"
 
 namespace svla {
 
@@ -45,12 +45,22 @@ struct GemmPlan {
   int splits = 1;
   int red = GEMM_RED_NONE;
   int m_tiles = 1, n_tiles = 1;
+  bool persistent = false;  // one CTA per SM walking the tiles, double-buffered accumulators
+  int ctas = 0;             // grid of the persistent kernel
+};
+
+// operand-ring depth of the persistent kernel: as many stages as fit in the
+// 227 KB of dynamic shared memory a CTA may use (barriers and alignment slack aside)
+template <int BN>
+struct PersistentStages {
+  static constexpr int value = (232448 - 2048) / (GEMM_BM * GEMM_BK * 2 + BN * GEMM_BK * 2);
 };
 
 constexpr int NUM_SMS_B200 = 148;
 
 // Tile, stage and split-K plan of one GEMM.
-//  * enough 128 x 256 / 128 x 128 tiles to fill the 148 SMs: no split;
+//  * M > 384 rows, or enough wide tiles to fill the 148 SMs: the persistent
+//    kernel (one CTA per SM, double-buffered accumulators), no split;
 //  * otherwise (the batch-1 and prefix shapes) 128 x 64 or 128 x 32 tiles with
 //    K split over a thread-block cluster of up to 8 CTAs, so that about one
 //    wave of CTAs streams the weights; 4 stages keep the CTA small enough for
@@ -63,6 +73,29 @@ inline GemmPlan plan_gemm(int M, int N, int K, int forced_splits, int min_bn = 3
   const int KB = (K + GEMM_BK - 1) / GEMM_BK;
   p.m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
   auto tiles = [&](int bn) { return p.m_tiles * ((N + bn - 1) / bn); };
+  if (forced_splits <= 1 && (p.m_tiles >= 4 || tiles(256) >= NUM_SMS_B200 || tiles(128) >= 100)) {
+    // persistent: a CTA's time is about (tiles it walks) x (operand bytes of
+    // one tile, 128 + BN rows of K); pick the width that minimises
+    // waves x (128 + BN), ties to the wider tile
+    const int cands[5] = {64, 96, 128, 192, 256};
+    long best = -1;
+    for (int bn : cands) {
+      if (min_bn == 64 && bn % 64) continue;
+      const int t = tiles(bn);
+      const long waves = (t + NUM_SMS_B200 - 1) / NUM_SMS_B200;
+      const long cost = waves * (GEMM_BM + bn);
+      if (best < 0 || cost <= best) {
+        best = cost;
+        p.bn = bn;
+      }
+    }
+    p.n_tiles = (N + p.bn - 1) / p.bn;
+    p.persistent = true;
+    p.splits = 1;
+    const int t = p.m_tiles * p.n_tiles;
+    p.ctas = t < NUM_SMS_B200 ? t : NUM_SMS_B200;
+    return p;
+  }
   auto clamp_splits = [&](int sp) {
     if (sp > KB) sp = KB;
     if (sp > GEMM_MAX_CLUSTER) sp = GEMM_MAX_CLUSTER;
@@ -89,6 +122,62 @@ inline GemmPlan plan_gemm(int M, int N, int K, int forced_splits, int min_bn = 3
 }
 
 inline int gemm_min_bn(int epi) { return (epi == GE_SWIGLU || epi == GE_QKV_ROPE64) ? 64 : 32; }
+
+template <int BN, int EPI>
+inline cudaError_t launch_persistent_inst(const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& args,
+                                          int ctas, cudaStream_t s) {
+  constexpr int ST = PersistentStages<BN>::value;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = GemmCfg<BN, ST>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_tc_persistent_kernel<BN, EPI, ST>, ta, tw, args);
+}
+
+template <int BN>
+inline cudaError_t dispatch_persistent(int epi, const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& a,
+                                       int ctas, cudaStream_t s) {
+  switch (epi) {
+    case GE_F32: return launch_persistent_inst<BN, GE_F32>(ta, tw, a, ctas, s);
+    case GE_BF16: return launch_persistent_inst<BN, GE_BF16>(ta, tw, a, ctas, s);
+    case GE_ADD_F32: return launch_persistent_inst<BN, GE_ADD_F32>(ta, tw, a, ctas, s);
+    case GE_SILU_BF16: return launch_persistent_inst<BN, GE_SILU_BF16>(ta, tw, a, ctas, s);
+    case GE_QKV_ROPE32: return launch_persistent_inst<BN, GE_QKV_ROPE32>(ta, tw, a, ctas, s);
+  }
+  if constexpr (BN % 64 == 0) {
+    if (epi == GE_SWIGLU) return launch_persistent_inst<BN, GE_SWIGLU>(ta, tw, a, ctas, s);
+    if (epi == GE_QKV_ROPE64) return launch_persistent_inst<BN, GE_QKV_ROPE64>(ta, tw, a, ctas, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int BN>
+inline cudaError_t set_attrs_persistent() {
+  constexpr int ST = PersistentStages<BN>::value;
+  const int smem = (int)GemmCfg<BN, ST>::SMEM;
+  cudaError_t e = cudaSuccess;
+#define SVLA_SETP(EPI)                                                                                       \
+  if (e == cudaSuccess)                                                                                      \
+    e = cudaFuncSetAttribute(gemm_tc_persistent_kernel<BN, EPI, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             smem);
+  SVLA_SETP(GE_F32)
+  SVLA_SETP(GE_BF16)
+  SVLA_SETP(GE_ADD_F32)
+  SVLA_SETP(GE_SILU_BF16)
+  SVLA_SETP(GE_QKV_ROPE32)
+  if constexpr (BN % 64 == 0) {
+    SVLA_SETP(GE_SWIGLU)
+    SVLA_SETP(GE_QKV_ROPE64)
+  }
+#undef SVLA_SETP
+  return e;
+}
 
 inline size_t gemm_partials_bytes(const GemmPlan& p) {
   if (p.red != GEMM_RED_GLOBAL) return 0;
@@ -156,7 +245,12 @@ inline cudaError_t set_attrs_inst() {
 }
 
 inline cudaError_t gemm_set_attrs() {
-  cudaError_t e = set_attrs_inst<32, 4>();
+  cudaError_t e = set_attrs_persistent<64>();
+  if (e == cudaSuccess) e = set_attrs_persistent<96>();
+  if (e == cudaSuccess) e = set_attrs_persistent<128>();
+  if (e == cudaSuccess) e = set_attrs_persistent<192>();
+  if (e == cudaSuccess) e = set_attrs_persistent<256>();
+  if (e == cudaSuccess) e = set_attrs_inst<32, 4>();
   if (e == cudaSuccess) e = set_attrs_inst<64, 4>();
   if (e == cudaSuccess) e = set_attrs_inst<128, 6>();
   if (e == cudaSuccess) e = set_attrs_inst<256, 4>();
@@ -176,6 +270,16 @@ inline cudaError_t run_gemm(int epi, const void* A, int lda, const void* W, int 
   args.partials = partials;
   args.counters = counters;
   args.red_mode = p.red;
+  if (p.persistent) {
+    switch (p.bn) {
+      case 64: return dispatch_persistent<64>(epi, ta, tw, args, p.ctas, s);
+      case 96: return dispatch_persistent<96>(epi, ta, tw, args, p.ctas, s);
+      case 128: return dispatch_persistent<128>(epi, ta, tw, args, p.ctas, s);
+      case 192: return dispatch_persistent<192>(epi, ta, tw, args, p.ctas, s);
+      case 256: return dispatch_persistent<256>(epi, ta, tw, args, p.ctas, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   dim3 grid(p.n_tiles, p.m_tiles, p.splits);
   const int cz = p.red == GEMM_RED_CLUSTER ? p.splits : 1;
   if (p.bn == 32 && p.stages == 4) return dispatch_epi<32, 4>(epi, ta, tw, args, grid, cz, s);

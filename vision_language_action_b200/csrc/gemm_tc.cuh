@@ -51,6 +51,19 @@ struct GemmArgs {
   const int* pos;        // per-row position, or null: row % pos_mod
   int pos_mod;
   const float2* rope_cs; // [pos][head_dim/2] (cos, sin)
+  // Fused RMSNorm (reading 8), producer side (GE_F32 / GE_ADD_F32): also store
+  // bf16(out) to rb_out and each row's sum of squares over this tile's columns
+  // to ss_out[n_blk * ss_ld + m].
+  bf16* rb_out;
+  int ld_rb;
+  float* ss_out;
+  // Consumer side: scale row m of the accumulator by
+  // rsqrt(sum_{t < ss_tiles} ss_in[t * ss_ld + m] * norm_inv_dim + norm_eps); the
+  // norm's gain is folded into W. A is then the bf16 copy of the raw residual.
+  const float* ss_in;
+  int ss_tiles;
+  int ss_ld;
+  float norm_inv_dim, norm_eps;
   // split-K
   float* partials;       // [tiles][splits][128][BN]   (red_mode GEMM_RED_GLOBAL)
   int* counters;         // [tiles], zero between launches
@@ -83,8 +96,8 @@ struct GemmCfg {
   static constexpr uint32_t B_BYTES = BN * GEMM_BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
-  // ring + barriers/flags area + alignment slack
-  static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 256 + 1024;
+  // ring + barriers/flags (512 B) + row factors (512 B) + alignment slack
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 1024 + 1024;
   // two CTAs per SM when they fit, so a dependent GEMM can start next to this one
   static constexpr int MIN_BLOCKS = SMEM <= 113 * 1024 ? 2 : 1;
   static constexpr size_t RED_TILE = (size_t)GEMM_BM * (BN + 4) * sizeof(float);
@@ -154,6 +167,7 @@ template <int BN>
 struct AccSource {
   uint32_t taddr_row;
   const float* smem_row;  // null: read TMEM
+  float scale = 1.f;      // fused RMSNorm row factor
   SVLA_DEV void get(int c, float (&v)[16]) const {
     if (smem_row == nullptr) {
       tmem_ld16(taddr_row + (uint32_t)c, v);
@@ -168,8 +182,18 @@ struct AccSource {
         v[4 * i + 3] = t.w;
       }
     }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] *= scale;
   }
 };
+
+// Fused RMSNorm row factor of row m (1 when the GEMM consumes no norm).
+SVLA_DEV float norm_row_scale(const GemmArgs& a, int m, bool row_ok) {
+  if (a.ss_in == nullptr || !row_ok) return 1.f;
+  float s = 0.f;
+  for (int t = 0; t < a.ss_tiles; ++t) s += __ldg(a.ss_in + (size_t)t * a.ss_ld + m);
+  return rsqrtf(s * a.norm_inv_dim + a.norm_eps);
+}
 
 // Split-K reduction by the last CTA of a tile: the 128 epilogue threads sum
 // the partial tiles [split][128][BN] in split order (coalesced float4 loads,
@@ -202,7 +226,8 @@ SVLA_DEV void reduce_partials(const float* tile_part, int splits, int rows, floa
 }
 
 template <int BN, int EPI>
-SVLA_DEV void run_epilogue(const GemmArgs& a, const AccSource<BN>& src, int m, int n0, bool row_ok) {
+SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, bool row_ok, float row_scale) {
+  src.scale = row_scale;
   // tcgen05.ld is warp-collective: every lane walks the same columns; only
   // rows inside M store.
   if constexpr (EPI == GE_SWIGLU) {
@@ -265,6 +290,7 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, const AccSource<BN>& src, int m, i
       for (int c = 0; c < HD; c += 16) store16_bf16(dst + c, *reinterpret_cast<float(*)[16]>(x + c), 16);
     }
   } else {
+    float ss = 0.f;  // sum of squares of this row's outputs in this tile (fused RMSNorm)
 #pragma unroll 1
     for (int c = 0; c < BN; c += 16) {
       float v[16];
@@ -273,10 +299,30 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, const AccSource<BN>& src, int m, i
       if (!row_ok || col >= a.N) continue;
       const int ncols = a.N - col;
       add_bias16(v, a.bias, col, a.N);
-      if constexpr (EPI == GE_F32) {
-        store16_f32(reinterpret_cast<float*>(a.out) + (size_t)m * a.ldo + col, v, ncols);
-      } else if constexpr (EPI == GE_ADD_F32) {
-        add16_f32(reinterpret_cast<float*>(a.out) + (size_t)m * a.ldo + col, v, ncols);
+      if constexpr (EPI == GE_F32 || EPI == GE_ADD_F32) {
+        float* dst = reinterpret_cast<float*>(a.out) + (size_t)m * a.ldo + col;
+        if constexpr (EPI == GE_ADD_F32) {
+          if (ncols >= 16) {
+            const float4* d4 = reinterpret_cast<const float4*>(dst);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float4 o = d4[i];
+              v[4 * i] += o.x;
+              v[4 * i + 1] += o.y;
+              v[4 * i + 2] += o.z;
+              v[4 * i + 3] += o.w;
+            }
+          } else {
+            for (int i = 0; i < ncols; ++i) v[i] += dst[i];
+          }
+        }
+        store16_f32(dst, v, ncols);
+        if (a.rb_out) {
+          store16_bf16(a.rb_out + (size_t)m * a.ld_rb + col, v, ncols);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (i < ncols) ss = fmaf(v[i], v[i], ss);
+        }
       } else if constexpr (EPI == GE_BF16) {
         store16_bf16(reinterpret_cast<bf16*>(a.out) + (size_t)m * a.ldo + col, v, ncols);
       } else if constexpr (EPI == GE_SILU_BF16) {
@@ -284,6 +330,9 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, const AccSource<BN>& src, int m, i
         for (int i = 0; i < 16; ++i) v[i] = silu_f(v[i]);
         store16_bf16(reinterpret_cast<bf16*>(a.out) + (size_t)m * a.ldo + col, v, ncols);
       }
+    }
+    if constexpr (EPI == GE_F32 || EPI == GE_ADD_F32) {
+      if (a.ss_out && row_ok) a.ss_out[(size_t)(n0 / BN) * a.ss_ld + m] = ss;
     }
   }
 }
@@ -304,6 +353,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES>::MIN_BLOCKS)
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(bars + 2 * STAGES + 1);
   // misc[0] tmem base, misc[1] abort flag, misc[2] k-blocks issued, misc[3] k-blocks consumed,
   // misc[4] "this CTA reduces"
+  float* misc_scale = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 512);  // [128] row factors
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -407,6 +457,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES>::MIN_BLOCKS)
     const int m = m_blk * GEMM_BM + row;
     const bool row_ok = m < args.M;
     const int n0 = n_blk * BN;
+    const float rscale = norm_row_scale(args, m, row_ok);  // overlaps the main loop
+    misc_scale[row] = rscale;
     bool ok = mbar_wait(acc_bar, 0, lim);
     if (!ok) {
       misc[1] = 1;
@@ -420,7 +472,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES>::MIN_BLOCKS)
       src.taddr_row = tmem_base + ((uint32_t)(quad * 32) << 16);
       src.smem_row = nullptr;
       if (splits == 1) {
-        run_epilogue<BN, EPI>(args, src, m, n0, row_ok);
+        run_epilogue<BN, EPI>(args, src, m, n0, row_ok, rscale);
       } else if (C::CLUSTER_OK && args.red_mode == GEMM_RED_CLUSTER) {
         // stage this split's partial tile in shared memory (the operand ring is idle)
         float* red = reinterpret_cast<float*>(ring);
@@ -458,7 +510,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES>::MIN_BLOCKS)
           reduce_partials<BN>(tile_part, splits, rows, red, threadIdx.x - 64);
           epi_bar();
           src.smem_row = red + row * (BN + 4);
-          run_epilogue<BN, EPI>(args, src, m, n0, row_ok);
+          run_epilogue<BN, EPI>(args, src, m, n0, row_ok, rscale);
           if (threadIdx.x == 64) args.counters[tile] = 0;  // re-arm for the next launch
         }
       }
@@ -517,7 +569,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES>::MIN_BLOCKS)
           AccSource<BN> src;
           src.taddr_row = 0;
           src.smem_row = fin + row * (BN + 4);
-          run_epilogue<BN, EPI>(args, src, m, n_blk * BN, true);
+          run_epilogue<BN, EPI>(args, src, m, n_blk * BN, true, misc_scale[row]);
         }
       }
       cluster_sync();  // peers have finished reading this CTA's partial tile

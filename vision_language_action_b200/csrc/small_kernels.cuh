@@ -67,6 +67,30 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const void* __restrict__ x
 }
 
 // ---------------------------------------------------------------------------
+// Start of the prefix residual stream: x = float(embeds) and, for the first
+// layer's fused RMSNorm, each row's sum of squares (one warp per row).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) residual_init_kernel(const uint16_t* __restrict__ emb, float* __restrict__ x,
+                                                            float* __restrict__ ss, int M, int D) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= M) return;
+  float acc = 0.f;
+  for (int c = lane; c < D / 4; c += 32) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(emb + (size_t)warp * D) + c);
+    const float4 t = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                                 __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+    reinterpret_cast<float4*>(x + (size_t)warp * D)[c] = t;
+    acc += t.x * t.x + t.y * t.y + t.z * t.z + t.w * t.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) ss[warp] = acc;
+}
+
+// ---------------------------------------------------------------------------
 // Prefix positions (reading 2): pos[b, i] = (sum_{j <= i} valid[b, j]) - 1.
 // One warp per query; a query with no valid token records
 // SVLA_ERR_EMPTY_PREFIX (reading 1: every row needs a visible key).

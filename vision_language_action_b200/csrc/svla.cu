@@ -153,6 +153,18 @@ __global__ void interleave_gu_kernel(const uint16_t* __restrict__ src, uint16_t*
   for (int k = threadIdx.x; k < K; k += blockDim.x) dst[(size_t)r * K + k] = src[(size_t)sr * K + k];
 }
 
+// W[n, k] <- bf16(W[n, k] * g[k]): folds an RMSNorm gain into the projection
+// that consumes the normalised activations (the GEMM epilogue applies the
+// per-row 1/rms factor).
+__global__ void fold_gain_kernel(uint16_t* __restrict__ w, const uint16_t* __restrict__ g, int rows, int cols) {
+  const size_t n = (size_t)rows * cols;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const float v = __uint_as_float(((uint32_t)w[i]) << 16) * __uint_as_float(((uint32_t)g[i % cols]) << 16);
+    const __nv_bfloat16 b = __float2bfloat16_rn(v);
+    w[i] = *reinterpret_cast<const uint16_t*>(&b);
+  }
+}
+
 __global__ void bf16_to_f32_kernel(const uint16_t* __restrict__ src, float* __restrict__ dst, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) dst[i] = __uint_as_float(((uint32_t)src[i]) << 16);
@@ -179,6 +191,7 @@ struct svla_handle {
   float* p_x = nullptr;
   bf16 *p_y = nullptr, *p_q = nullptr, *p_o = nullptr, *p_h = nullptr;
   int* p_pos = nullptr;
+  float* p_ss = nullptr;  // fused RMSNorm: per-(n-tile, row) sums of squares of the residual
   float* p_part = nullptr;
   int* p_cnt = nullptr;
   // denoise workspace
@@ -186,6 +199,7 @@ struct svla_handle {
   bf16 *e_y = nullptr, *e_q = nullptr, *e_k = nullptr, *e_v = nullptr, *e_o = nullptr, *e_h = nullptr;
   bf16 *e_a = nullptr, *e_h1 = nullptr, *kvx = nullptr;
   float* e_c = nullptr;
+  float* e_ss = nullptr;
   float* e_part = nullptr;
   int* e_cnt = nullptr;
   float* noise_buf = nullptr;
@@ -201,6 +215,7 @@ namespace {
 
 constexpr size_t PART_BYTES = (size_t)NUM_SMS_B200 * GEMM_BM * 256 * sizeof(float);
 constexpr int CNT_INTS = 4096;
+constexpr int SS_TILES_MAX = 128;  // n-tiles of a residual-producing GEMM (width <= 2048 at >= 16-wide tiles)
 
 svla_status fail(svla_handle* h, svla_status s, const std::string& msg) {
   const std::string m = std::string(status_str(s)) + ": " + msg;
@@ -306,6 +321,27 @@ cudaError_t attention(const bf16* q, int ldq, const bf16* k, const bf16* v, int 
     if (e_ != cudaSuccess) return e_;         \
   } while (0)
 
+// ---- fused RMSNorm plumbing ------------------------------------------------
+// The GEMM that writes a residual stream also writes its bf16 copy `rb` and the
+// per-(n-tile, row) sums of squares `ss`; the next GEMM takes `rb` as A (its
+// weights carry the norm gain) and scales row m by rsqrt(sum ss / D + eps).
+int residual_tiles(int M, int N, int K) { return plan_gemm(M, N, K, 0, gemm_min_bn(GE_ADD_F32)).n_tiles; }
+
+void norm_producer(GemmArgs& a, bf16* rb, int ld, float* ss, int M) {
+  a.rb_out = rb;
+  a.ld_rb = ld;
+  a.ss_out = ss;
+  a.ss_ld = M;
+}
+
+void norm_consumer(GemmArgs& a, const float* ss, int tiles, int M, int D, float eps) {
+  a.ss_in = ss;
+  a.ss_tiles = tiles;
+  a.ss_ld = M;
+  a.norm_inv_dim = 1.f / (float)D;
+  a.norm_eps = eps;
+}
+
 // ---- prefill schedule -------------------------------------------------------
 cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pad, int B, int L, void* kv,
                            cudaStream_t s) {
@@ -314,15 +350,16 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
   const int qw = c.p_heads * hd, kvw = c.p_kv_heads * hd;
   bf16* cache = reinterpret_cast<bf16*>(kv);
   const size_t layer_elems = (size_t)B * L * kvw;
+  bf16* rb = h->p_y;  // bf16 copy of the residual stream
   SVLA_TRY(launch_pdl(positions_kernel, dim3((B + 7) / 8), dim3(256), 0, s, pad, B, L, h->p_pos, h->status));
+  SVLA_TRY(launch_pdl(residual_init_kernel, dim3((M + 7) / 8), dim3(256), 0, s,
+                      reinterpret_cast<const uint16_t*>(embeds), h->p_x, h->p_ss, M, D));
+  const int o_tiles = residual_tiles(M, D, qw), d_tiles = residual_tiles(M, D, c.p_ffn);
   for (int l = 0; l < c.p_layers; ++l) {
     const Entry* e = &h->lay.p[9 * l];
     bf16* Kl = cache + (size_t)l * layer_elems;
     bf16* Vl = cache + (size_t)(c.p_layers + l) * layer_elems;
-    if (l == 0)
-      SVLA_TRY(rmsnorm(embeds, true, h->p_x, h->W(e[0].off), M, D, c.rms_eps, h->p_y, s));
-    else
-      SVLA_TRY(rmsnorm(h->p_x, false, nullptr, h->W(e[0].off), M, D, c.rms_eps, h->p_y, s));
+    // QKV of RMSNorm(x): the residual's bf16 copy (the embeddings themselves on layer 0)
     GemmArgs qa = out_args(nullptr, 0);
     qa.q_out = h->p_q;
     qa.ldq = qw;
@@ -334,16 +371,21 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
     qa.pos = h->p_pos;
     qa.pos_mod = 1;
     qa.rope_cs = h->rope_cs;
-    SVLA_TRY(gemm(h, hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32, h->p_y, D, h->W(e[1].off), D, M, qw + 2 * kvw, D, qa,
+    norm_consumer(qa, h->p_ss, l == 0 ? 1 : d_tiles, M, D, c.rms_eps);
+    const bf16* xin = l == 0 ? reinterpret_cast<const bf16*>(embeds) : rb;
+    SVLA_TRY(gemm(h, hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32, xin, D, h->W(e[1].off), D, M, qw + 2 * kvw, D, qa,
                   h->p_part, h->p_cnt, s));
     if (l == c.p_layers - 1) break;  // nothing reads the last layer's attention / MLP output
     SVLA_TRY(attention(h->p_q, qw, Kl, Vl, kvw, pad, B, c.p_heads, c.p_kv_heads, hd, L, L, 0, h->p_o, qw, s));
-    SVLA_TRY(gemm(h, GE_ADD_F32, h->p_o, qw, h->W(e[4].off), qw, M, D, qw, out_args(h->p_x, D), h->p_part, h->p_cnt, s));
-    SVLA_TRY(rmsnorm(h->p_x, false, nullptr, h->W(e[5].off), M, D, c.rms_eps, h->p_y, s));
-    SVLA_TRY(gemm(h, GE_SWIGLU, h->p_y, D, h->W(e[6].off), D, M, 2 * c.p_ffn, D, out_args(h->p_h, c.p_ffn), h->p_part,
-                  h->p_cnt, s));
-    SVLA_TRY(gemm(h, GE_ADD_F32, h->p_h, c.p_ffn, h->W(e[8].off), c.p_ffn, M, D, c.p_ffn, out_args(h->p_x, D),
-                  h->p_part, h->p_cnt, s));
+    GemmArgs oa = out_args(h->p_x, D);
+    norm_producer(oa, rb, D, h->p_ss, M);
+    SVLA_TRY(gemm(h, GE_ADD_F32, h->p_o, qw, h->W(e[4].off), qw, M, D, qw, oa, h->p_part, h->p_cnt, s));
+    GemmArgs ga = out_args(h->p_h, c.p_ffn);
+    norm_consumer(ga, h->p_ss, o_tiles, M, D, c.rms_eps);
+    SVLA_TRY(gemm(h, GE_SWIGLU, rb, D, h->W(e[6].off), D, M, 2 * c.p_ffn, D, ga, h->p_part, h->p_cnt, s));
+    GemmArgs da = out_args(h->p_x, D);
+    norm_producer(da, rb, D, h->p_ss, M);
+    SVLA_TRY(gemm(h, GE_ADD_F32, h->p_h, c.p_ffn, h->W(e[8].off), c.p_ffn, M, D, c.p_ffn, da, h->p_part, h->p_cnt, s));
   }
   return cudaSuccess;
 }
@@ -357,6 +399,7 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
   const int Mp = B * L;
   const bf16* cache = reinterpret_cast<const bf16*>(kv);
   const size_t layer_elems = (size_t)Mp * pkvw;
+  bf16* rb = h->e_y;  // bf16 copy of the expert residual stream
   if (actions != noise) SVLA_TRY(cudaMemcpyAsync(actions, noise, (size_t)M * A * sizeof(float), cudaMemcpyDeviceToDevice, s));
   // hoisted cross K/V projection (once per query, not per step)
   for (int l = 1; l < c.e_layers; l += 2) {
@@ -371,6 +414,8 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
   const Layout& Lh = h->lay;
   int se_blocks = (M + SE_WARPS - 1) / SE_WARPS;
   if (se_blocks > 2 * NUM_SMS_B200) se_blocks = 2 * NUM_SMS_B200;
+  const int t2_tiles = residual_tiles(M, E, E), o_tiles = residual_tiles(M, E, qw);
+  const int d_tiles = residual_tiles(M, E, c.e_ffn);
   for (int k = 0; k < n_steps; ++k) {
     StepBeginArgs sb;
     sb.x = actions;
@@ -388,14 +433,15 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
     sb.c_out = h->e_c;
     sb.nA = (M + 7) / 8;
     SVLA_TRY(launch_pdl(step_begin_kernel, dim3(sb.nA + (E + 7) / 8), dim3(256), 0, s, sb));
-    // time MLP: h1 = silu(W_t1[:, :E] a + c), r = W_t2 h1 + b_t2
+    // time MLP: h1 = silu(W_t1[:, :E] a + c), r = W_t2 h1 + b_t2 (the residual stream starts here)
     SVLA_TRY(gemm(h, GE_SILU_BF16, h->e_a, E, h->W(Lh.w_t1.off), 2 * E, M, E, E, out_args(h->e_h1, E, h->e_c),
                   h->e_part, h->e_cnt, s));
-    SVLA_TRY(gemm(h, GE_F32, h->e_h1, E, h->W(Lh.w_t2.off), E, M, E, E, out_args(h->e_r, E, h->b_t2_f32), h->e_part,
-                  h->e_cnt, s));
+    GemmArgs ta = out_args(h->e_r, E, h->b_t2_f32);
+    norm_producer(ta, rb, E, h->e_ss, M);
+    SVLA_TRY(gemm(h, GE_F32, h->e_h1, E, h->W(Lh.w_t2.off), E, M, E, E, ta, h->e_part, h->e_cnt, s));
     for (int l = 0; l < c.e_layers; ++l) {
       const Entry* e = &Lh.e[9 * l];
-      SVLA_TRY(rmsnorm(h->e_r, false, nullptr, h->W(e[0].off), M, E, c.rms_eps, h->e_y, s));
+      const int in_tiles = l == 0 ? t2_tiles : d_tiles;
       if (l % 2 == 0) {
         GemmArgs qa = out_args(nullptr, 0);
         qa.q_out = h->e_q;
@@ -408,24 +454,29 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
         qa.pos = nullptr;
         qa.pos_mod = H;  // chunk positions 0..H-1 (reading 4)
         qa.rope_cs = h->rope_cs;
-        SVLA_TRY(gemm(h, hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32, h->e_y, E, h->W(e[1].off), E, M, qw + 2 * kvw, E,
-                      qa, h->e_part, h->e_cnt, s));
+        norm_consumer(qa, h->e_ss, in_tiles, M, E, c.rms_eps);
+        SVLA_TRY(gemm(h, hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32, rb, E, h->W(e[1].off), E, M, qw + 2 * kvw, E, qa,
+                      h->e_part, h->e_cnt, s));
         SVLA_TRY(attention(h->e_q, qw, h->e_k, h->e_v, kvw, nullptr, B, c.e_heads, c.e_kv_heads, hd, H, H, 1, h->e_o,
                            qw, s));
       } else {
-        SVLA_TRY(gemm(h, GE_BF16, h->e_y, E, h->W(e[1].off), E, M, qw, E, out_args(h->e_q, qw), h->e_part, h->e_cnt,
-                      s));
+        GemmArgs qa = out_args(h->e_q, qw);
+        norm_consumer(qa, h->e_ss, in_tiles, M, E, c.rms_eps);
+        SVLA_TRY(gemm(h, GE_BF16, rb, E, h->W(e[1].off), E, M, qw, E, qa, h->e_part, h->e_cnt, s));
         const bf16* kx = h->kvx + (size_t)(l / 2) * 2 * Mp * kvw;
         SVLA_TRY(attention(h->e_q, qw, kx, kx + (size_t)Mp * kvw, kvw, pad, B, c.e_heads, c.e_kv_heads, hd, H, L, 0,
                            h->e_o, qw, s));
       }
-      SVLA_TRY(gemm(h, GE_ADD_F32, h->e_o, qw, h->W(e[4].off), qw, M, E, qw, out_args(h->e_r, E), h->e_part,
-                    h->e_cnt, s));
-      SVLA_TRY(rmsnorm(h->e_r, false, nullptr, h->W(e[5].off), M, E, c.rms_eps, h->e_y, s));
-      SVLA_TRY(gemm(h, GE_SWIGLU, h->e_y, E, h->W(e[6].off), E, M, 2 * c.e_ffn, E, out_args(h->e_h, c.e_ffn),
-                    h->e_part, h->e_cnt, s));
-      SVLA_TRY(gemm(h, GE_ADD_F32, h->e_h, c.e_ffn, h->W(e[8].off), c.e_ffn, M, E, c.e_ffn, out_args(h->e_r, E),
-                    h->e_part, h->e_cnt, s));
+      GemmArgs oa = out_args(h->e_r, E);
+      norm_producer(oa, rb, E, h->e_ss, M);
+      SVLA_TRY(gemm(h, GE_ADD_F32, h->e_o, qw, h->W(e[4].off), qw, M, E, qw, oa, h->e_part, h->e_cnt, s));
+      GemmArgs ga = out_args(h->e_h, c.e_ffn);
+      norm_consumer(ga, h->e_ss, o_tiles, M, E, c.rms_eps);
+      SVLA_TRY(gemm(h, GE_SWIGLU, rb, E, h->W(e[6].off), E, M, 2 * c.e_ffn, E, ga, h->e_part, h->e_cnt, s));
+      GemmArgs da = out_args(h->e_r, E);
+      norm_producer(da, rb, E, h->e_ss, M);
+      SVLA_TRY(gemm(h, GE_ADD_F32, h->e_h, c.e_ffn, h->W(e[8].off), c.e_ffn, M, E, c.e_ffn, da, h->e_part, h->e_cnt,
+                    s));
     }
     StepEndArgs se;
     se.r = h->e_r;
@@ -566,6 +617,23 @@ svla_status svla_create(const svla_config* cfg, const void* blob, size_t blob_by
     cudaFree(tmp);
     if (e != cudaSuccess) return bail(e, "gate/up layout");
   }
+  // fold the RMSNorm gains into the projections that consume the normalised
+  // activations: QKV (in_norm) and gate/up (post_norm) of every layer, and the
+  // expert's q projection on cross-attention layers
+  for (int l = 0; l < c.p_layers + c.e_layers && e == cudaSuccess; ++l) {
+    const bool pre = l < c.p_layers;
+    const Entry* en = pre ? &lay.p[9 * l] : &lay.e[9 * (l - c.p_layers)];
+    const int K = pre ? c.p_width : c.e_width;
+    const int F = pre ? c.p_ffn : c.e_ffn;
+    const int qrows = pre ? (c.p_heads + 2 * c.p_kv_heads) * c.head_dim
+                          : ((l - c.p_layers) % 2 == 0 ? (c.e_heads + 2 * c.e_kv_heads) * c.head_dim
+                                                       : c.e_heads * c.head_dim);
+    fold_gain_kernel<<<512, 256>>>(h->w + en[1].off, h->w + en[0].off, qrows, K);
+    fold_gain_kernel<<<512, 256>>>(h->w + en[6].off, h->w + en[5].off, 2 * F, K);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return bail(e, "gain folding");
   if ((e = halloc(h, &h->b_t2_f32, c.e_width)) != cudaSuccess) return bail(e, "bias");
   bf16_to_f32_kernel<<<(c.e_width + 255) / 256, 256>>>(h->w + lay.b_t2.off, h->b_t2_f32, c.e_width);
   // RoPE table (reading 3), computed in double on the host
@@ -604,6 +672,8 @@ svla_status svla_create(const svla_config* cfg, const void* blob, size_t blob_by
   if ((e = halloc(h, &h->p_o, Mp * pq)) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->p_h, Mp * c.p_ffn)) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->p_pos, Mp)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->p_ss, (size_t)SS_TILES_MAX * Mp)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_ss, (size_t)SS_TILES_MAX * Me)) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->e_r, Me * c.e_width)) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->e_y, Me * c.e_width)) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->e_q, Me * eq)) != cudaSuccess) return bail(e, "workspace");
