@@ -34,9 +34,11 @@ import synth  # noqa: E402
 METRIC = "ms per 50-action chunk (b=1)"
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM bytes (read + write) per launch of the GEMM kernel from the ncu capture
-# summarised in profiles/; None until a capture of the current kernel exists.
-NCU_TRAFFIC_PER_LAUNCH = None
+# DRAM bytes (read + write) per launch of the batch-1 GEMM kernel: mean of the
+# three launches of the ncu --set full capture summarised in
+# profiles/gemm_tc_kernel_smolvla_b1.md. Set to None whenever the kernel changes
+# until it is captured again.
+NCU_TRAFFIC_PER_LAUNCH = 3.70e6
 
 
 def _peaks():
