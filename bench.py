@@ -38,7 +38,7 @@ L2_BYTES = 126 * 1024 * 1024
 # three launches of the ncu --set full capture summarised in
 # profiles/gemm_tc_kernel_smolvla_b1.md. Set to None whenever the kernel changes
 # until it is captured again.
-NCU_TRAFFIC_PER_LAUNCH = 3.70e6
+NCU_TRAFFIC_PER_LAUNCH = None
 
 
 def _peaks():

@@ -40,6 +40,7 @@ def gemm(epi, A, W, C, bias=None, splits=0, status=None):
 SHAPES = [
     (1, 320, 64), (50, 720, 960), (50, 1600, 720), (63, 960, 720), (64, 320, 320), (65, 720, 2048),
     (177, 1600, 960), (177, 960, 2560), (1600, 4096, 720), (1600, 720, 2048), (300, 96, 128),
+    (513, 720, 960), (2568, 1600, 960), (5664, 5120, 960),
 ]
 
 

@@ -36,12 +36,13 @@ struct AttnArgs {
 constexpr int ATT_BQ = 64;
 constexpr int ATT_BK = 64;
 constexpr int ATT_THREADS = 128;
+constexpr int ATT_NBUF = 2;  // key/value tiles in flight (double buffering)
 
 template <int HD>
 struct AttnCfg {
   static constexpr int LDS = HD + 8;  // padded smem row (elements): conflict-free ldmatrix
   static constexpr int TILE = ATT_BK * LDS;
-  static constexpr size_t SMEM = (size_t)(ATT_BQ * LDS + 4 * TILE) * 2 + 2 * ATT_BK;
+  static constexpr size_t SMEM = (size_t)(ATT_BQ * LDS + 2 * ATT_NBUF * TILE) * 2 + ATT_NBUF * ATT_BK;
 };
 
 SVLA_DEV void cp_async16(uint32_t dst, const void* src, bool pred) {
@@ -83,9 +84,9 @@ __global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a
 
   extern __shared__ __align__(16) uint8_t att_smem[];
   bf16* sQ = reinterpret_cast<bf16*>(att_smem);
-  bf16* sK = sQ + ATT_BQ * LDS;       // [2][64][LDS]
-  bf16* sV = sK + 2 * C::TILE;        // [2][64][LDS]
-  uint8_t* sF = reinterpret_cast<uint8_t*>(sV + 2 * C::TILE);  // [2][64] key flags
+  bf16* sK = sQ + ATT_BQ * LDS;           // [NBUF][64][LDS]
+  bf16* sV = sK + ATT_NBUF * C::TILE;     // [NBUF][64][LDS]
+  uint8_t* sF = reinterpret_cast<uint8_t*>(sV + ATT_NBUF * C::TILE);  // [NBUF][64] key flags
 
   griddep_launch_dependents();
   griddep_wait();
@@ -126,8 +127,12 @@ __global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a
       sF[buf * ATT_BK + tid] = f;
     }
   };
-  load_kv(0, 0);
-  cp_async_commit();
+  // tiles 0 .. NBUF-1 in flight (group 0 also carries Q); one commit group per tile
+#pragma unroll
+  for (int t = 0; t < ATT_NBUF; ++t) {
+    if (t < nkt) load_kv(t, t);
+    cp_async_commit();
+  }
 
   const int g = lane >> 2, t4 = lane & 3;
   const int row0 = q0 + warp * 16 + g;  // this thread's rows: row0 and row0 + 8
@@ -140,14 +145,8 @@ __global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a
   float l_run[2] = {0.f, 0.f};
 
   for (int kt = 0; kt < nkt; ++kt) {
-    const int buf = kt & 1;
-    if (kt + 1 < nkt) {
-      load_kv(kt + 1, buf ^ 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
+    const int buf = kt % ATT_NBUF;
+    cp_async_wait<ATT_NBUF - 1>();  // tile kt (and Q) have landed; later tiles may still fly
     __syncthreads();
     if (kt == 0) {
       // Q fragments (A operand, row-major 16 x 16 per k-step)
@@ -243,7 +242,9 @@ __global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a
         mma_bf16_16816(o[2 * nd2 + 1], pa[kk], b2, b3);
       }
     }
-    __syncthreads();  // this buffer is refilled by the next iteration's prefetch
+    __syncthreads();  // every warp is done with this buffer: refill it with tile kt + NBUF
+    if (kt + ATT_NBUF < nkt) load_kv(kt + ATT_NBUF, buf);
+    cp_async_commit();
   }
 
   // finish: row sums across the quad, normalise, store bf16

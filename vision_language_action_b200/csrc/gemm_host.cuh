@@ -4,6 +4,7 @@
 
 #include <mutex>
 
+#include "gemm_pair.cuh"
 #include "gemm_persistent.cuh"
 
 namespace svla {
@@ -46,7 +47,8 @@ struct GemmPlan {
   int red = GEMM_RED_NONE;
   int m_tiles = 1, n_tiles = 1;
   bool persistent = false;  // one CTA per SM walking the tiles, double-buffered accumulators
-  int ctas = 0;             // grid of the persistent kernel
+  bool pair = false;        // persistent CTA pairs (cta_group::2) on 256 x BN tiles
+  int ctas = 0;             // grid of the persistent kernel (CTAs, twice the pairs for `pair`)
 };
 
 // operand-ring depth of the persistent kernel: as many stages as fit in the
@@ -94,6 +96,26 @@ inline GemmPlan plan_gemm(int M, int N, int K, int forced_splits, int min_bn = 3
     p.splits = 1;
     const int t = p.m_tiles * p.n_tiles;
     p.ctas = t < NUM_SMS_B200 ? t : NUM_SMS_B200;
+    // CTA pairs: per CTA a 128 x BN block moves 128 + BN/2 rows of K per stage.
+    // Measured on B200 they win on wide outputs at large M (12800 x 4096 x 720:
+    // 702 vs 633 TFLOP/s; 5664 x 5120 x 960: 813 vs 368) and lose at M = 1600 and
+    // on narrow N (wave quantisation), so they are used only there.
+    if (M >= 4096 && N >= 2048) {
+      const int m2 = (M + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
+      const int pairs_max = NUM_SMS_B200 / 2;
+      for (int bn : {128, 256}) {
+        const int tp = m2 * ((N + bn - 1) / bn);
+        const long waves = (tp + pairs_max - 1) / pairs_max;
+        const long cost = waves * (GEMM_BM + bn / 2);
+        if (cost <= best) {
+          best = cost;
+          p.bn = bn;
+          p.pair = true;
+          p.n_tiles = (N + bn - 1) / bn;
+          p.ctas = 2 * (tp < pairs_max ? tp : pairs_max);
+        }
+      }
+    }
     return p;
   }
   auto clamp_splits = [&](int sp) {
@@ -138,6 +160,59 @@ inline cudaError_t launch_persistent_inst(const CUtensorMap& ta, const CUtensorM
   cfg.attrs = at;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, gemm_tc_persistent_kernel<BN, EPI, ST>, ta, tw, args);
+}
+
+template <int BN, int EPI>
+inline cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& args, int ctas,
+                                    cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = PairCfg<BN>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = 2;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, gemm_tc_pair_kernel<BN, EPI>, ta, tw, args);
+}
+
+template <int BN>
+inline cudaError_t dispatch_pair(int epi, const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& a, int ctas,
+                                 cudaStream_t s) {
+  switch (epi) {
+    case GE_F32: return launch_pair_inst<BN, GE_F32>(ta, tw, a, ctas, s);
+    case GE_BF16: return launch_pair_inst<BN, GE_BF16>(ta, tw, a, ctas, s);
+    case GE_ADD_F32: return launch_pair_inst<BN, GE_ADD_F32>(ta, tw, a, ctas, s);
+    case GE_SILU_BF16: return launch_pair_inst<BN, GE_SILU_BF16>(ta, tw, a, ctas, s);
+    case GE_SWIGLU: return launch_pair_inst<BN, GE_SWIGLU>(ta, tw, a, ctas, s);
+    case GE_QKV_ROPE64: return launch_pair_inst<BN, GE_QKV_ROPE64>(ta, tw, a, ctas, s);
+    case GE_QKV_ROPE32: return launch_pair_inst<BN, GE_QKV_ROPE32>(ta, tw, a, ctas, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int BN>
+inline cudaError_t set_attrs_pair() {
+  const int smem = (int)PairCfg<BN>::SMEM;
+  cudaError_t e = cudaSuccess;
+#define SVLA_SETQ(EPI)                                                                                       \
+  if (e == cudaSuccess)                                                                                      \
+    e = cudaFuncSetAttribute(gemm_tc_pair_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  SVLA_SETQ(GE_F32)
+  SVLA_SETQ(GE_BF16)
+  SVLA_SETQ(GE_ADD_F32)
+  SVLA_SETQ(GE_SILU_BF16)
+  SVLA_SETQ(GE_SWIGLU)
+  SVLA_SETQ(GE_QKV_ROPE64)
+  SVLA_SETQ(GE_QKV_ROPE32)
+#undef SVLA_SETQ
+  return e;
 }
 
 template <int BN>
@@ -245,7 +320,9 @@ inline cudaError_t set_attrs_inst() {
 }
 
 inline cudaError_t gemm_set_attrs() {
-  cudaError_t e = set_attrs_persistent<64>();
+  cudaError_t e = set_attrs_pair<128>();
+  if (e == cudaSuccess) e = set_attrs_pair<256>();
+  if (e == cudaSuccess) e = set_attrs_persistent<64>();
   if (e == cudaSuccess) e = set_attrs_persistent<96>();
   if (e == cudaSuccess) e = set_attrs_persistent<128>();
   if (e == cudaSuccess) e = set_attrs_persistent<192>();
@@ -262,7 +339,7 @@ inline cudaError_t run_gemm(int epi, const void* A, int lda, const void* W, int 
                             GemmArgs args, const GemmPlan& p, float* partials, int* counters, cudaStream_t s) {
   CUtensorMap ta, tw;
   if (!make_tmap_bf16(&ta, A, M, K, lda, GEMM_BM)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16(&tw, W, N, K, ldw, p.bn)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tw, W, N, K, ldw, p.pair ? p.bn / 2 : p.bn)) return cudaErrorInvalidValue;
   if (p.red == GEMM_RED_GLOBAL && (!partials || !counters)) return cudaErrorInvalidValue;
   args.M = M;
   args.N = N;
@@ -270,6 +347,11 @@ inline cudaError_t run_gemm(int epi, const void* A, int lda, const void* W, int 
   args.partials = partials;
   args.counters = counters;
   args.red_mode = p.red;
+  if (p.pair) {
+    if (p.bn == 128) return dispatch_pair<128>(epi, ta, tw, args, p.ctas, s);
+    if (p.bn == 256) return dispatch_pair<256>(epi, ta, tw, args, p.ctas, s);
+    return cudaErrorInvalidValue;
+  }
   if (p.persistent) {
     switch (p.bn) {
       case 64: return dispatch_persistent<64>(epi, ta, tw, args, p.ctas, s);

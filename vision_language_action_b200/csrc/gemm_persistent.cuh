@@ -171,6 +171,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int mb, nb;
       tile_mn((int)blockIdx.x + tc * (int)gridDim.x, mb, nb);
       const int m = mb * GEMM_BM + row;
+      prefetch_epilogue_inputs<BN, EPI>(args, m, nb * BN, m < args.M);
       const float rscale = norm_row_scale(args, m, m < args.M);  // before the accumulator is ready
       bool ok = mbar_wait(accf_bar(buf), aph, lim);
       if (!ok) {

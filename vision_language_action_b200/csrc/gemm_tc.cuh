@@ -187,6 +187,20 @@ struct AccSource {
   }
 };
 
+// The residual-add epilogue reads its row segment of the output: start that
+// read (into L1) as soon as the earlier kernels are complete, long before the
+// accumulator is ready.
+template <int BN, int EPI>
+SVLA_DEV void prefetch_epilogue_inputs(const GemmArgs& a, int m, int n0, bool row_ok) {
+  if constexpr (EPI == GE_ADD_F32) {
+    if (row_ok && n0 < a.N) {
+      const float* p = reinterpret_cast<const float*>(a.out) + (size_t)m * a.ldo + n0;
+#pragma unroll
+      for (int c = 0; c < BN; c += 32) prefetch_l1(p + c);
+    }
+  }
+}
+
 // Fused RMSNorm row factor of row m (1 when the GEMM consumes no norm).
 SVLA_DEV float norm_row_scale(const GemmArgs& a, int m, bool row_ok) {
   if (a.ss_in == nullptr || !row_ok) return 1.f;
@@ -457,6 +471,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES>::MIN_BLOCKS)
     const int m = m_blk * GEMM_BM + row;
     const bool row_ok = m < args.M;
     const int n0 = n_blk * BN;
+    prefetch_epilogue_inputs<BN, EPI>(args, m, n0, row_ok);
     const float rscale = norm_row_scale(args, m, row_ok);  // overlaps the main loop
     misc_scale[row] = rscale;
     bool ok = mbar_wait(acc_bar, 0, lim);

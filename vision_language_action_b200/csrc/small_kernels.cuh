@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(256) residual_init_kernel(const uint16_t* __re
   const int lane = threadIdx.x & 31;
   if (warp >= M) return;
   float acc = 0.f;
+#pragma unroll 8
   for (int c = lane; c < D / 4; c += 32) {
     const uint2 u = __ldg(reinterpret_cast<const uint2*>(emb + (size_t)warp * D) + c);
     const float4 t = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
@@ -192,8 +193,25 @@ __global__ void __launch_bounds__(256) step_begin_kernel(const StepBeginArgs p) 
     const int o = ((int)blockIdx.x - p.nA) * 8 + warp;
     float acc = 0.f;
     if (o < p.De) {
-      const uint16_t* wr = reinterpret_cast<const uint16_t*>(p.w_t1) + (size_t)o * 2 * p.De + p.De;
-      for (int i = lane; i < p.De; i += 32) acc = fmaf(bf2f(wr[i]), es[i], acc);
+      // W_t1[o, De:] as 16-byte chunks (De is a multiple of 16), all loads issued first
+      const uint4* wr = reinterpret_cast<const uint4*>(p.w_t1 + (size_t)o * 2 * p.De + p.De);
+      const int n8 = p.De / 8;
+      uint4 w[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (lane + 32 * u < n8) w[u] = __ldg(wr + lane + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = lane + 32 * u;
+        if (c < n8) {
+          const uint32_t q[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            acc = fmaf(__uint_as_float(q[k] << 16), es[8 * c + 2 * k], acc);
+            acc = fmaf(__uint_as_float(q[k] & 0xffff0000u), es[8 * c + 2 * k + 1], acc);
+          }
+        }
+      }
 #pragma unroll
       for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
     }
@@ -244,7 +262,20 @@ __global__ void __launch_bounds__(256) step_end_kernel(const StepEndArgs p) {
   {
     const int n16 = p.A * p.De / 8;  // 16-byte chunks (A * De is a multiple of 8)
     const uint4* src = reinterpret_cast<const uint4*>(p.w_out);
-    for (int i = threadIdx.x; i < n16; i += blockDim.x) reinterpret_cast<uint4*>(se_w)[i] = __ldg(src + i);
+    // batches of 8 independent loads per thread, so the copy is not a chain of round trips
+    for (int i0 = threadIdx.x; i0 < n16; i0 += 8 * blockDim.x) {
+      uint4 t[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n16) t[u] = __ldg(src + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n16) reinterpret_cast<uint4*>(se_w)[i] = t[u];
+      }
+    }
   }
   __syncthreads();
   griddep_wait();
