@@ -48,6 +48,7 @@ struct GemmPlan {
   int m_tiles = 1, n_tiles = 1;
   bool persistent = false;  // one CTA per SM walking the tiles, double-buffered accumulators
   bool pair = false;        // persistent CTA pairs (cta_group::2) on 256 x BN tiles
+  int a_rows = GEMM_BM;     // 64: batch-1 variant, 64-row A box and every k-block in flight
   int ctas = 0;             // grid of the persistent kernel (CTAs, twice the pairs for `pair`)
 };
 
@@ -129,6 +130,33 @@ inline GemmPlan plan_gemm(int M, int N, int K, int forced_splits, int min_bn = 3
   } else if (tiles(128) >= 100) {
     p.bn = 128;
     p.stages = 6;
+  } else if (M <= 64 && forced_splits <= 0) {
+    // batch 1: 64-row A boxes, 6 (BN 64) / 8 (BN 32) stages hold all of a CTA's
+    // k-blocks; the most CTAs within one wave, then the fewest splits
+    int best_ctas = -1;
+    for (int bn : {64, 32}) {
+      if (bn < min_bn) continue;
+      const int t = (N + bn - 1) / bn;
+      const int st = bn == 64 ? 6 : 8;
+      for (int sp = 1; sp <= GEMM_MAX_CLUSTER && sp <= KB; ++sp) {
+        if ((KB + sp - 1) / sp > st) continue;
+        const int c = t * sp;
+        if (c > NUM_SMS_B200) break;
+        if (c > best_ctas || (c == best_ctas && sp < p.splits)) {
+          best_ctas = c;
+          p.bn = bn;
+          p.stages = st;
+          p.splits = sp;
+        }
+      }
+    }
+    if (best_ctas < 0) {  // K too deep for one pass: the 128-row configuration below
+      p.bn = 64;
+      p.stages = 4;
+      p.splits = 1;
+    } else {
+      p.a_rows = 64;
+    }
   } else {
     const int t64 = tiles(64), t32 = tiles(32);
     const int s64 = clamp_splits(NUM_SMS_B200 / t64), s32 = clamp_splits(NUM_SMS_B200 / t32);
@@ -261,13 +289,13 @@ inline size_t gemm_partials_bytes(const GemmPlan& p) {
 
 // One instance: launched with programmatic stream serialization (PDL) and, for
 // the cluster reduction, a (1, 1, splits) cluster.
-template <int BN, int ST, int EPI>
+template <int BN, int ST, int EPI, int AR = GEMM_BM>
 inline cudaError_t launch_gemm_inst(const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& args, dim3 grid,
                                     int cluster_z, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(GEMM_THREADS);
-  cfg.dynamicSmemBytes = GemmCfg<BN, ST>::SMEM;
+  cfg.dynamicSmemBytes = GemmCfg<BN, ST, AR>::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute at[2];
   int n = 0;
@@ -283,31 +311,31 @@ inline cudaError_t launch_gemm_inst(const CUtensorMap& ta, const CUtensorMap& tw
   }
   cfg.attrs = at;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, EPI, ST>, ta, tw, args);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, EPI, ST, AR>, ta, tw, args);
 }
 
-template <int BN, int ST>
+template <int BN, int ST, int AR = GEMM_BM>
 inline cudaError_t dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& a, dim3 g,
                                 int cz, cudaStream_t s) {
   switch (epi) {
-    case GE_F32: return launch_gemm_inst<BN, ST, GE_F32>(ta, tw, a, g, cz, s);
-    case GE_BF16: return launch_gemm_inst<BN, ST, GE_BF16>(ta, tw, a, g, cz, s);
-    case GE_ADD_F32: return launch_gemm_inst<BN, ST, GE_ADD_F32>(ta, tw, a, g, cz, s);
-    case GE_SILU_BF16: return launch_gemm_inst<BN, ST, GE_SILU_BF16>(ta, tw, a, g, cz, s);
-    case GE_SWIGLU: return launch_gemm_inst<BN, ST, GE_SWIGLU>(ta, tw, a, g, cz, s);
-    case GE_QKV_ROPE64: return launch_gemm_inst<BN, ST, GE_QKV_ROPE64>(ta, tw, a, g, cz, s);
-    case GE_QKV_ROPE32: return launch_gemm_inst<BN, ST, GE_QKV_ROPE32>(ta, tw, a, g, cz, s);
+    case GE_F32: return launch_gemm_inst<BN, ST, GE_F32, AR>(ta, tw, a, g, cz, s);
+    case GE_BF16: return launch_gemm_inst<BN, ST, GE_BF16, AR>(ta, tw, a, g, cz, s);
+    case GE_ADD_F32: return launch_gemm_inst<BN, ST, GE_ADD_F32, AR>(ta, tw, a, g, cz, s);
+    case GE_SILU_BF16: return launch_gemm_inst<BN, ST, GE_SILU_BF16, AR>(ta, tw, a, g, cz, s);
+    case GE_SWIGLU: return launch_gemm_inst<BN, ST, GE_SWIGLU, AR>(ta, tw, a, g, cz, s);
+    case GE_QKV_ROPE64: return launch_gemm_inst<BN, ST, GE_QKV_ROPE64, AR>(ta, tw, a, g, cz, s);
+    case GE_QKV_ROPE32: return launch_gemm_inst<BN, ST, GE_QKV_ROPE32, AR>(ta, tw, a, g, cz, s);
   }
   return cudaErrorInvalidValue;
 }
 
-template <int BN, int ST>
+template <int BN, int ST, int AR = GEMM_BM>
 inline cudaError_t set_attrs_inst() {
   cudaError_t e = cudaSuccess;
-  const int smem = (int)GemmCfg<BN, ST>::SMEM;
+  const int smem = (int)GemmCfg<BN, ST, AR>::SMEM;
 #define SVLA_SET(EPI)                                                                                         \
   if (e == cudaSuccess)                                                                                       \
-    e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, ST, AR>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   SVLA_SET(GE_F32)
   SVLA_SET(GE_BF16)
   SVLA_SET(GE_ADD_F32)
@@ -327,6 +355,8 @@ inline cudaError_t gemm_set_attrs() {
   if (e == cudaSuccess) e = set_attrs_persistent<128>();
   if (e == cudaSuccess) e = set_attrs_persistent<192>();
   if (e == cudaSuccess) e = set_attrs_persistent<256>();
+  if (e == cudaSuccess) e = set_attrs_inst<32, 8, 64>();
+  if (e == cudaSuccess) e = set_attrs_inst<64, 6, 64>();
   if (e == cudaSuccess) e = set_attrs_inst<32, 4>();
   if (e == cudaSuccess) e = set_attrs_inst<64, 4>();
   if (e == cudaSuccess) e = set_attrs_inst<128, 6>();
@@ -338,7 +368,7 @@ inline cudaError_t gemm_set_attrs() {
 inline cudaError_t run_gemm(int epi, const void* A, int lda, const void* W, int ldw, int M, int N, int K,
                             GemmArgs args, const GemmPlan& p, float* partials, int* counters, cudaStream_t s) {
   CUtensorMap ta, tw;
-  if (!make_tmap_bf16(&ta, A, M, K, lda, GEMM_BM)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&ta, A, M, K, lda, p.a_rows)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&tw, W, N, K, ldw, p.pair ? p.bn / 2 : p.bn)) return cudaErrorInvalidValue;
   if (p.red == GEMM_RED_GLOBAL && (!partials || !counters)) return cudaErrorInvalidValue;
   args.M = M;
@@ -364,6 +394,11 @@ inline cudaError_t run_gemm(int epi, const void* A, int lda, const void* W, int 
   }
   dim3 grid(p.n_tiles, p.m_tiles, p.splits);
   const int cz = p.red == GEMM_RED_CLUSTER ? p.splits : 1;
+  if (p.a_rows == 64) {
+    if (p.bn == 32 && p.stages == 8) return dispatch_epi<32, 8, 64>(epi, ta, tw, args, grid, cz, s);
+    if (p.bn == 64 && p.stages == 6) return dispatch_epi<64, 6, 64>(epi, ta, tw, args, grid, cz, s);
+    return cudaErrorInvalidValue;
+  }
   if (p.bn == 32 && p.stages == 4) return dispatch_epi<32, 4>(epi, ta, tw, args, grid, cz, s);
   if (p.bn == 64 && p.stages == 4) return dispatch_epi<64, 4>(epi, ta, tw, args, grid, cz, s);
   if (p.bn == 128 && p.stages == 6) return dispatch_epi<128, 6>(epi, ta, tw, args, grid, cz, s);

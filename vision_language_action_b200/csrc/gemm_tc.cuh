@@ -89,15 +89,23 @@ constexpr int GEMM_BK = 64;
 constexpr int GEMM_THREADS = 192;
 constexpr unsigned long long GEMM_DRAIN_NS = 2000000000ull;  // fixed limit for the drain path
 
-template <int BN, int STAGES_>
+// A_ROWS = 64 (M <= 64 only): the A box covers 64 rows, so a stage is smaller
+// and every k-block of a batch-1 CTA fits in flight at once. The M = 128 MMA
+// then reads rows 64..127 from the bytes after the A box (the stage's W tile,
+// the next stage, and for the last stage a pad at the end of the ring): those
+// accumulator rows are never stored.
+template <int BN, int STAGES_, int A_ROWS_ = GEMM_BM>
 struct GemmCfg {
   static constexpr int STAGES = STAGES_;
-  static constexpr uint32_t A_BYTES = GEMM_BM * GEMM_BK * 2;
+  static constexpr int A_ROWS = A_ROWS_;
+  static constexpr uint32_t A_BYTES = A_ROWS * GEMM_BK * 2;
   static constexpr uint32_t B_BYTES = BN * GEMM_BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t RING_PAD = (GEMM_BM - A_ROWS) * GEMM_BK * 2;
+  static constexpr uint32_t RING_BYTES = STAGES * STAGE_BYTES + RING_PAD;
   static constexpr uint32_t TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
-  // ring + barriers/flags (512 B) + row factors (512 B) + alignment slack
-  static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 1024 + 1024;
+  // ring (+ pad) + barriers/flags (512 B) + row factors (512 B) + alignment slack
+  static constexpr size_t SMEM = (size_t)RING_BYTES + 1024 + 1024;
   // two CTAs per SM when they fit, so a dependent GEMM can start next to this one
   static constexpr int MIN_BLOCKS = SMEM <= 113 * 1024 ? 2 : 1;
   static constexpr size_t RED_TILE = (size_t)GEMM_BM * (BN + 4) * sizeof(float);
@@ -354,20 +362,20 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, 
 // named barrier over the 4 epilogue warps (ids 2..5)
 SVLA_DEV void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int BN, int EPI, int STAGES>
-__global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES>::MIN_BLOCKS)
+template <int BN, int EPI, int STAGES, int A_ROWS = GEMM_BM>
+__global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES, A_ROWS>::MIN_BLOCKS)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                    const GemmArgs args) {
-  using C = GemmCfg<BN, STAGES>;
+  using C = GemmCfg<BN, STAGES, A_ROWS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES);
   // bars[0..S) full, [S..2S) empty, [2S] accumulator ready
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(bars + 2 * STAGES + 1);
   // misc[0] tmem base, misc[1] abort flag, misc[2] k-blocks issued, misc[3] k-blocks consumed,
   // misc[4] "this CTA reduces"
-  float* misc_scale = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 512);  // [128] row factors
+  float* misc_scale = reinterpret_cast<float*>(smem + C::RING_BYTES + 512);  // [128] row factors
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
