@@ -128,6 +128,20 @@ SVLA_API svla_status svla_denoise(svla_handle* h, const void* kv_cache, const ui
                          int B, int L, const float* noise, int H, int n_steps,
                          float* actions, float* trace, void* stream);
 
+/* svla_denoise with the gradient-free prefix overwrite at a chunk junction
+ * ("Paper vs hardware 11: SmolVLA" §What I ran: the actions that run during
+ * the inference delay are taken from the previous chunk, which removes most of
+ * the jump at the handover). After every Euler step the first d rows of each
+ * query's state are set to t·noise + (1 − t)·prefix, t the time reached, so
+ * the chunk is denoised conditioned on them and ends with exactly `prefix`.
+ *   prefix: device float32 [B, d, action_dim]; 0 <= d <= H (d = 0: svla_denoise).
+ *   actions must not alias noise when d > 0 (the overwrite reads the noise).
+ * Other arguments as svla_denoise; the trace holds the overwritten states. */
+SVLA_API svla_status svla_denoise_prefix(svla_handle* h, const void* kv_cache, const uint8_t* pad_mask,
+                                         int B, int L, const float* noise, int H, int n_steps,
+                                         const float* prefix, int d, float* actions, float* trace,
+                                         void* stream);
+
 /* Draw the noise, prefill, denoise, on one stream.
  * Noise: Philox4x32-10 keyed by seed (key = {seed low 32, seed high 32}),
  * counter {block, query, 0, 0}; element e of a query's [H, A] noise is lane

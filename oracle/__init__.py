@@ -32,6 +32,6 @@ checkpoint is unpinned: no weights or activation dumps exist here.
 """
 from .model import (  # noqa: F401
     load_weights, rms_norm, rope, attention, silu, prefix_positions, prefill,
-    time_embedding, velocity, denoise, sample, oracle_joint, cross_kv,
+    time_embedding, velocity, denoise, denoise_prefix_overwrite, sample, oracle_joint, cross_kv,
 )
 from .philox import philox4x32_10, gaussian_noise  # noqa: F401

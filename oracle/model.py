@@ -26,6 +26,9 @@ below; the numbers are used wherever a reading is cited):
 13. Euler: t_0 = 1, dt = -1/N, v evaluated at (x_k, t_k), t_k = 1 + k dt,
     x_{k+1} = x_k + dt v_k; the output is x_N ("noeira docs, SmolVLA"
     §Architecture: x_t = t eps + (1 - t) a, target eps - a).
+17. Prefix overwrite at a chunk junction: after each Euler step the first d
+    rows of the state are the flow path of the previous chunk's d actions at
+    the time reached (see ``denoise_prefix_overwrite``).
 
 Optional ``emulate_bf16`` rounds to bf16 at the points where the GPU stores
 bf16 (normalised activations, q/k/v, attention output, SwiGLU output, time-MLP
@@ -252,6 +255,40 @@ def denoise(W, s, K, V, valid, noise: np.ndarray, n_steps: int,
         t = 1.0 + k * dt
         v = velocity(W, s, x, t, K, V, valid, emulate_bf16)
         x = x + dt * v
+        vs.append(v)
+        xs.append(x.copy())
+    return np.stack(vs), np.stack(xs), x
+
+
+def denoise_prefix_overwrite(W, s, K, V, valid, noise: np.ndarray, n_steps: int,
+                             a_prev: np.ndarray, emulate_bf16: bool = False):
+    """Euler denoise with the gradient-free prefix overwrite at a chunk junction.
+
+    "Paper vs hardware 11: SmolVLA" §What I ran: the first d actions of a new
+    chunk run during the inference delay, and overwriting that prefix with the
+    previous chunk's actions removes most of the jump at the junction.
+    Reading 17: after every Euler step (and so before every later velocity
+    evaluation) the first d rows of the state are set to the flow path of the
+    known actions, x_t[:d] = t eps[:d] + (1 - t) a_prev (x_t = t eps + (1 - t) a,
+    "noeira docs, SmolVLA" §Architecture), with t the time the step reached;
+    the final chunk therefore starts with exactly a_prev. At t = 1 the
+    overwrite is the noise itself, so step 0 is unchanged. a_prev is [d, A],
+    0 <= d <= H. Returns (vs, xs, x) like ``denoise``; xs holds the states
+    after the overwrite.
+    """
+    a_prev = np.asarray(a_prev, dtype=F64)
+    d = a_prev.shape[0]
+    eps = np.array(noise, dtype=F64)
+    dt = -1.0 / n_steps
+    x = eps.copy()
+    vs, xs = [], []
+    for k in range(n_steps):
+        t = 1.0 + k * dt
+        v = velocity(W, s, x, t, K, V, valid, emulate_bf16)
+        x = x + dt * v
+        t_next = 1.0 + (k + 1) * dt
+        if d:
+            x[:d] = t_next * eps[:d] + (1.0 - t_next) * a_prev
         vs.append(v)
         xs.append(x.copy())
     return np.stack(vs), np.stack(xs), x

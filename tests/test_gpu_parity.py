@@ -189,3 +189,49 @@ def test_sample_noise_matches_philox_and_denoise(tiny):
     a2, _ = tiny.m.denoise(kv, tiny.valid, noise, tiny.wl.n_steps)
     torch.cuda.synchronize()
     assert torch.equal(a2, actions)
+
+
+# ---------------------------------------------------------------------------
+# prefix overwrite at a chunk junction (reading 17)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("wl_name,d,queries", [("tiny", 3, (0,)), ("smolvla_b1", 7, (0,)),
+                                               ("smolvla_b32", 7, (5, 31))])
+def test_prefix_overwrite_parity(wl_name, d, queries):
+    import oracle
+    r = Run(wl_name)
+    try:
+        wl, s = r.wl, r.s
+        g = torch.Generator(device="cpu").manual_seed(17)
+        prefix = torch.randn(r.B, d, s.action_dim, generator=g).to(DEV)
+        a, tr = r.m.denoise_prefix(r.kv, r.valid, r.noise, wl.n_steps, prefix, trace=True)
+        a0, _ = r.m.denoise_prefix(r.kv, r.valid, r.noise, wl.n_steps, prefix[:, :0].contiguous())
+        torch.cuda.synchronize()
+        assert torch.equal(a0, r.actions)                       # d = 0 is plain denoise
+        assert torch.equal(a[:, :d], prefix)                     # the chunk starts with the given actions
+        W = H.oracle_weights(wl_name)
+        inp = H.inputs(wl_name)
+        trn = tr.cpu().numpy()
+        for b in queries:
+            emb = synth.bf16_bits_to_f32(inp["embeds"][b]).astype(np.float64)
+            K, V = oracle.prefill(W, s, emb, inp["valid"][b])
+            vs, xs, x = oracle.denoise_prefix_overwrite(W, s, K, V, inp["valid"][b],
+                                                        inp["noise"][b].astype(np.float64), wl.n_steps,
+                                                        prefix[b].cpu().numpy().astype(np.float64))
+            got = a[b].cpu().numpy()
+            assert H.max_abs(got, x) <= H.CHUNK_MAX_ABS and H.rel_l2(got, x) <= H.CHUNK_REL_L2, (b, H.max_abs(got, x))
+            for k in range(wl.n_steps):
+                assert H.max_abs(trn[k, 1, b], xs[k]) <= H.CHUNK_MAX_ABS, (b, k)
+    finally:
+        r.close()
+        gc.collect()
+
+
+def test_prefix_overwrite_argument_errors(tiny):
+    p = torch.zeros(1, tiny.wl.H + 1, tiny.s.action_dim, device=DEV)
+    with pytest.raises(_abi.SvlaError) as e:
+        tiny.m.denoise_prefix(tiny.kv, tiny.valid, tiny.noise, 2, p)
+    assert e.value.status == _abi.SVLA_ERR_SHAPE
+    x = tiny.noise.clone()
+    with pytest.raises(_abi.SvlaError) as e:
+        tiny.m.denoise_prefix(tiny.kv, tiny.valid, x, 2, p[:, :2].contiguous(), actions=x)
+    assert e.value.status == _abi.SVLA_ERR_ARG

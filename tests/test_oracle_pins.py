@@ -306,3 +306,46 @@ def test_bf16_emulation_stays_close():
     _, _, _, _, xe = oracle.sample(W, s, emb, valid, noise, wl.n_steps, emulate_bf16=True)
     d = np.abs(x - xe).max()
     assert 0 < d < 2e-2
+
+
+# --------------------------------------------------------------------------
+# prefix overwrite at a chunk junction (reading 17)
+# --------------------------------------------------------------------------
+def test_prefix_overwrite_with_no_prefix_is_plain_denoise():
+    s, W, emb, valid, noise, wl = _tiny(random_affine=True)
+    K, V = oracle.prefill(W, s, emb, valid)
+    a = oracle.denoise(W, s, K, V, valid, noise, wl.n_steps)
+    b = oracle.denoise_prefix_overwrite(W, s, K, V, valid, noise, wl.n_steps, np.zeros((0, s.action_dim)))
+    for u, w in zip(a, b):
+        assert np.array_equal(u, w)
+
+
+@pytest.mark.parametrize("n_steps", [3, 4, 10])
+def test_prefix_overwrite_lands_on_the_previous_actions(n_steps):
+    """t reaches exactly 0, so the flow path t eps + (1 - t) a_prev ends on a_prev."""
+    s, W, emb, valid, noise, wl = _tiny(random_affine=True)
+    K, V = oracle.prefill(W, s, emb, valid)
+    rng = np.random.default_rng(3)
+    a_prev = rng.standard_normal((3, s.action_dim))
+    vs, xs, x = oracle.denoise_prefix_overwrite(W, s, K, V, valid, noise, n_steps, a_prev)
+    assert np.array_equal(x[:3], a_prev)
+    assert not np.allclose(x[3:], oracle.denoise(W, s, K, V, valid, noise, n_steps)[2][3:])  # conditioning
+
+
+def test_prefix_overwrite_constant_velocity_closed_form():
+    """With v = c everywhere: rows past the prefix move linearly, prefix rows
+    follow the flow path of the given actions, step by step, exactly."""
+    s, W, emb, valid, _, wl = _tiny()
+    W = dict(W)
+    A = s.action_dim
+    c = np.array([0.5, -1.25, 2.0, 0.0, -0.375, 1.0, 3.5, -2.0])[:A]
+    W["w_out"] = np.zeros_like(W["w_out"])
+    W["b_out"] = c
+    x0 = (np.arange(wl.H * A).reshape(wl.H, A) % 7 - 3) * 0.25
+    a_prev = (np.arange(2 * A).reshape(2, A) % 5 - 2) * 0.5
+    K, V = oracle.prefill(W, s, emb, valid)
+    vs, xs, x = oracle.denoise_prefix_overwrite(W, s, K, V, valid, x0, 4, a_prev)
+    for k in range(4):
+        t = 1.0 - 0.25 * (k + 1)
+        assert np.array_equal(xs[k][2:], x0[2:] + (k + 1) * (-0.25) * c)
+        assert np.array_equal(xs[k][:2], t * x0[:2] + (1 - t) * a_prev)

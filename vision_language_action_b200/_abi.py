@@ -42,6 +42,7 @@ SIGNATURES = {
     "svla_blob_bytes": (_S, [ctypes.POINTER(SvlaConfig)]),
     "svla_prefill": (_I, [_P, _P, _P, _I, _I, _P, _P]),
     "svla_denoise": (_I, [_P, _P, _P, _I, _I, _P, _I, _I, _P, _P, _P]),
+    "svla_denoise_prefix": (_I, [_P, _P, _P, _I, _I, _P, _I, _I, _P, _I, _P, _P, _P]),
     "svla_sample": (_I, [_P, _P, _P, _I, _I, ctypes.c_uint64, _I, _I, _P, _P, _P, _P]),
     "svla_device_status": (_I, [_P, _P]),
     "svla_last_error": (ctypes.c_char_p, [_P]),

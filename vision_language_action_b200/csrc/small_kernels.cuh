@@ -236,6 +236,12 @@ struct StepEndArgs {
   float* x;                // [M, A] in/out
   float* trace_v;          // [M, A] or null
   float* trace_x;          // [M, A] or null
+  // prefix overwrite at a chunk junction (reading 17): rows j < d of every
+  // query's chunk become t_next * noise + (1 - t_next) * prefix[b, j]
+  const float* prefix;     // [B, d, A] or null
+  const float* noise;      // [M, A] (the state at t = 1)
+  int d, H;
+  float t_next;
 };
 
 constexpr int SE_WARPS = 8;
@@ -332,7 +338,13 @@ __global__ void __launch_bounds__(256) step_end_kernel(const StepEndArgs p) {
       const int o = o0 + lane;
       if (o < p.A) {
         const float vv = v + bf2f(reinterpret_cast<const uint16_t*>(p.b_out)[o]);
-        const float xn = p.x[(size_t)m * p.A + o] + p.dt * vv;
+        float xn = p.x[(size_t)m * p.A + o] + p.dt * vv;
+        if (p.prefix) {
+          const int b = m / p.H, j = m % p.H;
+          if (j < p.d)
+            xn = p.t_next * p.noise[(size_t)m * p.A + o] +
+                 (1.0f - p.t_next) * p.prefix[((size_t)b * p.d + j) * p.A + o];
+        }
         p.x[(size_t)m * p.A + o] = xn;
         if (p.trace_v) p.trace_v[(size_t)m * p.A + o] = vv;
         if (p.trace_x) p.trace_x[(size_t)m * p.A + o] = xn;

@@ -392,7 +392,7 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
 
 // ---- denoise schedule -------------------------------------------------------
 cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise, int H,
-                           int n_steps, float* actions, float* trace, cudaStream_t s) {
+                           int n_steps, float* actions, float* trace, const float* prefix, int d, cudaStream_t s) {
   const svla_config& c = h->cfg;
   const int M = B * H, E = c.e_width, hd = c.head_dim, A = c.action_dim;
   const int qw = c.e_heads * hd, kvw = c.e_kv_heads * hd, pkvw = c.p_kv_heads * hd;
@@ -491,6 +491,11 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
     se.x = actions;
     se.trace_v = trace ? trace + (size_t)(2 * k) * M * A : nullptr;
     se.trace_x = trace ? trace + (size_t)(2 * k + 1) * M * A : nullptr;
+    se.prefix = d > 0 ? prefix : nullptr;
+    se.noise = noise;
+    se.d = d;
+    se.H = H;
+    se.t_next = 1.0f - (float)(k + 1) / (float)n_steps;
     SVLA_TRY(launch_pdl(step_end_kernel, dim3(se_blocks), dim3(256), (size_t)A * E * 2, s, se));
   }
   return cudaSuccess;
@@ -727,22 +732,42 @@ svla_status svla_prefill(svla_handle* h, const void* embeds, const uint8_t* pad,
                    "prefill");
 }
 
-svla_status svla_denoise(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise, int H,
-                         int n_steps, float* actions, float* trace, void* stream) {
+static svla_status denoise_impl(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise,
+                                int H, int n_steps, const float* prefix, int d, float* actions, float* trace,
+                                void* stream) {
   if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
   if (!kv || !pad || !noise || !actions) return fail(h, SVLA_ERR_ARG, "null pointer");
   if (B < 1 || L < 1 || B > h->cfg.max_batch || L > h->cfg.max_prefix)
     return fail(h, SVLA_ERR_SHAPE, "B or L outside [1, max_batch] x [1, max_prefix]");
   if (H < 1 || H > h->cfg.max_chunk) return fail(h, SVLA_ERR_SHAPE, "H outside [1, max_chunk]");
   if (n_steps < 1 || n_steps > 1000) return fail(h, SVLA_ERR_SHAPE, "n_steps outside [1, 1000]");
+  if (d < 0 || d > H) return fail(h, SVLA_ERR_SHAPE, "prefix length d outside [0, H]");
+  if (d > 0 && !prefix) return fail(h, SVLA_ERR_ARG, "null prefix with d > 0");
+  if (d > 0 && (const void*)noise == (const void*)actions)
+    return fail(h, SVLA_ERR_ARG, "the prefix overwrite needs the noise: actions must not alias noise");
   DeviceGuard dg(h->device);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   std::vector<uint64_t> key = {2, (uint64_t)B, (uint64_t)L, (uint64_t)H, (uint64_t)n_steps,
                                (uint64_t)(uintptr_t)kv, (uint64_t)(uintptr_t)pad, (uint64_t)(uintptr_t)noise,
-                               (uint64_t)(uintptr_t)actions, (uint64_t)(uintptr_t)trace, g_wait_ns.load()};
+                               (uint64_t)(uintptr_t)actions, (uint64_t)(uintptr_t)trace, g_wait_ns.load(),
+                               (uint64_t)(uintptr_t)(d > 0 ? prefix : nullptr), (uint64_t)d};
   return run_graph(
-      h, key, [&](cudaStream_t cs) { return record_denoise(h, kv, pad, B, L, noise, H, n_steps, actions, trace, cs); },
+      h, key,
+      [&](cudaStream_t cs) {
+        return record_denoise(h, kv, pad, B, L, noise, H, n_steps, actions, trace, d > 0 ? prefix : nullptr, d, cs);
+      },
       s, "denoise");
+}
+
+svla_status svla_denoise(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise, int H,
+                         int n_steps, float* actions, float* trace, void* stream) {
+  return denoise_impl(h, kv, pad, B, L, noise, H, n_steps, nullptr, 0, actions, trace, stream);
+}
+
+svla_status svla_denoise_prefix(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise,
+                                int H, int n_steps, const float* prefix, int d, float* actions, float* trace,
+                                void* stream) {
+  return denoise_impl(h, kv, pad, B, L, noise, H, n_steps, prefix, d, actions, trace, stream);
 }
 
 svla_status svla_sample(svla_handle* h, const void* embeds, const uint8_t* pad, int B, int L, uint64_t seed, int H,

@@ -113,6 +113,24 @@ class SmolVLA:
         _abi.check(st, self.h)
         return actions, tr
 
+    def denoise_prefix(self, kv_cache: torch.Tensor, pad_mask: torch.Tensor, noise: torch.Tensor, n_steps: int,
+                       prefix: torch.Tensor, actions: Optional[torch.Tensor] = None, trace: bool = False,
+                       stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+        """Denoise with the first prefix.shape[1] actions of each query's chunk
+        overwritten along the flow path of ``prefix`` ([B, d, A] fp32)."""
+        B, H, A = noise.shape
+        L = pad_mask.shape[1]
+        d = prefix.shape[1]
+        if actions is None:
+            actions = torch.empty_like(noise)
+        tr = None
+        if trace:
+            tr = torch.empty((n_steps, 2, B, H, A), dtype=torch.float32, device=noise.device)
+        st = self.lib.svla_denoise_prefix(self.h, _ptr(kv_cache), _ptr(pad_mask), B, L, _ptr(noise), H, n_steps,
+                                          _ptr(prefix), d, _ptr(actions), _ptr(tr), _stream(stream))
+        _abi.check(st, self.h)
+        return actions, tr
+
     def sample(self, embeds: torch.Tensor, pad_mask: torch.Tensor, seed: int, H: int, n_steps: int,
                kv_cache: Optional[torch.Tensor] = None, return_noise: bool = False, stream=None):
         B, L = pad_mask.shape
