@@ -235,3 +235,56 @@ def test_prefix_overwrite_argument_errors(tiny):
     with pytest.raises(_abi.SvlaError) as e:
         tiny.m.denoise_prefix(tiny.kv, tiny.valid, x, 2, p[:, :2].contiguous(), actions=x)
     assert e.value.status == _abi.SVLA_ERR_ARG
+
+
+# ---------------------------------------------------------------------------
+# edge cases on the tiny model: degenerate and ragged sizes
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,L,Hc,n_steps,mask", [
+    (1, 1, 1, 1, "all"),          # one prefix token, one action row, one Euler step
+    (2, 9, 3, 2, "one_middle"),   # a single valid token amid padding
+    (3, 65, 17, 4, "ragged"),     # ragged tiles in every dimension, per-query pad patterns
+    (1, 130, 64, 3, "lead_pad"),  # leading padding (positions start at the first valid token)
+])
+def test_tiny_edge_cases(B, L, Hc, n_steps, mask):
+    import oracle
+    s = synth.SHAPES["tiny"]
+    _, wb, blob = H_weights_tiny()
+    rng = np.random.default_rng(B * 1000 + L * 10 + Hc)
+    emb_bits = synth.f32_to_bf16_bits(rng.standard_normal((B, L, s.p_width), dtype=np.float32))
+    noise = rng.standard_normal((B, Hc, s.action_dim), dtype=np.float32)
+    valid = np.ones((B, L), np.uint8)
+    if mask == "one_middle":
+        valid[:] = 0
+        valid[:, L // 2] = 1
+    elif mask == "ragged":
+        valid[0, 60:] = 0
+        valid[1, 3:20] = 0
+        valid[2, ::3] = 0
+    elif mask == "lead_pad":
+        valid[0, :40] = 0
+    m = SmolVLA(s, blob, max_batch=B, max_prefix=L, max_chunk=Hc)
+    try:
+        e = torch.from_numpy(emb_bits.view(np.int16)).to(DEV).view(torch.bfloat16)
+        v = torch.from_numpy(valid).to(DEV)
+        n = torch.from_numpy(noise).to(DEV)
+        kv = m.prefill(e, v)
+        a, _ = m.denoise(kv, v, n, n_steps)
+        assert m.device_status() == _abi.SVLA_OK
+        kvn = kv.float().cpu().numpy().reshape(2, s.p_layers, B, L, s.p_kv_heads, s.head_dim)
+        W = oracle.load_weights(wb)
+        for b in range(B):
+            emb = synth.bf16_bits_to_f32(emb_bits[b]).astype(np.float64)
+            K, V, _, _, x = oracle.sample(W, s, emb, valid[b], noise[b].astype(np.float64), n_steps)
+            ok = valid[b].astype(bool)
+            for l in range(s.p_layers):
+                assert H.rel_l2(kvn[0, l, b][ok], K[l][ok]) <= H.KV_REL_L2
+                assert H.rel_l2(kvn[1, l, b][ok], V[l][ok]) <= H.KV_REL_L2
+            got = a[b].cpu().numpy()
+            assert H.max_abs(got, x) <= H.CHUNK_MAX_ABS and H.rel_l2(got, x) <= H.CHUNK_REL_L2, (b, H.max_abs(got, x))
+    finally:
+        m.close()
+
+
+def H_weights_tiny():
+    return H.weights("tiny")
