@@ -372,6 +372,11 @@ def ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = float(t.item())
 
+    # the two calls of a step timed on their own (same warm-up and step count)
+    ms_pre = time_steps(lambda: m.prefill(d["embeds"], d["valid"], d["kv"]), args.steps, args.warmup, barrier)
+    ms_den = time_steps(lambda: m.denoise(d["kv"], d["valid"], d["noise"], wl.n_steps, actions=d["actions"]),
+                        args.steps, args.warmup, barrier)
+
     hbm_bytes, gflops, aflops = chunk_work(s, wl.B, wl.L, wl.H, wl.n_steps)
     chunk_s = value * 1e-3 * world  # per-rank chunk latency in s
     roof = gemm_roofline(s, wl.B, wl.L, wl.H, wl.n_steps, f"cuda:{dev}", hbm_peak)
@@ -431,6 +436,8 @@ def ours(args, rank, world, local_rank):
             "cpu_baseline": cpu,
             "e2e": {"value": round(ms_e2e / (args.steps * chunks_per_step), 4), "unit": "ms",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "breakdown": {"prefill_ms": round(ms_pre / args.steps, 4), "denoise_ms": round(ms_den / args.steps, 4),
+                          "note": "each call timed alone on rank 0, same steps and warm-up"},
             "gpu_launches": launches_per_chunk(s, wl.n_steps) * args.steps,
             "clocks": clk,
             "secondary": secondary,

@@ -142,6 +142,29 @@ SVLA_API svla_status svla_denoise_prefix(svla_handle* h, const void* kv_cache, c
                                          const float* prefix, int d, float* actions, float* trace,
                                          void* stream);
 
+/* Which implementation runs the denoise of svla_denoise, svla_denoise_prefix
+ * and svla_sample on this handle. Both compute the same path (same readings,
+ * same bf16 rounding points); each is bitwise run-to-run deterministic and both
+ * meet the parity tolerances, but they round in different orders, so their
+ * results differ in the last bits.
+ *   SVLA_DENOISE_AUTO   (default) FUSED when svla_denoise_fused_supported, else GRAPH.
+ *   SVLA_DENOISE_GRAPH  one CUDA graph: the hoisted cross K/V projection, then
+ *                       ~85 dependent kernels per Euler step; any shape.
+ *   SVLA_DENOISE_FUSED  the hoisted projection, then ONE persistent kernel for
+ *                       all steps (one CTA per SM, cooperative launch, the
+ *                       dependent steps as stages separated by grid barriers);
+ *                       needs B * H <= 64 and H <= 64, else the denoise call
+ *                       returns SVLA_ERR_UNSUPPORTED.
+ * Returns SVLA_ERR_ARG for another value or a null handle. */
+#define SVLA_DENOISE_AUTO   0
+#define SVLA_DENOISE_GRAPH  1
+#define SVLA_DENOISE_FUSED  2
+SVLA_API svla_status svla_set_denoise_path(svla_handle* h, int path);
+
+/* 1 if the persistent denoise kernel takes batch B with chunk length H on
+ * this handle (B * H <= 64, H <= 64, within the handle's limits), else 0. */
+SVLA_API int svla_denoise_fused_supported(const svla_handle* h, int B, int H);
+
 /* Draw the noise, prefill, denoise, on one stream.
  * Noise: Philox4x32-10 keyed by seed (key = {seed low 32, seed high 32}),
  * counter {block, query, 0, 0}; element e of a query's [H, A] noise is lane

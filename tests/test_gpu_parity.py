@@ -31,13 +31,14 @@ DEV = "cuda:0"
 class Run:
     """GPU run of a workload: handle, device inputs, K/V, chunk and trace."""
 
-    def __init__(self, wl_name, random_affine=False, B=None):
+    def __init__(self, wl_name, random_affine=False, B=None, path=_abi.DENOISE_AUTO):
         wl = synth.WORKLOADS[wl_name]
         s, _, blob = H.weights(wl_name, random_affine)
         inp = H.inputs(wl_name)
         self.wl, self.s = wl, s
         self.B = wl.B if B is None else B
         self.m = SmolVLA(s, blob, max_batch=self.B, max_prefix=wl.L, max_chunk=wl.H)
+        self.m.set_denoise_path(path)
         self.valid = torch.from_numpy(inp["valid"][:self.B]).to(DEV)
         self.noise = torch.from_numpy(inp["noise"][:self.B]).to(DEV)
         if wl.prefix_kind == "kv_given":
@@ -80,6 +81,9 @@ def check_query(run: Run, b: int, random_affine=False):
     assert H.rel_l2(got, x) <= H.CHUNK_REL_L2, (wl.name, b, H.rel_l2(got, x))
 
 
+PATHS = {"graph": _abi.DENOISE_GRAPH, "fused": _abi.DENOISE_FUSED}
+
+
 @pytest.fixture(scope="module")
 def tiny():
     r = Run("tiny")
@@ -87,21 +91,29 @@ def tiny():
     r.close()
 
 
-def test_tiny_parity(tiny):
-    check_query(tiny, 0)
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_tiny_parity(path):
+    r = Run("tiny", path=PATHS[path])
+    try:
+        check_query(r, 0)
+    finally:
+        r.close()
 
 
-def test_tiny_random_affine_parity():
-    r = Run("tiny", random_affine=True)
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_tiny_random_affine_parity(path):
+    r = Run("tiny", random_affine=True, path=PATHS[path])
     try:
         check_query(r, 0, random_affine=True)
     finally:
         r.close()
 
 
-def test_smolvla_b1_parity():
-    r = Run("smolvla_b1")
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_smolvla_b1_parity(path):
+    r = Run("smolvla_b1", path=PATHS[path])
     try:
+        assert r.m.fused_supported(1, r.wl.H)
         check_query(r, 0)
         # run-to-run bitwise determinism of prefill and denoise
         kv2 = r.m.prefill(r.embeds, r.valid)
@@ -115,7 +127,8 @@ def test_smolvla_b1_parity():
 
 
 def test_smolvla_b32_parity_and_batch_invariance():
-    r = Run("smolvla_b32")
+    # batch invariance of one implementation: the graph path at B = 32 and B = 1
+    r = Run("smolvla_b32", path=_abi.DENOISE_GRAPH)
     try:
         for b in (0, 13, 31):
             check_query(r, b)
@@ -194,11 +207,12 @@ def test_sample_noise_matches_philox_and_denoise(tiny):
 # ---------------------------------------------------------------------------
 # prefix overwrite at a chunk junction (reading 17)
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("wl_name,d,queries", [("tiny", 3, (0,)), ("smolvla_b1", 7, (0,)),
-                                               ("smolvla_b32", 7, (5, 31))])
-def test_prefix_overwrite_parity(wl_name, d, queries):
+@pytest.mark.parametrize("wl_name,d,queries,path", [
+    ("tiny", 3, (0,), "graph"), ("tiny", 3, (0,), "fused"), ("smolvla_b1", 7, (0,), "graph"),
+    ("smolvla_b1", 7, (0,), "fused"), ("smolvla_b32", 7, (5, 31), "graph")])
+def test_prefix_overwrite_parity(wl_name, d, queries, path):
     import oracle
-    r = Run(wl_name)
+    r = Run(wl_name, path=PATHS[path])
     try:
         wl, s = r.wl, r.s
         g = torch.Generator(device="cpu").manual_seed(17)
@@ -240,13 +254,14 @@ def test_prefix_overwrite_argument_errors(tiny):
 # ---------------------------------------------------------------------------
 # edge cases on the tiny model: degenerate and ragged sizes
 # ---------------------------------------------------------------------------
+@pytest.mark.parametrize("path", sorted(PATHS))
 @pytest.mark.parametrize("B,L,Hc,n_steps,mask", [
     (1, 1, 1, 1, "all"),          # one prefix token, one action row, one Euler step
     (2, 9, 3, 2, "one_middle"),   # a single valid token amid padding
     (3, 65, 17, 4, "ragged"),     # ragged tiles in every dimension, per-query pad patterns
     (1, 130, 64, 3, "lead_pad"),  # leading padding (positions start at the first valid token)
 ])
-def test_tiny_edge_cases(B, L, Hc, n_steps, mask):
+def test_tiny_edge_cases(B, L, Hc, n_steps, mask, path):
     import oracle
     s = synth.SHAPES["tiny"]
     _, wb, blob = H_weights_tiny()
@@ -265,6 +280,8 @@ def test_tiny_edge_cases(B, L, Hc, n_steps, mask):
         valid[0, :40] = 0
     m = SmolVLA(s, blob, max_batch=B, max_prefix=L, max_chunk=Hc)
     try:
+        assert m.fused_supported(B, Hc)  # every case here has B * H <= 64
+        m.set_denoise_path(PATHS[path])
         e = torch.from_numpy(emb_bits.view(np.int16)).to(DEV).view(torch.bfloat16)
         v = torch.from_numpy(valid).to(DEV)
         n = torch.from_numpy(noise).to(DEV)
@@ -288,3 +305,56 @@ def test_tiny_edge_cases(B, L, Hc, n_steps, mask):
 
 def H_weights_tiny():
     return H.weights("tiny")
+
+
+# ---------------------------------------------------------------------------
+# the persistent denoise kernel: selection rules and its bounded waits
+# ---------------------------------------------------------------------------
+def test_fused_path_selection(tiny):
+    m = tiny.m
+    assert m.fused_supported(1, tiny.wl.H)
+    assert not m.fused_supported(1, 65)            # more than 64 chunk rows of one query
+    with pytest.raises(_abi.SvlaError) as e:
+        m.set_denoise_path(7)
+    assert e.value.status == _abi.SVLA_ERR_ARG
+
+
+def test_fused_unsupported_shape_is_rejected():
+    s, _, blob = H.weights("tiny")
+    m = SmolVLA(s, blob, max_batch=9, max_prefix=24, max_chunk=8)
+    try:
+        assert not m.fused_supported(9, 8)          # 72 rows
+        m.set_denoise_path(_abi.DENOISE_FUSED)
+        kv = m.new_kv_cache(9, 24)
+        kv.zero_()
+        v = torch.ones(9, 24, dtype=torch.uint8, device=DEV)
+        n = torch.zeros(9, 8, s.action_dim, device=DEV)
+        with pytest.raises(_abi.SvlaError) as e:
+            m.denoise(kv, v, n, 2)
+        assert e.value.status == _abi.SVLA_ERR_UNSUPPORTED
+    finally:
+        m.close()
+
+
+def test_fused_timeout_reports_and_recovers(tiny):
+    """A wait limit of 0 makes the first unsatisfied wait (a grid barrier or a
+    weight slot) give up: the kernel records SVLA_ERR_TIMEOUT, every CTA leaves
+    through the abort word, and the next launch with the normal limit is exact."""
+    m = tiny.m
+    m.set_denoise_path(_abi.DENOISE_FUSED)
+    try:
+        ref, _ = m.denoise(tiny.kv, tiny.valid, tiny.noise, tiny.wl.n_steps)
+        assert m.device_status() == _abi.SVLA_OK
+        lib = _abi.load()
+        lib.svla_set_wait_limit_ns(0)
+        try:
+            m.denoise(tiny.kv, tiny.valid, tiny.noise, tiny.wl.n_steps)
+            st = m.device_status()
+        finally:
+            lib.svla_set_wait_limit_ns(1_000_000_000)
+        assert st == _abi.SVLA_ERR_TIMEOUT
+        again, _ = m.denoise(tiny.kv, tiny.valid, tiny.noise, tiny.wl.n_steps)
+        assert m.device_status() == _abi.SVLA_OK
+        assert torch.equal(again, ref)
+    finally:
+        m.set_denoise_path(_abi.DENOISE_AUTO)

@@ -54,7 +54,11 @@ SIGNATURES = {
     "svla_op_attention": (_I, [_P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
     "svla_op_rmsnorm": (_I, [_P, _P, _I, _I, ctypes.c_float, _P, _P]),
     "svla_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "svla_set_denoise_path": (_I, [_P, _I]),
+    "svla_denoise_fused_supported": (_I, [_P, _I, _I]),
 }
+
+DENOISE_AUTO, DENOISE_GRAPH, DENOISE_FUSED = 0, 1, 2
 
 _lib = None
 

@@ -31,6 +31,10 @@ struct AttnArgs {
   int ldo;
   int n_q, n_kv, Lq, Lk, causal;
   float scale_log2;  // log2(e) / sqrt(hd)
+  // Output layout: o_pc == 0: row-major with ldo. Otherwise column planes of
+  // o_pc columns: element (row m = b * Lq + i, column c) of the [o_M, n_q * HD]
+  // output is at out[((c / o_pc) * o_M + m) * (o_pc + 8) + c % o_pc].
+  int o_pc = 0, o_M = 0;
 };
 
 constexpr int ATT_BQ = 64;
@@ -38,11 +42,11 @@ constexpr int ATT_BK = 64;
 constexpr int ATT_THREADS = 128;
 constexpr int ATT_NBUF = 2;  // key/value tiles in flight (double buffering)
 
-template <int HD>
+template <int HD, int NBUF = ATT_NBUF>
 struct AttnCfg {
   static constexpr int LDS = HD + 8;  // padded smem row (elements): conflict-free ldmatrix
   static constexpr int TILE = ATT_BK * LDS;
-  static constexpr size_t SMEM = (size_t)(ATT_BQ * LDS + 2 * ATT_NBUF * TILE) * 2 + ATT_NBUF * ATT_BK;
+  static constexpr size_t SMEM = (size_t)(ATT_BQ * LDS + 2 * NBUF * TILE) * 2 + NBUF * ATT_BK;
 };
 
 SVLA_DEV void cp_async16(uint32_t dst, const void* src, bool pred) {
@@ -74,26 +78,29 @@ SVLA_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int HD>
-__global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a) {
-  using C = AttnCfg<HD>;
+// barrier over the ATT_THREADS threads that run one attention block
+SVLA_DEV void att_sync(int bar_id) { asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(ATT_THREADS) : "memory"); }
+
+// One (64-row query block qb, query head h, query b) block of attention, run
+// by ATT_THREADS consecutive threads (tid = 0..127 among them) that
+// synchronise on named barrier `bar_id`; `smem` holds AttnCfg<HD, NBUF>::SMEM
+// bytes; NBUF key/value tiles are in flight at a time.
+template <int HD, int NBUF = ATT_NBUF>
+SVLA_DEV void attention_block(const AttnArgs& a, int qb, int h, int b, uint8_t* smem, int tid, int bar_id) {
+  using C = AttnCfg<HD, NBUF>;
   constexpr int LDS = C::LDS;
   constexpr int KS = HD / 16;  // k-steps of q.k
   constexpr int ND = HD / 8;   // 8-wide output column blocks
   constexpr int CPR = HD / 8;  // 16-byte chunks per row
 
-  extern __shared__ __align__(16) uint8_t att_smem[];
-  bf16* sQ = reinterpret_cast<bf16*>(att_smem);
+  bf16* sQ = reinterpret_cast<bf16*>(smem);
   bf16* sK = sQ + ATT_BQ * LDS;           // [NBUF][64][LDS]
-  bf16* sV = sK + ATT_NBUF * C::TILE;     // [NBUF][64][LDS]
-  uint8_t* sF = reinterpret_cast<uint8_t*>(sV + ATT_NBUF * C::TILE);  // [NBUF][64] key flags
+  bf16* sV = sK + NBUF * C::TILE;     // [NBUF][64][LDS]
+  uint8_t* sF = reinterpret_cast<uint8_t*>(sV + NBUF * C::TILE);  // [NBUF][64] key flags
 
-  griddep_launch_dependents();
-  griddep_wait();
-  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g_kv = h / (a.n_q / a.n_kv);
   const int q0 = qb * ATT_BQ;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int warp = tid >> 5, lane = tid & 31;
 
   const bf16* qbase = a.q + (size_t)b * a.Lq * a.ldq + (size_t)h * HD;
   const bf16* kbase = a.k + (size_t)b * a.Lk * a.ldkv + (size_t)g_kv * HD;
@@ -129,7 +136,7 @@ __global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a
   };
   // tiles 0 .. NBUF-1 in flight (group 0 also carries Q); one commit group per tile
 #pragma unroll
-  for (int t = 0; t < ATT_NBUF; ++t) {
+  for (int t = 0; t < NBUF; ++t) {
     if (t < nkt) load_kv(t, t);
     cp_async_commit();
   }
@@ -145,9 +152,9 @@ __global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a
   float l_run[2] = {0.f, 0.f};
 
   for (int kt = 0; kt < nkt; ++kt) {
-    const int buf = kt % ATT_NBUF;
-    cp_async_wait<ATT_NBUF - 1>();  // tile kt (and Q) have landed; later tiles may still fly
-    __syncthreads();
+    const int buf = kt % NBUF;
+    cp_async_wait<NBUF - 1>();  // tile kt (and Q) have landed; later tiles may still fly
+    att_sync(bar_id);
     if (kt == 0) {
       // Q fragments (A operand, row-major 16 x 16 per k-step)
 #pragma unroll
@@ -242,8 +249,8 @@ __global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a
         mma_bf16_16816(o[2 * nd2 + 1], pa[kk], b2, b3);
       }
     }
-    __syncthreads();  // every warp is done with this buffer: refill it with tile kt + NBUF
-    if (kt + ATT_NBUF < nkt) load_kv(kt + ATT_NBUF, buf);
+    att_sync(bar_id);  // every warp is done with this buffer: refill it with tile kt + NBUF
+    if (kt + NBUF < nkt) load_kv(kt + NBUF, buf);
     cp_async_commit();
   }
 
@@ -255,17 +262,33 @@ __global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a
   }
   const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
   const float inv1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
-  bf16* obase = a.out + (size_t)b * a.Lq * a.ldo + (size_t)h * HD;
 #pragma unroll
   for (int nd = 0; nd < ND; ++nd) {
     const int c = nd * 8 + 2 * t4;
+    bf16* col_base;
+    size_t row_pitch;
+    if (a.o_pc == 0) {
+      col_base = a.out + (size_t)b * a.Lq * a.ldo + (size_t)h * HD + c;
+      row_pitch = a.ldo;
+    } else {
+      const int col = h * HD + c, pl = col / a.o_pc;
+      col_base = a.out + ((size_t)pl * a.o_M + (size_t)b * a.Lq) * (a.o_pc + 8) + (col - pl * a.o_pc);
+      row_pitch = a.o_pc + 8;
+    }
     if (row0 < a.Lq)
-      *reinterpret_cast<uint32_t*>(obase + (size_t)row0 * a.ldo + c) =
-          pack_bf16x2(o[nd][0] * inv0, o[nd][1] * inv0);
+      *reinterpret_cast<uint32_t*>(col_base + (size_t)row0 * row_pitch) = pack_bf16x2(o[nd][0] * inv0, o[nd][1] * inv0);
     if (row0 + 8 < a.Lq)
-      *reinterpret_cast<uint32_t*>(obase + (size_t)(row0 + 8) * a.ldo + c) =
+      *reinterpret_cast<uint32_t*>(col_base + (size_t)(row0 + 8) * row_pitch) =
           pack_bf16x2(o[nd][2] * inv1, o[nd][3] * inv1);
   }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(ATT_THREADS) attention_kernel(const AttnArgs a) {
+  extern __shared__ __align__(16) uint8_t att_smem[];
+  griddep_launch_dependents();
+  griddep_wait();
+  attention_block<HD>(a, blockIdx.x, blockIdx.y, blockIdx.z, att_smem, threadIdx.x, 1);
 }
 
 }  // namespace svla

@@ -11,6 +11,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <list>
 #include <utility>
@@ -19,6 +20,7 @@
 #include <vector>
 
 #include "attention.cuh"
+#include "denoise_fused.cuh"
 #include "gemm_host.cuh"
 #include "small_kernels.cuh"
 
@@ -27,6 +29,7 @@ using namespace svla;
 namespace {
 
 std::atomic<unsigned long long> g_wait_ns{1000000000ull};
+constexpr int FD_SMEM_MAX = 232448 - 1024;  // dynamic shared memory of the persistent denoise kernel
 thread_local std::string t_last_error = "no error";
 
 const char* status_str(svla_status s) {
@@ -61,6 +64,10 @@ cudaError_t ensure_attrs(int dev) {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(attention_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)AttnCfg<32>::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(denoise_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, FD_SMEM_MAX);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(denoise_fused_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, FD_SMEM_MAX);
   if (e == cudaSuccess && !encode_fn()) e = cudaErrorNotSupported;  // resolve outside any capture
   if (e == cudaSuccess) g_attr_done[dev] = true;
   return e;
@@ -170,6 +177,43 @@ __global__ void bf16_to_f32_kernel(const uint16_t* __restrict__ src, float* __re
   if (i < n) dst[i] = __uint_as_float(((uint32_t)src[i]) << 16);
 }
 
+// Offsets (elements) of the persistent kernel's padded weight copy.
+struct FusedWeights {
+  std::vector<size_t> qkv, o, gu, d;
+  size_t t1a = 0, t2 = 0, total = 0;
+};
+
+FusedWeights fused_weight_layout(const svla_config& c) {
+  FusedWeights F;
+  const size_t E = c.e_width, qw = (size_t)c.e_heads * c.head_dim, kvw = (size_t)c.e_kv_heads * c.head_dim;
+  size_t off = 0;
+  auto add = [&](size_t rows, size_t K) {
+    const size_t o = off;
+    off += rows * (K + 8);
+    return o;
+  };
+  for (int l = 0; l < c.e_layers; ++l) {
+    F.qkv.push_back(add(l % 2 == 0 ? qw + 2 * kvw : qw, E));
+    F.o.push_back(add(E, qw));
+    F.gu.push_back(add(2 * (size_t)c.e_ffn, E));
+    F.d.push_back(add(E, c.e_ffn));
+  }
+  F.t1a = add(E, E);
+  F.t2 = add(E, E);
+  F.total = off;
+  return F;
+}
+
+// dst[r, :cols] = src[r * src_ld : + cols] with row pitch cols + 8 (pad columns zero)
+__global__ void pad_rows_kernel(const uint16_t* __restrict__ src, size_t src_ld, uint16_t* __restrict__ dst,
+                                int rows, int cols) {
+  const size_t dld = (size_t)cols + 8, n = (size_t)rows * dld;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = i / dld, c = i % dld;
+    dst[i] = c < (size_t)cols ? src[r * src_ld + c] : (uint16_t)0;
+  }
+}
+
 struct GraphEntry {
   std::vector<uint64_t> key;
   cudaGraphExec_t exec = nullptr;
@@ -203,12 +247,18 @@ struct svla_handle {
   float* e_part = nullptr;
   int* e_cnt = nullptr;
   float* noise_buf = nullptr;
+  unsigned* fd_sync = nullptr;  // persistent denoise: barrier counter, abort word
+  uint16_t* fw = nullptr;       // persistent denoise: expert GEMM weights with row pitch K + 8
+  FusedWeights fwl;
+  int denoise_path = SVLA_DENOISE_AUTO;
+  int num_sms = 0;
   cudaStream_t cap = nullptr;  // capture stream
   std::list<GraphEntry> graphs;
   std::vector<void*> allocs;
   std::string last_error = "no error";
 
   const bf16* W(size_t off) const { return reinterpret_cast<const bf16*>(w + off); }
+  const bf16* FW(size_t off) const { return reinterpret_cast<const bf16*>(fw + off); }
 };
 
 namespace {
@@ -391,8 +441,127 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
 }
 
 // ---- denoise schedule -------------------------------------------------------
+// Plan of the persistent denoise kernel for M = B * H chunk rows: two weight
+// slots (the largest job slice: w rows of K + 8 bf16), the activation region
+// (each GEMM operand staged whole, or as two planes of a column split that
+// fits), the k-half reduction buffer, the row scales, the row-stage vectors
+// and four mbarriers.
+struct FusedPlan {
+  int slot_bytes = 0, a_bytes = 0;
+  int p_e = 1, p_o = 1, p_h = 1;  // column planes of the E-, q- and ffn-wide operands
+  size_t smem = 0;
+};
+
+size_t fused_misc_bytes(const svla_config& c) {
+  return 4 * 4 * 4 * 32 * sizeof(float) + FD_MAX_M * sizeof(float) + ((size_t)c.e_width + 128) * sizeof(float) + 32;
+}
+
+bool fused_plan(const svla_config& c, int M, FusedPlan* fp) {
+  const int E = c.e_width, qw = c.e_heads * c.head_dim;
+  auto sl = [](int w, int K) { return (size_t)w * (K + 8) * 2; };
+  size_t slot = std::max({sl(8, E), sl(16, E), sl(8, qw), sl(32, E), sl(8, c.e_ffn)});
+  slot = (slot + 127) / 128 * 128;
+  const size_t misc = fused_misc_bytes(c);
+  if (2 * slot + misc + AttnCfg<64, FD_ATT_NBUF>::SMEM > (size_t)FD_SMEM_MAX) return false;
+  const size_t budget = (size_t)FD_SMEM_MAX - 2 * slot - misc;
+  // attention blocks and the row stage's W_out, W_in share the region
+  size_t need = std::max({AttnCfg<64, FD_ATT_NBUF>::SMEM, AttnCfg<32, FD_ATT_NBUF>::SMEM, (size_t)4 * c.action_dim * E});
+  auto planes = [&](int K, int* P) {
+    for (int q = 1; q <= FD_MAX_PLANES; q *= 2) {
+      if (K % (16 * q)) return false;
+      const size_t plane = (size_t)M * (K / q + 8) * 2;
+      const size_t region = q == 1 ? plane : 2 * plane;
+      if (region <= budget) {
+        *P = q;
+        need = std::max(need, region);
+        return true;
+      }
+    }
+    return false;
+  };
+  FusedPlan f;
+  if (!planes(E, &f.p_e) || !planes(qw, &f.p_o) || !planes(c.e_ffn, &f.p_h)) return false;
+  f.slot_bytes = (int)slot;
+  f.a_bytes = (int)((need + 127) / 128 * 128);
+  f.smem = 2 * slot + f.a_bytes + misc;
+  if (f.smem > (size_t)FD_SMEM_MAX) return false;
+  if (fp) *fp = f;
+  return true;
+}
+
+bool fused_ok(const svla_handle* h, int B, int H) {
+  const svla_config& c = h->cfg;
+  if (B < 1 || H < 1 || B > c.max_batch || H > c.max_chunk) return false;
+  if ((long long)B * H > FD_MAX_M || H > ATT_BQ || H > ATT_BK) return false;
+  if (c.e_layers > FD_MAX_LAYERS || c.e_ffn % 32 || c.e_width % 16) return false;
+  if (h->num_sms < 1 || !h->fw) return false;
+  return fused_plan(c, B * H, nullptr);
+}
+
+cudaError_t launch_fused(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise, int H,
+                         int n_steps, float* actions, float* trace, const float* prefix, int d, cudaStream_t s) {
+  (void)kv;
+  const svla_config& c = h->cfg;
+  const Layout& Lh = h->lay;
+  const int Mp = B * L, kvw = c.e_kv_heads * c.head_dim;
+  FdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = B; a.H = H; a.L = L; a.M = B * H; a.E = c.e_width; a.A = c.action_dim; a.hd = c.head_dim;
+  a.nq = c.e_heads; a.nkv = c.e_kv_heads; a.ffn = c.e_ffn; a.n_steps = n_steps; a.n_layers = c.e_layers;
+  a.eps = c.rms_eps;
+  a.dt = -1.0f / (float)n_steps;
+  a.noise = noise; a.x = actions; a.trace = trace; a.prefix = d > 0 ? prefix : nullptr; a.d = d; a.pad = pad;
+  FusedPlan fp;
+  if (!fused_plan(c, B * H, &fp)) return cudaErrorInvalidValue;
+  const FusedWeights& F = h->fwl;
+  a.w_in = h->W(Lh.w_in.off); a.b_in = h->W(Lh.b_in.off); a.w_t1 = h->W(Lh.w_t1.off);
+  a.b_t1 = h->W(Lh.b_t1.off); a.b_t2 = h->b_t2_f32;
+  a.w_t1a = h->FW(F.t1a); a.w_t2 = h->FW(F.t2);
+  a.final_norm = h->W(Lh.final_norm.off); a.w_out = h->W(Lh.w_out.off); a.b_out = h->W(Lh.b_out.off);
+  for (int l = 0; l < c.e_layers; ++l) {
+    const Entry* e = &Lh.e[9 * l];
+    FdLayer& fl = a.layer[l];
+    (void)e;
+    fl.w_qkv = h->FW(F.qkv[l]);
+    fl.w_o = h->FW(F.o[l]);
+    fl.w_gu = h->FW(F.gu[l]);
+    fl.w_d = h->FW(F.d[l]);
+    if (l % 2 == 1) {
+      fl.kx = h->kvx + (size_t)(l / 2) * 2 * Mp * kvw;
+      fl.vx = fl.kx + (size_t)Mp * kvw;
+    }
+  }
+  a.rope_cs = h->rope_cs; a.inv_period = h->inv_period;
+  const int qw = c.e_heads * c.head_dim;
+  a.r = h->e_r;
+  a.rb = FdAct{h->e_y, c.e_width, fp.p_e};
+  a.a = FdAct{h->e_a, c.e_width, fp.p_e};
+  a.h1 = FdAct{h->e_h1, c.e_width, fp.p_e};
+  a.o = FdAct{h->e_o, qw, fp.p_o};
+  a.hh = FdAct{h->e_h, c.e_ffn, fp.p_h};
+  a.q = h->e_q; a.k = h->e_k; a.v = h->e_v; a.c = h->e_c;
+  a.sync = h->fd_sync; a.status = h->status; a.wait_ns = g_wait_ns.load();
+  a.slot_bytes = fp.slot_bytes;
+  a.a_bytes = fp.a_bytes;
+  const size_t smem = fp.smem;
+  SVLA_TRY(cudaMemsetAsync(h->fd_sync, 0, 2 * sizeof(unsigned), s));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(h->num_sms);
+  cfg.blockDim = dim3(FD_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident at once: the grid barriers need it
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return c.head_dim == 64 ? cudaLaunchKernelEx(&cfg, denoise_fused_kernel<64>, a)
+                          : cudaLaunchKernelEx(&cfg, denoise_fused_kernel<32>, a);
+}
+
 cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise, int H,
-                           int n_steps, float* actions, float* trace, const float* prefix, int d, cudaStream_t s) {
+                           int n_steps, float* actions, float* trace, const float* prefix, int d, bool fused,
+                           cudaStream_t s) {
   const svla_config& c = h->cfg;
   const int M = B * H, E = c.e_width, hd = c.head_dim, A = c.action_dim;
   const int qw = c.e_heads * hd, kvw = c.e_kv_heads * hd, pkvw = c.p_kv_heads * hd;
@@ -411,6 +580,7 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
     SVLA_TRY(gemm(h, GE_BF16, cache + (size_t)(c.p_layers + l) * layer_elems, pkvw, h->W(e[3].off), pkvw, Mp, kvw,
                   pkvw, out_args(vx, kvw), h->e_part, h->e_cnt, s));
   }
+  if (fused) return launch_fused(h, kv, pad, B, L, noise, H, n_steps, actions, trace, prefix, d, s);
   const Layout& Lh = h->lay;
   int se_blocks = (M + SE_WARPS - 1) / SE_WARPS;
   if (se_blocks > 2 * NUM_SMS_B200) se_blocks = 2 * NUM_SMS_B200;
@@ -639,6 +809,29 @@ svla_status svla_create(const svla_config* cfg, const void* blob, size_t blob_by
   }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return bail(e, "gain folding");
+  // the persistent denoise kernel's copy of the expert GEMM weights (row pitch K + 8)
+  {
+    h->fwl = fused_weight_layout(c);
+    const FusedWeights& F = h->fwl;
+    if ((e = halloc(h, &h->fw, F.total)) != cudaSuccess) return bail(e, "fused weights");
+    const size_t E = c.e_width, qw = (size_t)c.e_heads * c.head_dim, kvw = (size_t)c.e_kv_heads * c.head_dim;
+    for (int l = 0; l < c.e_layers && e == cudaSuccess; ++l) {
+      const Entry* en = &lay.e[9 * l];
+      pad_rows_kernel<<<512, 256>>>(h->w + en[1].off, E, h->fw + F.qkv[l], (int)(l % 2 == 0 ? qw + 2 * kvw : qw),
+                                    (int)E);
+      pad_rows_kernel<<<512, 256>>>(h->w + en[4].off, qw, h->fw + F.o[l], (int)E, (int)qw);
+      pad_rows_kernel<<<512, 256>>>(h->w + en[6].off, E, h->fw + F.gu[l], 2 * c.e_ffn, (int)E);
+      pad_rows_kernel<<<512, 256>>>(h->w + en[8].off, c.e_ffn, h->fw + F.d[l], (int)E, c.e_ffn);
+      e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+      pad_rows_kernel<<<512, 256>>>(h->w + lay.w_t1.off, 2 * E, h->fw + F.t1a, (int)E, (int)E);
+      pad_rows_kernel<<<512, 256>>>(h->w + lay.w_t2.off, E, h->fw + F.t2, (int)E, (int)E);
+      e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return bail(e, "fused weights");
+  }
   if ((e = halloc(h, &h->b_t2_f32, c.e_width)) != cudaSuccess) return bail(e, "bias");
   bf16_to_f32_kernel<<<(c.e_width + 255) / 256, 256>>>(h->w + lay.b_t2.off, h->b_t2_f32, c.e_width);
   // RoPE table (reading 3), computed in double on the host
@@ -680,18 +873,21 @@ svla_status svla_create(const svla_config* cfg, const void* blob, size_t blob_by
   if ((e = halloc(h, &h->p_ss, (size_t)SS_TILES_MAX * Mp)) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->e_ss, (size_t)SS_TILES_MAX * Me)) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->e_r, Me * c.e_width)) != cudaSuccess) return bail(e, "workspace");
-  if ((e = halloc(h, &h->e_y, Me * c.e_width)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_y, Me * (c.e_width + 8 * FD_MAX_PLANES))) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->e_q, Me * eq)) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->e_k, Me * ekv)) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->e_v, Me * ekv)) != cudaSuccess) return bail(e, "workspace");
-  if ((e = halloc(h, &h->e_o, Me * eq)) != cudaSuccess) return bail(e, "workspace");
-  if ((e = halloc(h, &h->e_h, Me * c.e_ffn)) != cudaSuccess) return bail(e, "workspace");
-  if ((e = halloc(h, &h->e_a, Me * c.e_width)) != cudaSuccess) return bail(e, "workspace");
-  if ((e = halloc(h, &h->e_h1, Me * c.e_width)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_o, Me * (eq + 8 * FD_MAX_PLANES))) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_h, Me * (c.e_ffn + 8 * FD_MAX_PLANES))) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_a, Me * (c.e_width + 8 * FD_MAX_PLANES))) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->e_h1, Me * (c.e_width + 8 * FD_MAX_PLANES))) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->e_c, (size_t)c.e_width)) != cudaSuccess) return bail(e, "workspace");
   if ((e = halloc(h, &h->kvx, (size_t)((c.e_layers + 1) / 2) * 2 * Mp * ekv)) != cudaSuccess)
     return bail(e, "workspace");
   if ((e = halloc(h, &h->noise_buf, Me * c.action_dim)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = halloc(h, &h->fd_sync, 2)) != cudaSuccess) return bail(e, "workspace");
+  if ((e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess)
+    return bail(e, "device attributes");
   if ((e = halloc(h, reinterpret_cast<uint8_t**>(&h->p_part), PART_BYTES)) != cudaSuccess) return bail(e, "split-K");
   if ((e = halloc(h, reinterpret_cast<uint8_t**>(&h->e_part), PART_BYTES)) != cudaSuccess) return bail(e, "split-K");
   if ((e = halloc(h, &h->p_cnt, CNT_INTS)) != cudaSuccess) return bail(e, "split-K");
@@ -745,16 +941,21 @@ static svla_status denoise_impl(svla_handle* h, const void* kv, const uint8_t* p
   if (d > 0 && !prefix) return fail(h, SVLA_ERR_ARG, "null prefix with d > 0");
   if (d > 0 && (const void*)noise == (const void*)actions)
     return fail(h, SVLA_ERR_ARG, "the prefix overwrite needs the noise: actions must not alias noise");
+  const bool can_fuse = fused_ok(h, B, H);
+  if (h->denoise_path == SVLA_DENOISE_FUSED && !can_fuse)
+    return fail(h, SVLA_ERR_UNSUPPORTED, "the persistent denoise kernel needs B * H <= 64 and H <= 64");
+  const bool fused = can_fuse && h->denoise_path != SVLA_DENOISE_GRAPH;
   DeviceGuard dg(h->device);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  std::vector<uint64_t> key = {2, (uint64_t)B, (uint64_t)L, (uint64_t)H, (uint64_t)n_steps,
+  std::vector<uint64_t> key = {fused ? 3u : 2u, (uint64_t)B, (uint64_t)L, (uint64_t)H, (uint64_t)n_steps,
                                (uint64_t)(uintptr_t)kv, (uint64_t)(uintptr_t)pad, (uint64_t)(uintptr_t)noise,
                                (uint64_t)(uintptr_t)actions, (uint64_t)(uintptr_t)trace, g_wait_ns.load(),
                                (uint64_t)(uintptr_t)(d > 0 ? prefix : nullptr), (uint64_t)d};
   return run_graph(
       h, key,
       [&](cudaStream_t cs) {
-        return record_denoise(h, kv, pad, B, L, noise, H, n_steps, actions, trace, d > 0 ? prefix : nullptr, d, cs);
+        return record_denoise(h, kv, pad, B, L, noise, H, n_steps, actions, trace, d > 0 ? prefix : nullptr, d, fused,
+                              cs);
       },
       s, "denoise");
 }
@@ -791,6 +992,16 @@ svla_status svla_sample(svla_handle* h, const void* embeds, const uint8_t* pad, 
   if (st != SVLA_OK) return st;
   return svla_denoise(h, kv, pad, B, L, noise, H, n_steps, actions, nullptr, stream);
 }
+
+svla_status svla_set_denoise_path(svla_handle* h, int path) {
+  if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
+  if (path != SVLA_DENOISE_AUTO && path != SVLA_DENOISE_GRAPH && path != SVLA_DENOISE_FUSED)
+    return fail(h, SVLA_ERR_ARG, "path must be SVLA_DENOISE_AUTO, _GRAPH or _FUSED");
+  h->denoise_path = path;
+  return SVLA_OK;
+}
+
+int svla_denoise_fused_supported(const svla_handle* h, int B, int H) { return h && fused_ok(h, B, H) ? 1 : 0; }
 
 svla_status svla_device_status(svla_handle* h, void* stream) {
   if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");

@@ -143,6 +143,13 @@ class SmolVLA:
         _abi.check(st, self.h)
         return (actions, kv_cache, noise) if return_noise else (actions, kv_cache)
 
+    def set_denoise_path(self, path: int) -> None:
+        """_abi.DENOISE_AUTO (default), DENOISE_GRAPH or DENOISE_FUSED."""
+        _abi.check(self.lib.svla_set_denoise_path(self.h, path), self.h)
+
+    def fused_supported(self, B: int, H: int) -> bool:
+        return bool(self.lib.svla_denoise_fused_supported(self.h, B, H))
+
     def device_status(self, stream=None) -> int:
         """Synchronise the stream; return (and clear) the device-side status."""
         return int(self.lib.svla_device_status(self.h, _stream(stream)))
