@@ -162,7 +162,9 @@ SVLA_API svla_status svla_denoise_prefix(svla_handle* h, const void* kv_cache, c
 SVLA_API svla_status svla_set_denoise_path(svla_handle* h, int path);
 
 /* 1 if the persistent denoise kernel takes batch B with chunk length H on
- * this handle (B * H <= 64, H <= 64, within the handle's limits), else 0. */
+ * this handle for every prefix length up to max_prefix (B * H <= 64, H <= 64,
+ * within the handle's limits, and a head's prefix keys and values fit in
+ * shared memory), else 0. */
 SVLA_API int svla_denoise_fused_supported(const svla_handle* h, int B, int H);
 
 /* Draw the noise, prefill, denoise, on one stream.

@@ -51,8 +51,7 @@ constexpr int FD_THREADS = 256;
 constexpr int FD_MAX_M = 64;    // chunk rows handled (B * H)
 constexpr int FD_MAX_LAYERS = 32;
 constexpr int FD_MAX_PLANES = 8;
-constexpr int FD_PIPE_TID = 128;
-constexpr int FD_ATT_NBUF = 4;    // key/value tiles of the cross-attention in flight at once  // the thread that refills the weight slots (warp 4, idle in epilogues)
+constexpr int FD_PIPE_TID = 128;  // the thread that refills the weight slots (warp 4, idle in epilogues)
 
 enum FdEpi : int { FD_SILU_BIAS = 0, FD_RES_INIT, FD_QKV_ROPE, FD_Q, FD_RES_ADD, FD_SWIGLU };
 
@@ -67,6 +66,7 @@ struct FdAct {
 };
 
 SVLA_DEV size_t fd_act_off(const FdAct& a, int M, int m, int c) {
+  if (a.P == 1) return (size_t)m * (a.K + 8) + c;
   const int kp = a.K / a.P, q = c / kp;
   return ((size_t)q * M + m) * (kp + 8) + (c - q * kp);
 }
@@ -185,11 +185,15 @@ SVLA_DEV void fd_job_rows(const FdArgs& p, const FdGemm& s, int j, int& r0, int&
 // ---------------------------------------------------------------------------
 // small PTX helpers
 // ---------------------------------------------------------------------------
-SVLA_DEV unsigned ld_acquire_u32(const unsigned* p) {
+SVLA_DEV unsigned ld_relaxed_u32(const unsigned* p) {
   unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+SVLA_DEV void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+SVLA_DEV void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 SVLA_DEV void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -215,12 +219,12 @@ SVLA_DEV bool fd_grid_sync(const FdArgs& p, unsigned idx, int* flag) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    __threadfence();
-    atomicAdd(p.sync, 1u);
+    // release: this CTA's writes (ordered before this thread by the barrier above)
+    red_release_add(p.sync, 1u);
     const unsigned target = (idx + 1) * gridDim.x;
     uint64_t t0 = 0;
     for (uint32_t i = 1;; ++i) {
-      if (ld_acquire_u32(p.sync) >= target) break;
+      if (ld_relaxed_u32(p.sync) >= target) break;
       if (*reinterpret_cast<volatile unsigned*>(p.sync + 1) != 0) { ok = 0; break; }
       if ((i & 63u) == 0) {
         const uint64_t now = globaltimer_ns();
@@ -234,7 +238,7 @@ SVLA_DEV bool fd_grid_sync(const FdArgs& p, unsigned idx, int* flag) {
         }
       }
     }
-    __threadfence();
+    fence_acquire_gpu();  // acquire: the other CTAs' writes before their arrivals
     *flag = ok;
   }
   __syncthreads();
@@ -289,6 +293,9 @@ SVLA_DEV void fd_issue(const FdArgs& p, FdPipe& pp, uint8_t* slots, uint32_t bar
 // elements this thread holds are added to ss (rows g and g + 8 of the m-tile):
 // the RMSNorm statistics come for free from the operand registers.
 // ---------------------------------------------------------------------------
+// x * sigmoid(x) with the fast (approximate, 2 ulp) division
+SVLA_DEV float fd_silu(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+
 SVLA_DEV float sq_bf16x2(uint32_t u) {
   const float lo = __uint_as_float(u << 16), hi = __uint_as_float(u & 0xffff0000u);
   return fmaf(lo, lo, hi * hi);
@@ -515,7 +522,7 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, u
         const float g0 = acc[t][2 * hr] * sc[hr], g1 = acc[t][2 * hr + 1] * sc[hr];
         const float u0 = acc[t + 2][2 * hr] * sc[hr], u1 = acc[t + 2][2 * hr + 1] * sc[hr];
         *reinterpret_cast<uint32_t*>(p.hh.ptr + fd_act_off(p.hh, M, m, gcol + 8 * t + 2 * t4)) =
-            pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+            pack_bf16x2(fd_silu(g0) * u0, fd_silu(g1) * u1);
       }
     }
   } else {
@@ -527,8 +534,8 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, u
       if (m >= M) continue;
       float v0 = acc[0][2 * hr] * sc[hr], v1 = acc[0][2 * hr + 1] * sc[hr];
       if (s.epi == FD_SILU_BIAS) {
-        v0 = silu_f(v0 + pre[hr][0].x);
-        v1 = silu_f(v1 + pre[hr][0].y);
+        v0 = fd_silu(v0 + pre[hr][0].x);
+        v1 = fd_silu(v1 + pre[hr][0].y);
         *reinterpret_cast<uint32_t*>(p.h1.ptr + fd_act_off(p.h1, M, m, col)) = pack_bf16x2(v0, v1);
       } else if (s.epi == FD_Q) {
         *reinterpret_cast<uint32_t*>(p.q + (size_t)m * (p.nq * HD) + col) = pack_bf16x2(v0, v1);
@@ -544,6 +551,185 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, u
 }
 
 // ---------------------------------------------------------------------------
+// Attention of the small-batch chunk (the same definition as attention_block:
+// softmax(q k^T / sqrt(hd) + mask) v, GQA, causal self-attention over the chunk
+// or cross-attention to valid prefix keys) with the work of one (query b, head
+// h) split finer: a job is 16 query rows, and the CTA's 8 warps split that
+// job's keys in chunks of 16 (warp w takes chunks w, w + 8, ..), each keeping
+// its own running max, sum and output; the 8 partial states are merged in
+// shared memory in warp order (deterministic). At batch 1 this spreads a
+// layer's attention over B * heads * ceil(H / 16) CTAs and all their warps.
+// Shared memory: Q [16][HD + 8], K and V [Lk][HD + 8] (bf16), key flags [Lk],
+// the merge buffers [8][16][HD] fp32 + [8][16][2] fp32.
+// ---------------------------------------------------------------------------
+template <int HD>
+__host__ __device__ inline size_t fd_att_smem(int Lk) {
+  const int lk = (Lk + 15) & ~15;
+  return (size_t)(16 + 2 * lk) * (HD + 8) * 2 + lk + 8 * 16 * HD * 4 + 8 * 16 * 2 * 4;
+}
+
+template <int HD>
+SVLA_DEV void fd_attention_job(const AttnArgs& a, int b, int h, int i0, uint8_t* smem) {
+  constexpr int LDS = HD + 8, KS = HD / 16, ND = HD / 8, CPR = HD / 8;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int g_kv = h / (a.n_q / a.n_kv);
+  const int nrow = min(16, a.Lq - i0);
+  const int lk = a.causal ? min(a.Lk, i0 + 16) : a.Lk;  // keys any row of this job can see
+  const int lkp = (lk + 15) & ~15;
+  bf16* sQ = reinterpret_cast<bf16*>(smem);
+  bf16* sK = sQ + 16 * LDS;
+  bf16* sV = sK + (size_t)lkp * LDS;
+  uint8_t* sF = reinterpret_cast<uint8_t*>(sV + (size_t)lkp * LDS);
+  float* sO = reinterpret_cast<float*>(smem + (fd_att_smem<HD>(a.Lk) - 8 * 16 * HD * 4 - 8 * 16 * 2 * 4));
+  float* sML = sO + 8 * 16 * HD;
+
+  const bf16* qbase = a.q + ((size_t)b * a.Lq + i0) * a.ldq + (size_t)h * HD;
+  const bf16* kbase = a.k + (size_t)b * a.Lk * a.ldkv + (size_t)g_kv * HD;
+  const bf16* vbase = a.v + (size_t)b * a.Lk * a.ldkv + (size_t)g_kv * HD;
+  for (int i = tid; i < 16 * CPR; i += FD_THREADS) {
+    const int r = i / CPR, c = i % CPR;
+    const bool ok = r < nrow;
+    cp_async16(smem_u32(sQ + r * LDS + c * 8), qbase + (size_t)(ok ? r : 0) * a.ldq + c * 8, ok);
+  }
+  for (int i = tid; i < lkp * CPR; i += FD_THREADS) {
+    const int r = i / CPR, c = i % CPR;
+    const bool ok = r < lk;
+    const size_t off = (size_t)(ok ? r : 0) * a.ldkv + c * 8;
+    cp_async16(smem_u32(sK + r * LDS + c * 8), kbase + off, ok);
+    cp_async16(smem_u32(sV + r * LDS + c * 8), vbase + off, ok);
+  }
+  for (int j = tid; j < lkp; j += FD_THREADS)
+    sF[j] = (j < lk) ? (a.key_valid ? a.key_valid[(size_t)b * a.Lk + j] : (uint8_t)1) : (uint8_t)0;
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  uint32_t qa[KS][4];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int mi = lane >> 3;
+    ldsm_x4(smem_u32(sQ + ((mi & 1) * 8 + (lane & 7)) * LDS + ks * 16 + (mi >> 1) * 8), qa[ks][0], qa[ks][1],
+            qa[ks][2], qa[ks][3]);
+  }
+  float o[ND][4];
+#pragma unroll
+  for (int i = 0; i < ND; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  const int row_a = i0 + g, row_b = i0 + g + 8;  // query positions of this thread's rows
+  for (int ch = warp; ch * 16 < lk; ch += 8) {
+    const int k0 = ch * 16;
+    float sc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int mi = lane >> 3;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(smem_u32(sK + (k0 + (mi >> 1) * 8 + (lane & 7)) * LDS + ks * 16 + (mi & 1) * 8), b0, b1, b2, b3);
+      mma_bf16_16816(sc[0], qa[ks], b0, b1);
+      mma_bf16_16816(sc[1], qa[ks], b2, b3);
+    }
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = k0 + nt * 8 + 2 * t4 + (e & 1);
+        const int row = (e >> 1) ? row_b : row_a;
+        bool vis = sF[j] != 0;
+        if (a.causal) vis = vis && (j <= row);
+        const float v = vis ? sc[nt][e] * a.scale_log2 : -INFINITY;
+        sc[nt][e] = v;
+        mx[e >> 1] = fmaxf(mx[e >> 1], v);
+      }
+    float muse[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+      const float m_new = fmaxf(m_run[r], mx[r]);
+      muse[r] = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = exp2f(m_run[r] - muse[r]);
+      m_run[r] = m_new;
+      l_run[r] *= alpha;
+#pragma unroll
+      for (int i = 0; i < ND; ++i) {
+        o[i][2 * r] *= alpha;
+        o[i][2 * r + 1] *= alpha;
+      }
+    }
+    uint32_t pa[4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const float p0 = exp2f(sc[nt][0] - muse[0]), p1 = exp2f(sc[nt][1] - muse[0]);
+      const float p2 = exp2f(sc[nt][2] - muse[1]), p3 = exp2f(sc[nt][3] - muse[1]);
+      l_run[0] += p0 + p1;
+      l_run[1] += p2 + p3;
+      pa[nt * 2 + 0] = pack_bf16x2(p0, p1);
+      pa[nt * 2 + 1] = pack_bf16x2(p2, p3);
+    }
+#pragma unroll
+    for (int nd2 = 0; nd2 < ND / 2; ++nd2) {
+      const int mi = lane >> 3;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(smem_u32(sV + (k0 + (mi & 1) * 8 + (lane & 7)) * LDS + nd2 * 16 + (mi >> 1) * 8), b0, b1, b2, b3);
+      mma_bf16_16816(o[2 * nd2], pa, b0, b1);
+      mma_bf16_16816(o[2 * nd2 + 1], pa, b2, b3);
+    }
+  }
+  // this warp's partial state: running max, sum over its keys, unnormalised output
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+    l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+  }
+  float* myO = sO + warp * 16 * HD;
+#pragma unroll
+  for (int nd = 0; nd < ND; ++nd) {
+    const int c = nd * 8 + 2 * t4;
+    *reinterpret_cast<float2*>(myO + g * HD + c) = make_float2(o[nd][0], o[nd][1]);
+    *reinterpret_cast<float2*>(myO + (g + 8) * HD + c) = make_float2(o[nd][2], o[nd][3]);
+  }
+  if (t4 == 0) {
+    sML[(warp * 16 + g) * 2] = m_run[0];
+    sML[(warp * 16 + g) * 2 + 1] = l_run[0];
+    sML[(warp * 16 + g + 8) * 2] = m_run[1];
+    sML[(warp * 16 + g + 8) * 2 + 1] = l_run[1];
+  }
+  __syncthreads();
+  // merge the 8 partial states (warp order), normalise, store bf16 pairs
+  for (int idx = tid; idx < 16 * (HD / 2); idx += FD_THREADS) {
+    const int r = idx / (HD / 2), c = 2 * (idx % (HD / 2));
+    if (r >= nrow) continue;
+    float mmax = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) mmax = fmaxf(mmax, sML[(w * 16 + r) * 2]);
+    const float muse = (mmax == -INFINITY) ? 0.f : mmax;
+    float l = 0.f, v0 = 0.f, v1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const float f = exp2f(sML[(w * 16 + r) * 2] - muse);
+      l += f * sML[(w * 16 + r) * 2 + 1];
+      const float2 ov = *reinterpret_cast<const float2*>(sO + (w * 16 + r) * HD + c);
+      v0 += f * ov.x;
+      v1 += f * ov.y;
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const int m = b * a.Lq + i0 + r, col = h * HD + c;
+    bf16* dst;
+    if (a.o_pc == 0) {
+      dst = a.out + (size_t)m * a.ldo + col;
+    } else {
+      const int pl = col / a.o_pc;
+      dst = a.out + ((size_t)pl * a.o_M + m) * (a.o_pc + 8) + (col - pl * a.o_pc);
+    }
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(v0 * inv, v1 * inv);
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
 // row stage: end of step k_end (if >= 0) and start of step k_begin (if < n),
 // rows m = blockIdx.x, blockIdx.x + gridDim.x, ..:
 //   v = RMSNorm(r) W_out^T + b_out, x += dt v (trace, prefix overwrite), then
@@ -551,6 +737,11 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, u
 // Weight rows are read as 16-byte vectors, all of a warp's loads issued before
 // its arithmetic.
 // ---------------------------------------------------------------------------
+// bytes of the row stage's staged weights (W_out, W_in, b_in, final_norm, b_out), rounded to 16
+__host__ __device__ inline size_t fd_row_stage_bytes(int E, int A) {
+  return (((size_t)4 * A * E + 4 * E + 2 * A) + 15) / 16 * 16;
+}
+
 SVLA_DEV bool fd_row_stage(const FdArgs& p, int k_end, int k_begin, float* fbuf, uint8_t* ubuf, FdPipe& pp,
                            uint32_t bar_base, int* flag) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -559,18 +750,34 @@ SVLA_DEV bool fd_row_stage(const FdArgs& p, int k_end, int k_begin, float* fbuf,
   float* y = fbuf;           // [E]
   float* xs = fbuf + E;      // [A]
   float* red = xs + 64;      // [8]
-  // W_out [A, E] and W_in [E, A] staged in shared memory (one bulk copy each)
+  // W_out [A, E], W_in [E, A], b_in [E], final_norm [E], b_out [A] staged in
+  // shared memory (one bulk copy each)
   const uint16_t* sw_out = reinterpret_cast<const uint16_t*>(ubuf);
   const uint16_t* sw_in = sw_out + (size_t)A * E;
+  const uint16_t* sb_in = sw_in + (size_t)A * E;
+  const uint16_t* sgain = sb_in + E;
+  const uint16_t* sb_out = sgain + E;
+  float* sx = reinterpret_cast<float*>(ubuf + fd_row_stage_bytes(E, A));  // [3][A]: x, noise, prefix rows
   if (tid == 0) {
     const uint32_t bar = bar_base + 16, bytes = (uint32_t)A * E * 2;
-    mbar_arrive_expect_tx(bar, 2 * bytes);
+    mbar_arrive_expect_tx(bar, 2 * bytes + 4 * E + 2 * A);
     bulk_load(smem_u32(sw_out), p.w_out, bytes, bar);
     bulk_load(smem_u32(sw_in), p.w_in, bytes, bar);
+    bulk_load(smem_u32(sb_in), p.b_in, 2 * E, bar);
+    bulk_load(smem_u32(sgain), p.final_norm, 2 * E, bar);
+    bulk_load(smem_u32(sb_out), p.b_out, 2 * A, bar);
     ++pp.a_iss[0];
   }
   bool staged = false;
   for (int m = blockIdx.x; m < M; m += gridDim.x) {
+    // this row's state (and the prefix-overwrite inputs), fetched while the weights land
+    for (int o = tid; o < A; o += FD_THREADS) {
+      sx[o] = __ldcg(p.x + (size_t)m * A + o);
+      if (p.prefix && k_end >= 0 && (m % p.H) < p.d) {
+        sx[A + o] = p.noise[(size_t)m * A + o];
+        sx[2 * A + o] = p.prefix[((size_t)(m / p.H) * p.d + (m % p.H)) * A + o];
+      }
+    }
     if (k_end >= 0) {
       // final RMSNorm of the residual row
       float ss = 0.f;
@@ -603,8 +810,7 @@ SVLA_DEV bool fd_row_stage(const FdArgs& p, int k_end, int k_begin, float* fbuf,
 #pragma unroll
       for (int w = 0; w < FD_THREADS / 32; ++w) tot += red[w];
       const float inv = rsqrtf(tot / (float)E + p.eps);
-      for (int c = tid; c < E; c += FD_THREADS)
-        y[c] *= inv * bf2f(reinterpret_cast<const uint16_t*>(p.final_norm)[c]);
+      for (int c = tid; c < E; c += FD_THREADS) y[c] *= inv * bf2f(sgain[c]);
       __syncthreads();
       // action_out + Euler: warp w handles outputs w, w + 8, ..
       for (int o = warp; o < A; o += FD_THREADS / 32) {
@@ -623,13 +829,11 @@ SVLA_DEV bool fd_row_stage(const FdArgs& p, int k_end, int k_begin, float* fbuf,
 #pragma unroll
         for (int sft = 16; sft > 0; sft >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, sft);
         if (lane == 0) {
-          const float vv = dot + bf2f(reinterpret_cast<const uint16_t*>(p.b_out)[o]);
-          float xn = __ldcg(p.x + (size_t)m * A + o) + p.dt * vv;
-          if (p.prefix) {
-            const int b = m / p.H, jr = m % p.H;
+          const float vv = dot + bf2f(sb_out[o]);
+          float xn = sx[o] + p.dt * vv;
+          if (p.prefix && (m % p.H) < p.d) {
             const float t_next = 1.0f - (float)(k_end + 1) / (float)p.n_steps;
-            if (jr < p.d)
-              xn = t_next * p.noise[(size_t)m * A + o] + (1.0f - t_next) * p.prefix[((size_t)b * p.d + jr) * A + o];
+            xn = t_next * sx[A + o] + (1.0f - t_next) * sx[2 * A + o];
           }
           p.x[(size_t)m * A + o] = xn;
           xs[o] = xn;
@@ -640,7 +844,7 @@ SVLA_DEV bool fd_row_stage(const FdArgs& p, int k_end, int k_begin, float* fbuf,
         }
       }
     } else {
-      for (int o = tid; o < A; o += FD_THREADS) xs[o] = __ldcg(p.x + (size_t)m * A + o);
+      for (int o = tid; o < A; o += FD_THREADS) xs[o] = sx[o];
     }
     __syncthreads();
     if (k_begin < p.n_steps) {
@@ -657,8 +861,7 @@ SVLA_DEV bool fd_row_stage(const FdArgs& p, int k_end, int k_begin, float* fbuf,
             acc = fmaf(xs[8 * c + 2 * e + 1], __uint_as_float(q[e] & 0xffff0000u), acc);
           }
         }
-        p.a.ptr[fd_act_off(p.a, M, m, o)] =
-            __float2bfloat16_rn(acc + bf2f(reinterpret_cast<const uint16_t*>(p.b_in)[o]));
+        p.a.ptr[fd_act_off(p.a, M, m, o)] = __float2bfloat16_rn(acc + bf2f(sb_in[o]));
       }
     }
     __syncthreads();
@@ -762,7 +965,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
       const FdGemm s = fd_gemm(p, g);
       if (gi == 0 && k + 1 < p.n_steps) {
         // rows of W_t1 for the next step's time vector (computed during layer 0's attention)
-        const int n_att = p.B * p.nq, G = (int)gridDim.x;
+        const int n_att = p.B * p.nq * ((p.H + 15) / 16), G = (int)gridDim.x;
         if (n_att < G)
           fd_time_c_prefetch(p, (int)blockIdx.x - n_att, G - n_att);
         else
@@ -803,15 +1006,15 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
         } else {
           at.k = p.layer[l].kx; at.v = p.layer[l].vx; at.key_valid = p.pad; at.Lk = p.L; at.causal = 0;
         }
-        const int n_att = p.B * p.nq;
+        const int rblk = (p.H + 15) / 16;
+        const int n_att = p.B * p.nq * rblk;
         for (int jb = blockIdx.x; jb < n_att; jb += gridDim.x) {
-          if (threadIdx.x < ATT_THREADS)
-            attention_block<HD, FD_ATT_NBUF>(at, 0, jb % p.nq, jb / p.nq, ubuf, threadIdx.x, 1);
-          __syncthreads();
+          const int rb_ = jb % rblk, hh_ = (jb / rblk) % p.nq, b_ = jb / (rblk * p.nq);
+          fd_attention_job<HD>(at, b_, hh_, 16 * rb_, ubuf);
         }
         if (l == 0 && k + 1 < p.n_steps) {
           // the next step's time vector (its T1 stage is far ahead): on the CTAs
-          // without an attention block when there are such CTAs
+          // without an attention job when there are such CTAs
           const int G = (int)gridDim.x;
           if (n_att < G)
             fd_time_c(p, k + 1, (int)blockIdx.x - n_att, G - n_att, fbuf);

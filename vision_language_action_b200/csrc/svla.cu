@@ -456,16 +456,19 @@ size_t fused_misc_bytes(const svla_config& c) {
   return 4 * 4 * 4 * 32 * sizeof(float) + FD_MAX_M * sizeof(float) + ((size_t)c.e_width + 128) * sizeof(float) + 32;
 }
 
-bool fused_plan(const svla_config& c, int M, FusedPlan* fp) {
+bool fused_plan(const svla_config& c, int M, int L, FusedPlan* fp) {
   const int E = c.e_width, qw = c.e_heads * c.head_dim;
   auto sl = [](int w, int K) { return (size_t)w * (K + 8) * 2; };
   size_t slot = std::max({sl(8, E), sl(16, E), sl(8, qw), sl(32, E), sl(8, c.e_ffn)});
   slot = (slot + 127) / 128 * 128;
   const size_t misc = fused_misc_bytes(c);
-  if (2 * slot + misc + AttnCfg<64, FD_ATT_NBUF>::SMEM > (size_t)FD_SMEM_MAX) return false;
+  if (2 * slot + misc > (size_t)FD_SMEM_MAX) return false;
   const size_t budget = (size_t)FD_SMEM_MAX - 2 * slot - misc;
-  // attention blocks and the row stage's W_out, W_in share the region
-  size_t need = std::max({AttnCfg<64, FD_ATT_NBUF>::SMEM, AttnCfg<32, FD_ATT_NBUF>::SMEM, (size_t)4 * c.action_dim * E});
+  // the attention jobs (all keys staged) and the row stage's W_out, W_in share the region
+  const size_t att = std::max(c.head_dim == 64 ? fd_att_smem<64>(L) : fd_att_smem<32>(L),
+                              c.head_dim == 64 ? fd_att_smem<64>(c.max_chunk) : fd_att_smem<32>(c.max_chunk));
+  size_t need = std::max(att, fd_row_stage_bytes(E, c.action_dim) + 3 * 64 * sizeof(float));
+  if (need > budget) return false;
   auto planes = [&](int K, int* P) {
     for (int q = 1; q <= FD_MAX_PLANES; q *= 2) {
       if (K % (16 * q)) return false;
@@ -489,13 +492,13 @@ bool fused_plan(const svla_config& c, int M, FusedPlan* fp) {
   return true;
 }
 
-bool fused_ok(const svla_handle* h, int B, int H) {
+bool fused_ok(const svla_handle* h, int B, int H, int L) {
   const svla_config& c = h->cfg;
   if (B < 1 || H < 1 || B > c.max_batch || H > c.max_chunk) return false;
   if ((long long)B * H > FD_MAX_M || H > ATT_BQ || H > ATT_BK) return false;
   if (c.e_layers > FD_MAX_LAYERS || c.e_ffn % 32 || c.e_width % 16) return false;
   if (h->num_sms < 1 || !h->fw) return false;
-  return fused_plan(c, B * H, nullptr);
+  return fused_plan(c, B * H, L, nullptr);
 }
 
 cudaError_t launch_fused(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise, int H,
@@ -512,7 +515,7 @@ cudaError_t launch_fused(svla_handle* h, const void* kv, const uint8_t* pad, int
   a.dt = -1.0f / (float)n_steps;
   a.noise = noise; a.x = actions; a.trace = trace; a.prefix = d > 0 ? prefix : nullptr; a.d = d; a.pad = pad;
   FusedPlan fp;
-  if (!fused_plan(c, B * H, &fp)) return cudaErrorInvalidValue;
+  if (!fused_plan(c, B * H, L, &fp)) return cudaErrorInvalidValue;
   const FusedWeights& F = h->fwl;
   a.w_in = h->W(Lh.w_in.off); a.b_in = h->W(Lh.b_in.off); a.w_t1 = h->W(Lh.w_t1.off);
   a.b_t1 = h->W(Lh.b_t1.off); a.b_t2 = h->b_t2_f32;
@@ -941,9 +944,10 @@ static svla_status denoise_impl(svla_handle* h, const void* kv, const uint8_t* p
   if (d > 0 && !prefix) return fail(h, SVLA_ERR_ARG, "null prefix with d > 0");
   if (d > 0 && (const void*)noise == (const void*)actions)
     return fail(h, SVLA_ERR_ARG, "the prefix overwrite needs the noise: actions must not alias noise");
-  const bool can_fuse = fused_ok(h, B, H);
+  const bool can_fuse = fused_ok(h, B, H, L);
   if (h->denoise_path == SVLA_DENOISE_FUSED && !can_fuse)
-    return fail(h, SVLA_ERR_UNSUPPORTED, "the persistent denoise kernel needs B * H <= 64 and H <= 64");
+    return fail(h, SVLA_ERR_UNSUPPORTED,
+                "the persistent denoise kernel needs B * H <= 64, H <= 64 and the prefix keys in shared memory");
   const bool fused = can_fuse && h->denoise_path != SVLA_DENOISE_GRAPH;
   DeviceGuard dg(h->device);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -1001,7 +1005,9 @@ svla_status svla_set_denoise_path(svla_handle* h, int path) {
   return SVLA_OK;
 }
 
-int svla_denoise_fused_supported(const svla_handle* h, int B, int H) { return h && fused_ok(h, B, H) ? 1 : 0; }
+int svla_denoise_fused_supported(const svla_handle* h, int B, int H) {
+  return h && fused_ok(h, B, H, h->cfg.max_prefix) ? 1 : 0;
+}
 
 svla_status svla_device_status(svla_handle* h, void* stream) {
   if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
