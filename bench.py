@@ -34,11 +34,13 @@ import synth  # noqa: E402
 METRIC = "ms per 50-action chunk (b=1)"
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM bytes (read + write) per launch of the batch-1 GEMM kernel: mean of the
-# three launches of the ncu --set full capture summarised in
-# profiles/gemm_tc_kernel_smolvla_b1.md. Set to None whenever the kernel changes
-# until it is captured again.
-NCU_TRAFFIC_PER_LAUNCH = None
+# DRAM bytes (read + write) per launch from ncu captures, None whenever the
+# kernel has changed since its capture:
+#  - the batch-1 GEMM kernel (gemm_tc_kernel): mean of the three launches of
+#    the capture summarised in profiles/gemm_tc_kernel_smolvla_b1.md;
+#  - the persistent denoise kernel: profiles/denoise_fused_kernel_smolvla_b1.md.
+NCU_TRAFFIC_GEMM_B1 = 3.698e6
+NCU_TRAFFIC_FUSED = 1.9915e9
 
 
 def _peaks():
@@ -103,12 +105,34 @@ def chunk_work(s, B, L, H, n_steps):
     return hbm, flops, att
 
 
-def launches_per_chunk(s, n_steps):
+def launches_per_chunk(s, n_steps, fused):
     """Kernels libsvla launches for one prefill + denoise (the CUDA graphs' kernel nodes)."""
     pre = 2 + s.p_layers + 4 * (s.p_layers - 1)   # positions, residual init, QKV per layer, attn/O/GU/D
     hoist = 2 * (s.e_layers // 2)
+    if fused:
+        return pre + hoist + 1                     # the whole Euler loop is one persistent kernel
     step = 1 + 2 + 5 * s.e_layers + 1              # step begin, time MLP, 5 per layer, step end
     return pre + hoist + n_steps * step
+
+
+def denoise_bytes(s, B, L, H, n_steps):
+    """Algorithmic HBM bytes of one svla_denoise call: the hoisted cross K/V
+    projection (odd-layer cache read, W_k/W_v, K'/V' written) once, then per
+    Euler step every expert weight the step multiplies by (streamed from HBM:
+    196 MB do not stay in the 126 MB L2) and the projected K'/V' it reads."""
+    man = dict(synth.manifest(s))
+    nbytes = lambda n: 2 * int(np.prod(man[n]))  # noqa: E731
+    kvw = s.p_kv_heads * s.head_dim
+    n_odd = s.e_layers // 2
+    kvx = n_odd * 2 * B * L * s.e_kv_width * 2
+    hoist = n_odd * 2 * B * L * kvw * 2 + kvx
+    step_w = 0
+    for l in range(s.e_layers):
+        names = ["in_norm", "wq", "wo", "post_norm", "wg", "wu", "wd"] + (["wk", "wv"] if l % 2 == 0 else [])
+        hoist += 0 if l % 2 == 0 else nbytes(f"e{l}.wk") + nbytes(f"e{l}.wv")
+        step_w += sum(nbytes(f"e{l}.{n}") for n in names)
+    step_w += sum(nbytes(n) for n in ("final_norm", "w_in", "b_in", "w_t1", "b_t1", "w_t2", "b_t2", "w_out", "b_out"))
+    return hoist + n_steps * (step_w + kvx)
 
 
 # ---------------------------------------------------------------------------
@@ -313,7 +337,7 @@ def gemm_roofline(s, B, L, H, n_steps, dev, hbm_peak):
     achieved = bytes_chunk / (t_chunk * 1e-3) / 1e9
     return {"bound": "hbm", "kernel": "gemm_tc_kernel", "achieved": round(achieved, 1), "peak": hbm_peak,
             "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-            "traffic": NCU_TRAFFIC_PER_LAUNCH,
+            "traffic": NCU_TRAFFIC_GEMM_B1,
             "launches_per_chunk": n_launch, "avg_launch_us": round(1e3 * t_chunk / n_launch, 2),
             "algorithmic_bytes_per_launch": int(bytes_chunk / n_launch),
             "gemm_ms_per_chunk": round(float(t_chunk), 4)}
@@ -379,7 +403,22 @@ def ours(args, rank, world, local_rank):
 
     hbm_bytes, gflops, aflops = chunk_work(s, wl.B, wl.L, wl.H, wl.n_steps)
     chunk_s = value * 1e-3 * world  # per-rank chunk latency in s
-    roof = gemm_roofline(s, wl.B, wl.L, wl.H, wl.n_steps, f"cuda:{dev}", hbm_peak)
+    fused = m.fused_supported(wl.B, wl.H)
+    graph_gemm = gemm_roofline(s, wl.B, wl.L, wl.H, wl.n_steps, f"cuda:{dev}", hbm_peak)
+    if fused:
+        # dominant kernel: the persistent denoise kernel, timed live as the denoise
+        # call it makes up (the call's graph also holds the 16 hoisted K'/V'
+        # projections, whose bytes are counted too)
+        dbytes = denoise_bytes(s, wl.B, wl.L, wl.H, wl.n_steps)
+        t_den = ms_den / args.steps * 1e-3
+        achieved = dbytes / t_den / 1e9
+        roof = {"bound": "hbm", "kernel": "denoise_fused_kernel", "achieved": round(achieved, 1), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": NCU_TRAFFIC_FUSED,
+                "algorithmic_bytes_per_launch": int(dbytes), "launch_ms": round(t_den * 1e3, 4),
+                "timed_as": "svla_denoise call (16 hoisted K'/V' projection GEMMs + denoise_fused_kernel), CUDA events",
+                "peak_kind": f"{peak_kind} HBM copy"}
+    else:
+        roof = graph_gemm
     m.close()
     del d
     torch.cuda.empty_cache()
@@ -438,7 +477,8 @@ def ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
             "breakdown": {"prefill_ms": round(ms_pre / args.steps, 4), "denoise_ms": round(ms_den / args.steps, 4),
                           "note": "each call timed alone on rank 0, same steps and warm-up"},
-            "gpu_launches": launches_per_chunk(s, wl.n_steps) * args.steps,
+            "gpu_launches": launches_per_chunk(s, wl.n_steps, fused) * args.steps,
+            "graph_gemm_roofline": graph_gemm if fused else None,
             "clocks": clk,
             "secondary": secondary,
         }
