@@ -125,6 +125,10 @@ struct FdGemm {
   int layer;
 };
 
+// Shared-memory copy of FdArgs::layer (dynamic indexing into the kernel
+// parameters would go through the constant cache on every job).
+__shared__ FdLayer fd_layers[FD_MAX_LAYERS];
+
 // GEMM stages per Euler step: time MLP (2), then QKV, O, gate/up, down per layer
 SVLA_DEV int fd_gemms_per_step(const FdArgs& p) { return 2 + 4 * p.n_layers; }
 
@@ -145,7 +149,7 @@ SVLA_DEV FdGemm fd_gemm(const FdArgs& p, int g) {
     return s;
   }
   const int l = (r - 2) / 4, sub = (r - 2) % 4;
-  const FdLayer& L = p.layer[l];
+  const FdLayer& L = fd_layers[l];
   s.layer = l;
   if (sub == 0) {
     s.A = p.rb; s.W = L.w_qkv; s.norm = true;
@@ -939,6 +943,8 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
   __shared__ FdPipe pp;
 
   const uint32_t bar_base = smem_u32(bars);
+  for (int l = threadIdx.x; l < p.n_layers; l += FD_THREADS) fd_layers[l] = p.layer[l];
+  __syncthreads();
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) mbar_init(bar_base + 8 * i, 1);
     fence_barrier_init();
@@ -973,7 +979,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
       }
       if (s.layer >= 0 && s.layer % 2 == 1 && (gi - 2) % 4 == 0 && blockIdx.x < 2 && threadIdx.x == 0) {
         // this layer's projected prefix keys / values, read by the attention after this stage
-        const FdLayer& Ly = p.layer[s.layer];
+        const FdLayer& Ly = fd_layers[s.layer];
         prefetch_l2_bulk(blockIdx.x == 0 ? Ly.kx : Ly.vx, (uint32_t)p.B * p.L * p.nkv * HD * 2);
       }
       if (gi == gps - 1 && blockIdx.x == 0 && threadIdx.x == 0) {
@@ -1004,7 +1010,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
         if (l % 2 == 0) {
           at.k = p.k; at.v = p.v; at.key_valid = nullptr; at.Lk = p.H; at.causal = 1;
         } else {
-          at.k = p.layer[l].kx; at.v = p.layer[l].vx; at.key_valid = p.pad; at.Lk = p.L; at.causal = 0;
+          at.k = fd_layers[l].kx; at.v = fd_layers[l].vx; at.key_valid = p.pad; at.Lk = p.L; at.causal = 0;
         }
         const int rblk = (p.H + 15) / 16;
         const int n_att = p.B * p.nq * rblk;

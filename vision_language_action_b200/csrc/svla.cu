@@ -29,7 +29,7 @@ using namespace svla;
 namespace {
 
 std::atomic<unsigned long long> g_wait_ns{1000000000ull};
-constexpr int FD_SMEM_MAX = 232448 - 1024;  // dynamic shared memory of the persistent denoise kernel
+constexpr int FD_SMEM_MAX = 232448 - 4096;  // dynamic shared memory of the persistent denoise kernel (static: <= 4 KB)
 thread_local std::string t_last_error = "no error";
 
 const char* status_str(svla_status s) {
