@@ -49,7 +49,9 @@ namespace svla {
 
 constexpr int FD_THREADS = 256;
 constexpr int FD_MAX_M = 64;    // chunk rows handled (B * H)
-constexpr int FD_MAX_LAYERS = 32;
+constexpr int FD_MAX_LAYERS = 24;
+constexpr int FD_MAX_GPS = 2 + 4 * FD_MAX_LAYERS;  // GEMM stages per Euler step
+constexpr int FD_MAX_JPS = 2;                       // jobs of one CTA in one GEMM stage
 constexpr int FD_MAX_PLANES = 8;
 constexpr int FD_PIPE_TID = 128;  // the thread that refills the weight slots (warp 4, idle in epilogues)
 
@@ -128,6 +130,16 @@ struct FdGemm {
 // Shared-memory copy of FdArgs::layer (dynamic indexing into the kernel
 // parameters would go through the constant cache on every job).
 __shared__ FdLayer fd_layers[FD_MAX_LAYERS];
+
+// The GEMM stages of one Euler step (the same every step) and this CTA's
+// weight-copy schedule for a step are built once at kernel start: the refill of
+// a weight slot and the start of a job are then table lookups instead of a
+// chain of dependent integer arithmetic on one thread.
+struct FdSlice {
+  const bf16* src0;   // first run of rows
+  const bf16* src1;   // second run of rows
+  uint32_t run_bytes;
+};
 
 // GEMM stages per Euler step: time MLP (2), then QKV, O, gate/up, down per layer
 SVLA_DEV int fd_gemms_per_step(const FdArgs& p) { return 2 + 4 * p.n_layers; }
@@ -218,9 +230,11 @@ SVLA_DEV void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
 // abandoned (abort word raised, or this wait ran out of time). Every thread
 // first orders its global stores before the bulk copies that other CTAs issue
 // after the barrier.
-SVLA_DEV bool fd_grid_sync(const FdArgs& p, unsigned idx, int* flag) {
+template <typename Hook>
+SVLA_DEV bool fd_grid_sync(const FdArgs& p, unsigned idx, int* flag, Hook&& while_waiting) {
   fence_proxy_async_global();
   __syncthreads();
+  while_waiting();  // work of threads other than 0 that overlaps the barrier
   if (threadIdx.x == 0) {
     int ok = 1;
     // release: this CTA's writes (ordered before this thread by the barrier above)
@@ -253,40 +267,34 @@ SVLA_DEV bool fd_grid_sync(const FdArgs& p, unsigned idx, int* flag) {
 // shared-memory state of the bulk-copy pipelines (thread 0 drives them)
 // ---------------------------------------------------------------------------
 struct FdPipe {
-  int next_g, next_j;      // next (GEMM stage, job) of this CTA whose weights are not yet issued
+  int jobs_per_step, total_jobs;  // this CTA's GEMM jobs per Euler step / in the launch
   int issued, consumed;    // weight slices issued / consumed so far (slot = count % 2)
-  int total_g;
+  int pending;             // consumed slices whose slot refill is deferred to the next barrier
   int a_iss[2], a_use[2];  // activation-buffer copies issued / waited for (mbarrier parity)
 };
 
-// advance (g, j) to this CTA's next job at or after it
-SVLA_DEV void fd_next_job(const FdArgs& p, int& g, int& j, int total_g) {
-  while (g < total_g) {
-    const FdGemm s = fd_gemm(p, g);
-    if (j < s.n_jobs) return;
-    ++g;
-    j = blockIdx.x;
-  }
-}
-
 // issue the weight slice of this CTA's next job into slot (issued % 2): two
-// bulk copies, one per run of rows; thread 0 only
-SVLA_DEV void fd_issue(const FdArgs& p, FdPipe& pp, uint8_t* slots, uint32_t bar_base) {
-  if (pp.next_g >= pp.total_g || pp.issued - pp.consumed >= 2) return;
-  const FdGemm s = fd_gemm(p, pp.next_g);
-  int r0, r1;
-  fd_job_rows(p, s, pp.next_j, r0, r1);
+// bulk copies, one per run of rows; one thread only
+SVLA_DEV void fd_issue(FdPipe& pp, const FdSlice* sched, uint8_t* slots, int slot_bytes, uint32_t bar_base) {
+  if (pp.issued >= pp.total_jobs || pp.issued - pp.consumed >= 2) return;
+  const FdSlice e = sched[pp.issued % pp.jobs_per_step];
   const int slot = pp.issued & 1;
   const uint32_t bar = bar_base + 8 * slot;
-  const uint32_t pitch = (uint32_t)(s.K + 8), run_bytes = (uint32_t)(s.w / 2) * pitch * 2;
-  const uint32_t dst = smem_u32(slots + (size_t)slot * p.slot_bytes);
-  fence_proxy_async_smem();  // generic-proxy reads of this slot are ordered before the async writes
-  mbar_arrive_expect_tx(bar, 2 * run_bytes);
-  bulk_load(dst, s.W + (size_t)r0 * pitch, run_bytes, bar);
-  bulk_load(dst + run_bytes, s.W + (size_t)r1 * pitch, run_bytes, bar);
+  const uint32_t dst = smem_u32(slots + (size_t)slot * slot_bytes);
+  // (the threads that read the slot ordered their reads with fence.proxy.async
+  // before the barrier that precedes this call)
+  mbar_arrive_expect_tx(bar, 2 * e.run_bytes);
+  bulk_load(dst, e.src0, e.run_bytes, bar);
+  bulk_load(dst + e.run_bytes, e.src1, e.run_bytes, bar);
   ++pp.issued;
-  pp.next_j += gridDim.x;
-  fd_next_job(p, pp.next_g, pp.next_j, pp.total_g);
+}
+
+// the deferred slot refill, run by FD_PIPE_TID while the CTA waits at a barrier
+SVLA_DEV void fd_refill(const FdArgs& p, FdPipe& pp, const FdSlice* sched, uint8_t* slots, uint32_t bar_base) {
+  if (threadIdx.x == FD_PIPE_TID && pp.pending) {
+    pp.pending = 0;
+    fd_issue(pp, sched, slots, p.slot_bytes, bar_base);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -351,7 +359,8 @@ SVLA_DEV void fd_mma_plane(const bf16* ab, int apitch, const uint8_t* wsl, int w
 // two buffers); all FD_THREADS threads take part.
 // ---------------------------------------------------------------------------
 template <int HD>
-SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, uint8_t* slots, uint32_t bar_base,
+SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, const FdSlice* sched, uint8_t* slots,
+                          uint32_t bar_base,
                           bf16* abuf, float* red, float* rscale, int* flag) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int M = p.M, K = s.K, P = s.A.P, Kp = K / P, apitch = Kp + 8;
@@ -372,6 +381,10 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, u
     fence_proxy_async_global();  // the activations were written by generic stores of other CTAs
     issue_plane(0);
     if (P > 1) issue_plane(1);
+    if (pp.issued <= pp.consumed && pp.pending) {  // a second job of one stage: no barrier in between
+      pp.pending = 0;
+      fd_issue(pp, sched, slots, p.slot_bytes, bar_base);
+    }
   }
 
   // epilogue inputs that do not depend on the products, fetched now so their
@@ -462,10 +475,10 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, u
   }
   __syncthreads();
   if (tid == FD_PIPE_TID) {
-    // the weight slot is free: a thread of warp 4 (idle in the epilogue)
-    // hands it the job after next
+    // the weight slot is free: its refill with the job after next is issued
+    // while this CTA waits at the next grid barrier (fd_refill)
     ++pp.consumed;
-    fd_issue(p, pp, slots, bar_base);
+    ++pp.pending;
   }
   if (kp != 0 || !mma_warp) return true;
 #pragma unroll
@@ -941,34 +954,50 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
   uint64_t* bars = reinterpret_cast<uint64_t*>(fbuf + p.E + 128);   // weight slots 0, 1; activation buffers 0, 1
   __shared__ int flag;
   __shared__ FdPipe pp;
+  __shared__ FdGemm stages[FD_MAX_GPS];
+  __shared__ FdSlice sched[FD_MAX_GPS * FD_MAX_JPS];
 
   const uint32_t bar_base = smem_u32(bars);
   for (int l = threadIdx.x; l < p.n_layers; l += FD_THREADS) fd_layers[l] = p.layer[l];
   __syncthreads();
+  const int gps = fd_gemms_per_step(p);
+  for (int g = threadIdx.x; g < gps; g += FD_THREADS) stages[g] = fd_gemm(p, g);
+  __syncthreads();
   if (threadIdx.x == 0) {
+    // this CTA's jobs of one step in order, with the rows each reads
+    int n = 0;
+    for (int g = 0; g < gps; ++g) {
+      const FdGemm& st = stages[g];
+      for (int j = blockIdx.x; j < st.n_jobs; j += gridDim.x) {
+        int r0, r1;
+        fd_job_rows(p, st, j, r0, r1);
+        const uint32_t pitch = (uint32_t)(st.K + 8);
+        sched[n].src0 = st.W + (size_t)r0 * pitch;
+        sched[n].src1 = st.W + (size_t)r1 * pitch;
+        sched[n].run_bytes = (uint32_t)(st.w / 2) * pitch * 2;
+        ++n;
+      }
+    }
     for (int i = 0; i < 4; ++i) mbar_init(bar_base + 8 * i, 1);
     fence_barrier_init();
     pp.a_iss[0] = pp.a_iss[1] = pp.a_use[0] = pp.a_use[1] = 0;
-    pp.total_g = p.n_steps * fd_gemms_per_step(p);
-    pp.next_g = 0;
-    pp.next_j = blockIdx.x;
-    pp.issued = pp.consumed = 0;
-    fd_next_job(p, pp.next_g, pp.next_j, pp.total_g);
-    fd_issue(p, pp, slots, bar_base);
-    fd_issue(p, pp, slots, bar_base);
+    pp.jobs_per_step = n;
+    pp.total_jobs = n * p.n_steps;
+    pp.issued = pp.consumed = pp.pending = 0;
+    fd_issue(pp, sched, slots, p.slot_bytes, bar_base);
+    fd_issue(pp, sched, slots, p.slot_bytes, bar_base);
   }
   __syncthreads();
 
   unsigned nbar = 0;
   bool alive = true;
+  auto refill = [&]() { fd_refill(p, pp, sched, slots, bar_base); };
   alive = fd_row_stage(p, -1, 0, fbuf, ubuf, pp, bar_base, &flag);
   fd_time_c(p, 0, blockIdx.x, gridDim.x, fbuf);
-  if (alive) alive = fd_grid_sync(p, nbar++, &flag);
-  const int gps = fd_gemms_per_step(p);
+  if (alive) alive = fd_grid_sync(p, nbar++, &flag, refill);
   for (int k = 0; k < p.n_steps && alive; ++k) {
     for (int gi = 0; gi < gps && alive; ++gi) {
-      const int g = k * gps + gi;
-      const FdGemm s = fd_gemm(p, g);
+      const FdGemm& s = stages[gi];
       if (gi == 0 && k + 1 < p.n_steps) {
         // rows of W_t1 for the next step's time vector (computed during layer 0's attention)
         const int n_att = p.B * p.nq * ((p.H + 15) / 16), G = (int)gridDim.x;
@@ -988,9 +1017,9 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
         prefetch_l2_bulk(p.w_in, (uint32_t)p.A * p.E * 2);
       }
       for (int j = blockIdx.x; j < s.n_jobs && alive; j += gridDim.x)
-        alive = fd_gemm_job<HD>(p, s, j, pp, slots, bar_base, reinterpret_cast<bf16*>(ubuf), red, rscale, &flag);
+        alive = fd_gemm_job<HD>(p, s, j, pp, sched, slots, bar_base, reinterpret_cast<bf16*>(ubuf), red, rscale, &flag);
       if (!alive) break;
-      alive = fd_grid_sync(p, nbar++, &flag);
+      alive = fd_grid_sync(p, nbar++, &flag, refill);
       if (!alive) break;
       if (s.layer >= 0 && (gi - 2) % 4 == 0) {
         // attention of this layer (after its QKV stage)
@@ -1027,12 +1056,12 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
           else
             fd_time_c(p, k + 1, (int)blockIdx.x, G, fbuf);
         }
-        alive = fd_grid_sync(p, nbar++, &flag);
+        alive = fd_grid_sync(p, nbar++, &flag, refill);
       }
     }
     if (!alive) break;
     alive = fd_row_stage(p, k, k + 1, fbuf, ubuf, pp, bar_base, &flag);
-    if (alive && k + 1 < p.n_steps) alive = fd_grid_sync(p, nbar++, &flag);
+    if (alive && k + 1 < p.n_steps) alive = fd_grid_sync(p, nbar++, &flag, refill);
   }
   // drain: wait (bounded) for this CTA's bulk copies still in flight
   if (threadIdx.x == 0) {

@@ -29,7 +29,7 @@ using namespace svla;
 namespace {
 
 std::atomic<unsigned long long> g_wait_ns{1000000000ull};
-constexpr int FD_SMEM_MAX = 232448 - 4096;  // dynamic shared memory of the persistent denoise kernel (static: <= 4 KB)
+constexpr int FD_SMEM_MAX = 232448 - 16384;  // dynamic shared memory of the persistent denoise kernel (static: < 16 KB)
 thread_local std::string t_last_error = "no error";
 
 const char* status_str(svla_status s) {
@@ -497,6 +497,11 @@ bool fused_ok(const svla_handle* h, int B, int H, int L) {
   if (B < 1 || H < 1 || B > c.max_batch || H > c.max_chunk) return false;
   if ((long long)B * H > FD_MAX_M || H > ATT_BQ || H > ATT_BK) return false;
   if (c.e_layers > FD_MAX_LAYERS || c.e_ffn % 32 || c.e_width % 16) return false;
+  {  // at most FD_MAX_JPS jobs of one GEMM stage per CTA
+    const int jobs = std::max({c.e_width / 8, (c.e_heads + 2 * c.e_kv_heads) * c.head_dim / 16,
+                               c.e_heads * c.head_dim / 8, c.e_ffn / 16});
+    if (jobs > FD_MAX_JPS * h->num_sms) return false;
+  }
   if (h->num_sms < 1 || !h->fw) return false;
   return fused_plan(c, B * H, L, nullptr);
 }
