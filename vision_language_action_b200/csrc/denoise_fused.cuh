@@ -53,6 +53,7 @@ constexpr int FD_MAX_LAYERS = 24;
 constexpr int FD_MAX_GPS = 2 + 4 * FD_MAX_LAYERS;  // GEMM stages per Euler step
 constexpr int FD_MAX_JPS = 2;                       // jobs of one CTA in one GEMM stage
 constexpr int FD_MAX_PLANES = 8;
+constexpr int FD_MAX_ABUF = 4;  // activation plane buffers
 constexpr int FD_PIPE_TID = 128;  // the thread that refills the weight slots (warp 4, idle in epilogues)
 
 enum FdEpi : int { FD_SILU_BIAS = 0, FD_RES_INIT, FD_QKV_ROPE, FD_Q, FD_RES_ADD, FD_SWIGLU };
@@ -65,6 +66,7 @@ enum FdEpi : int { FD_SILU_BIAS = 0, FD_RES_INIT, FD_QKV_ROPE, FD_Q, FD_RES_ADD,
 struct FdAct {
   bf16* ptr;
   int K, P;
+  int NB;  // shared-memory buffers its planes cycle through (planes in flight)
 };
 
 SVLA_DEV size_t fd_act_off(const FdAct& a, int M, int m, int c) {
@@ -270,7 +272,7 @@ struct FdPipe {
   int jobs_per_step, total_jobs;  // this CTA's GEMM jobs per Euler step / in the launch
   int issued, consumed;    // weight slices issued / consumed so far (slot = count % 2)
   int pending;             // consumed slices whose slot refill is deferred to the next barrier
-  int a_iss[2], a_use[2];  // activation-buffer copies issued / waited for (mbarrier parity)
+  int a_iss[FD_MAX_ABUF], a_use[FD_MAX_ABUF];  // activation-buffer copies issued / waited for
 };
 
 // issue the weight slice of this CTA's next job into slot (issued % 2): two
@@ -365,13 +367,14 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, c
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int M = p.M, K = s.K, P = s.A.P, Kp = K / P, apitch = Kp + 8;
   const uint32_t plane_bytes = (uint32_t)M * apitch * 2;
-  const uint32_t abar = bar_base + 16;  // activation buffers' mbarriers: abar, abar + 8
+  const uint32_t abar = bar_base + 16;  // activation buffers' mbarriers: abar + 8 b
+  const int NB = s.A.NB;
   const int slot = pp.consumed & 1;
   const uint8_t* wsl = slots + (size_t)slot * p.slot_bytes;
   const int wld = K + 8;  // staged W row (elements)
 
   auto issue_plane = [&](int q) {  // thread 0
-    const int buf = q & 1;
+    const int buf = q % NB;
     const uint32_t bar = abar + 8 * buf;
     mbar_arrive_expect_tx(bar, plane_bytes);
     bulk_load(smem_u32(abuf + (size_t)buf * M * apitch), s.A.ptr + (size_t)q * M * apitch, plane_bytes, bar);
@@ -379,8 +382,7 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, c
   };
   if (tid == 0) {
     fence_proxy_async_global();  // the activations were written by generic stores of other CTAs
-    issue_plane(0);
-    if (P > 1) issue_plane(1);
+    for (int q = 0; q < NB && q < P; ++q) issue_plane(q);
     if (pp.issued <= pp.consumed && pp.pending) {  // a second job of one stage: no barrier in between
       pp.pending = 0;
       fd_issue(pp, sched, slots, p.slot_bytes, bar_base);
@@ -421,7 +423,7 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, c
   float ss[2] = {0.f, 0.f};  // norm: squares of this thread's A elements, rows g and g + 8
 
   for (int q = 0; q < P; ++q) {
-    const int buf = q & 1;
+    const int buf = q % NB;
     if (tid == 0) {
       bool ok = true;
       if (q == 0) ok = mbar_wait(bar_base + 8 * slot, (uint32_t)((pp.consumed >> 1) & 1), p.wait_ns);
@@ -448,7 +450,7 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, c
     // re-filled by the async proxy: order this thread's generic reads first
     fence_proxy_async_smem();
     __syncthreads();
-    if (tid == 0 && q + 2 < P) issue_plane(q + 2);
+    if (tid == 0 && q + NB < P) issue_plane(q + NB);
   }
 
   float acc[4][4];
@@ -951,7 +953,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
   float* red = reinterpret_cast<float*>(ubuf + p.a_bytes);          // [4 m-tiles][4 n-tiles][4][32]
   float* rscale = red + 4 * 4 * 4 * 32;                             // [64]
   float* fbuf = rscale + FD_MAX_M;                                  // [E + 64 + 8] row stage
-  uint64_t* bars = reinterpret_cast<uint64_t*>(fbuf + p.E + 128);   // weight slots 0, 1; activation buffers 0, 1
+  uint64_t* bars = reinterpret_cast<uint64_t*>(fbuf + p.E + 128);   // weight slots 0, 1; activation buffers 0..3
   __shared__ int flag;
   __shared__ FdPipe pp;
   __shared__ FdGemm stages[FD_MAX_GPS];
@@ -978,9 +980,9 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
         ++n;
       }
     }
-    for (int i = 0; i < 4; ++i) mbar_init(bar_base + 8 * i, 1);
+    for (int i = 0; i < 2 + FD_MAX_ABUF; ++i) mbar_init(bar_base + 8 * i, 1);
     fence_barrier_init();
-    pp.a_iss[0] = pp.a_iss[1] = pp.a_use[0] = pp.a_use[1] = 0;
+    for (int b = 0; b < FD_MAX_ABUF; ++b) pp.a_iss[b] = pp.a_use[b] = 0;
     pp.jobs_per_step = n;
     pp.total_jobs = n * p.n_steps;
     pp.issued = pp.consumed = pp.pending = 0;
@@ -1067,7 +1069,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
   if (threadIdx.x == 0) {
     for (int c = pp.consumed; c < pp.issued; ++c)
       (void)mbar_wait(bar_base + 8 * (c & 1), (uint32_t)((c >> 1) & 1), 1000000ull);
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < FD_MAX_ABUF; ++b)
       for (int u = pp.a_use[b]; u < pp.a_iss[b]; ++u)
         (void)mbar_wait(bar_base + 16 + 8 * b, (uint32_t)(u & 1), 1000000ull);
   }
