@@ -49,11 +49,8 @@ namespace svla {
 
 constexpr int FD_THREADS = 256;
 constexpr int FD_MAX_M = 64;    // chunk rows handled (B * H)
-constexpr int FD_MAX_LAYERS = 24;
-constexpr int FD_MAX_GPS = 2 + 4 * FD_MAX_LAYERS;  // GEMM stages per Euler step
-constexpr int FD_MAX_JPS = 2;                       // jobs of one CTA in one GEMM stage
+constexpr int FD_MAX_LAYERS = 32;
 constexpr int FD_MAX_PLANES = 8;
-constexpr int FD_MAX_ABUF = 4;  // activation plane buffers
 constexpr int FD_PIPE_TID = 128;  // the thread that refills the weight slots (warp 4, idle in epilogues)
 
 enum FdEpi : int { FD_SILU_BIAS = 0, FD_RES_INIT, FD_QKV_ROPE, FD_Q, FD_RES_ADD, FD_SWIGLU };
@@ -66,7 +63,6 @@ enum FdEpi : int { FD_SILU_BIAS = 0, FD_RES_INIT, FD_QKV_ROPE, FD_Q, FD_RES_ADD,
 struct FdAct {
   bf16* ptr;
   int K, P;
-  int NB;  // shared-memory buffers its planes cycle through (planes in flight)
 };
 
 SVLA_DEV size_t fd_act_off(const FdAct& a, int M, int m, int c) {
@@ -132,16 +128,6 @@ struct FdGemm {
 // Shared-memory copy of FdArgs::layer (dynamic indexing into the kernel
 // parameters would go through the constant cache on every job).
 __shared__ FdLayer fd_layers[FD_MAX_LAYERS];
-
-// The GEMM stages of one Euler step (the same every step) and this CTA's
-// weight-copy schedule for a step are built once at kernel start: the refill of
-// a weight slot and the start of a job are then table lookups instead of a
-// chain of dependent integer arithmetic on one thread.
-struct FdSlice {
-  const bf16* src0;   // first run of rows
-  const bf16* src1;   // second run of rows
-  uint32_t run_bytes;
-};
 
 // GEMM stages per Euler step: time MLP (2), then QKV, O, gate/up, down per layer
 SVLA_DEV int fd_gemms_per_step(const FdArgs& p) { return 2 + 4 * p.n_layers; }
@@ -232,11 +218,9 @@ SVLA_DEV void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
 // abandoned (abort word raised, or this wait ran out of time). Every thread
 // first orders its global stores before the bulk copies that other CTAs issue
 // after the barrier.
-template <typename Hook>
-SVLA_DEV bool fd_grid_sync(const FdArgs& p, unsigned idx, int* flag, Hook&& while_waiting) {
+SVLA_DEV bool fd_grid_sync(const FdArgs& p, unsigned idx, int* flag) {
   fence_proxy_async_global();
   __syncthreads();
-  while_waiting();  // work of threads other than 0 that overlaps the barrier
   if (threadIdx.x == 0) {
     int ok = 1;
     // release: this CTA's writes (ordered before this thread by the barrier above)
@@ -269,34 +253,40 @@ SVLA_DEV bool fd_grid_sync(const FdArgs& p, unsigned idx, int* flag, Hook&& whil
 // shared-memory state of the bulk-copy pipelines (thread 0 drives them)
 // ---------------------------------------------------------------------------
 struct FdPipe {
-  int jobs_per_step, total_jobs;  // this CTA's GEMM jobs per Euler step / in the launch
+  int next_g, next_j;      // next (GEMM stage, job) of this CTA whose weights are not yet issued
   int issued, consumed;    // weight slices issued / consumed so far (slot = count % 2)
-  int pending;             // consumed slices whose slot refill is deferred to the next barrier
-  int a_iss[FD_MAX_ABUF], a_use[FD_MAX_ABUF];  // activation-buffer copies issued / waited for
+  int total_g;
+  int a_iss[2], a_use[2];  // activation-buffer copies issued / waited for (mbarrier parity)
 };
 
-// issue the weight slice of this CTA's next job into slot (issued % 2): two
-// bulk copies, one per run of rows; one thread only
-SVLA_DEV void fd_issue(FdPipe& pp, const FdSlice* sched, uint8_t* slots, int slot_bytes, uint32_t bar_base) {
-  if (pp.issued >= pp.total_jobs || pp.issued - pp.consumed >= 2) return;
-  const FdSlice e = sched[pp.issued % pp.jobs_per_step];
-  const int slot = pp.issued & 1;
-  const uint32_t bar = bar_base + 8 * slot;
-  const uint32_t dst = smem_u32(slots + (size_t)slot * slot_bytes);
-  // (the threads that read the slot ordered their reads with fence.proxy.async
-  // before the barrier that precedes this call)
-  mbar_arrive_expect_tx(bar, 2 * e.run_bytes);
-  bulk_load(dst, e.src0, e.run_bytes, bar);
-  bulk_load(dst + e.run_bytes, e.src1, e.run_bytes, bar);
-  ++pp.issued;
+// advance (g, j) to this CTA's next job at or after it
+SVLA_DEV void fd_next_job(const FdArgs& p, int& g, int& j, int total_g) {
+  while (g < total_g) {
+    const FdGemm s = fd_gemm(p, g);
+    if (j < s.n_jobs) return;
+    ++g;
+    j = blockIdx.x;
+  }
 }
 
-// the deferred slot refill, run by FD_PIPE_TID while the CTA waits at a barrier
-SVLA_DEV void fd_refill(const FdArgs& p, FdPipe& pp, const FdSlice* sched, uint8_t* slots, uint32_t bar_base) {
-  if (threadIdx.x == FD_PIPE_TID && pp.pending) {
-    pp.pending = 0;
-    fd_issue(pp, sched, slots, p.slot_bytes, bar_base);
-  }
+// issue the weight slice of this CTA's next job into slot (issued % 2): two
+// bulk copies, one per run of rows; thread 0 only
+SVLA_DEV void fd_issue(const FdArgs& p, FdPipe& pp, uint8_t* slots, uint32_t bar_base) {
+  if (pp.next_g >= pp.total_g || pp.issued - pp.consumed >= 2) return;
+  const FdGemm s = fd_gemm(p, pp.next_g);
+  int r0, r1;
+  fd_job_rows(p, s, pp.next_j, r0, r1);
+  const int slot = pp.issued & 1;
+  const uint32_t bar = bar_base + 8 * slot;
+  const uint32_t pitch = (uint32_t)(s.K + 8), run_bytes = (uint32_t)(s.w / 2) * pitch * 2;
+  const uint32_t dst = smem_u32(slots + (size_t)slot * p.slot_bytes);
+  fence_proxy_async_smem();  // generic-proxy reads of this slot are ordered before the async writes
+  mbar_arrive_expect_tx(bar, 2 * run_bytes);
+  bulk_load(dst, s.W + (size_t)r0 * pitch, run_bytes, bar);
+  bulk_load(dst + run_bytes, s.W + (size_t)r1 * pitch, run_bytes, bar);
+  ++pp.issued;
+  pp.next_j += gridDim.x;
+  fd_next_job(p, pp.next_g, pp.next_j, pp.total_g);
 }
 
 // ---------------------------------------------------------------------------
@@ -361,20 +351,18 @@ SVLA_DEV void fd_mma_plane(const bf16* ab, int apitch, const uint8_t* wsl, int w
 // two buffers); all FD_THREADS threads take part.
 // ---------------------------------------------------------------------------
 template <int HD>
-SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, const FdSlice* sched, uint8_t* slots,
-                          uint32_t bar_base,
+SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, uint8_t* slots, uint32_t bar_base,
                           bf16* abuf, float* red, float* rscale, int* flag) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int M = p.M, K = s.K, P = s.A.P, Kp = K / P, apitch = Kp + 8;
   const uint32_t plane_bytes = (uint32_t)M * apitch * 2;
-  const uint32_t abar = bar_base + 16;  // activation buffers' mbarriers: abar + 8 b
-  const int NB = s.A.NB;
+  const uint32_t abar = bar_base + 16;  // activation buffers' mbarriers: abar, abar + 8
   const int slot = pp.consumed & 1;
   const uint8_t* wsl = slots + (size_t)slot * p.slot_bytes;
   const int wld = K + 8;  // staged W row (elements)
 
   auto issue_plane = [&](int q) {  // thread 0
-    const int buf = q % NB;
+    const int buf = q & 1;
     const uint32_t bar = abar + 8 * buf;
     mbar_arrive_expect_tx(bar, plane_bytes);
     bulk_load(smem_u32(abuf + (size_t)buf * M * apitch), s.A.ptr + (size_t)q * M * apitch, plane_bytes, bar);
@@ -382,11 +370,8 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, c
   };
   if (tid == 0) {
     fence_proxy_async_global();  // the activations were written by generic stores of other CTAs
-    for (int q = 0; q < NB && q < P; ++q) issue_plane(q);
-    if (pp.issued <= pp.consumed && pp.pending) {  // a second job of one stage: no barrier in between
-      pp.pending = 0;
-      fd_issue(pp, sched, slots, p.slot_bytes, bar_base);
-    }
+    issue_plane(0);
+    if (P > 1) issue_plane(1);
   }
 
   // epilogue inputs that do not depend on the products, fetched now so their
@@ -423,7 +408,7 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, c
   float ss[2] = {0.f, 0.f};  // norm: squares of this thread's A elements, rows g and g + 8
 
   for (int q = 0; q < P; ++q) {
-    const int buf = q % NB;
+    const int buf = q & 1;
     if (tid == 0) {
       bool ok = true;
       if (q == 0) ok = mbar_wait(bar_base + 8 * slot, (uint32_t)((pp.consumed >> 1) & 1), p.wait_ns);
@@ -450,7 +435,7 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, c
     // re-filled by the async proxy: order this thread's generic reads first
     fence_proxy_async_smem();
     __syncthreads();
-    if (tid == 0 && q + NB < P) issue_plane(q + NB);
+    if (tid == 0 && q + 2 < P) issue_plane(q + 2);
   }
 
   float acc[4][4];
@@ -477,10 +462,10 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, c
   }
   __syncthreads();
   if (tid == FD_PIPE_TID) {
-    // the weight slot is free: its refill with the job after next is issued
-    // while this CTA waits at the next grid barrier (fd_refill)
+    // the weight slot is free: a thread of warp 4 (idle in the epilogue)
+    // hands it the job after next
     ++pp.consumed;
-    ++pp.pending;
+    fd_issue(p, pp, slots, bar_base);
   }
   if (kp != 0 || !mma_warp) return true;
 #pragma unroll
@@ -953,53 +938,37 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
   float* red = reinterpret_cast<float*>(ubuf + p.a_bytes);          // [4 m-tiles][4 n-tiles][4][32]
   float* rscale = red + 4 * 4 * 4 * 32;                             // [64]
   float* fbuf = rscale + FD_MAX_M;                                  // [E + 64 + 8] row stage
-  uint64_t* bars = reinterpret_cast<uint64_t*>(fbuf + p.E + 128);   // weight slots 0, 1; activation buffers 0..3
+  uint64_t* bars = reinterpret_cast<uint64_t*>(fbuf + p.E + 128);   // weight slots 0, 1; activation buffers 0, 1
   __shared__ int flag;
   __shared__ FdPipe pp;
-  __shared__ FdGemm stages[FD_MAX_GPS];
-  __shared__ FdSlice sched[FD_MAX_GPS * FD_MAX_JPS];
 
   const uint32_t bar_base = smem_u32(bars);
   for (int l = threadIdx.x; l < p.n_layers; l += FD_THREADS) fd_layers[l] = p.layer[l];
   __syncthreads();
-  const int gps = fd_gemms_per_step(p);
-  for (int g = threadIdx.x; g < gps; g += FD_THREADS) stages[g] = fd_gemm(p, g);
-  __syncthreads();
   if (threadIdx.x == 0) {
-    // this CTA's jobs of one step in order, with the rows each reads
-    int n = 0;
-    for (int g = 0; g < gps; ++g) {
-      const FdGemm& st = stages[g];
-      for (int j = blockIdx.x; j < st.n_jobs; j += gridDim.x) {
-        int r0, r1;
-        fd_job_rows(p, st, j, r0, r1);
-        const uint32_t pitch = (uint32_t)(st.K + 8);
-        sched[n].src0 = st.W + (size_t)r0 * pitch;
-        sched[n].src1 = st.W + (size_t)r1 * pitch;
-        sched[n].run_bytes = (uint32_t)(st.w / 2) * pitch * 2;
-        ++n;
-      }
-    }
-    for (int i = 0; i < 2 + FD_MAX_ABUF; ++i) mbar_init(bar_base + 8 * i, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(bar_base + 8 * i, 1);
     fence_barrier_init();
-    for (int b = 0; b < FD_MAX_ABUF; ++b) pp.a_iss[b] = pp.a_use[b] = 0;
-    pp.jobs_per_step = n;
-    pp.total_jobs = n * p.n_steps;
-    pp.issued = pp.consumed = pp.pending = 0;
-    fd_issue(pp, sched, slots, p.slot_bytes, bar_base);
-    fd_issue(pp, sched, slots, p.slot_bytes, bar_base);
+    pp.a_iss[0] = pp.a_iss[1] = pp.a_use[0] = pp.a_use[1] = 0;
+    pp.total_g = p.n_steps * fd_gemms_per_step(p);
+    pp.next_g = 0;
+    pp.next_j = blockIdx.x;
+    pp.issued = pp.consumed = 0;
+    fd_next_job(p, pp.next_g, pp.next_j, pp.total_g);
+    fd_issue(p, pp, slots, bar_base);
+    fd_issue(p, pp, slots, bar_base);
   }
   __syncthreads();
 
   unsigned nbar = 0;
   bool alive = true;
-  auto refill = [&]() { fd_refill(p, pp, sched, slots, bar_base); };
   alive = fd_row_stage(p, -1, 0, fbuf, ubuf, pp, bar_base, &flag);
   fd_time_c(p, 0, blockIdx.x, gridDim.x, fbuf);
-  if (alive) alive = fd_grid_sync(p, nbar++, &flag, refill);
+  if (alive) alive = fd_grid_sync(p, nbar++, &flag);
+  const int gps = fd_gemms_per_step(p);
   for (int k = 0; k < p.n_steps && alive; ++k) {
     for (int gi = 0; gi < gps && alive; ++gi) {
-      const FdGemm& s = stages[gi];
+      const int g = k * gps + gi;
+      const FdGemm s = fd_gemm(p, g);
       if (gi == 0 && k + 1 < p.n_steps) {
         // rows of W_t1 for the next step's time vector (computed during layer 0's attention)
         const int n_att = p.B * p.nq * ((p.H + 15) / 16), G = (int)gridDim.x;
@@ -1019,9 +988,9 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
         prefetch_l2_bulk(p.w_in, (uint32_t)p.A * p.E * 2);
       }
       for (int j = blockIdx.x; j < s.n_jobs && alive; j += gridDim.x)
-        alive = fd_gemm_job<HD>(p, s, j, pp, sched, slots, bar_base, reinterpret_cast<bf16*>(ubuf), red, rscale, &flag);
+        alive = fd_gemm_job<HD>(p, s, j, pp, slots, bar_base, reinterpret_cast<bf16*>(ubuf), red, rscale, &flag);
       if (!alive) break;
-      alive = fd_grid_sync(p, nbar++, &flag, refill);
+      alive = fd_grid_sync(p, nbar++, &flag);
       if (!alive) break;
       if (s.layer >= 0 && (gi - 2) % 4 == 0) {
         // attention of this layer (after its QKV stage)
@@ -1058,18 +1027,18 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
           else
             fd_time_c(p, k + 1, (int)blockIdx.x, G, fbuf);
         }
-        alive = fd_grid_sync(p, nbar++, &flag, refill);
+        alive = fd_grid_sync(p, nbar++, &flag);
       }
     }
     if (!alive) break;
     alive = fd_row_stage(p, k, k + 1, fbuf, ubuf, pp, bar_base, &flag);
-    if (alive && k + 1 < p.n_steps) alive = fd_grid_sync(p, nbar++, &flag, refill);
+    if (alive && k + 1 < p.n_steps) alive = fd_grid_sync(p, nbar++, &flag);
   }
   // drain: wait (bounded) for this CTA's bulk copies still in flight
   if (threadIdx.x == 0) {
     for (int c = pp.consumed; c < pp.issued; ++c)
       (void)mbar_wait(bar_base + 8 * (c & 1), (uint32_t)((c >> 1) & 1), 1000000ull);
-    for (int b = 0; b < FD_MAX_ABUF; ++b)
+    for (int b = 0; b < 2; ++b)
       for (int u = pp.a_use[b]; u < pp.a_iss[b]; ++u)
         (void)mbar_wait(bar_base + 16 + 8 * b, (uint32_t)(u & 1), 1000000ull);
   }

@@ -29,7 +29,7 @@ using namespace svla;
 namespace {
 
 std::atomic<unsigned long long> g_wait_ns{1000000000ull};
-constexpr int FD_SMEM_MAX = 232448 - 16384;  // dynamic shared memory of the persistent denoise kernel (static: < 16 KB)
+constexpr int FD_SMEM_MAX = 232448 - 4096;  // dynamic shared memory of the persistent denoise kernel (static: <= 4 KB)
 thread_local std::string t_last_error = "no error";
 
 const char* status_str(svla_status s) {
@@ -448,14 +448,12 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
 // and four mbarriers.
 struct FusedPlan {
   int slot_bytes = 0, a_bytes = 0;
-  int p_e = 1, p_o = 1, p_h = 1;     // column planes of the E-, q- and ffn-wide operands
-  int nb_e = 1, nb_o = 1, nb_h = 1;  // plane buffers (planes in flight) of each
+  int p_e = 1, p_o = 1, p_h = 1;  // column planes of the E-, q- and ffn-wide operands
   size_t smem = 0;
 };
 
 size_t fused_misc_bytes(const svla_config& c) {
-  return 4 * 4 * 4 * 32 * sizeof(float) + FD_MAX_M * sizeof(float) + ((size_t)c.e_width + 128) * sizeof(float) +
-         8 * (2 + FD_MAX_ABUF);
+  return 4 * 4 * 4 * 32 * sizeof(float) + FD_MAX_M * sizeof(float) + ((size_t)c.e_width + 128) * sizeof(float) + 32;
 }
 
 bool fused_plan(const svla_config& c, int M, int L, FusedPlan* fp) {
@@ -471,35 +469,21 @@ bool fused_plan(const svla_config& c, int M, int L, FusedPlan* fp) {
                               c.head_dim == 64 ? fd_att_smem<64>(c.max_chunk) : fd_att_smem<32>(c.max_chunk));
   size_t need = std::max(att, fd_row_stage_bytes(E, c.action_dim) + 3 * 64 * sizeof(float));
   if (need > budget) return false;
-  // one plane when the operand fits whole; otherwise the fewest planes that
-  // can be double-buffered (every plane costs a synchronisation round: more,
-  // smaller planes measured slower), with as many buffers as fit (up to four)
-  auto planes = [&](int K, int* P, int* NB) {
-    if ((size_t)M * (K + 8) * 2 <= budget) {
-      *P = 1;
-      *NB = 1;
-      need = std::max(need, (size_t)M * (K + 8) * 2);
-      return true;
-    }
-    int best_q = 0, best_nb = 0;
-    for (int q = 2; q <= FD_MAX_PLANES; q *= 2) {
-      if (K % (16 * q)) break;
+  auto planes = [&](int K, int* P) {
+    for (int q = 1; q <= FD_MAX_PLANES; q *= 2) {
+      if (K % (16 * q)) return false;
       const size_t plane = (size_t)M * (K / q + 8) * 2;
-      const int nb = (int)std::min<size_t>({budget / plane, (size_t)FD_MAX_ABUF, (size_t)q});
-      if (nb >= 2) {
-        best_q = q;
-        best_nb = nb;
-        break;
+      const size_t region = q == 1 ? plane : 2 * plane;
+      if (region <= budget) {
+        *P = q;
+        need = std::max(need, region);
+        return true;
       }
     }
-    if (!best_q) return false;
-    *P = best_q;
-    *NB = best_nb;
-    need = std::max(need, best_nb * (size_t)M * (K / best_q + 8) * 2);
-    return true;
+    return false;
   };
   FusedPlan f;
-  if (!planes(E, &f.p_e, &f.nb_e) || !planes(qw, &f.p_o, &f.nb_o) || !planes(c.e_ffn, &f.p_h, &f.nb_h)) return false;
+  if (!planes(E, &f.p_e) || !planes(qw, &f.p_o) || !planes(c.e_ffn, &f.p_h)) return false;
   f.slot_bytes = (int)slot;
   f.a_bytes = (int)((need + 127) / 128 * 128);
   f.smem = 2 * slot + f.a_bytes + misc;
@@ -513,11 +497,6 @@ bool fused_ok(const svla_handle* h, int B, int H, int L) {
   if (B < 1 || H < 1 || B > c.max_batch || H > c.max_chunk) return false;
   if ((long long)B * H > FD_MAX_M || H > ATT_BQ || H > ATT_BK) return false;
   if (c.e_layers > FD_MAX_LAYERS || c.e_ffn % 32 || c.e_width % 16) return false;
-  {  // at most FD_MAX_JPS jobs of one GEMM stage per CTA
-    const int jobs = std::max({c.e_width / 8, (c.e_heads + 2 * c.e_kv_heads) * c.head_dim / 16,
-                               c.e_heads * c.head_dim / 8, c.e_ffn / 16});
-    if (jobs > FD_MAX_JPS * h->num_sms) return false;
-  }
   if (h->num_sms < 1 || !h->fw) return false;
   return fused_plan(c, B * H, L, nullptr);
 }
@@ -558,11 +537,11 @@ cudaError_t launch_fused(svla_handle* h, const void* kv, const uint8_t* pad, int
   a.rope_cs = h->rope_cs; a.inv_period = h->inv_period;
   const int qw = c.e_heads * c.head_dim;
   a.r = h->e_r;
-  a.rb = FdAct{h->e_y, c.e_width, fp.p_e, fp.nb_e};
-  a.a = FdAct{h->e_a, c.e_width, fp.p_e, fp.nb_e};
-  a.h1 = FdAct{h->e_h1, c.e_width, fp.p_e, fp.nb_e};
-  a.o = FdAct{h->e_o, qw, fp.p_o, fp.nb_o};
-  a.hh = FdAct{h->e_h, c.e_ffn, fp.p_h, fp.nb_h};
+  a.rb = FdAct{h->e_y, c.e_width, fp.p_e};
+  a.a = FdAct{h->e_a, c.e_width, fp.p_e};
+  a.h1 = FdAct{h->e_h1, c.e_width, fp.p_e};
+  a.o = FdAct{h->e_o, qw, fp.p_o};
+  a.hh = FdAct{h->e_h, c.e_ffn, fp.p_h};
   a.q = h->e_q; a.k = h->e_k; a.v = h->e_v; a.c = h->e_c;
   a.sync = h->fd_sync; a.status = h->status; a.wait_ns = g_wait_ns.load();
   a.slot_bytes = fp.slot_bytes;
