@@ -35,3 +35,4 @@ from .model import (  # noqa: F401
     time_embedding, velocity, denoise, denoise_prefix_overwrite, sample, oracle_joint, cross_kv,
 )
 from .philox import philox4x32_10, gaussian_noise  # noqa: F401
+from .assembly import pixel_shuffle, connector, state_token, assemble_prefix  # noqa: F401

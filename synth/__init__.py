@@ -30,7 +30,8 @@ import numpy as np
 __all__ = [
     "ModelShape", "Workload", "SHAPES", "WORKLOADS", "manifest", "param_count",
     "gen_weights", "pack_blob", "gen_inputs", "f32_to_bf16_bits",
-    "bf16_bits_to_f32", "pack_kv_cache", "kv_cache_elems",
+    "bf16_bits_to_f32", "pack_kv_cache", "kv_cache_elems", "AssemblyShape", "ASSEMBLY_SHAPES",
+    "assembly_manifest", "gen_assembly_weights", "pack_assembly_blob", "gen_assembly_inputs",
 ]
 
 
@@ -289,3 +290,71 @@ def gen_inputs(wl: Workload, B: int | None = None) -> Dict[str, np.ndarray]:
     else:
         out["embeds"] = np.stack(embeds)
     return out
+
+
+# --------------------------------------------------------------------------
+# Prefix assembly upstream of the prefill: the connector (pixel shuffle of the
+# vision tower's patch grid, then a linear map to the LM width) and the state
+# projection ("noeira docs, SmolVLA" §Architecture: SigLIP width 768 on a
+# 512x512 image in 16x16 patches -> 32 x 32 patches, pixel shuffle x4 -> 64
+# tokens per image, linear to 960; "Paper vs hardware 11: SmolVLA" §claims:
+# the state projected to one prefix token). The state width 32 matches the
+# padded action width.
+# --------------------------------------------------------------------------
+@dataclass(frozen=True)
+class AssemblyShape:
+    vis_width: int     # C: channels of a patch feature
+    grid: int          # patches per image side
+    shuffle: int       # r: pixel-shuffle factor
+    state_dim: int     # S
+    n_img: int         # cameras per query
+    text_len: int      # T: text tokens (padded)
+
+    @property
+    def tokens_per_image(self) -> int:
+        return (self.grid // self.shuffle) ** 2
+
+    @property
+    def conn_in(self) -> int:
+        return self.shuffle * self.shuffle * self.vis_width
+
+
+ASSEMBLY_SHAPES: Dict[str, AssemblyShape] = {
+    "tiny": AssemblyShape(vis_width=16, grid=8, shuffle=2, state_dim=8, n_img=2, text_len=6),
+    "smolvla": AssemblyShape(vis_width=768, grid=32, shuffle=4, state_dim=32, n_img=2, text_len=48),
+}
+
+
+def assembly_manifest(a: AssemblyShape, width: int) -> List[Tuple[str, Tuple[int, ...]]]:
+    """Blob order of the assembly weights: W_c [width, r*r*C], W_s [width, S], b_s [width]."""
+    return [("w_conn", (width, a.conn_in)), ("w_state", (width, a.state_dim)), ("b_state", (width,))]
+
+
+def gen_assembly_weights(a: AssemblyShape, width: int, seed: int, std: float = 0.02) -> Dict[str, np.ndarray]:
+    """Seeded assembly weights as bf16 bits (the state bias N(0, std) too, so it is exercised)."""
+    rng = np.random.default_rng([seed, 0xA55E])
+    return {n: f32_to_bf16_bits(np.float32(std) * rng.standard_normal(shp, dtype=np.float32))
+            for n, shp in assembly_manifest(a, width)}
+
+
+def pack_assembly_blob(a: AssemblyShape, width: int, w: Dict[str, np.ndarray]) -> np.ndarray:
+    return np.concatenate([np.asarray(w[n], np.uint16).reshape(-1) for n, _ in assembly_manifest(a, width)])
+
+
+def gen_assembly_inputs(a: AssemblyShape, width: int, B: int, seed: int) -> Dict[str, np.ndarray]:
+    """Seeded inputs of one batch: ``vis`` (bf16 bits [B, n_img, grid^2, C]),
+    ``text`` (bf16 bits [B, T, width]), ``text_valid`` (uint8 [B, T], a
+    per-query count of leading valid tokens in [1, T]) and ``state`` (float32
+    [B, S])."""
+    out = {"vis": [], "text": [], "text_valid": [], "state": []}
+    for b in range(B):
+        qr = np.random.default_rng([seed, 0xA55F, b])
+        out["vis"].append(f32_to_bf16_bits(qr.standard_normal((a.n_img, a.grid * a.grid, a.vis_width),
+                                                              dtype=np.float32)))
+        out["text"].append(f32_to_bf16_bits(qr.standard_normal((a.text_len, width), dtype=np.float32)))
+        n = int(qr.integers(1, a.text_len + 1))
+        tv = np.zeros(a.text_len, np.uint8)
+        tv[:n] = 1
+        out["text_valid"].append(tv)
+        out["state"].append(qr.standard_normal(a.state_dim, dtype=np.float32))
+    return {k: np.stack(v) for k, v in out.items()}
