@@ -40,7 +40,7 @@ L2_BYTES = 126 * 1024 * 1024
 #    the capture summarised in profiles/gemm_tc_kernel_smolvla_b1.md;
 #  - the persistent denoise kernel: profiles/denoise_fused_kernel_smolvla_b1.md.
 NCU_TRAFFIC_GEMM_B1 = 3.698e6
-NCU_TRAFFIC_FUSED = 1.9915e9
+NCU_TRAFFIC_FUSED = 1.991e9
 
 
 def _peaks():
@@ -401,6 +401,27 @@ def ours(args, rank, world, local_rank):
     ms_den = time_steps(lambda: m.denoise(d["kv"], d["valid"], d["noise"], wl.n_steps, actions=d["actions"]),
                         args.steps, args.warmup, barrier)
 
+    # prefix assembly upstream of the step (connector + state token, svla_assemble_prefix),
+    # timed alone: the headline step starts from the assembled prefix embeddings
+    asm = None
+    ash = synth.ASSEMBLY_SHAPES["smolvla"]
+    if wl.L == ash.n_img * ash.tokens_per_image + ash.text_len + 1:
+        wbits = synth.gen_assembly_weights(ash, s.p_width, wl.seed)
+        m.set_assembly(synth.pack_assembly_blob(ash, s.p_width, wbits), ash.vis_width, ash.grid, ash.shuffle,
+                       ash.state_dim, ash.n_img)
+        ai = synth.gen_assembly_inputs(ash, s.p_width, wl.B, wl.seed)
+        av = torch.from_numpy(ai["vis"].view(np.int16)).to(f"cuda:{dev}").view(torch.bfloat16)
+        at = torch.from_numpy(ai["text"].view(np.int16)).to(f"cuda:{dev}").view(torch.bfloat16)
+        atv = torch.from_numpy(ai["text_valid"]).to(f"cuda:{dev}")
+        ast = torch.from_numpy(ai["state"]).to(f"cuda:{dev}")
+        ms_asm = time_steps(lambda: m.assemble_prefix(av, at, atv, ast), args.steps, args.warmup, barrier)
+        conn_w = 2 * s.p_width * ash.conn_in
+        asm_bytes = conn_w + 2 * 2 * wl.B * ash.n_img * ash.grid * ash.grid * ash.vis_width \
+            + 2 * wl.B * wl.L * s.p_width
+        asm = {"assemble_ms": round(ms_asm / args.steps, 4), "images": ash.n_img,
+               "algorithmic_bytes": int(asm_bytes),
+               "note": "pixel-shuffle gather + connector GEMM (12288 -> 960) + state token and layout, 3 kernels"}
+
     hbm_bytes, gflops, aflops = chunk_work(s, wl.B, wl.L, wl.H, wl.n_steps)
     chunk_s = value * 1e-3 * world  # per-rank chunk latency in s
     fused = m.fused_supported(wl.B, wl.H)
@@ -477,6 +498,7 @@ def ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
             "breakdown": {"prefill_ms": round(ms_pre / args.steps, 4), "denoise_ms": round(ms_den / args.steps, 4),
                           "note": "each call timed alone on rank 0, same steps and warm-up"},
+            "prefix_assembly": asm,
             "gpu_launches": launches_per_chunk(s, wl.n_steps, fused) * args.steps,
             "graph_gemm_roofline": graph_gemm if fused else None,
             "clocks": clk,

@@ -178,6 +178,36 @@ SVLA_API svla_status svla_sample(svla_handle* h, const void* prefix_embeds, cons
                         int B, int L, uint64_t seed, int H, int n_steps,
                         void* kv_cache, float* noise_out, float* actions, void* stream);
 
+/* Prefix assembly upstream of the prefill ("noeira docs, SmolVLA"
+ * §Architecture: the connector — pixel shuffle of the vision tower's patch
+ * grid, then a linear projection to the LM width — and a prefix of the camera
+ * images, the tokenised instruction and one state token; "Paper vs hardware
+ * 11: SmolVLA" §claims: the state projected to one token). Pixel shuffle x r
+ * is the space-to-depth of the g x g patch grid: output token (i, j)
+ * concatenates the r x r block of patches (r i + a, r j + b) in row-major
+ * (a, b) order; the state token is W_s s + b_s in fp32, stored bf16; the
+ * prefix is [image tokens in camera order | text tokens | state token].
+ *
+ * svla_set_assembly: blob = bf16 [W_c (p_width x r*r*vis_width) | W_s
+ *   (p_width x state_dim) | b_s (p_width)], host or device memory, copied
+ *   (svla_assembly_blob_bytes gives its size; another size is
+ *   SVLA_ERR_BLOB_SIZE). vis_width a multiple of 8, grid a multiple of
+ *   shuffle, 1 <= state_dim <= 64; allocates the workspace for max_batch x
+ *   max_images images. Call once, outside any stream capture.
+ * svla_assemble_prefix: vis device bf16 [B][n_img][grid*grid][vis_width]
+ *   (row-major patch index); text device bf16 [B][T][p_width] with text_valid
+ *   device u8 [B][T] (both may be NULL when T = 0); state device f32
+ *   [B][state_dim]; writes embeds device bf16 [B][L][p_width] and pad device
+ *   u8 [B][L], L = n_img (grid/shuffle)^2 + T + 1 — the inputs of
+ *   svla_prefill. Stream-ordered; 1 <= B <= max_batch, 1 <= n_img <=
+ *   max_images. */
+SVLA_API size_t svla_assembly_blob_bytes(int p_width, int vis_width, int shuffle, int state_dim);
+SVLA_API svla_status svla_set_assembly(svla_handle* h, const void* blob, size_t blob_bytes, int vis_width,
+                                       int grid, int shuffle, int state_dim, int max_images);
+SVLA_API svla_status svla_assemble_prefix(svla_handle* h, const void* vis, const void* text,
+                                          const uint8_t* text_valid, const float* state, int B, int n_img,
+                                          int T, void* embeds, uint8_t* pad, void* stream);
+
 /* Synchronise `stream`, then return and clear the device status word of the
  * handle's device (SVLA_OK, SVLA_ERR_EMPTY_PREFIX, SVLA_ERR_TIMEOUT) — or
  * SVLA_ERR_CUDA if the synchronisation itself failed. */

@@ -110,3 +110,15 @@ def test_gemm_plan_workspace_rules():
     assert lib.svla_op_gemm_workspace_bytes(50, 720, 2048, 1) == 0
     # more than 8 forced splits reduce through a global workspace
     assert lib.svla_op_gemm_workspace_bytes(50, 720, 2048, 16) > 0
+
+
+@pytest.mark.parametrize("shape", ["tiny", "smolvla"])
+def test_assembly_blob_bytes_and_null_handle(shape):
+    lib = _abi.load()
+    s = synth.SHAPES[shape]
+    a = synth.ASSEMBLY_SHAPES[shape]
+    n = sum(int(np.prod(shp)) for _, shp in synth.assembly_manifest(a, s.p_width))
+    assert lib.svla_assembly_blob_bytes(s.p_width, a.vis_width, a.shuffle, a.state_dim) == 2 * n
+    assert lib.svla_assembly_blob_bytes(0, a.vis_width, a.shuffle, a.state_dim) == 0
+    assert lib.svla_set_assembly(None, None, 0, 8, 8, 2, 8, 1) == _abi.SVLA_ERR_ARG
+    assert lib.svla_assemble_prefix(None, None, None, None, None, 1, 1, 0, None, None, None) == _abi.SVLA_ERR_ARG

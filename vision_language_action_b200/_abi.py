@@ -55,6 +55,9 @@ SIGNATURES = {
     "svla_op_rmsnorm": (_I, [_P, _P, _I, _I, ctypes.c_float, _P, _P]),
     "svla_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "svla_set_denoise_path": (_I, [_P, _I]),
+    "svla_assembly_blob_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "svla_set_assembly": (_I, [_P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I]),
+    "svla_assemble_prefix": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "svla_denoise_fused_supported": (_I, [_P, _I, _I]),
 }
 

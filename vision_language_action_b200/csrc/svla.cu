@@ -19,6 +19,7 @@
 #include <string>
 #include <vector>
 
+#include "assembly.cuh"
 #include "attention.cuh"
 #include "denoise_fused.cuh"
 #include "gemm_host.cuh"
@@ -251,6 +252,11 @@ struct svla_handle {
   uint16_t* fw = nullptr;       // persistent denoise: expert GEMM weights with row pitch K + 8
   FusedWeights fwl;
   int denoise_path = SVLA_DENOISE_AUTO;
+  // prefix assembly (svla_set_assembly): connector and state-projection weights, workspaces
+  uint16_t* asm_w = nullptr;   // W_c [p_width, r*r*C] | W_s [p_width, S] | b_s [p_width]
+  uint16_t* asm_a = nullptr;   // gathered connector operand [max_batch * max_images * tpi, r*r*C]
+  uint16_t* asm_out = nullptr; // connector output [max_batch * max_images * tpi, p_width]
+  int asm_C = 0, asm_grid = 0, asm_r = 0, asm_S = 0, asm_max_img = 0;
   int num_sms = 0;
   cudaStream_t cap = nullptr;  // capture stream
   std::list<GraphEntry> graphs;
@@ -1007,6 +1013,78 @@ svla_status svla_set_denoise_path(svla_handle* h, int path) {
 
 int svla_denoise_fused_supported(const svla_handle* h, int B, int H) {
   return h && fused_ok(h, B, H, h->cfg.max_prefix) ? 1 : 0;
+}
+
+size_t svla_assembly_blob_bytes(int p_width, int vis_width, int shuffle, int state_dim) {
+  if (p_width < 1 || vis_width < 1 || shuffle < 1 || state_dim < 1) return 0;
+  return (size_t)2 * p_width * ((size_t)shuffle * shuffle * vis_width + state_dim + 1);
+}
+
+svla_status svla_set_assembly(svla_handle* h, const void* blob, size_t blob_bytes, int vis_width, int grid,
+                              int shuffle, int state_dim, int max_images) {
+  if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
+  if (!blob) return fail(h, SVLA_ERR_ARG, "null blob");
+  if (vis_width < 8 || vis_width % 8 || shuffle < 1 || grid < shuffle || grid % shuffle || state_dim < 1 ||
+      state_dim > 64 || max_images < 1)
+    return fail(h, SVLA_ERR_SHAPE,
+                "vis_width a multiple of 8, grid a multiple of shuffle, 1 <= state_dim <= 64, max_images >= 1");
+  const int D = h->cfg.p_width;
+  const size_t want = svla_assembly_blob_bytes(D, vis_width, shuffle, state_dim);
+  if (blob_bytes != want) return fail(h, SVLA_ERR_BLOB_SIZE, "assembly blob size mismatch");
+  DeviceGuard dg(h->device);
+  const size_t K = (size_t)shuffle * shuffle * vis_width, tpi = (size_t)(grid / shuffle) * (grid / shuffle);
+  const size_t rows = (size_t)h->cfg.max_batch * max_images * tpi;
+  cudaError_t e;
+  if ((e = halloc(h, &h->asm_w, want / 2)) != cudaSuccess) return cuda_fail(h, e, "assembly weights");
+  if ((e = cudaMemcpy(h->asm_w, blob, want, cudaMemcpyDefault)) != cudaSuccess) return cuda_fail(h, e, "assembly weights");
+  if ((e = halloc(h, &h->asm_a, rows * K)) != cudaSuccess) return cuda_fail(h, e, "assembly workspace");
+  if ((e = halloc(h, &h->asm_out, rows * D)) != cudaSuccess) return cuda_fail(h, e, "assembly workspace");
+  h->asm_C = vis_width;
+  h->asm_grid = grid;
+  h->asm_r = shuffle;
+  h->asm_S = state_dim;
+  h->asm_max_img = max_images;
+  return SVLA_OK;
+}
+
+svla_status svla_assemble_prefix(svla_handle* h, const void* vis, const void* text, const uint8_t* text_valid,
+                                 const float* state, int B, int n_img, int T, void* embeds, uint8_t* pad,
+                                 void* stream) {
+  if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
+  if (!h->asm_w) return fail(h, SVLA_ERR_ARG, "no assembly weights: call svla_set_assembly first");
+  if (!vis || !state || !embeds || !pad || (T > 0 && (!text || !text_valid))) return fail(h, SVLA_ERR_ARG, "null pointer");
+  if (B < 1 || B > h->cfg.max_batch || n_img < 1 || n_img > h->asm_max_img || T < 0)
+    return fail(h, SVLA_ERR_SHAPE, "B, n_img or T outside the handle's limits");
+  DeviceGuard dg(h->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int D = h->cfg.p_width, r = h->asm_r, g = h->asm_grid, C = h->asm_C, S = h->asm_S;
+  const int tpi = (g / r) * (g / r), K = r * r * C, M = B * n_img * tpi;
+  const long long chunks = (long long)M * K / 8;
+  const int blocks = (int)std::min<long long>((chunks + 255) / 256, 8LL * NUM_SMS_B200);
+  cudaError_t e = launch_pdl(pixel_shuffle_kernel, dim3(blocks), dim3(256), 0, s,
+                             reinterpret_cast<const uint16_t*>(vis), B * n_img, g, r, C, h->asm_a);
+  if (e == cudaSuccess)
+    e = gemm(h, GE_BF16, reinterpret_cast<const bf16*>(h->asm_a), K, reinterpret_cast<const bf16*>(h->asm_w), K, M, D,
+             K, out_args(h->asm_out, D), h->p_part, h->p_cnt, s);
+  if (e == cudaSuccess) {
+    AssembleArgs a;
+    a.conn = h->asm_out;
+    a.text = reinterpret_cast<const uint16_t*>(text);
+    a.text_valid = text_valid;
+    a.state = state;
+    a.w_state = h->asm_w + (size_t)D * K;
+    a.b_state = a.w_state + (size_t)D * S;
+    a.n_vis = n_img * tpi;
+    a.T = T;
+    a.D = D;
+    a.S = S;
+    a.L = a.n_vis + T + 1;
+    a.out = reinterpret_cast<uint16_t*>(embeds);
+    a.pad = pad;
+    e = launch_pdl(assemble_kernel, dim3(a.L, B), dim3(128), 0, s, a);
+  }
+  if (e != cudaSuccess) return cuda_fail(h, e, "assemble prefix");
+  return SVLA_OK;
 }
 
 svla_status svla_device_status(svla_handle* h, void* stream) {

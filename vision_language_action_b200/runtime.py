@@ -143,6 +143,37 @@ class SmolVLA:
         _abi.check(st, self.h)
         return (actions, kv_cache, noise) if return_noise else (actions, kv_cache)
 
+    def set_assembly(self, blob, vis_width: int, grid: int, shuffle: int, state_dim: int, max_images: int) -> None:
+        """Connector + state-projection weights (bf16 blob: W_c | W_s | b_s)."""
+        import numpy as np
+        if isinstance(blob, torch.Tensor):
+            t = blob.contiguous()
+            ptr, nbytes, keep = t.data_ptr(), t.numel() * t.element_size(), t
+        else:
+            keep = np.ascontiguousarray(blob)
+            ptr, nbytes = keep.ctypes.data, keep.nbytes
+        st = self.lib.svla_set_assembly(self.h, ctypes.c_void_p(ptr), nbytes, vis_width, grid, shuffle, state_dim,
+                                        max_images)
+        del keep
+        _abi.check(st, self.h)
+        self.asm = (grid, shuffle)
+
+    def assemble_prefix(self, vis: torch.Tensor, text: torch.Tensor, text_valid: torch.Tensor, state: torch.Tensor,
+                        stream=None):
+        """vis bf16 [B, n_img, grid^2, C], text bf16 [B, T, p_width], text_valid u8 [B, T],
+        state f32 [B, S] -> (embeds bf16 [B, L, p_width], pad u8 [B, L])."""
+        B, n_img = vis.shape[0], vis.shape[1]
+        T = text.shape[1]
+        grid, r = self.asm
+        L = n_img * (grid // r) ** 2 + T + 1
+        embeds = torch.empty((B, L, self.cfg.p_width), dtype=torch.bfloat16, device=vis.device)
+        pad = torch.empty((B, L), dtype=torch.uint8, device=vis.device)
+        st = self.lib.svla_assemble_prefix(self.h, _ptr(vis), _ptr(text) if T else None,
+                                           _ptr(text_valid) if T else None, _ptr(state), B, n_img, T,
+                                           _ptr(embeds), _ptr(pad), _stream(stream))
+        _abi.check(st, self.h)
+        return embeds, pad
+
     def set_denoise_path(self, path: int) -> None:
         """_abi.DENOISE_AUTO (default), DENOISE_GRAPH or DENOISE_FUSED."""
         _abi.check(self.lib.svla_set_denoise_path(self.h, path), self.h)
