@@ -259,6 +259,22 @@ def gpu_setup(wl_name, dev, B=None):
     return m, wl, host, d
 
 
+def max_over_ranks(x: float, world: int, device: str) -> float:
+    """The largest value of x over the ranks (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def ms_per_chunk(ms_total_max: float, steps: int, batch_per_rank: int, world: int) -> float:
+    """Job-level metric: the timed region (max over ranks) over every chunk all ranks produced."""
+    return ms_total_max / (steps * batch_per_rank * world)
+
+
 def time_steps(fn, steps, warmup, barrier):
     import torch
     for _ in range(warmup):
@@ -368,13 +384,10 @@ def ours(args, rank, world, local_rank):
     st = m.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after the timed region")
-    if world > 1:
-        t = torch.tensor([ms_total], device=f"cuda:{dev}")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, f"cuda:{dev}")
     ms_step = ms_total / args.steps
     chunks_per_step = wl.B * world
-    value = ms_total / (args.steps * chunks_per_step)
+    value = ms_per_chunk(ms_total, args.steps, wl.B, world)
 
     # end to end through the public API with host buffers: H2D inputs, both calls, D2H actions
     out_host = torch.empty_like(host["noise"]).pin_memory()
@@ -390,11 +403,7 @@ def ours(args, rank, world, local_rank):
         out_host.copy_(d["actions"], non_blocking=True)
         torch.cuda.current_stream().synchronize()
 
-    ms_e2e = time_steps(e2e_step, args.steps, args.warmup, barrier)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=f"cuda:{dev}")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(time_steps(e2e_step, args.steps, args.warmup, barrier), world, f"cuda:{dev}")
 
     # the two calls of a step timed on their own (same warm-up and step count)
     ms_pre = time_steps(lambda: m.prefill(d["embeds"], d["valid"], d["kv"]), args.steps, args.warmup, barrier)
