@@ -259,6 +259,8 @@ struct svla_handle {
   int asm_C = 0, asm_grid = 0, asm_r = 0, asm_S = 0, asm_max_img = 0;
   int num_sms = 0;
   cudaStream_t cap = nullptr;  // capture stream
+  cudaStream_t side[4] = {};   // branches of the hoisted projections inside the denoise graph
+  cudaEvent_t fork = nullptr, join[4] = {};
   std::list<GraphEntry> graphs;
   std::vector<void*> allocs;
   std::string last_error = "no error";
@@ -303,6 +305,14 @@ void free_all(svla_handle* h) {
   for (void* p : h->allocs) cudaFree(p);
   h->allocs.clear();
   if (h->cap) cudaStreamDestroy(h->cap);
+  for (int i = 0; i < 4; ++i) {
+    if (h->side[i]) cudaStreamDestroy(h->side[i]);
+    if (h->join[i]) cudaEventDestroy(h->join[i]);
+    h->side[i] = nullptr;
+    h->join[i] = nullptr;
+  }
+  if (h->fork) cudaEventDestroy(h->fork);
+  h->fork = nullptr;
   h->cap = nullptr;
 }
 
@@ -579,15 +589,31 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
   const size_t layer_elems = (size_t)Mp * pkvw;
   bf16* rb = h->e_y;  // bf16 copy of the expert residual stream
   if (actions != noise) SVLA_TRY(cudaMemcpyAsync(actions, noise, (size_t)M * A * sizeof(float), cudaMemcpyDeviceToDevice, s));
-  // hoisted cross K/V projection (once per query, not per step)
+  // hoisted cross K/V projection (once per query, not per step). The 2 x (e_layers / 2)
+  // GEMMs are independent and each fills only part of the GPU at batch 1: they run as
+  // 4 parallel branches of the graph (fork / join events), unless their plan needs the
+  // shared split-K workspace (then one after another).
+  const bool par = plan_gemm(Mp, kvw, pkvw, 0, gemm_min_bn(GE_BF16)).red != GEMM_RED_GLOBAL;
+  if (par) {
+    SVLA_TRY(cudaEventRecord(h->fork, s));
+    for (int i = 0; i < 4; ++i) SVLA_TRY(cudaStreamWaitEvent(h->side[i], h->fork, 0));
+  }
+  int branch = 0;
   for (int l = 1; l < c.e_layers; l += 2) {
     const Entry* e = &h->lay.e[9 * l];
     bf16* kx = h->kvx + (size_t)(l / 2) * 2 * Mp * kvw;
     bf16* vx = kx + (size_t)Mp * kvw;
+    cudaStream_t sk = par ? h->side[branch++ % 4] : s, sv = par ? h->side[branch++ % 4] : s;
     SVLA_TRY(gemm(h, GE_BF16, cache + (size_t)l * layer_elems, pkvw, h->W(e[2].off), pkvw, Mp, kvw, pkvw,
-                  out_args(kx, kvw), h->e_part, h->e_cnt, s));
+                  out_args(kx, kvw), h->e_part, h->e_cnt, sk));
     SVLA_TRY(gemm(h, GE_BF16, cache + (size_t)(c.p_layers + l) * layer_elems, pkvw, h->W(e[3].off), pkvw, Mp, kvw,
-                  pkvw, out_args(vx, kvw), h->e_part, h->e_cnt, s));
+                  pkvw, out_args(vx, kvw), h->e_part, h->e_cnt, sv));
+  }
+  if (par) {
+    for (int i = 0; i < 4; ++i) {
+      SVLA_TRY(cudaEventRecord(h->join[i], h->side[i]));
+      SVLA_TRY(cudaStreamWaitEvent(s, h->join[i], 0));
+    }
   }
   if (fused) return launch_fused(h, kv, pad, B, L, noise, H, n_steps, actions, trace, prefix, d, s);
   const Layout& Lh = h->lay;
@@ -904,6 +930,12 @@ svla_status svla_create(const svla_config* cfg, const void* blob, size_t blob_by
   cudaMemset(h->p_cnt, 0, CNT_INTS * sizeof(int));
   cudaMemset(h->e_cnt, 0, CNT_INTS * sizeof(int));
   if ((e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking)) != cudaSuccess) return bail(e, "stream");
+  for (int i = 0; i < 4 && e == cudaSuccess; ++i) {
+    e = cudaStreamCreateWithFlags(&h->side[i], cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->join[i], cudaEventDisableTiming);
+  }
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming);
+  if (e != cudaSuccess) return bail(e, "streams");
   if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(e, "create");
   *out = h;
   return SVLA_OK;
