@@ -733,6 +733,18 @@ SVLA_DEV void fd_attention_job(const AttnArgs& a, int b, int h, int i0, uint8_t*
   __syncthreads();
 }
 
+// The same attention job as a kernel of the graph path: one CTA per (query b,
+// head h, 16 query rows), blockIdx.x = (b * n_q + h) * ceil(Lq / 16) + row block;
+// output as AttnArgs gives it (o_pc == 0: row-major [B * Lq, ldo]).
+template <int HD>
+__global__ void __launch_bounds__(FD_THREADS) attention_rows_kernel(const AttnArgs a) {
+  extern __shared__ __align__(16) uint8_t att_rows_smem[];
+  griddep_launch_dependents();
+  griddep_wait();
+  const int rblk = (a.Lq + 15) / 16, j = blockIdx.x;
+  fd_attention_job<HD>(a, j / (rblk * a.n_q), (j / rblk) % a.n_q, 16 * (j % rblk), att_rows_smem);
+}
+
 // ---------------------------------------------------------------------------
 // row stage: end of step k_end (if >= 0) and start of step k_begin (if < n),
 // rows m = blockIdx.x, blockIdx.x + gridDim.x, ..:

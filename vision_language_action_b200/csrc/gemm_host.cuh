@@ -158,8 +158,18 @@ inline GemmPlan plan_gemm(int M, int N, int K, int forced_splits, int min_bn = 3
       p.a_rows = 64;
     }
   } else {
+    // two CTAs of this configuration fit on an SM (4 stages, <= 113 KB), so one
+    // wave holds 2 x SMs CTAs; a split keeps >= 3 k-blocks (below that the
+    // cluster reduction costs more than it saves: measured at M = 177, K = 320
+    // one split took 3.6 us against 5.2 us with five; at N = 960, K = 2560 eight
+    // splits took 10.8 us against 12.2 us with four)
     const int t64 = tiles(64), t32 = tiles(32);
-    const int s64 = clamp_splits(NUM_SMS_B200 / t64), s32 = clamp_splits(NUM_SMS_B200 / t32);
+    auto fit = [&](int t) {
+      int sp = clamp_splits(2 * NUM_SMS_B200 / t);
+      while (sp > 1 && KB / sp < 3) --sp;
+      return sp;
+    };
+    const int s64 = fit(t64), s32 = fit(t32);
     const int c64 = t64 * s64, c32 = t32 * s32;
     p.bn = (c64 >= 120 || c64 >= c32 || min_bn > 32) ? 64 : 32;
     p.stages = 4;

@@ -30,7 +30,8 @@ using namespace svla;
 namespace {
 
 std::atomic<unsigned long long> g_wait_ns{1000000000ull};
-constexpr int FD_SMEM_MAX = 232448 - 4096;  // dynamic shared memory of the persistent denoise kernel (static: <= 4 KB)
+constexpr int FD_SMEM_MAX = 232448 - 4096;
+constexpr int ATT_ROWS_SMEM_MAX = 200 * 1024;  // the split-key attention kernel stages all keys of a head  // dynamic shared memory of the persistent denoise kernel (static: <= 4 KB)
 thread_local std::string t_last_error = "no error";
 
 const char* status_str(svla_status s) {
@@ -65,6 +66,10 @@ cudaError_t ensure_attrs(int dev) {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(attention_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)AttnCfg<32>::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attention_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_ROWS_SMEM_MAX);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attention_rows_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_ROWS_SMEM_MAX);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(denoise_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, FD_SMEM_MAX);
   if (e == cudaSuccess)
@@ -377,6 +382,15 @@ cudaError_t attention(const bf16* q, int ldq, const bf16* k, const bf16* v, int 
   a.causal = causal;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)hd));
   dim3 grid((Lq + ATT_BQ - 1) / ATT_BQ, nq, B);
+  // Few blocks (batch 1): one CTA per 16 query rows with the keys split over its
+  // 8 warps, so a head's work spreads over 4x more CTAs; every such CTA stages
+  // all of the head's keys, so larger batches keep the 64-row blocks.
+  const size_t rows_smem = hd == 64 ? fd_att_smem<64>(Lk) : fd_att_smem<32>(Lk);
+  if ((long long)grid.x * nq * B < 2 * NUM_SMS_B200 && rows_smem <= (size_t)ATT_ROWS_SMEM_MAX) {
+    const dim3 g2((unsigned)((long long)B * nq * ((Lq + 15) / 16)));
+    if (hd == 64) return launch_pdl(attention_rows_kernel<64>, g2, dim3(FD_THREADS), rows_smem, s, a);
+    return launch_pdl(attention_rows_kernel<32>, g2, dim3(FD_THREADS), rows_smem, s, a);
+  }
   if (hd == 64) return launch_pdl(attention_kernel<64>, grid, dim3(ATT_THREADS), AttnCfg<64>::SMEM, s, a);
   return launch_pdl(attention_kernel<32>, grid, dim3(ATT_THREADS), AttnCfg<32>::SMEM, s, a);
 }
