@@ -40,7 +40,7 @@ L2_BYTES = 126 * 1024 * 1024
 #    the capture summarised in profiles/gemm_tc_kernel_smolvla_b1.md;
 #  - the persistent denoise kernel: profiles/denoise_fused_kernel_smolvla_b1.md.
 NCU_TRAFFIC_GEMM_B1 = 3.698e6
-NCU_TRAFFIC_FUSED = 1.991e9
+NCU_TRAFFIC_FUSED = 1.9916e9
 
 
 def _peaks():
