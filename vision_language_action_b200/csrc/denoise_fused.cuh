@@ -9,38 +9,42 @@
 //
 //   per step k (t = 1 - k / n):
 //     a   = x W_in^T + b_in                       (row stage, CUDA cores)
-//     c   = W_t1[:, E:] e(t) + b_t1               (row stage, all CTAs)
+//     c   = W_t1[:, E:] e(t) + b_t1               (computed one step ahead, on the
+//                                                  CTAs idle during layer 0's attention)
 //     h1  = silu(a W_t1[:, :E]^T + c)             (GEMM stage)
 //     r   = h1 W_t2^T + b_t2                      (GEMM stage: residual stream)
 //     16 x [ QKV (RMSNorm, RoPE) | attention | O (+ r) | gate/up (RMSNorm,
 //            SwiGLU) | down (+ r) ]                (5 stages per layer)
-//     v   = RMSNorm(r) W_out^T + b_out; x += dt v (row stage)
+//     v   = RMSNorm(r) W_out^T + b_out; x += dt v (row stage, with the next a)
 //
-// At this batch the path is a chain of ~850 dependent steps of a few
+// At this batch the path is a chain of ~830 dependent stages of a few
 // microseconds each; HBM streaming (200 MB of expert weights per step) is far
 // from the bound. The design therefore cuts the cost of each dependency:
-//   - a stage boundary is a grid barrier (one atomic per CTA, one poller per
-//     CTA), not a kernel boundary;
+//   - a stage boundary is a grid barrier (a release reduction per CTA, one
+//     relaxed poller per CTA), not a kernel boundary;
 //   - weights never depend on activations: every CTA streams the weight slice
 //     of its next GEMM job into a free shared-memory slot with bulk async
-//     copies (cp.async.bulk, no multicast) while the current stages run, so a
-//     GEMM stage's critical path is only: barrier, activation rows from L2,
-//     the products, the epilogue;
+//     copies (cp.async.bulk, no multicast) while earlier stages run, so a GEMM
+//     stage's critical path is: barrier, one bulk copy of the activation
+//     operand (kept in padded column planes for that), the products, the
+//     epilogue;
 //   - GEMM jobs are 8/16/32-column slices of W over the full K (no split-K, no
 //     reduction between CTAs): the <= 64 activation rows are tiny, the weight
-//     slice is the large operand. At <= 64 rows the tensor work of a job is a
-//     few hundred warp-level mma.sync m16n8k16 (bf16 in, fp32 accumulate): the
-//     MMA path is not where the time goes, so the register-level MMA is used
-//     rather than tcgen05 (no TMEM allocation or commit round trips in the
-//     chain); the batched path keeps the tcgen05 GEMMs.
+//     slice is the large operand. The products are warp-level mma.sync
+//     m16n8k16 (bf16 in, fp32 accumulate): a tcgen05 variant of the job
+//     (M = 64, N = w) was measured slower, its K/16 tiny MMAs being issue-bound
+//     on one thread; the batched path keeps the tcgen05 GEMMs;
+//   - attention jobs are (query, head, 16 rows) with the keys split over the
+//     CTA's 8 warps.
 // RMSNorm (reading 8) is applied on the consumer side: the activation operand
 // is the bf16 copy of the residual, each GEMM job sums its rows' squares from
-// the staged rows and scales the accumulator rows by rsqrt(mean + eps); the
-// gains are folded into the QKV and gate/up weights at create.
+// the A fragments it multiplies and scales the accumulator rows by
+// rsqrt(mean + eps); the gains are folded into the QKV and gate/up weights.
 //
-// Every wait is bounded (grid barrier and weight-slot mbarriers): on time-out
-// the CTA records SVLA_ERR_TIMEOUT, raises the abort word, drains its bulk
-// copies and returns; the other CTAs see the abort word at their next barrier.
+// Every wait is bounded (grid barrier and the mbarriers of the bulk copies): on
+// time-out the CTA records SVLA_ERR_TIMEOUT, raises the abort word, drains its
+// bulk copies and returns; the other CTAs see the abort word at their next
+// barrier.
 #pragma once
 
 #include "attention.cuh"
