@@ -36,3 +36,4 @@ from .model import (  # noqa: F401
 )
 from .philox import philox4x32_10, gaussian_noise  # noqa: F401
 from .assembly import pixel_shuffle, connector, state_token, assemble_prefix  # noqa: F401
+from .quant import quantize_affine8, dequantize_affine8, quantize_prefix  # noqa: F401
