@@ -105,6 +105,21 @@ def chunk_work(s, B, L, H, n_steps):
     return hbm, flops, att
 
 
+def prefix_projection_bytes(s, bits):
+    """Bytes of the prefix projections one prefill reads (the last layer stops
+    after its QKV): bf16 weights, or int8 codes plus a bf16 (alpha, beta) pair
+    per 64 weights (the vlm-8bit preset)."""
+    D, hd = s.p_width, s.head_dim
+    mats = [((s.p_heads + 2 * s.p_kv_heads) * hd, D), (D, s.p_heads * hd), (2 * s.p_ffn, D), (D, s.p_ffn)]
+    tot = 0
+    for l in range(s.p_layers):
+        for i, (N, K) in enumerate(mats):
+            if l == s.p_layers - 1 and i > 0:
+                break
+            tot += 2 * N * K if bits == 16 else N * K + N * (K // 64) * 4
+    return tot
+
+
 def launches_per_chunk(s, n_steps, fused):
     """Kernels libsvla launches for one prefill + denoise (the CUDA graphs' kernel nodes)."""
     pre = 2 + s.p_layers + 4 * (s.p_layers - 1)   # positions, residual init, QKV per layer, attn/O/GU/D
@@ -238,14 +253,14 @@ def reference_arm(args, rank):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
-def gpu_setup(wl_name, dev, B=None):
+def gpu_setup(wl_name, dev, B=None, prefix_int8=False):
     import torch
     from vision_language_action_b200.runtime import SmolVLA
     wl = synth.WORKLOADS[wl_name]
     s = wl.model
     B = wl.B if B is None else B
     blob = synth.pack_blob(s, synth.gen_weights(s, wl.seed))
-    m = SmolVLA(s, blob, max_batch=B, max_prefix=wl.L, max_chunk=wl.H, device=dev)
+    m = SmolVLA(s, blob, max_batch=B, max_prefix=wl.L, max_chunk=wl.H, device=dev, prefix_int8=prefix_int8)
     del blob
     inp = synth.gen_inputs(wl, B=B)
     host = {
@@ -359,6 +374,47 @@ def gemm_roofline(s, B, L, H, n_steps, dev, hbm_peak):
             "gemm_ms_per_chunk": round(float(t_chunk), 4)}
 
 
+def int8_prefix(args, dev, barrier, hbm_peak, peak_kind):
+    """The vlm-8bit preset (weight-only int8 prefix projections) at batch 1 and
+    batch 32: prefill and chunk times on one handle, switched between its int8
+    and dense prefix weights, and the int8 prefill's bytes against HBM."""
+    out = {"preset": "vlm-8bit: prefix projections int8, affine groups of 64 (bf16 alpha, beta); expert bf16"}
+    for name in ("smolvla_b1", "smolvla_b32"):
+        m, wl, _, d = gpu_setup(name, dev, prefix_int8=True)
+        s = wl.model
+        steps = args.steps if wl.B == 1 else max(3, args.steps // 2)
+
+        def pre():
+            m.prefill(d["embeds"], d["valid"], d["kv"])
+
+        def chunk():
+            pre()
+            m.denoise(d["kv"], d["valid"], d["noise"], wl.n_steps, actions=d["actions"])
+
+        t8 = time_steps(pre, steps, args.warmup, barrier) / steps
+        c8 = time_steps(chunk, steps, args.warmup, barrier) / steps
+        m.set_prefix_weights(16)
+        t16 = time_steps(pre, steps, args.warmup, barrier) / steps
+        m.set_prefix_weights(8)
+        if m.device_status() != 0:
+            raise RuntimeError("device status after the int8 prefill timing")
+        m.close()
+        del d
+        w8, w16 = prefix_projection_bytes(s, 8), prefix_projection_bytes(s, 16)
+        pre_bytes = chunk_work(s, wl.B, wl.L, wl.H, 0)[0] - w16 + w8
+        achieved = pre_bytes / (t8 * 1e-3) / 1e9
+        out[name] = {"prefill_ms": round(t8, 4), "prefill_ms_dense_same_handle": round(t16, 4),
+                     "chunk_ms": round(c8 / wl.B, 4) if wl.B == 1 else None,
+                     "chunks_per_s": round(wl.B / (c8 * 1e-3), 2) if wl.B > 1 else None,
+                     "projection_bytes_int8": int(w8), "projection_bytes_bf16": int(w16),
+                     "prefill_roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                                          "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                                          "algorithmic_bytes": int(pre_bytes), "peak_kind": peak_kind}}
+    import torch
+    torch.cuda.empty_cache()
+    return out
+
+
 def ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -453,6 +509,8 @@ def ours(args, rank, world, local_rank):
     del d
     torch.cuda.empty_cache()
 
+    q8 = None if args.no_int8 else int8_prefix(args, dev, barrier, hbm_peak, peak_kind)
+
     secondary = None
     if not args.no_secondary:
         m3, wl3, host3, d3 = gpu_setup("smolvla_b32", dev)
@@ -508,6 +566,7 @@ def ours(args, rank, world, local_rank):
             "breakdown": {"prefill_ms": round(ms_pre / args.steps, 4), "denoise_ms": round(ms_den / args.steps, 4),
                           "note": "each call timed alone on rank 0, same steps and warm-up"},
             "prefix_assembly": asm,
+            "int8_prefix": q8,
             "gpu_launches": launches_per_chunk(s, wl.n_steps, fused) * args.steps,
             "graph_gemm_roofline": graph_gemm if fused else None,
             "clocks": clk,
@@ -524,6 +583,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-int8", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

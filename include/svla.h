@@ -89,6 +89,31 @@ typedef struct svla_config {
 SVLA_API svla_status svla_create(const svla_config* cfg, const void* blob, size_t blob_bytes,
                         int device, svla_handle** out);
 
+/* svla_create with options. flags is a bitwise OR of:
+ *   SVLA_CREATE_PREFIX_INT8  also build the weight-only int8 copy of the prefix
+ *     LM's projections (the "vlm-8bit" preset of the mlx-smolvla PyPI page,
+ *     §Run a checkpoint) and select it for svla_prefill; the dense bf16
+ *     weights stay resident, so svla_set_prefix_weights can switch back.
+ *     Scheme (the page names the preset only; these are readings): every group
+ *     of 64 consecutive input weights of one output row of W_q, W_k, W_v, W_o,
+ *     W_g, W_u, W_d gets lo = min, hi = max, alpha = bf16((hi - lo) / 255),
+ *     beta = lo and codes q = clamp(rint((w - beta) / alpha), 0, 255) (0 when
+ *     alpha = 0), each step an IEEE fp32 operation rounded to nearest even; the
+ *     GEMMs use w^ = bf16(alpha q + beta) (times the folded RMSNorm gain, as the
+ *     dense path does). Norm gains, the expert and the heads stay bf16.
+ *     Needs p_width and p_ffn multiples of 64 (they are, by check_config).
+ * flags = 0 is svla_create. Unknown flag bits: SVLA_ERR_ARG. */
+#define SVLA_CREATE_PREFIX_INT8 1u
+SVLA_API svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob_bytes,
+                           int device, unsigned flags, svla_handle** out);
+
+/* Prefix weights svla_prefill uses from the next call on: 16 = dense bf16
+ * (default), 8 = the int8 copy (SVLA_ERR_UNSUPPORTED unless the handle was
+ * created with SVLA_CREATE_PREFIX_INT8). Other values: SVLA_ERR_ARG. */
+SVLA_API svla_status svla_set_prefix_weights(svla_handle* h, int bits);
+/* The prefix weight width svla_prefill uses (16 or 8); 0 for a NULL handle. */
+SVLA_API int svla_prefix_weights(const svla_handle* h);
+
 /* Free everything the handle owns (synchronises its device first). NULL is ok. */
 SVLA_API svla_status svla_destroy(svla_handle* h);
 
@@ -260,6 +285,29 @@ SVLA_API int svla_op_gemm_splits(int M, int N, int K);
 SVLA_API svla_status svla_op_attention(const void* q, int ldq, const void* k, const void* v, int ldkv,
                               const uint8_t* key_valid, int B, int n_q, int n_kv, int hd,
                               int Lq, int Lk, int causal, void* out, int ldo, void* stream);
+
+/* The vlm-8bit quantiser (svla_create_ex, SVLA_CREATE_PREFIX_INT8) on one matrix.
+ *   W:  device bf16 [N, K], row stride ldw >= K elements (even), 4-byte aligned.
+ *   q:  device uint8 [N, K] codes, row stride ldq >= K bytes (even).
+ *   ab: device bf16 [K/64][N][2]: (alpha, beta) of row n, group g at (g, n).
+ *   K % 64 == 0, N >= 1; weights must be finite. Asynchronous on `stream`. */
+SVLA_API svla_status svla_op_quantize_affine8(const void* W, int ldw, int N, int K, void* q, int ldq,
+                                     void* ab, void* stream);
+
+/* C[M, N] = A[M, K] · W^[N, K]^T with W^[n, k] = bf16(bf16(alpha q + beta) * g[k])
+ * on the tcgen05 tensor cores (the int8 weights are dequantised in shared
+ * memory, fp32 accumulation). Epilogues and C as svla_op_gemm.
+ *   A: device bf16, row stride lda >= K (multiple of 8), 16-byte aligned.
+ *   q, ab: as written by svla_op_quantize_affine8 (ldq a multiple of 16).
+ *   gain: NULL (g = 1) or device bf16 [K], 16-byte aligned.
+ *   K % 64 == 0, N % 8 == 0. splits: 0 = choose, else 1..8 (cluster split-K;
+ *   no workspace). status: as svla_op_gemm. */
+SVLA_API svla_status svla_op_gemm_w8(int epilogue, const void* A, int lda, const void* q, int ldq,
+                            const void* ab, const void* gain, int M, int N, int K, void* C, int ldc,
+                            const float* bias, int splits, int* status, void* stream);
+/* The K-split count svla_op_gemm_w8 picks for splits = 0, and its tile width. */
+SVLA_API int svla_op_gemm_w8_splits(int M, int N, int K);
+SVLA_API int svla_op_gemm_w8_tile_n(int M, int N, int K);
 
 /* RMSNorm (reading 8): y(bf16)[M, D] = x(f32)[M, D] / sqrt(mean(x^2) + eps) * g(bf16)[D]. */
 SVLA_API svla_status svla_op_rmsnorm(const float* x, const void* g, int M, int D, float eps,

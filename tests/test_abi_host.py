@@ -122,3 +122,41 @@ def test_assembly_blob_bytes_and_null_handle(shape):
     assert lib.svla_assembly_blob_bytes(0, a.vis_width, a.shuffle, a.state_dim) == 0
     assert lib.svla_set_assembly(None, None, 0, 8, 8, 2, 8, 1) == _abi.SVLA_ERR_ARG
     assert lib.svla_assemble_prefix(None, None, None, None, None, 1, 1, 0, None, None, None) == _abi.SVLA_ERR_ARG
+
+
+def test_int8_argument_checks_and_plan():
+    lib = _abi.load()
+    p = ctypes.c_void_p(16)
+    s = synth.SHAPES["tiny"]
+    blob = np.zeros(16, np.uint16)
+    h = ctypes.c_void_p()
+    cfg = config_from_shape(s, 1, 24, 8)
+    assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, 2,
+                              ctypes.byref(h)) == _abi.SVLA_ERR_ARG
+    cfg = config_from_shape(s.replace(p_heads=3, p_kv_heads=1), 1, 24, 8)  # O projection K = 96
+    assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0,
+                              _abi.CREATE_PREFIX_INT8, ctypes.byref(h)) == _abi.SVLA_ERR_SHAPE
+    assert lib.svla_set_prefix_weights(None, 8) == _abi.SVLA_ERR_ARG
+    assert lib.svla_prefix_weights(None) == 0
+    # quantiser: K a multiple of 64, aligned pointers
+    assert lib.svla_op_quantize_affine8(p, 96, 4, 96, p, 96, p, None) == _abi.SVLA_ERR_SHAPE
+    assert lib.svla_op_quantize_affine8(None, 64, 4, 64, p, 64, p, None) == _abi.SVLA_ERR_ARG
+    assert lib.svla_op_quantize_affine8(ctypes.c_void_p(18), 64, 4, 64, p, 64, p, None) == _abi.SVLA_ERR_ARG
+    # int8 GEMM: epilogue, K % 64, N % 8, splits <= 8, 16-byte alignment
+    args = lambda **kw: dict(dict(epi=0, lda=64, ldq=64, g=None, M=4, N=8, K=64, ldc=8, sp=0), **kw)
+    def call(a):
+        return lib.svla_op_gemm_w8(a["epi"], p, a["lda"], p, a["ldq"], p, a["g"], a["M"], a["N"], a["K"], p,
+                                   a["ldc"], None, a["sp"], None, None)
+    assert call(args(epi=9)) == _abi.SVLA_ERR_ARG
+    assert call(args(K=96, lda=96, ldq=96)) == _abi.SVLA_ERR_SHAPE
+    assert call(args(N=12, ldc=12)) == _abi.SVLA_ERR_SHAPE
+    assert call(args(sp=9)) == _abi.SVLA_ERR_SHAPE
+    assert call(args(ldq=72)) == _abi.SVLA_ERR_SHAPE
+    assert call(args(g=ctypes.c_void_p(24))) == _abi.SVLA_ERR_ARG
+    # at the batch-1 prefill's shapes the int8 plan splits K like the dense plan
+    # (same partial-sum order); large M takes 128-wide tiles without a split
+    for (M, N, K) in [(177, 1600, 960), (177, 960, 960), (177, 5120, 960), (177, 960, 2560), (354, 960, 2560)]:
+        assert lib.svla_op_gemm_w8_splits(M, N, K) == lib.svla_op_gemm_splits(M, N, K), (M, N, K)
+    assert lib.svla_op_gemm_w8_splits(5664, 5120, 960) == 1
+    assert lib.svla_op_gemm_w8_tile_n(5664, 5120, 960) == 128
+    assert lib.svla_op_gemm_w8_splits(177, 1600, 100) == 0

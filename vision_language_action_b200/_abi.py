@@ -37,6 +37,9 @@ _S = ctypes.c_size_t
 # name -> (restype, argtypes)
 SIGNATURES = {
     "svla_create": (_I, [ctypes.POINTER(SvlaConfig), _P, _S, _I, ctypes.POINTER(_P)]),
+    "svla_create_ex": (_I, [ctypes.POINTER(SvlaConfig), _P, _S, _I, ctypes.c_uint, ctypes.POINTER(_P)]),
+    "svla_set_prefix_weights": (_I, [_P, _I]),
+    "svla_prefix_weights": (_I, [_P]),
     "svla_destroy": (_I, [_P]),
     "svla_kv_cache_bytes": (_S, [_P, _I, _I]),
     "svla_blob_bytes": (_S, [ctypes.POINTER(SvlaConfig)]),
@@ -59,9 +62,14 @@ SIGNATURES = {
     "svla_set_assembly": (_I, [_P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I]),
     "svla_assemble_prefix": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "svla_denoise_fused_supported": (_I, [_P, _I, _I]),
+    "svla_op_quantize_affine8": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
+    "svla_op_gemm_w8": (_I, [_I, _P, _I, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P]),
+    "svla_op_gemm_w8_splits": (_I, [_I, _I, _I]),
+    "svla_op_gemm_w8_tile_n": (_I, [_I, _I, _I]),
 }
 
 DENOISE_AUTO, DENOISE_GRAPH, DENOISE_FUSED = 0, 1, 2
+CREATE_PREFIX_INT8 = 1
 
 _lib = None
 

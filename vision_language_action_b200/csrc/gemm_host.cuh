@@ -6,6 +6,7 @@
 
 #include "gemm_pair.cuh"
 #include "gemm_persistent.cuh"
+#include "gemm_w8.cuh"
 
 namespace svla {
 
@@ -357,6 +358,163 @@ inline cudaError_t set_attrs_inst() {
   return e;
 }
 
+// ---------------------------------------------------------------------------
+// weight-only int8 GEMM (gemm_w8.cuh)
+// ---------------------------------------------------------------------------
+
+// 2-D uint8 tensor [rows, cols] (row stride ld_bytes), box {64, box_rows}, no
+// swizzle (the dequantising threads read it), zero fill outside the tensor.
+inline bool make_tmap_u8(CUtensorMap* m, const void* ptr, int rows, int cols, size_t ld_bytes, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)GEMM_BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The (alpha, beta) pairs [K/64][N][2] bf16 as a 2-D tensor [K/64, 2N]; box
+// {2 box_n, 1}: the pairs of box_n rows for one k-block.
+inline bool make_tmap_pairs(CUtensorMap* m, const void* ptr, int N, int groups, int box_n) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)2 * N, (cuuint64_t)groups};
+  cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+  cuuint32_t box[2] = {(cuuint32_t)(2 * box_n), 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Plan of the int8 GEMM: many tiles -> 128-wide tiles, one split; otherwise
+// the dense kernel's small-M rule (64- or 32-wide tiles, two CTAs per SM, K
+// split over a cluster so that a split keeps >= 3 k-blocks). With the same
+// tile width and splits as the dense plan, the partial sums are added in the
+// same order, so an int8 GEMM equals the dense GEMM on the dequantised weights.
+inline GemmPlan plan_gemm_w8(int M, int N, int K, int forced_splits, int min_bn = 32) {
+  GemmPlan p;
+  const int KB = K / GEMM_BK;
+  p.m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
+  auto tiles = [&](int bn) { return p.m_tiles * ((N + bn - 1) / bn); };
+  auto clamp_splits = [&](int sp) {
+    if (sp > KB) sp = KB;
+    if (sp > GEMM_MAX_CLUSTER) sp = GEMM_MAX_CLUSTER;
+    return sp < 1 ? 1 : sp;
+  };
+  if (forced_splits <= 1 && (p.m_tiles >= 4 || tiles(128) >= 100)) {
+    p.bn = 128;
+    p.stages = 4;
+    p.splits = 1;
+  } else {
+    const int t64 = tiles(64), t32 = tiles(32);
+    auto fit = [&](int t) {
+      int sp = clamp_splits(2 * NUM_SMS_B200 / t);
+      while (sp > 1 && KB / sp < 3) --sp;
+      return sp;
+    };
+    const int s64 = fit(t64), s32 = fit(t32);
+    const int c64 = t64 * s64, c32 = t32 * s32;
+    p.bn = (c64 >= 120 || c64 >= c32 || min_bn > 32) ? 64 : 32;
+    p.stages = p.bn == 64 ? 3 : 4;
+    p.splits = p.bn == 64 ? s64 : s32;
+  }
+  if (forced_splits > 0) p.splits = clamp_splits(forced_splits);
+  p.n_tiles = (N + p.bn - 1) / p.bn;
+  p.red = p.splits > 1 ? GEMM_RED_CLUSTER : GEMM_RED_NONE;
+  return p;
+}
+
+template <int BN, int ST, int EPI>
+inline cudaError_t launch_w8_inst(const CUtensorMap& ta, const CUtensorMap& tq, const CUtensorMap& ts,
+                                  const GemmArgs& args, const uint16_t* gain, dim3 grid, int cluster_z,
+                                  cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = W8Cfg<BN, ST>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  int n = 0;
+  at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_z > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = 1;
+    at[n].val.clusterDim.y = 1;
+    at[n].val.clusterDim.z = (unsigned)cluster_z;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, gemm_w8_kernel<BN, EPI, ST>, ta, tq, ts, args, gain);
+}
+
+template <int BN, int ST>
+inline cudaError_t dispatch_w8(int epi, const CUtensorMap& ta, const CUtensorMap& tq, const CUtensorMap& ts,
+                               const GemmArgs& a, const uint16_t* gain, dim3 g, int cz, cudaStream_t s) {
+  switch (epi) {
+    case GE_F32: return launch_w8_inst<BN, ST, GE_F32>(ta, tq, ts, a, gain, g, cz, s);
+    case GE_BF16: return launch_w8_inst<BN, ST, GE_BF16>(ta, tq, ts, a, gain, g, cz, s);
+    case GE_ADD_F32: return launch_w8_inst<BN, ST, GE_ADD_F32>(ta, tq, ts, a, gain, g, cz, s);
+    case GE_SILU_BF16: return launch_w8_inst<BN, ST, GE_SILU_BF16>(ta, tq, ts, a, gain, g, cz, s);
+    case GE_QKV_ROPE32: return launch_w8_inst<BN, ST, GE_QKV_ROPE32>(ta, tq, ts, a, gain, g, cz, s);
+  }
+  if constexpr (BN % 64 == 0) {
+    if (epi == GE_SWIGLU) return launch_w8_inst<BN, ST, GE_SWIGLU>(ta, tq, ts, a, gain, g, cz, s);
+    if (epi == GE_QKV_ROPE64) return launch_w8_inst<BN, ST, GE_QKV_ROPE64>(ta, tq, ts, a, gain, g, cz, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int BN, int ST>
+inline cudaError_t set_attrs_w8() {
+  const int smem = (int)W8Cfg<BN, ST>::SMEM;
+  cudaError_t e = cudaSuccess;
+#define SVLA_SETW(EPI)                                                                                       \
+  if (e == cudaSuccess)                                                                                      \
+    e = cudaFuncSetAttribute(gemm_w8_kernel<BN, EPI, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  SVLA_SETW(GE_F32)
+  SVLA_SETW(GE_BF16)
+  SVLA_SETW(GE_ADD_F32)
+  SVLA_SETW(GE_SILU_BF16)
+  SVLA_SETW(GE_QKV_ROPE32)
+  if constexpr (BN % 64 == 0) {
+    SVLA_SETW(GE_SWIGLU)
+    SVLA_SETW(GE_QKV_ROPE64)
+  }
+#undef SVLA_SETW
+  return e;
+}
+
+// Full launch of the int8 GEMM. Q: codes [N, K] (row stride ldq bytes); ab:
+// (alpha, beta) pairs [K/64][N][2]; gain: bf16 [K] or null. K % 64 == 0 and
+// N % 4 == 0 (TMA strides), checked by the callers.
+inline cudaError_t run_gemm_w8(int epi, const void* A, int lda, const uint8_t* Q, size_t ldq, const uint16_t* ab,
+                               const uint16_t* gain, int M, int N, int K, GemmArgs args, const GemmPlan& p,
+                               cudaStream_t s) {
+  CUtensorMap ta, tq, ts;
+  if (!make_tmap_bf16(&ta, A, M, K, lda, GEMM_BM)) return cudaErrorInvalidValue;
+  if (!make_tmap_u8(&tq, Q, N, K, ldq, p.bn)) return cudaErrorInvalidValue;
+  if (!make_tmap_pairs(&ts, ab, N, K / W8_GROUP, p.bn)) return cudaErrorInvalidValue;
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.partials = nullptr;
+  args.counters = nullptr;
+  args.red_mode = p.red;
+  const dim3 grid(p.n_tiles, p.m_tiles, p.splits);
+  const int cz = p.red == GEMM_RED_CLUSTER ? p.splits : 1;
+  if (p.bn == 32 && p.stages == 4) return dispatch_w8<32, 4>(epi, ta, tq, ts, args, gain, grid, cz, s);
+  if (p.bn == 64 && p.stages == 3) return dispatch_w8<64, 3>(epi, ta, tq, ts, args, gain, grid, cz, s);
+  if (p.bn == 128 && p.stages == 4) return dispatch_w8<128, 4>(epi, ta, tq, ts, args, gain, grid, cz, s);
+  return cudaErrorInvalidValue;
+}
+
 inline cudaError_t gemm_set_attrs() {
   cudaError_t e = set_attrs_pair<128>();
   if (e == cudaSuccess) e = set_attrs_pair<256>();
@@ -371,6 +529,9 @@ inline cudaError_t gemm_set_attrs() {
   if (e == cudaSuccess) e = set_attrs_inst<64, 4>();
   if (e == cudaSuccess) e = set_attrs_inst<128, 6>();
   if (e == cudaSuccess) e = set_attrs_inst<256, 4>();
+  if (e == cudaSuccess) e = set_attrs_w8<32, 4>();
+  if (e == cudaSuccess) e = set_attrs_w8<64, 3>();
+  if (e == cudaSuccess) e = set_attrs_w8<128, 4>();
   return e;
 }
 

@@ -362,6 +362,115 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, 
 // named barrier over the 4 epilogue warps (ids 2..5)
 SVLA_DEV void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Epilogue warps, accumulator complete: run the epilogue (one split), or hand
+// this split's partial tile to the cluster or global-workspace reduction.
+template <int BN, int EPI, bool CLUSTER_OK>
+SVLA_DEV void gemm_accumulator_out(const GemmArgs& args, uint32_t tmem_base, uint8_t* ring, volatile uint32_t* misc,
+                                   int quad, int row, int m, int n0, bool row_ok, float rscale, int m_blk, int n_blk,
+                                   int split, int splits) {
+  AccSource<BN> src;
+  src.taddr_row = tmem_base + ((uint32_t)(quad * 32) << 16);
+  src.smem_row = nullptr;
+  if (splits == 1) {
+    run_epilogue<BN, EPI>(args, src, m, n0, row_ok, rscale);
+  } else if (CLUSTER_OK && args.red_mode == GEMM_RED_CLUSTER) {
+    // stage this split's partial tile in shared memory (the operand ring is idle)
+    float* red = reinterpret_cast<float*>(ring);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tmem_ld16(src.taddr_row + (uint32_t)c, v);
+      float4* d = reinterpret_cast<float4*>(red + row * (BN + 4) + c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+  } else {
+    const int tile = m_blk * gridDim.x + n_blk;
+    float* tile_part = args.partials + (size_t)tile * splits * GEMM_BM * BN;
+    // 1) this split's partial rows
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tmem_ld16(src.taddr_row + (uint32_t)c, v);
+      if (row_ok) store16_f32(tile_part + ((size_t)split * GEMM_BM + row) * BN + c, v, 16);
+    }
+    __threadfence();
+    epi_bar();
+    if (threadIdx.x == 64) {
+      const int old = atomicAdd(args.counters + tile, 1);
+      misc[4] = (old == splits - 1) ? 1u : 0u;
+    }
+    epi_bar();
+    if (misc[4]) {
+      // 2) last CTA: sum all splits in split order into shared memory (the
+      //    operand ring is idle now), then run the epilogue from there
+      __threadfence();
+      float* red = reinterpret_cast<float*>(ring);
+      const int rows = min(GEMM_BM, args.M - m_blk * GEMM_BM);
+      reduce_partials<BN>(tile_part, splits, rows, red, threadIdx.x - 64);
+      epi_bar();
+      src.smem_row = red + row * (BN + 4);
+      run_epilogue<BN, EPI>(args, src, m, n0, row_ok, rscale);
+      if (threadIdx.x == 64) args.counters[tile] = 0;  // re-arm for the next launch
+    }
+  }
+}
+
+// Cluster split-K tail, run by every thread of every CTA of the cluster after
+// the main loop: CTA r sums rows r, r + S, .. of the peers' staged partial
+// tiles in split order and runs their epilogue.
+template <int BN, int EPI, bool CLUSTER_OK>
+SVLA_DEV void gemm_cluster_reduce(const GemmArgs& args, uint8_t* ring, volatile uint32_t* misc,
+                                  const float* misc_scale, int m_blk, int n_blk, int splits) {
+  if constexpr (CLUSTER_OK) {
+    if (args.red_mode == GEMM_RED_CLUSTER && splits > 1) {
+      // Every thread of every CTA of the cluster reaches both barriers exactly
+      // once, whatever happened before (no early exit exists in this kernel).
+      cluster_sync();
+      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+      if (warp >= 2) {
+        const int t = threadIdx.x - 64;
+        const uint32_t rank = cluster_ctarank();
+        const int rows = min(GEMM_BM, args.M - m_blk * GEMM_BM);
+        float* red = reinterpret_cast<float*>(ring);
+        float* fin = red + GEMM_BM * (BN + 4);
+        const uint32_t red_s = smem_u32(red);
+        constexpr int V4 = BN / 4;
+        const int my_rows = (rows - (int)rank + splits - 1) / splits;
+        for (int item = t; item < my_rows * V4; item += 128) {
+          const int r = (int)rank + splits * (item / V4), c4 = item % V4;
+          const uint32_t off = (uint32_t)((r * (BN + 4) + 4 * c4) * 4);
+          float4 part[GEMM_MAX_CLUSTER];
+#pragma unroll
+          for (int p = 0; p < GEMM_MAX_CLUSTER; ++p)
+            if (p < splits) part[p] = ld_dsmem_f4(dsmem_addr(red_s + off, (uint32_t)p));
+          float4 acc = part[0];
+#pragma unroll
+          for (int p = 1; p < GEMM_MAX_CLUSTER; ++p) {
+            if (p < splits) {
+              acc.x += part[p].x;
+              acc.y += part[p].y;
+              acc.z += part[p].z;
+              acc.w += part[p].w;
+            }
+          }
+          *reinterpret_cast<float4*>(fin + r * (BN + 4) + 4 * c4) = acc;
+        }
+        epi_bar();
+        const int row = (warp & 3) * 32 + lane;
+        const int m = m_blk * GEMM_BM + row;
+        if (misc[1] == 0 && row < rows && row % splits == (int)rank) {
+          AccSource<BN> src;
+          src.taddr_row = 0;
+          src.smem_row = fin + row * (BN + 4);
+          run_epilogue<BN, EPI>(args, src, m, n_blk * BN, true, misc_scale[row]);
+        }
+      }
+      cluster_sync();  // peers have finished reading this CTA's partial tile
+    }
+  }
+}
+
 template <int BN, int EPI, int STAGES, int A_ROWS = GEMM_BM>
 __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES, A_ROWS>::MIN_BLOCKS)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
@@ -490,54 +599,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES, A_ROWS>::MIN
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
     const bool aborted = misc[1] != 0;
-    if (ok && !aborted) {
-      AccSource<BN> src;
-      src.taddr_row = tmem_base + ((uint32_t)(quad * 32) << 16);
-      src.smem_row = nullptr;
-      if (splits == 1) {
-        run_epilogue<BN, EPI>(args, src, m, n0, row_ok, rscale);
-      } else if (C::CLUSTER_OK && args.red_mode == GEMM_RED_CLUSTER) {
-        // stage this split's partial tile in shared memory (the operand ring is idle)
-        float* red = reinterpret_cast<float*>(ring);
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          float v[16];
-          tmem_ld16(src.taddr_row + (uint32_t)c, v);
-          float4* d = reinterpret_cast<float4*>(red + row * (BN + 4) + c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        }
-      } else {
-        const int tile = m_blk * gridDim.x + n_blk;
-        float* tile_part = args.partials + (size_t)tile * splits * GEMM_BM * BN;
-        // 1) this split's partial rows
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          float v[16];
-          tmem_ld16(src.taddr_row + (uint32_t)c, v);
-          if (row_ok) store16_f32(tile_part + ((size_t)split * GEMM_BM + row) * BN + c, v, 16);
-        }
-        __threadfence();
-        epi_bar();
-        if (threadIdx.x == 64) {
-          const int old = atomicAdd(args.counters + tile, 1);
-          misc[4] = (old == splits - 1) ? 1u : 0u;
-        }
-        epi_bar();
-        if (misc[4]) {
-          // 2) last CTA: sum all splits in split order into shared memory (the
-          //    operand ring is idle now), then run the epilogue from there
-          __threadfence();
-          float* red = reinterpret_cast<float*>(ring);
-          const int rows = min(GEMM_BM, args.M - m_blk * GEMM_BM);
-          reduce_partials<BN>(tile_part, splits, rows, red, threadIdx.x - 64);
-          epi_bar();
-          src.smem_row = red + row * (BN + 4);
-          run_epilogue<BN, EPI>(args, src, m, n0, row_ok, rscale);
-          if (threadIdx.x == 64) args.counters[tile] = 0;  // re-arm for the next launch
-        }
-      }
-    }
+    if (ok && !aborted)
+      gemm_accumulator_out<BN, EPI, C::CLUSTER_OK>(args, tmem_base, ring, misc, quad, row, m, n0, row_ok, rscale,
+                                                   m_blk, n_blk, split, splits);
     tc_fence_before();
   }
 
@@ -552,52 +616,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES, A_ROWS>::MIN
     if (threadIdx.x == 32) mbar_wait(acc_bar, 0, GEMM_DRAIN_NS);
     __syncthreads();
   }
-  if constexpr (C::CLUSTER_OK) {
-    if (args.red_mode == GEMM_RED_CLUSTER && splits > 1) {
-      // Every thread of every CTA of the cluster reaches both barriers exactly
-      // once, whatever happened before (no early exit exists in this kernel).
-      cluster_sync();
-      if (warp >= 2) {
-        const int t = threadIdx.x - 64;
-        const uint32_t rank = cluster_ctarank();
-        const int rows = min(GEMM_BM, args.M - m_blk * GEMM_BM);
-        float* red = reinterpret_cast<float*>(ring);
-        float* fin = red + GEMM_BM * (BN + 4);
-        const uint32_t red_s = smem_u32(red);
-        constexpr int V4 = BN / 4;
-        const int my_rows = (rows - (int)rank + splits - 1) / splits;
-        for (int item = t; item < my_rows * V4; item += 128) {
-          const int r = (int)rank + splits * (item / V4), c4 = item % V4;
-          const uint32_t off = (uint32_t)((r * (BN + 4) + 4 * c4) * 4);
-          float4 part[GEMM_MAX_CLUSTER];
-#pragma unroll
-          for (int p = 0; p < GEMM_MAX_CLUSTER; ++p)
-            if (p < splits) part[p] = ld_dsmem_f4(dsmem_addr(red_s + off, (uint32_t)p));
-          float4 acc = part[0];
-#pragma unroll
-          for (int p = 1; p < GEMM_MAX_CLUSTER; ++p) {
-            if (p < splits) {
-              acc.x += part[p].x;
-              acc.y += part[p].y;
-              acc.z += part[p].z;
-              acc.w += part[p].w;
-            }
-          }
-          *reinterpret_cast<float4*>(fin + r * (BN + 4) + 4 * c4) = acc;
-        }
-        epi_bar();
-        const int row = (warp & 3) * 32 + lane;
-        const int m = m_blk * GEMM_BM + row;
-        if (misc[1] == 0 && row < rows && row % splits == (int)rank) {
-          AccSource<BN> src;
-          src.taddr_row = 0;
-          src.smem_row = fin + row * (BN + 4);
-          run_epilogue<BN, EPI>(args, src, m, n_blk * BN, true, misc_scale[row]);
-        }
-      }
-      cluster_sync();  // peers have finished reading this CTA's partial tile
-    }
-  }
+  gemm_cluster_reduce<BN, EPI, C::CLUSTER_OK>(args, ring, misc, misc_scale, m_blk, n_blk, splits);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);

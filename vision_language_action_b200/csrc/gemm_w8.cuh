@@ -1,0 +1,325 @@
+// Weight-only int8 GEMM on the tcgen05 tensor cores, and the quantiser that
+// produces its weights (the vlm-8bit preset of the mlx-smolvla PyPI page,
+// §Run a checkpoint: the prefix LM's projections in 8 bits, activations bf16).
+//
+//   C[M, N] = A[M, K] · W^[N, K]^T,   W^[n, k] = bf16(bf16(alpha q + beta) * g[k])
+//
+// Quantisation: affine groups of 64 consecutive input weights of one output
+// row; per group lo = min, hi = max, alpha = bf16((hi - lo) / 255), beta = lo,
+// code q = clamp(rint((w - beta) / alpha), 0, 255), every step an IEEE fp32
+// operation rounded to nearest even. g is the RMSNorm gain folded into a
+// projection that consumes normalised activations (1 where there is none), so
+// the operand equals the dense path's folded weight computed from W^.
+//
+// Storage: codes uint8 [N, K] row-major; (alpha, beta) as bf16 pairs in a
+// group-major array [K/64][N][2], so the pairs of one k-block of a tile are
+// one contiguous TMA box.
+//
+// CTA (same roles as the dense kernel, one more stage of work):
+//   warp 0      : TMA producer: A (bf16, 128-byte swizzle), the int8 code tile
+//                 [BN][64] and its BN (alpha, beta) pairs, into a ring.
+//   warp 1      : TMEM allocation; one lane issues tcgen05.mma (kind::f16) on
+//                 A and the dequantised tile, commits each stage.
+//   warps 2..5  : during the main loop they dequantise each stage's codes into
+//                 a bf16 tile in the 128-byte-swizzled K-major layout that TMA
+//                 would have written, then (after the loop) run the epilogue.
+// The int8 tiles arrive on their own barrier, so the dequantisation of the
+// first stages overlaps the wait for the producer kernel of A.
+#pragma once
+
+#include "gemm_tc.cuh"
+
+namespace svla {
+
+constexpr int W8_GROUP = 64;  // = GEMM_BK: one (alpha, beta) pair per row and k-block
+
+template <int BN, int STAGES_>
+struct W8Cfg {
+  static constexpr int STAGES = STAGES_;
+  static constexpr uint32_t A_BYTES = GEMM_BM * GEMM_BK * 2;
+  static constexpr uint32_t B_BYTES = BN * GEMM_BK * 2;  // dequantised tile (bf16)
+  static constexpr uint32_t Q_BYTES = BN * GEMM_BK;      // codes
+  static constexpr uint32_t S_BYTES = BN * 4;            // (alpha, beta) pairs
+  static constexpr uint32_t STAGE_BYTES = (A_BYTES + B_BYTES + Q_BYTES + S_BYTES + 1023) / 1024 * 1024;
+  static constexpr uint32_t RING_BYTES = STAGES * STAGE_BYTES;
+  static constexpr uint32_t TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
+  // ring + barriers/flags (512 B) + row factors (512 B) + alignment slack
+  static constexpr size_t SMEM = (size_t)RING_BYTES + 1024 + 1024;
+  static constexpr int MIN_BLOCKS = SMEM <= 113 * 1024 ? 2 : 1;
+  static constexpr size_t RED_TILE = (size_t)GEMM_BM * (BN + 4) * sizeof(float);
+  static constexpr bool CLUSTER_OK = 2 * RED_TILE <= (size_t)RING_BYTES;
+  static_assert(BN % 32 == 0 && BN <= 128, "the (alpha, beta) box holds at most 256 bf16");
+  static_assert(4 * STAGES + 1 <= 60, "barriers and flags share 512 bytes");
+  static_assert(CLUSTER_OK, "split-K of the int8 GEMM reduces over a cluster only");
+};
+
+SVLA_DEV void fence_proxy_async_cta() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+SVLA_DEV float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// Code byte j of the word as a float: 2^23 + q assembled in the bits, minus 2^23.
+template <int J>
+SVLA_DEV float code_f(uint32_t word) {
+  return __uint_as_float(__byte_perm(word, 0x4B000000u, 0x7540u + J)) - 8388608.f;
+}
+
+// 16 codes (one 16-byte chunk of a row) -> 16 operand values, packed bf16x2.
+SVLA_DEV void dequant16(uint4 qv, float al, float be, const float (&g)[16], bool has_gain, uint32_t (&out)[8]) {
+  const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float v[4] = {fmaf(al, code_f<0>(w[i]), be), fmaf(al, code_f<1>(w[i]), be), fmaf(al, code_f<2>(w[i]), be),
+                  fmaf(al, code_f<3>(w[i]), be)};
+    if (has_gain) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = bf16_round(v[j]) * g[4 * i + j];
+    }
+    out[2 * i] = pack_bf16x2(v[0], v[1]);
+    out[2 * i + 1] = pack_bf16x2(v[2], v[3]);
+  }
+}
+
+template <int BN, int EPI, int STAGES>
+__global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
+    gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
+                   const __grid_constant__ CUtensorMap tmS, const GemmArgs args, const uint16_t* __restrict__ gain) {
+  using C = W8Cfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES);
+  // bars[0..S) A full, [S..2S) codes full, [2S..3S) dequantised, [3S..4S) empty, [4S] accumulator
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(bars + 4 * STAGES + 1);
+  // misc[0] tmem base, misc[1] abort flag, misc[2] stages issued, misc[3] stages consumed,
+  // misc[4] "this CTA reduces"
+  float* misc_scale = reinterpret_cast<float*>(smem + C::RING_BYTES + 512);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_blk = blockIdx.x, m_blk = blockIdx.y, split = blockIdx.z, splits = gridDim.z;
+  const int KB = args.K / GEMM_BK;
+  const int kb0 = (int)(((long long)split * KB) / splits);
+  const int kb1 = (int)(((long long)(split + 1) * KB) / splits);
+  const int nkb = kb1 - kb0;
+
+  auto a_full = [&](int s) { return smem_u32(bars + s); };
+  auto q_full = [&](int s) { return smem_u32(bars + STAGES + s); };
+  auto deq_bar = [&](int s) { return smem_u32(bars + 2 * STAGES + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + 3 * STAGES + s); };
+  const uint32_t acc_bar = smem_u32(bars + 4 * STAGES);
+  auto stage = [&](int s) { return ring + (size_t)s * C::STAGE_BYTES; };
+
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(a_full(s), 1);
+      mbar_init(q_full(s), 1);
+      mbar_init(deq_bar(s), 128);  // every dequantising thread arrives
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(acc_bar, 1);
+    misc[1] = 0;
+    misc[2] = 0;
+    misc[3] = 0;
+    misc[4] = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmS);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)&misc[0]), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = misc[0];
+  const unsigned long long lim = args.wait_ns;
+  const int n0 = n_blk * BN;
+
+  auto issue_codes = [&](int i) {
+    const int s = i % STAGES;
+    uint8_t* st = stage(s);
+    mbar_arrive_expect_tx(q_full(s), C::Q_BYTES + C::S_BYTES);
+    tma_load_2d(smem_u32(st + C::A_BYTES + C::B_BYTES), &tmQ, q_full(s), (kb0 + i) * GEMM_BK, n0);
+    tma_load_2d(smem_u32(st + C::A_BYTES + C::B_BYTES + C::Q_BYTES), &tmS, q_full(s), 2 * n0, kb0 + i);
+  };
+  auto issue_a = [&](int i) {
+    const int s = i % STAGES;
+    mbar_arrive_expect_tx(a_full(s), C::A_BYTES);
+    tma_load_2d(smem_u32(stage(s)), &tmA, a_full(s), (kb0 + i) * GEMM_BK, m_blk * GEMM_BM);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // the weights do not depend on earlier kernels: the first stages' codes
+      // are requested before waiting for the producer of A
+      const int pre = nkb < STAGES ? nkb : STAGES;
+      for (int i = 0; i < pre; ++i) issue_codes(i);
+      griddep_wait();
+      for (int i = 0; i < pre; ++i) issue_a(i);
+      misc[2] = pre;
+      for (int i = pre; i < nkb; ++i) {
+        if (misc[1]) break;
+        const int s = i % STAGES;
+        if (!mbar_wait(empty_bar(s), ((uint32_t)(i / STAGES) & 1u) ^ 1u, lim)) {
+          misc[1] = 1;
+          set_status(args.status, SVLA_ERR_TIMEOUT);
+          break;
+        }
+        issue_codes(i);
+        issue_a(i);
+        misc[2] = i + 1;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, BN);
+      for (int i = 0; i < nkb; ++i) {
+        if (misc[1]) break;
+        const int s = i % STAGES;
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+        if (!mbar_wait(a_full(s), ph, lim) || !mbar_wait(deq_bar(s), ph, lim)) {
+          misc[1] = 1;
+          set_status(args.status, SVLA_ERR_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(stage(s));
+        const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+        for (int k = 0; k < GEMM_BK / 16; ++k) {
+          tc_mma_bf16(tmem_base, smem_desc_sw128(sa + 32 * k), smem_desc_sw128(sb + 32 * k), IDESC,
+                      (i > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit(empty_bar(s));
+        misc[3] = i + 1;
+      }
+      tc_commit(acc_bar);  // always: lets waiters know every issued MMA finished
+    }
+  } else {
+    // ---------------- dequantisation (main loop), then the epilogue ----------------
+    const int t = threadIdx.x - 64;
+    for (int i = 0; i < nkb; ++i) {
+      if (misc[1]) break;
+      const int s = i % STAGES;
+      if (!mbar_wait(q_full(s), (uint32_t)(i / STAGES) & 1u, lim)) {
+        misc[1] = 1;
+        set_status(args.status, SVLA_ERR_TIMEOUT);
+        break;
+      }
+      uint8_t* st = stage(s);
+      const uint8_t* qs = st + C::A_BYTES + C::B_BYTES;
+      const uint32_t* ps = reinterpret_cast<const uint32_t*>(st + C::A_BYTES + C::B_BYTES + C::Q_BYTES);
+      uint8_t* bs = st + C::A_BYTES;
+      const int k0 = (kb0 + i) * GEMM_BK;
+      // item = (row r, 16-code chunk c): 16 operand values = logical 16-byte
+      // chunks 2c, 2c + 1 of the row's 128 bytes, stored at chunk ^ (r % 8)
+      for (int item = t; item < BN * 4; item += 128) {
+        const int r = item >> 2, c = item & 3;
+        const uint4 qv = *reinterpret_cast<const uint4*>(qs + r * GEMM_BK + 16 * c);
+        const uint32_t ab = ps[r];
+        const float al = bf2f((uint16_t)(ab & 0xFFFFu)), be = bf2f((uint16_t)(ab >> 16));
+        float g[16];
+        if (gain) {
+          const uint4* gp = reinterpret_cast<const uint4*>(gain + k0 + 16 * c);
+          const uint4 g0 = __ldg(gp), g1 = __ldg(gp + 1);
+          const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            g[2 * j] = bf2f((uint16_t)(gw[j] & 0xFFFFu));
+            g[2 * j + 1] = bf2f((uint16_t)(gw[j] >> 16));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) g[j] = 1.f;
+        }
+        uint32_t o[8];
+        dequant16(qv, al, be, g, gain != nullptr, o);
+        uint8_t* row = bs + r * 128;
+        const int sw = r & 7;
+        *reinterpret_cast<uint4*>(row + (((2 * c) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+      fence_proxy_async_cta();  // generic stores -> visible to the tensor cores' async proxy
+      mbar_arrive(deq_bar(s));
+    }
+    griddep_wait();  // outputs, residuals, biases and positions come from earlier kernels
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int m = m_blk * GEMM_BM + row;
+    const bool row_ok = m < args.M;
+    prefetch_epilogue_inputs<BN, EPI>(args, m, n0, row_ok);
+    const float rscale = norm_row_scale(args, m, row_ok);
+    misc_scale[row] = rscale;
+    bool ok = mbar_wait(acc_bar, 0, lim);
+    if (!ok) {
+      misc[1] = 1;
+      set_status(args.status, SVLA_ERR_TIMEOUT);
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    const bool aborted = misc[1] != 0;
+    if (ok && !aborted)
+      gemm_accumulator_out<BN, EPI, C::CLUSTER_OK>(args, tmem_base, ring, misc, quad, row, m, n0, row_ok, rscale,
+                                                   m_blk, n_blk, split, splits);
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (misc[1]) {
+    // time-out path: let every issued TMA copy land and every MMA finish
+    if (threadIdx.x == 0) {
+      const int issued = (int)misc[2], consumed = (int)misc[3];
+      for (int i = consumed; i < issued; ++i) {
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+        mbar_wait(a_full(i % STAGES), ph, GEMM_DRAIN_NS);
+        mbar_wait(q_full(i % STAGES), ph, GEMM_DRAIN_NS);
+      }
+    }
+    if (threadIdx.x == 32) mbar_wait(acc_bar, 0, GEMM_DRAIN_NS);
+    __syncthreads();
+  }
+  gemm_cluster_reduce<BN, EPI, C::CLUSTER_OK>(args, ring, misc, misc_scale, m_blk, n_blk, splits);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// One warp per (row n, group g): lanes hold inputs 2 lane, 2 lane + 1 of the group.
+//   W: bf16 [N, K] (row stride ldw, even); q: uint8 [N, K] (row stride ldq);
+//   ab: bf16 pairs [K/64][N][2].
+__global__ void __launch_bounds__(256) quantize_affine8_kernel(const uint16_t* __restrict__ W, size_t ldw, int N,
+                                                               int K, uint8_t* __restrict__ q, size_t ldq,
+                                                               uint16_t* __restrict__ ab) {
+  const int G = K / W8_GROUP;
+  const long long wid = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= (long long)N * G) return;  // whole warps exit together
+  const int n = (int)(wid / G), g = (int)(wid % G);
+  const uint32_t v = *reinterpret_cast<const uint32_t*>(W + (size_t)n * ldw + (size_t)g * W8_GROUP + 2 * lane);
+  const float w0 = bf2f((uint16_t)(v & 0xFFFFu)), w1 = bf2f((uint16_t)(v >> 16));
+  float lo = fminf(w0, w1), hi = fmaxf(w0, w1);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  const float al = bf16_round(__fdiv_rn(__fsub_rn(hi, lo), 255.f));
+  auto code = [&](float w) -> uint32_t {
+    if (!(al > 0.f)) return 0u;
+    const float c = rintf(__fdiv_rn(__fsub_rn(w, lo), al));
+    return (uint32_t)fminf(fmaxf(c, 0.f), 255.f);
+  };
+  const uint32_t c0 = code(w0), c1 = code(w1);
+  *reinterpret_cast<uint16_t*>(q + (size_t)n * ldq + (size_t)g * W8_GROUP + 2 * lane) = (uint16_t)(c0 | (c1 << 8));
+  if (lane == 0) {
+    const __nv_bfloat16 a = __float2bfloat16_rn(al), b = __float2bfloat16_rn(lo);
+    ab[((size_t)g * N + n) * 2] = *reinterpret_cast<const uint16_t*>(&a);
+    ab[((size_t)g * N + n) * 2 + 1] = *reinterpret_cast<const uint16_t*>(&b);
+  }
+}
+
+}  // namespace svla

@@ -220,6 +220,13 @@ __global__ void pad_rows_kernel(const uint16_t* __restrict__ src, size_t src_ld,
   }
 }
 
+// One int8 prefix projection: codes [N, K] at q_off, (alpha, beta) pairs
+// [K/64][N][2] bf16 at ab_off (byte offsets into the handle's int8 buffer).
+struct Q8Mat {
+  size_t q_off = 0, ab_off = 0;
+  int N = 0, K = 0;
+};
+
 struct GraphEntry {
   std::vector<uint64_t> key;
   cudaGraphExec_t exec = nullptr;
@@ -257,6 +264,10 @@ struct svla_handle {
   uint16_t* fw = nullptr;       // persistent denoise: expert GEMM weights with row pitch K + 8
   FusedWeights fwl;
   int denoise_path = SVLA_DENOISE_AUTO;
+  // weight-only int8 prefix (svla_create_ex with SVLA_CREATE_PREFIX_INT8)
+  uint8_t* q8 = nullptr;     // codes and (alpha, beta) pairs of the prefix projections
+  std::vector<Q8Mat> q8m;    // per prefix layer: QKV, O, gate/up (interleaved rows), down
+  int prefix_bits = 16;      // weights svla_prefill uses
   // prefix assembly (svla_set_assembly): connector and state-projection weights, workspaces
   uint16_t* asm_w = nullptr;   // W_c [p_width, r*r*C] | W_s [p_width, S] | b_s [p_width]
   uint16_t* asm_a = nullptr;   // gathered connector operand [max_batch * max_images * tpi, r*r*C]
@@ -348,6 +359,16 @@ cudaError_t gemm(svla_handle* h, int epi, const bf16* A, int lda, const bf16* W,
   return run_gemm(epi, A, lda, W, ldw, M, N, K, args, p, part, cnt, s);
 }
 
+// one GEMM of the prefill on the int8 weights (gain: the folded RMSNorm gain, or null)
+cudaError_t gemm8(svla_handle* h, int epi, const bf16* A, int lda, const Q8Mat& w, const uint16_t* gain, int M,
+                  GemmArgs args, cudaStream_t s) {
+  GemmPlan p = plan_gemm_w8(M, w.N, w.K, 0, gemm_min_bn(epi));
+  args.status = h->status;
+  args.wait_ns = g_wait_ns.load();
+  return run_gemm_w8(epi, A, lda, h->q8 + w.q_off, (size_t)w.K, reinterpret_cast<const uint16_t*>(h->q8 + w.ab_off),
+                     gain, M, w.N, w.K, args, p, s);
+}
+
 GemmArgs out_args(void* out, int ldo, const float* bias = nullptr) {
   GemmArgs a;
   memset(&a, 0, sizeof(a));
@@ -434,9 +455,17 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
   SVLA_TRY(launch_pdl(positions_kernel, dim3((B + 7) / 8), dim3(256), 0, s, pad, B, L, h->p_pos, h->status));
   SVLA_TRY(launch_pdl(residual_init_kernel, dim3((M + 7) / 8), dim3(256), 0, s,
                       reinterpret_cast<const uint16_t*>(embeds), h->p_x, h->p_ss, M, D));
-  const int o_tiles = residual_tiles(M, D, qw), d_tiles = residual_tiles(M, D, c.p_ffn);
+  const bool q8 = h->prefix_bits == 8;
+  // n-tiles of the residual-producing GEMMs = the norm statistics' tiles
+  auto res_tiles = [&](int N, int K) {
+    return q8 ? plan_gemm_w8(M, N, K, 0, gemm_min_bn(GE_ADD_F32)).n_tiles : residual_tiles(M, N, K);
+  };
+  const int o_tiles = res_tiles(D, qw), d_tiles = res_tiles(D, c.p_ffn);
   for (int l = 0; l < c.p_layers; ++l) {
     const Entry* e = &h->lay.p[9 * l];
+    const Q8Mat* qm = q8 ? &h->q8m[4 * l] : nullptr;
+    const uint16_t* in_gain = h->w + e[0].off;
+    const uint16_t* post_gain = h->w + e[5].off;
     bf16* Kl = cache + (size_t)l * layer_elems;
     bf16* Vl = cache + (size_t)(c.p_layers + l) * layer_elems;
     // QKV of RMSNorm(x): the residual's bf16 copy (the embeddings themselves on layer 0)
@@ -453,19 +482,24 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
     qa.rope_cs = h->rope_cs;
     norm_consumer(qa, h->p_ss, l == 0 ? 1 : d_tiles, M, D, c.rms_eps);
     const bf16* xin = l == 0 ? reinterpret_cast<const bf16*>(embeds) : rb;
-    SVLA_TRY(gemm(h, hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32, xin, D, h->W(e[1].off), D, M, qw + 2 * kvw, D, qa,
-                  h->p_part, h->p_cnt, s));
+    const int qkv_epi = hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32;
+    SVLA_TRY(q8 ? gemm8(h, qkv_epi, xin, D, qm[0], in_gain, M, qa, s)
+                : gemm(h, qkv_epi, xin, D, h->W(e[1].off), D, M, qw + 2 * kvw, D, qa, h->p_part, h->p_cnt, s));
     if (l == c.p_layers - 1) break;  // nothing reads the last layer's attention / MLP output
     SVLA_TRY(attention(h->p_q, qw, Kl, Vl, kvw, pad, B, c.p_heads, c.p_kv_heads, hd, L, L, 0, h->p_o, qw, s));
     GemmArgs oa = out_args(h->p_x, D);
     norm_producer(oa, rb, D, h->p_ss, M);
-    SVLA_TRY(gemm(h, GE_ADD_F32, h->p_o, qw, h->W(e[4].off), qw, M, D, qw, oa, h->p_part, h->p_cnt, s));
+    SVLA_TRY(q8 ? gemm8(h, GE_ADD_F32, h->p_o, qw, qm[1], nullptr, M, oa, s)
+                : gemm(h, GE_ADD_F32, h->p_o, qw, h->W(e[4].off), qw, M, D, qw, oa, h->p_part, h->p_cnt, s));
     GemmArgs ga = out_args(h->p_h, c.p_ffn);
     norm_consumer(ga, h->p_ss, o_tiles, M, D, c.rms_eps);
-    SVLA_TRY(gemm(h, GE_SWIGLU, rb, D, h->W(e[6].off), D, M, 2 * c.p_ffn, D, ga, h->p_part, h->p_cnt, s));
+    SVLA_TRY(q8 ? gemm8(h, GE_SWIGLU, rb, D, qm[2], post_gain, M, ga, s)
+                : gemm(h, GE_SWIGLU, rb, D, h->W(e[6].off), D, M, 2 * c.p_ffn, D, ga, h->p_part, h->p_cnt, s));
     GemmArgs da = out_args(h->p_x, D);
     norm_producer(da, rb, D, h->p_ss, M);
-    SVLA_TRY(gemm(h, GE_ADD_F32, h->p_h, c.p_ffn, h->W(e[8].off), c.p_ffn, M, D, c.p_ffn, da, h->p_part, h->p_cnt, s));
+    SVLA_TRY(q8 ? gemm8(h, GE_ADD_F32, h->p_h, c.p_ffn, qm[3], nullptr, M, da, s)
+                : gemm(h, GE_ADD_F32, h->p_h, c.p_ffn, h->W(e[8].off), c.p_ffn, M, D, c.p_ffn, da, h->p_part,
+                       h->p_cnt, s));
   }
   return cudaSuccess;
 }
@@ -793,8 +827,16 @@ size_t svla_blob_bytes(const svla_config* cfg) {
 }
 
 svla_status svla_create(const svla_config* cfg, const void* blob, size_t blob_bytes, int device, svla_handle** out) {
+  return svla_create_ex(cfg, blob, blob_bytes, device, 0u, out);
+}
+
+svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob_bytes, int device, unsigned flags,
+                           svla_handle** out) {
   if (out) *out = nullptr;
   if (!cfg || !blob || !out) return fail(nullptr, SVLA_ERR_ARG, "null argument");
+  if (flags & ~SVLA_CREATE_PREFIX_INT8) return fail(nullptr, SVLA_ERR_ARG, "unknown flag bits");
+  if ((flags & SVLA_CREATE_PREFIX_INT8) && (cfg->p_heads * cfg->head_dim) % 64)
+    return fail(nullptr, SVLA_ERR_SHAPE, "int8 prefix weights need p_heads * head_dim to be a multiple of 64");
   if (const char* why = check_config(*cfg)) return fail(nullptr, SVLA_ERR_SHAPE, why);
   Layout lay = make_layout(*cfg);
   if (blob_bytes != lay.total * 2)
@@ -840,6 +882,44 @@ svla_status svla_create(const svla_config* cfg, const void* blob, size_t blob_by
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     cudaFree(tmp);
     if (e != cudaSuccess) return bail(e, "gate/up layout");
+  }
+  // vlm-8bit: quantise the prefix projections (gate/up already interleaved)
+  // before the gains are folded into the dense copy
+  if (flags & SVLA_CREATE_PREFIX_INT8) {
+    size_t off = 0;
+    auto add = [&](int N, int K) {
+      Q8Mat m;
+      m.N = N;
+      m.K = K;
+      m.q_off = off;
+      off += ((size_t)N * K + 255) / 256 * 256;
+      m.ab_off = off;
+      off += ((size_t)N * (K / W8_GROUP) * 4 + 255) / 256 * 256;
+      return m;
+    };
+    const int D = c.p_width, qw = c.p_heads * c.head_dim, kvw = c.p_kv_heads * c.head_dim;
+    for (int l = 0; l < c.p_layers; ++l) {
+      h->q8m.push_back(add(qw + 2 * kvw, D));
+      h->q8m.push_back(add(D, qw));
+      h->q8m.push_back(add(2 * c.p_ffn, D));
+      h->q8m.push_back(add(D, c.p_ffn));
+    }
+    if ((e = halloc(h, &h->q8, off)) != cudaSuccess) return bail(e, "int8 weights");
+    for (int l = 0; l < c.p_layers && e == cudaSuccess; ++l) {
+      const Entry* en = &lay.p[9 * l];
+      const size_t src[4] = {en[1].off, en[4].off, en[6].off, en[8].off};
+      for (int i = 0; i < 4 && e == cudaSuccess; ++i) {
+        const Q8Mat& m = h->q8m[4 * l + i];
+        const long long warps = (long long)m.N * (m.K / W8_GROUP);
+        quantize_affine8_kernel<<<(unsigned)((warps + 7) / 8), 256>>>(
+            h->w + src[i], (size_t)m.K, m.N, m.K, h->q8 + m.q_off, (size_t)m.K,
+            reinterpret_cast<uint16_t*>(h->q8 + m.ab_off));
+        e = cudaGetLastError();
+      }
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return bail(e, "int8 quantisation");
+    h->prefix_bits = 8;
   }
   // fold the RMSNorm gains into the projections that consume the normalised
   // activations: QKV (in_norm) and gate/up (post_norm) of every layer, and the
@@ -978,7 +1058,7 @@ svla_status svla_prefill(svla_handle* h, const void* embeds, const uint8_t* pad,
   DeviceGuard dg(h->device);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   std::vector<uint64_t> key = {1, (uint64_t)B, (uint64_t)L, (uint64_t)(uintptr_t)embeds, (uint64_t)(uintptr_t)pad,
-                               (uint64_t)(uintptr_t)kv, g_wait_ns.load()};
+                               (uint64_t)(uintptr_t)kv, g_wait_ns.load(), (uint64_t)h->prefix_bits};
   return run_graph(h, key, [&](cudaStream_t cs) { return record_prefill(h, embeds, pad, B, L, kv, cs); }, s,
                    "prefill");
 }
@@ -1056,6 +1136,17 @@ svla_status svla_set_denoise_path(svla_handle* h, int path) {
   h->denoise_path = path;
   return SVLA_OK;
 }
+
+svla_status svla_set_prefix_weights(svla_handle* h, int bits) {
+  if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
+  if (bits != 16 && bits != 8) return fail(h, SVLA_ERR_ARG, "bits must be 16 or 8");
+  if (bits == 8 && !h->q8)
+    return fail(h, SVLA_ERR_UNSUPPORTED, "the handle has no int8 prefix weights (create it with SVLA_CREATE_PREFIX_INT8)");
+  h->prefix_bits = bits;
+  return SVLA_OK;
+}
+
+int svla_prefix_weights(const svla_handle* h) { return h ? h->prefix_bits : 0; }
 
 int svla_denoise_fused_supported(const svla_handle* h, int B, int H) {
   return h && fused_ok(h, B, H, h->cfg.max_prefix) ? 1 : 0;
@@ -1199,6 +1290,56 @@ svla_status svla_op_gemm(int epilogue, const void* A, int lda, const void* W, in
   a.wait_ns = g_wait_ns.load();
   cudaError_t e = run_gemm(epi, A, lda, W, ldw, M, N, K, a, p, part, cnt, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(nullptr, e, "gemm launch");
+  return SVLA_OK;
+}
+
+svla_status svla_op_quantize_affine8(const void* W, int ldw, int N, int K, void* q, int ldq, void* ab, void* stream) {
+  if (!W || !q || !ab) return fail(nullptr, SVLA_ERR_ARG, "null pointer");
+  if (N < 1 || K < W8_GROUP || K % W8_GROUP || ldw < K || ldq < K || ldw % 2 || ldq % 2)
+    return fail(nullptr, SVLA_ERR_SHAPE, "bad sizes or strides (K a multiple of 64, even strides)");
+  if ((uintptr_t)W & 3 || (uintptr_t)q & 1 || (uintptr_t)ab & 3)
+    return fail(nullptr, SVLA_ERR_ARG, "W and ab must be 4-byte aligned, q 2-byte aligned");
+  const long long warps = (long long)N * (K / W8_GROUP);
+  quantize_affine8_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint16_t*>(W), (size_t)ldw, N, K, reinterpret_cast<uint8_t*>(q), (size_t)ldq,
+      reinterpret_cast<uint16_t*>(ab));
+  if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return cuda_fail(nullptr, e, "quantize launch");
+  return SVLA_OK;
+}
+
+int svla_op_gemm_w8_splits(int M, int N, int K) {
+  if (M < 1 || N < 1 || K < W8_GROUP || K % W8_GROUP) return 0;
+  return plan_gemm_w8(M, N, K, 0).splits;
+}
+
+int svla_op_gemm_w8_tile_n(int M, int N, int K) {
+  if (M < 1 || N < 1 || K < W8_GROUP || K % W8_GROUP) return 0;
+  return plan_gemm_w8(M, N, K, 0).bn;
+}
+
+svla_status svla_op_gemm_w8(int epilogue, const void* A, int lda, const void* q, int ldq, const void* ab,
+                            const void* gain, int M, int N, int K, void* C, int ldc, const float* bias, int splits,
+                            int* status, void* stream) {
+  const int epi = epi_code(epilogue);
+  if (epi < 0) return fail(nullptr, SVLA_ERR_ARG, "unknown epilogue");
+  if (!A || !q || !ab || !C) return fail(nullptr, SVLA_ERR_ARG, "null pointer");
+  if (M < 1 || N < 8 || N % 8 || K < W8_GROUP || K % W8_GROUP || splits < 0 || splits > GEMM_MAX_CLUSTER ||
+      lda < K || lda % 8 || ldq < K || ldq % 16 || ldc < N || (epi != GE_F32 && epi != GE_ADD_F32 ? ldc % 8 : ldc % 4))
+    return fail(nullptr, SVLA_ERR_SHAPE, "bad sizes or strides");
+  if (((uintptr_t)A | (uintptr_t)q | (uintptr_t)ab | (uintptr_t)C | (uintptr_t)gain) & 15)
+    return fail(nullptr, SVLA_ERR_ARG, "pointers must be 16-byte aligned");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!device_is_sm100(dev)) return fail(nullptr, SVLA_ERR_UNSUPPORTED, "device is not sm_100 (B200)");
+  if (cudaError_t e = ensure_attrs(dev); e != cudaSuccess) return cuda_fail(nullptr, e, "kernel attributes");
+  GemmPlan p = plan_gemm_w8(M, N, K, splits);
+  GemmArgs a = out_args(C, ldc, bias);
+  a.status = status;
+  a.wait_ns = g_wait_ns.load();
+  cudaError_t e = run_gemm_w8(epi, A, lda, reinterpret_cast<const uint8_t*>(q), (size_t)ldq,
+                              reinterpret_cast<const uint16_t*>(ab), reinterpret_cast<const uint16_t*>(gain), M, N, K,
+                              a, p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(nullptr, e, "gemm_w8 launch");
   return SVLA_OK;
 }
 

@@ -44,10 +44,12 @@ class SmolVLA:
 
     ``blob`` is the flat bf16 weight blob in manifest order, as a numpy uint16
     array, a torch uint16/bfloat16 tensor (host or CUDA), or raw bytes.
+    ``prefix_int8`` builds the weight-only int8 copy of the prefix LM's
+    projections (the vlm-8bit preset) and selects it for the prefill.
     """
 
     def __init__(self, shape, blob, max_batch: int, max_prefix: int, max_chunk: int,
-                 device: int = 0):
+                 device: int = 0, prefix_int8: bool = False):
         self.lib = _abi.load()
         self.cfg = config_from_shape(shape, max_batch, max_prefix, max_chunk)
         self.action_dim = shape.action_dim
@@ -62,8 +64,9 @@ class SmolVLA:
             ptr, nbytes = arr.ctypes.data, arr.nbytes
             self._blob_keep = arr
         h = ctypes.c_void_p()
-        st = self.lib.svla_create(ctypes.byref(self.cfg), ctypes.c_void_p(ptr), nbytes, device,
-                                  ctypes.byref(h))
+        flags = _abi.CREATE_PREFIX_INT8 if prefix_int8 else 0
+        st = self.lib.svla_create_ex(ctypes.byref(self.cfg), ctypes.c_void_p(ptr), nbytes, device, flags,
+                                     ctypes.byref(h))
         self._blob_keep = None
         _abi.check(st, None)
         self.h = h
@@ -177,6 +180,14 @@ class SmolVLA:
     def set_denoise_path(self, path: int) -> None:
         """_abi.DENOISE_AUTO (default), DENOISE_GRAPH or DENOISE_FUSED."""
         _abi.check(self.lib.svla_set_denoise_path(self.h, path), self.h)
+
+    def set_prefix_weights(self, bits: int) -> None:
+        """16 = dense bf16 prefix weights, 8 = the int8 copy (needs prefix_int8=True)."""
+        _abi.check(self.lib.svla_set_prefix_weights(self.h, bits), self.h)
+
+    @property
+    def prefix_weights(self) -> int:
+        return int(self.lib.svla_prefix_weights(self.h))
 
     def fused_supported(self, B: int, H: int) -> bool:
         return bool(self.lib.svla_denoise_fused_supported(self.h, B, H))
