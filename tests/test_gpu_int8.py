@@ -261,18 +261,22 @@ def test_int8_prefill_and_chunk_match_oracle(wl_name, queries):
         m.close()
 
 
-def test_int8_prefill_bitwise_equals_dense_prefill_on_dequantised_blob():
-    """At batch 1 every int8 GEMM takes the dense GEMM's plan, and its operand is
-    exactly the dense path's folded weight computed from w^: the K/V caches agree
-    bit for bit. Switching the int8 handle back to its dense weights reproduces
-    the dense handle given the original blob."""
-    wl = synth.WORKLOADS["smolvla_b1"]
-    s, _, blob = H.weights("smolvla_b1")
-    _, blob_q = dequantised_model("smolvla_b1")
-    embeds, valid, _ = device_inputs("smolvla_b1", 1)
-    m8 = SmolVLA(s, blob, max_batch=1, max_prefix=wl.L, max_chunk=wl.H, prefix_int8=True)
-    mq = SmolVLA(s, blob_q, max_batch=1, max_prefix=wl.L, max_chunk=wl.H)
-    md = SmolVLA(s, blob, max_batch=1, max_prefix=wl.L, max_chunk=wl.H)
+@pytest.mark.parametrize("wl_name", ["smolvla_b1", "smolvla_b32"])
+def test_int8_prefill_bitwise_equals_dense_prefill_on_dequantised_blob(wl_name):
+    """Batch 1: every int8 GEMM is the fused kernel with the dense GEMM's plan;
+    batch 32: every projection is dequantised into a buffer and the dense GEMM
+    runs on it. Either way the operand is exactly the dense path's folded weight
+    computed from w^, so the K/V caches agree bit for bit with the dense prefill
+    given the dequantised blob. Switching the int8 handle back to its dense
+    weights reproduces the dense handle given the original blob."""
+    wl = synth.WORKLOADS[wl_name]
+    s, _, blob = H.weights(wl_name)
+    _, blob_q = dequantised_model(wl_name)
+    embeds, valid, _ = device_inputs(wl_name, wl.B)
+    kw = dict(max_batch=wl.B, max_prefix=wl.L, max_chunk=wl.H)
+    m8 = SmolVLA(s, blob, prefix_int8=True, **kw)
+    mq = SmolVLA(s, blob_q, **kw)
+    md = SmolVLA(s, blob, **kw)
     try:
         kv8 = m8.prefill(embeds, valid)
         kvq = mq.prefill(embeds, valid)
@@ -281,6 +285,7 @@ def test_int8_prefill_bitwise_equals_dense_prefill_on_dequantised_blob():
         kv16 = m8.prefill(embeds, valid)
         m8.set_prefix_weights(8)
         kv8b = m8.prefill(embeds, valid)
+        assert m8.device_status() == _abi.SVLA_OK
         torch.cuda.synchronize()
         assert torch.equal(kv8.view(torch.int16), kvq.view(torch.int16))
         assert torch.equal(kv16.view(torch.int16), kvd.view(torch.int16))

@@ -186,7 +186,7 @@ inline int gemm_min_bn(int epi) { return (epi == GE_SWIGLU || epi == GE_QKV_ROPE
 
 template <int BN, int EPI>
 inline cudaError_t launch_persistent_inst(const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& args,
-                                          int ctas, cudaStream_t s) {
+                                          int ctas, cudaStream_t s, bool pdl) {
   constexpr int ST = PersistentStages<BN>::value;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
@@ -195,7 +195,7 @@ inline cudaError_t launch_persistent_inst(const CUtensorMap& ta, const CUtensorM
   cfg.stream = s;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = at;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, gemm_tc_persistent_kernel<BN, EPI, ST>, ta, tw, args);
@@ -203,7 +203,7 @@ inline cudaError_t launch_persistent_inst(const CUtensorMap& ta, const CUtensorM
 
 template <int BN, int EPI>
 inline cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& args, int ctas,
-                                    cudaStream_t s) {
+                                    cudaStream_t s, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
   cfg.blockDim = dim3(GEMM_THREADS);
@@ -211,7 +211,7 @@ inline cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tw
   cfg.stream = s;
   cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   at[1].id = cudaLaunchAttributeClusterDimension;
   at[1].val.clusterDim.x = 2;
   at[1].val.clusterDim.y = 1;
@@ -223,15 +223,15 @@ inline cudaError_t launch_pair_inst(const CUtensorMap& ta, const CUtensorMap& tw
 
 template <int BN>
 inline cudaError_t dispatch_pair(int epi, const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& a, int ctas,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, bool pdl) {
   switch (epi) {
-    case GE_F32: return launch_pair_inst<BN, GE_F32>(ta, tw, a, ctas, s);
-    case GE_BF16: return launch_pair_inst<BN, GE_BF16>(ta, tw, a, ctas, s);
-    case GE_ADD_F32: return launch_pair_inst<BN, GE_ADD_F32>(ta, tw, a, ctas, s);
-    case GE_SILU_BF16: return launch_pair_inst<BN, GE_SILU_BF16>(ta, tw, a, ctas, s);
-    case GE_SWIGLU: return launch_pair_inst<BN, GE_SWIGLU>(ta, tw, a, ctas, s);
-    case GE_QKV_ROPE64: return launch_pair_inst<BN, GE_QKV_ROPE64>(ta, tw, a, ctas, s);
-    case GE_QKV_ROPE32: return launch_pair_inst<BN, GE_QKV_ROPE32>(ta, tw, a, ctas, s);
+    case GE_F32: return launch_pair_inst<BN, GE_F32>(ta, tw, a, ctas, s, pdl);
+    case GE_BF16: return launch_pair_inst<BN, GE_BF16>(ta, tw, a, ctas, s, pdl);
+    case GE_ADD_F32: return launch_pair_inst<BN, GE_ADD_F32>(ta, tw, a, ctas, s, pdl);
+    case GE_SILU_BF16: return launch_pair_inst<BN, GE_SILU_BF16>(ta, tw, a, ctas, s, pdl);
+    case GE_SWIGLU: return launch_pair_inst<BN, GE_SWIGLU>(ta, tw, a, ctas, s, pdl);
+    case GE_QKV_ROPE64: return launch_pair_inst<BN, GE_QKV_ROPE64>(ta, tw, a, ctas, s, pdl);
+    case GE_QKV_ROPE32: return launch_pair_inst<BN, GE_QKV_ROPE32>(ta, tw, a, ctas, s, pdl);
   }
   return cudaErrorInvalidValue;
 }
@@ -256,17 +256,17 @@ inline cudaError_t set_attrs_pair() {
 
 template <int BN>
 inline cudaError_t dispatch_persistent(int epi, const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& a,
-                                       int ctas, cudaStream_t s) {
+                                       int ctas, cudaStream_t s, bool pdl) {
   switch (epi) {
-    case GE_F32: return launch_persistent_inst<BN, GE_F32>(ta, tw, a, ctas, s);
-    case GE_BF16: return launch_persistent_inst<BN, GE_BF16>(ta, tw, a, ctas, s);
-    case GE_ADD_F32: return launch_persistent_inst<BN, GE_ADD_F32>(ta, tw, a, ctas, s);
-    case GE_SILU_BF16: return launch_persistent_inst<BN, GE_SILU_BF16>(ta, tw, a, ctas, s);
-    case GE_QKV_ROPE32: return launch_persistent_inst<BN, GE_QKV_ROPE32>(ta, tw, a, ctas, s);
+    case GE_F32: return launch_persistent_inst<BN, GE_F32>(ta, tw, a, ctas, s, pdl);
+    case GE_BF16: return launch_persistent_inst<BN, GE_BF16>(ta, tw, a, ctas, s, pdl);
+    case GE_ADD_F32: return launch_persistent_inst<BN, GE_ADD_F32>(ta, tw, a, ctas, s, pdl);
+    case GE_SILU_BF16: return launch_persistent_inst<BN, GE_SILU_BF16>(ta, tw, a, ctas, s, pdl);
+    case GE_QKV_ROPE32: return launch_persistent_inst<BN, GE_QKV_ROPE32>(ta, tw, a, ctas, s, pdl);
   }
   if constexpr (BN % 64 == 0) {
-    if (epi == GE_SWIGLU) return launch_persistent_inst<BN, GE_SWIGLU>(ta, tw, a, ctas, s);
-    if (epi == GE_QKV_ROPE64) return launch_persistent_inst<BN, GE_QKV_ROPE64>(ta, tw, a, ctas, s);
+    if (epi == GE_SWIGLU) return launch_persistent_inst<BN, GE_SWIGLU>(ta, tw, a, ctas, s, pdl);
+    if (epi == GE_QKV_ROPE64) return launch_persistent_inst<BN, GE_QKV_ROPE64>(ta, tw, a, ctas, s, pdl);
   }
   return cudaErrorInvalidValue;
 }
@@ -302,7 +302,7 @@ inline size_t gemm_partials_bytes(const GemmPlan& p) {
 // the cluster reduction, a (1, 1, splits) cluster.
 template <int BN, int ST, int EPI, int AR = GEMM_BM>
 inline cudaError_t launch_gemm_inst(const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& args, dim3 grid,
-                                    int cluster_z, cudaStream_t s) {
+                                    int cluster_z, cudaStream_t s, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(GEMM_THREADS);
@@ -311,7 +311,7 @@ inline cudaError_t launch_gemm_inst(const CUtensorMap& ta, const CUtensorMap& tw
   cudaLaunchAttribute at[2];
   int n = 0;
   at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[n].val.programmaticStreamSerializationAllowed = 1;
+  at[n].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   ++n;
   if (cluster_z > 1) {
     at[n].id = cudaLaunchAttributeClusterDimension;
@@ -327,15 +327,15 @@ inline cudaError_t launch_gemm_inst(const CUtensorMap& ta, const CUtensorMap& tw
 
 template <int BN, int ST, int AR = GEMM_BM>
 inline cudaError_t dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tw, const GemmArgs& a, dim3 g,
-                                int cz, cudaStream_t s) {
+                                int cz, cudaStream_t s, bool pdl) {
   switch (epi) {
-    case GE_F32: return launch_gemm_inst<BN, ST, GE_F32, AR>(ta, tw, a, g, cz, s);
-    case GE_BF16: return launch_gemm_inst<BN, ST, GE_BF16, AR>(ta, tw, a, g, cz, s);
-    case GE_ADD_F32: return launch_gemm_inst<BN, ST, GE_ADD_F32, AR>(ta, tw, a, g, cz, s);
-    case GE_SILU_BF16: return launch_gemm_inst<BN, ST, GE_SILU_BF16, AR>(ta, tw, a, g, cz, s);
-    case GE_SWIGLU: return launch_gemm_inst<BN, ST, GE_SWIGLU, AR>(ta, tw, a, g, cz, s);
-    case GE_QKV_ROPE64: return launch_gemm_inst<BN, ST, GE_QKV_ROPE64, AR>(ta, tw, a, g, cz, s);
-    case GE_QKV_ROPE32: return launch_gemm_inst<BN, ST, GE_QKV_ROPE32, AR>(ta, tw, a, g, cz, s);
+    case GE_F32: return launch_gemm_inst<BN, ST, GE_F32, AR>(ta, tw, a, g, cz, s, pdl);
+    case GE_BF16: return launch_gemm_inst<BN, ST, GE_BF16, AR>(ta, tw, a, g, cz, s, pdl);
+    case GE_ADD_F32: return launch_gemm_inst<BN, ST, GE_ADD_F32, AR>(ta, tw, a, g, cz, s, pdl);
+    case GE_SILU_BF16: return launch_gemm_inst<BN, ST, GE_SILU_BF16, AR>(ta, tw, a, g, cz, s, pdl);
+    case GE_SWIGLU: return launch_gemm_inst<BN, ST, GE_SWIGLU, AR>(ta, tw, a, g, cz, s, pdl);
+    case GE_QKV_ROPE64: return launch_gemm_inst<BN, ST, GE_QKV_ROPE64, AR>(ta, tw, a, g, cz, s, pdl);
+    case GE_QKV_ROPE32: return launch_gemm_inst<BN, ST, GE_QKV_ROPE32, AR>(ta, tw, a, g, cz, s, pdl);
   }
   return cudaErrorInvalidValue;
 }
@@ -395,6 +395,14 @@ inline bool make_tmap_pairs(CUtensorMap* m, const void* ptr, int N, int groups, 
 // split over a cluster so that a split keeps >= 3 k-blocks). With the same
 // tile width and splits as the dense plan, the partial sums are added in the
 // same order, so an int8 GEMM equals the dense GEMM on the dequantised weights.
+// Many output tiles (large M): every weight tile is needed by many m-tiles, so
+// the prefill dequantises such a matrix once into a bf16 buffer and runs the
+// dense GEMM on it instead of the fused kernel.
+inline bool w8_many_tiles(int M, int N) {
+  const int mt = (M + GEMM_BM - 1) / GEMM_BM;
+  return mt >= 4 || mt * ((N + 127) / 128) >= 100;
+}
+
 inline GemmPlan plan_gemm_w8(int M, int N, int K, int forced_splits, int min_bn = 32) {
   GemmPlan p;
   const int KB = K / GEMM_BK;
@@ -405,7 +413,7 @@ inline GemmPlan plan_gemm_w8(int M, int N, int K, int forced_splits, int min_bn 
     if (sp > GEMM_MAX_CLUSTER) sp = GEMM_MAX_CLUSTER;
     return sp < 1 ? 1 : sp;
   };
-  if (forced_splits <= 1 && (p.m_tiles >= 4 || tiles(128) >= 100)) {
+  if (forced_splits <= 1 && w8_many_tiles(M, N)) {
     p.bn = 128;
     p.stages = 4;
     p.splits = 1;
@@ -419,7 +427,7 @@ inline GemmPlan plan_gemm_w8(int M, int N, int K, int forced_splits, int min_bn 
     const int s64 = fit(t64), s32 = fit(t32);
     const int c64 = t64 * s64, c32 = t32 * s32;
     p.bn = (c64 >= 120 || c64 >= c32 || min_bn > 32) ? 64 : 32;
-    p.stages = p.bn == 64 ? 3 : 4;
+    p.stages = p.bn == 64 ? 4 : 5;
     p.splits = p.bn == 64 ? s64 : s32;
   }
   if (forced_splits > 0) p.splits = clamp_splits(forced_splits);
@@ -509,8 +517,8 @@ inline cudaError_t run_gemm_w8(int epi, const void* A, int lda, const uint8_t* Q
   args.red_mode = p.red;
   const dim3 grid(p.n_tiles, p.m_tiles, p.splits);
   const int cz = p.red == GEMM_RED_CLUSTER ? p.splits : 1;
-  if (p.bn == 32 && p.stages == 4) return dispatch_w8<32, 4>(epi, ta, tq, ts, args, gain, grid, cz, s);
-  if (p.bn == 64 && p.stages == 3) return dispatch_w8<64, 3>(epi, ta, tq, ts, args, gain, grid, cz, s);
+  if (p.bn == 32 && p.stages == 5) return dispatch_w8<32, 5>(epi, ta, tq, ts, args, gain, grid, cz, s);
+  if (p.bn == 64 && p.stages == 4) return dispatch_w8<64, 4>(epi, ta, tq, ts, args, gain, grid, cz, s);
   if (p.bn == 128 && p.stages == 4) return dispatch_w8<128, 4>(epi, ta, tq, ts, args, gain, grid, cz, s);
   return cudaErrorInvalidValue;
 }
@@ -529,15 +537,19 @@ inline cudaError_t gemm_set_attrs() {
   if (e == cudaSuccess) e = set_attrs_inst<64, 4>();
   if (e == cudaSuccess) e = set_attrs_inst<128, 6>();
   if (e == cudaSuccess) e = set_attrs_inst<256, 4>();
-  if (e == cudaSuccess) e = set_attrs_w8<32, 4>();
-  if (e == cudaSuccess) e = set_attrs_w8<64, 3>();
+  if (e == cudaSuccess) e = set_attrs_w8<32, 5>();
+  if (e == cudaSuccess) e = set_attrs_w8<64, 4>();
   if (e == cudaSuccess) e = set_attrs_w8<128, 4>();
   return e;
 }
 
-// Full launch: encode the maps and dispatch the plan's instance.
+// Full launch: encode the maps and dispatch the plan's instance. pdl = false
+// launches without programmatic stream serialization: the kernel then starts
+// after the previous kernel completes, for a W the previous kernel writes (the
+// kernel streams W before its dependency wait).
 inline cudaError_t run_gemm(int epi, const void* A, int lda, const void* W, int ldw, int M, int N, int K,
-                            GemmArgs args, const GemmPlan& p, float* partials, int* counters, cudaStream_t s) {
+                            GemmArgs args, const GemmPlan& p, float* partials, int* counters, cudaStream_t s,
+                            bool pdl = true) {
   CUtensorMap ta, tw;
   if (!make_tmap_bf16(&ta, A, M, K, lda, p.a_rows)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&tw, W, N, K, ldw, p.pair ? p.bn / 2 : p.bn)) return cudaErrorInvalidValue;
@@ -549,31 +561,31 @@ inline cudaError_t run_gemm(int epi, const void* A, int lda, const void* W, int 
   args.counters = counters;
   args.red_mode = p.red;
   if (p.pair) {
-    if (p.bn == 128) return dispatch_pair<128>(epi, ta, tw, args, p.ctas, s);
-    if (p.bn == 256) return dispatch_pair<256>(epi, ta, tw, args, p.ctas, s);
+    if (p.bn == 128) return dispatch_pair<128>(epi, ta, tw, args, p.ctas, s, pdl);
+    if (p.bn == 256) return dispatch_pair<256>(epi, ta, tw, args, p.ctas, s, pdl);
     return cudaErrorInvalidValue;
   }
   if (p.persistent) {
     switch (p.bn) {
-      case 64: return dispatch_persistent<64>(epi, ta, tw, args, p.ctas, s);
-      case 96: return dispatch_persistent<96>(epi, ta, tw, args, p.ctas, s);
-      case 128: return dispatch_persistent<128>(epi, ta, tw, args, p.ctas, s);
-      case 192: return dispatch_persistent<192>(epi, ta, tw, args, p.ctas, s);
-      case 256: return dispatch_persistent<256>(epi, ta, tw, args, p.ctas, s);
+      case 64: return dispatch_persistent<64>(epi, ta, tw, args, p.ctas, s, pdl);
+      case 96: return dispatch_persistent<96>(epi, ta, tw, args, p.ctas, s, pdl);
+      case 128: return dispatch_persistent<128>(epi, ta, tw, args, p.ctas, s, pdl);
+      case 192: return dispatch_persistent<192>(epi, ta, tw, args, p.ctas, s, pdl);
+      case 256: return dispatch_persistent<256>(epi, ta, tw, args, p.ctas, s, pdl);
     }
     return cudaErrorInvalidValue;
   }
   dim3 grid(p.n_tiles, p.m_tiles, p.splits);
   const int cz = p.red == GEMM_RED_CLUSTER ? p.splits : 1;
   if (p.a_rows == 64) {
-    if (p.bn == 32 && p.stages == 8) return dispatch_epi<32, 8, 64>(epi, ta, tw, args, grid, cz, s);
-    if (p.bn == 64 && p.stages == 6) return dispatch_epi<64, 6, 64>(epi, ta, tw, args, grid, cz, s);
+    if (p.bn == 32 && p.stages == 8) return dispatch_epi<32, 8, 64>(epi, ta, tw, args, grid, cz, s, pdl);
+    if (p.bn == 64 && p.stages == 6) return dispatch_epi<64, 6, 64>(epi, ta, tw, args, grid, cz, s, pdl);
     return cudaErrorInvalidValue;
   }
-  if (p.bn == 32 && p.stages == 4) return dispatch_epi<32, 4>(epi, ta, tw, args, grid, cz, s);
-  if (p.bn == 64 && p.stages == 4) return dispatch_epi<64, 4>(epi, ta, tw, args, grid, cz, s);
-  if (p.bn == 128 && p.stages == 6) return dispatch_epi<128, 6>(epi, ta, tw, args, grid, cz, s);
-  if (p.bn == 256 && p.stages == 4) return dispatch_epi<256, 4>(epi, ta, tw, args, grid, cz, s);
+  if (p.bn == 32 && p.stages == 4) return dispatch_epi<32, 4>(epi, ta, tw, args, grid, cz, s, pdl);
+  if (p.bn == 64 && p.stages == 4) return dispatch_epi<64, 4>(epi, ta, tw, args, grid, cz, s, pdl);
+  if (p.bn == 128 && p.stages == 6) return dispatch_epi<128, 6>(epi, ta, tw, args, grid, cz, s, pdl);
+  if (p.bn == 256 && p.stages == 4) return dispatch_epi<256, 4>(epi, ta, tw, args, grid, cz, s, pdl);
   return cudaErrorInvalidValue;
 }
 

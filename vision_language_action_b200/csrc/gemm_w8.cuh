@@ -17,14 +17,17 @@
 //
 // CTA (same roles as the dense kernel, one more stage of work):
 //   warp 0      : TMA producer: A (bf16, 128-byte swizzle), the int8 code tile
-//                 [BN][64] and its BN (alpha, beta) pairs, into a ring.
+//                 [BN][64] and its BN (alpha, beta) pairs, into a STAGES ring.
 //   warp 1      : TMEM allocation; one lane issues tcgen05.mma (kind::f16) on
 //                 A and the dequantised tile, commits each stage.
 //   warps 2..5  : during the main loop they dequantise each stage's codes into
 //                 a bf16 tile in the 128-byte-swizzled K-major layout that TMA
 //                 would have written, then (after the loop) run the epilogue.
-// The int8 tiles arrive on their own barrier, so the dequantisation of the
-// first stages overlaps the wait for the producer kernel of A.
+// The dequantised tiles live in a ring of their own, two deep (a tile is only
+// alive between its dequantisation and its MMA), so the operand ring holds as
+// many stages as the dense kernel's at two CTAs per SM. The int8 tiles arrive
+// on their own barrier, so the dequantisation of the first stages overlaps the
+// wait for the producer kernel of A.
 #pragma once
 
 #include "gemm_tc.cuh"
@@ -37,11 +40,12 @@ template <int BN, int STAGES_>
 struct W8Cfg {
   static constexpr int STAGES = STAGES_;
   static constexpr uint32_t A_BYTES = GEMM_BM * GEMM_BK * 2;
-  static constexpr uint32_t B_BYTES = BN * GEMM_BK * 2;  // dequantised tile (bf16)
   static constexpr uint32_t Q_BYTES = BN * GEMM_BK;      // codes
   static constexpr uint32_t S_BYTES = BN * 4;            // (alpha, beta) pairs
-  static constexpr uint32_t STAGE_BYTES = (A_BYTES + B_BYTES + Q_BYTES + S_BYTES + 1023) / 1024 * 1024;
-  static constexpr uint32_t RING_BYTES = STAGES * STAGE_BYTES;
+  static constexpr uint32_t STAGE_BYTES = (A_BYTES + Q_BYTES + S_BYTES + 1023) / 1024 * 1024;
+  static constexpr int B_BUFS = 2;
+  static constexpr uint32_t B_BYTES = BN * GEMM_BK * 2;  // one dequantised tile (bf16), 1024-byte multiple
+  static constexpr uint32_t RING_BYTES = STAGES * STAGE_BYTES + B_BUFS * B_BYTES;
   static constexpr uint32_t TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
   // ring + barriers/flags (512 B) + row factors (512 B) + alignment slack
   static constexpr size_t SMEM = (size_t)RING_BYTES + 1024 + 1024;
@@ -49,7 +53,7 @@ struct W8Cfg {
   static constexpr size_t RED_TILE = (size_t)GEMM_BM * (BN + 4) * sizeof(float);
   static constexpr bool CLUSTER_OK = 2 * RED_TILE <= (size_t)RING_BYTES;
   static_assert(BN % 32 == 0 && BN <= 128, "the (alpha, beta) box holds at most 256 bf16");
-  static_assert(4 * STAGES + 1 <= 60, "barriers and flags share 512 bytes");
+  static_assert(3 * STAGES + 2 * B_BUFS + 1 <= 60, "barriers and flags share 512 bytes");
   static_assert(CLUSTER_OK, "split-K of the int8 GEMM reduces over a cluster only");
 };
 
@@ -88,8 +92,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES);
-  // bars[0..S) A full, [S..2S) codes full, [2S..3S) dequantised, [3S..4S) empty, [4S] accumulator
-  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(bars + 4 * STAGES + 1);
+  // bars[0..S) A full, [S..2S) codes full, [2S..3S) stage empty, then per dequantised
+  // buffer: full [3S, 3S+2), empty [3S+2, 3S+4); [3S+4] accumulator
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(bars + 3 * STAGES + 2 * C::B_BUFS + 1);
   // misc[0] tmem base, misc[1] abort flag, misc[2] stages issued, misc[3] stages consumed,
   // misc[4] "this CTA reduces"
   float* misc_scale = reinterpret_cast<float*>(smem + C::RING_BYTES + 512);
@@ -104,18 +109,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
 
   auto a_full = [&](int s) { return smem_u32(bars + s); };
   auto q_full = [&](int s) { return smem_u32(bars + STAGES + s); };
-  auto deq_bar = [&](int s) { return smem_u32(bars + 2 * STAGES + s); };
-  auto empty_bar = [&](int s) { return smem_u32(bars + 3 * STAGES + s); };
-  const uint32_t acc_bar = smem_u32(bars + 4 * STAGES);
+  auto empty_bar = [&](int s) { return smem_u32(bars + 2 * STAGES + s); };
+  auto b_full = [&](int b) { return smem_u32(bars + 3 * STAGES + b); };
+  auto b_empty = [&](int b) { return smem_u32(bars + 3 * STAGES + C::B_BUFS + b); };
+  const uint32_t acc_bar = smem_u32(bars + 3 * STAGES + 2 * C::B_BUFS);
   auto stage = [&](int s) { return ring + (size_t)s * C::STAGE_BYTES; };
+  auto bbuf = [&](int b) { return ring + (size_t)STAGES * C::STAGE_BYTES + (size_t)b * C::B_BYTES; };
 
   griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(a_full(s), 1);
       mbar_init(q_full(s), 1);
-      mbar_init(deq_bar(s), 128);  // every dequantising thread arrives
       mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < C::B_BUFS; ++b) {
+      mbar_init(b_full(b), 4);  // one arrival per dequantising warp
+      mbar_init(b_empty(b), 1);
     }
     mbar_init(acc_bar, 1);
     misc[1] = 0;
@@ -142,8 +152,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
     const int s = i % STAGES;
     uint8_t* st = stage(s);
     mbar_arrive_expect_tx(q_full(s), C::Q_BYTES + C::S_BYTES);
-    tma_load_2d(smem_u32(st + C::A_BYTES + C::B_BYTES), &tmQ, q_full(s), (kb0 + i) * GEMM_BK, n0);
-    tma_load_2d(smem_u32(st + C::A_BYTES + C::B_BYTES + C::Q_BYTES), &tmS, q_full(s), 2 * n0, kb0 + i);
+    tma_load_2d(smem_u32(st + C::A_BYTES), &tmQ, q_full(s), (kb0 + i) * GEMM_BK, n0);
+    tma_load_2d(smem_u32(st + C::A_BYTES + C::Q_BYTES), &tmS, q_full(s), 2 * n0, kb0 + i);
   };
   auto issue_a = [&](int i) {
     const int s = i % STAGES;
@@ -178,63 +188,74 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
       constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, BN);
       for (int i = 0; i < nkb; ++i) {
         if (misc[1]) break;
-        const int s = i % STAGES;
-        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-        if (!mbar_wait(a_full(s), ph, lim) || !mbar_wait(deq_bar(s), ph, lim)) {
+        const int s = i % STAGES, b = i % C::B_BUFS;
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u, bph = (uint32_t)(i / C::B_BUFS) & 1u;
+        if (!mbar_wait(a_full(s), ph, lim) || !mbar_wait(b_full(b), bph, lim)) {
           misc[1] = 1;
           set_status(args.status, SVLA_ERR_TIMEOUT);
           break;
         }
         tc_fence_after();
         const uint32_t sa = smem_u32(stage(s));
-        const uint32_t sb = sa + C::A_BYTES;
+        const uint32_t sb = smem_u32(bbuf(b));
 #pragma unroll
         for (int k = 0; k < GEMM_BK / 16; ++k) {
           tc_mma_bf16(tmem_base, smem_desc_sw128(sa + 32 * k), smem_desc_sw128(sb + 32 * k), IDESC,
                       (i > 0 || k > 0) ? 1u : 0u);
         }
         tc_commit(empty_bar(s));
+        tc_commit(b_empty(b));
         misc[3] = i + 1;
       }
       tc_commit(acc_bar);  // always: lets waiters know every issued MMA finished
     }
   } else {
     // ---------------- dequantisation (main loop), then the epilogue ----------------
+    // Control flow is uniform per warp (votes before every exit), so the warp
+    // can sync and arrive once per tile.
     const int t = threadIdx.x - 64;
+    const int c = t & 3;  // items t + 128 j: every item of a thread has chunk c
     for (int i = 0; i < nkb; ++i) {
-      if (misc[1]) break;
-      const int s = i % STAGES;
-      if (!mbar_wait(q_full(s), (uint32_t)(i / STAGES) & 1u, lim)) {
-        misc[1] = 1;
-        set_status(args.status, SVLA_ERR_TIMEOUT);
+      if (__any_sync(0xffffffffu, misc[1] != 0)) break;
+      const int s = i % STAGES, b = i % C::B_BUFS;
+      const int k0 = (kb0 + i) * GEMM_BK;
+      // the gain does not depend on the stage's data: load it before waiting
+      uint4 g0 = make_uint4(0u, 0u, 0u, 0u), g1 = g0;
+      if (gain) {
+        const uint4* gp = reinterpret_cast<const uint4*>(gain + k0 + 16 * c);
+        g0 = __ldg(gp);
+        g1 = __ldg(gp + 1);
+      }
+      bool ok = mbar_wait(q_full(s), (uint32_t)(i / STAGES) & 1u, lim);
+      ok = ok && mbar_wait(b_empty(b), ((uint32_t)(i / C::B_BUFS) & 1u) ^ 1u, lim);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) {
+          misc[1] = 1;
+          set_status(args.status, SVLA_ERR_TIMEOUT);
+        }
         break;
       }
-      uint8_t* st = stage(s);
-      const uint8_t* qs = st + C::A_BYTES + C::B_BYTES;
-      const uint32_t* ps = reinterpret_cast<const uint32_t*>(st + C::A_BYTES + C::B_BYTES + C::Q_BYTES);
-      uint8_t* bs = st + C::A_BYTES;
-      const int k0 = (kb0 + i) * GEMM_BK;
+      const uint8_t* st = stage(s);
+      const uint8_t* qs = st + C::A_BYTES;
+      const uint32_t* ps = reinterpret_cast<const uint32_t*>(st + C::A_BYTES + C::Q_BYTES);
+      uint8_t* bs = bbuf(b);
+      float g[16];
+      {
+        const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          g[2 * j] = gain ? bf2f((uint16_t)(gw[j] & 0xFFFFu)) : 1.f;
+          g[2 * j + 1] = gain ? bf2f((uint16_t)(gw[j] >> 16)) : 1.f;
+        }
+      }
       // item = (row r, 16-code chunk c): 16 operand values = logical 16-byte
       // chunks 2c, 2c + 1 of the row's 128 bytes, stored at chunk ^ (r % 8)
-      for (int item = t; item < BN * 4; item += 128) {
-        const int r = item >> 2, c = item & 3;
+#pragma unroll
+      for (int j = 0; j < BN * 4 / 128; ++j) {
+        const int r = (t + 128 * j) >> 2;
         const uint4 qv = *reinterpret_cast<const uint4*>(qs + r * GEMM_BK + 16 * c);
         const uint32_t ab = ps[r];
         const float al = bf2f((uint16_t)(ab & 0xFFFFu)), be = bf2f((uint16_t)(ab >> 16));
-        float g[16];
-        if (gain) {
-          const uint4* gp = reinterpret_cast<const uint4*>(gain + k0 + 16 * c);
-          const uint4 g0 = __ldg(gp), g1 = __ldg(gp + 1);
-          const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            g[2 * j] = bf2f((uint16_t)(gw[j] & 0xFFFFu));
-            g[2 * j + 1] = bf2f((uint16_t)(gw[j] >> 16));
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) g[j] = 1.f;
-        }
         uint32_t o[8];
         dequant16(qv, al, be, g, gain != nullptr, o);
         uint8_t* row = bs + r * 128;
@@ -243,7 +264,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
         *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
       }
       fence_proxy_async_cta();  // generic stores -> visible to the tensor cores' async proxy
-      mbar_arrive(deq_bar(s));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_full(b));
     }
     griddep_wait();  // outputs, residuals, biases and positions come from earlier kernels
     const int quad = warp & 3;
@@ -285,6 +307,45 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// Dequantise a whole matrix: out[n, k] = bf16(bf16(alpha q + beta) * g[k]), the
+// operand the fused kernel builds tile by tile. Used for GEMMs with many tiles
+// (large M), where the fused kernel would dequantise every weight tile once per
+// m-tile: the buffer (<= 10 MB for the prefix projections) is written once and
+// read from L2 by the dense GEMM that follows. One thread per 16 codes.
+__global__ void __launch_bounds__(256) dequant_affine8_kernel(const uint8_t* __restrict__ q,
+                                                              const uint16_t* __restrict__ ab,
+                                                              const uint16_t* __restrict__ gain, int N, int K,
+                                                              uint16_t* __restrict__ out) {
+  griddep_wait();  // the GEMM before may still be reading `out`
+  const int cpr = K / 16;
+  const long long total = (long long)N * cpr;
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(idx / cpr), k = (int)(idx % cpr) * 16;
+    const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + (size_t)n * K + k));
+    const uint32_t pr = __ldg(reinterpret_cast<const uint32_t*>(ab) + (size_t)(k / W8_GROUP) * N + n);
+    float g[16];
+    if (gain) {
+      const uint4* gp = reinterpret_cast<const uint4*>(gain + k);
+      const uint4 g0 = __ldg(gp), g1 = __ldg(gp + 1);
+      const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        g[2 * j] = bf2f((uint16_t)(gw[j] & 0xFFFFu));
+        g[2 * j + 1] = bf2f((uint16_t)(gw[j] >> 16));
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) g[j] = 1.f;
+    }
+    uint32_t o[8];
+    dequant16(qv, bf2f((uint16_t)(pr & 0xFFFFu)), bf2f((uint16_t)(pr >> 16)), g, gain != nullptr, o);
+    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)n * K + k);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
 

@@ -266,6 +266,7 @@ struct svla_handle {
   int denoise_path = SVLA_DENOISE_AUTO;
   // weight-only int8 prefix (svla_create_ex with SVLA_CREATE_PREFIX_INT8)
   uint8_t* q8 = nullptr;     // codes and (alpha, beta) pairs of the prefix projections
+  uint16_t* q8_deq = nullptr;  // one dequantised projection (bf16), for many-tile GEMMs
   std::vector<Q8Mat> q8m;    // per prefix layer: QKV, O, gate/up (interleaved rows), down
   int prefix_bits = 16;      // weights svla_prefill uses
   // prefix assembly (svla_set_assembly): connector and state-projection weights, workspaces
@@ -352,21 +353,35 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // one GEMM of the schedule
 cudaError_t gemm(svla_handle* h, int epi, const bf16* A, int lda, const bf16* W, int ldw, int M, int N, int K,
-                 GemmArgs args, float* part, int* cnt, cudaStream_t s) {
+                 GemmArgs args, float* part, int* cnt, cudaStream_t s, bool pdl = true) {
   GemmPlan p = plan_gemm(M, N, K, 0, gemm_min_bn(epi));
   args.status = h->status;
   args.wait_ns = g_wait_ns.load();
-  return run_gemm(epi, A, lda, W, ldw, M, N, K, args, p, part, cnt, s);
+  return run_gemm(epi, A, lda, W, ldw, M, N, K, args, p, part, cnt, s, pdl);
 }
 
-// one GEMM of the prefill on the int8 weights (gain: the folded RMSNorm gain, or null)
+// One GEMM of the prefill on the int8 weights (gain: the folded RMSNorm gain,
+// or null). Few tiles: the fused kernel dequantises tile by tile. Many tiles:
+// the matrix is dequantised once into the handle's bf16 buffer and the dense
+// GEMM (its plan, so its partial-sum order) runs on it, launched after the
+// dequantisation completes.
 cudaError_t gemm8(svla_handle* h, int epi, const bf16* A, int lda, const Q8Mat& w, const uint16_t* gain, int M,
-                  GemmArgs args, cudaStream_t s) {
+                  GemmArgs args, float* part, int* cnt, cudaStream_t s) {
+  const uint8_t* q = h->q8 + w.q_off;
+  const uint16_t* ab = reinterpret_cast<const uint16_t*>(h->q8 + w.ab_off);
+  if (w8_many_tiles(M, w.N)) {
+    const long long chunks = (long long)w.N * (w.K / 16);
+    const unsigned blocks = (unsigned)std::min<long long>((chunks + 255) / 256, 8LL * NUM_SMS_B200);
+    const cudaError_t e = launch_pdl(dequant_affine8_kernel, dim3(blocks), dim3(256), 0, s, q, ab, gain, w.N, w.K,
+                                     h->q8_deq);
+    if (e != cudaSuccess) return e;
+    return gemm(h, epi, A, lda, reinterpret_cast<const bf16*>(h->q8_deq), w.K, M, w.N, w.K, args, part, cnt, s,
+                /*pdl=*/false);
+  }
   GemmPlan p = plan_gemm_w8(M, w.N, w.K, 0, gemm_min_bn(epi));
   args.status = h->status;
   args.wait_ns = g_wait_ns.load();
-  return run_gemm_w8(epi, A, lda, h->q8 + w.q_off, (size_t)w.K, reinterpret_cast<const uint16_t*>(h->q8 + w.ab_off),
-                     gain, M, w.N, w.K, args, p, s);
+  return run_gemm_w8(epi, A, lda, q, (size_t)w.K, ab, gain, M, w.N, w.K, args, p, s);
 }
 
 GemmArgs out_args(void* out, int ldo, const float* bias = nullptr) {
@@ -458,7 +473,8 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
   const bool q8 = h->prefix_bits == 8;
   // n-tiles of the residual-producing GEMMs = the norm statistics' tiles
   auto res_tiles = [&](int N, int K) {
-    return q8 ? plan_gemm_w8(M, N, K, 0, gemm_min_bn(GE_ADD_F32)).n_tiles : residual_tiles(M, N, K);
+    return q8 && !w8_many_tiles(M, N) ? plan_gemm_w8(M, N, K, 0, gemm_min_bn(GE_ADD_F32)).n_tiles
+                                      : residual_tiles(M, N, K);
   };
   const int o_tiles = res_tiles(D, qw), d_tiles = res_tiles(D, c.p_ffn);
   for (int l = 0; l < c.p_layers; ++l) {
@@ -483,21 +499,21 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
     norm_consumer(qa, h->p_ss, l == 0 ? 1 : d_tiles, M, D, c.rms_eps);
     const bf16* xin = l == 0 ? reinterpret_cast<const bf16*>(embeds) : rb;
     const int qkv_epi = hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32;
-    SVLA_TRY(q8 ? gemm8(h, qkv_epi, xin, D, qm[0], in_gain, M, qa, s)
+    SVLA_TRY(q8 ? gemm8(h, qkv_epi, xin, D, qm[0], in_gain, M, qa, h->p_part, h->p_cnt, s)
                 : gemm(h, qkv_epi, xin, D, h->W(e[1].off), D, M, qw + 2 * kvw, D, qa, h->p_part, h->p_cnt, s));
     if (l == c.p_layers - 1) break;  // nothing reads the last layer's attention / MLP output
     SVLA_TRY(attention(h->p_q, qw, Kl, Vl, kvw, pad, B, c.p_heads, c.p_kv_heads, hd, L, L, 0, h->p_o, qw, s));
     GemmArgs oa = out_args(h->p_x, D);
     norm_producer(oa, rb, D, h->p_ss, M);
-    SVLA_TRY(q8 ? gemm8(h, GE_ADD_F32, h->p_o, qw, qm[1], nullptr, M, oa, s)
+    SVLA_TRY(q8 ? gemm8(h, GE_ADD_F32, h->p_o, qw, qm[1], nullptr, M, oa, h->p_part, h->p_cnt, s)
                 : gemm(h, GE_ADD_F32, h->p_o, qw, h->W(e[4].off), qw, M, D, qw, oa, h->p_part, h->p_cnt, s));
     GemmArgs ga = out_args(h->p_h, c.p_ffn);
     norm_consumer(ga, h->p_ss, o_tiles, M, D, c.rms_eps);
-    SVLA_TRY(q8 ? gemm8(h, GE_SWIGLU, rb, D, qm[2], post_gain, M, ga, s)
+    SVLA_TRY(q8 ? gemm8(h, GE_SWIGLU, rb, D, qm[2], post_gain, M, ga, h->p_part, h->p_cnt, s)
                 : gemm(h, GE_SWIGLU, rb, D, h->W(e[6].off), D, M, 2 * c.p_ffn, D, ga, h->p_part, h->p_cnt, s));
     GemmArgs da = out_args(h->p_x, D);
     norm_producer(da, rb, D, h->p_ss, M);
-    SVLA_TRY(q8 ? gemm8(h, GE_ADD_F32, h->p_h, c.p_ffn, qm[3], nullptr, M, da, s)
+    SVLA_TRY(q8 ? gemm8(h, GE_ADD_F32, h->p_h, c.p_ffn, qm[3], nullptr, M, da, h->p_part, h->p_cnt, s)
                 : gemm(h, GE_ADD_F32, h->p_h, c.p_ffn, h->W(e[8].off), c.p_ffn, M, D, c.p_ffn, da, h->p_part,
                        h->p_cnt, s));
   }
@@ -905,6 +921,9 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
       h->q8m.push_back(add(D, c.p_ffn));
     }
     if ((e = halloc(h, &h->q8, off)) != cudaSuccess) return bail(e, "int8 weights");
+    size_t max_nk = 0;
+    for (const Q8Mat& m : h->q8m) max_nk = std::max(max_nk, (size_t)m.N * m.K);
+    if ((e = halloc(h, &h->q8_deq, max_nk)) != cudaSuccess) return bail(e, "int8 dequantisation buffer");
     for (int l = 0; l < c.p_layers && e == cudaSuccess; ++l) {
       const Entry* en = &lay.p[9 * l];
       const size_t src[4] = {en[1].off, en[4].off, en[6].off, en[8].off};
