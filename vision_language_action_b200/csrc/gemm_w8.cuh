@@ -23,7 +23,7 @@
 //   warps 2..5  : during the main loop they dequantise each stage's codes into
 //                 a bf16 tile in the 128-byte-swizzled K-major layout that TMA
 //                 would have written, then (after the loop) run the epilogue.
-// The dequantised tiles live in a ring of their own, two deep (a tile is only
+// The dequantised tiles live in a ring of their own, three deep (a tile is only
 // alive between its dequantisation and its MMA), so the operand ring holds as
 // many stages as the dense kernel's at two CTAs per SM. The int8 tiles arrive
 // on their own barrier, so the dequantisation of the first stages overlaps the
@@ -43,7 +43,7 @@ struct W8Cfg {
   static constexpr uint32_t Q_BYTES = BN * GEMM_BK;      // codes
   static constexpr uint32_t S_BYTES = BN * 4;            // (alpha, beta) pairs
   static constexpr uint32_t STAGE_BYTES = (A_BYTES + Q_BYTES + S_BYTES + 1023) / 1024 * 1024;
-  static constexpr int B_BUFS = 2;
+  static constexpr int B_BUFS = 3;  // a deep-K CTA is bound by B_BUFS tiles per dequantise -> MMA -> commit trip
   static constexpr uint32_t B_BYTES = BN * GEMM_BK * 2;  // one dequantised tile (bf16), 1024-byte multiple
   static constexpr uint32_t RING_BYTES = STAGES * STAGE_BYTES + B_BUFS * B_BYTES;
   static constexpr uint32_t TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
@@ -61,25 +61,33 @@ SVLA_DEV void fence_proxy_async_cta() { asm volatile("fence.proxy.async.shared::
 
 SVLA_DEV float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
+// Two bf16 products, each rounded to nearest even: the product of two bf16
+// values is exact in fp32, so this equals bf16(float(a) * float(b)) per half.
+SVLA_DEV uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // Code byte j of the word as a float: 2^23 + q assembled in the bits, minus 2^23.
 template <int J>
 SVLA_DEV float code_f(uint32_t word) {
   return __uint_as_float(__byte_perm(word, 0x4B000000u, 0x7540u + J)) - 8388608.f;
 }
 
-// 16 codes (one 16-byte chunk of a row) -> 16 operand values, packed bf16x2.
-SVLA_DEV void dequant16(uint4 qv, float al, float be, const float (&g)[16], bool has_gain, uint32_t (&out)[8]) {
+// 16 codes (one 16-byte chunk of a row) -> 16 operand values, packed bf16x2:
+// w^ = bf16(alpha q + beta) (fp32 fma, alpha q exact), then times the gain pair
+// g2[j] (bf16x2, the same 16 inputs) where a gain is folded in.
+SVLA_DEV void dequant16(uint4 qv, float al, float be, const uint32_t (&g2)[8], bool has_gain, uint32_t (&out)[8]) {
   const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    float v[4] = {fmaf(al, code_f<0>(w[i]), be), fmaf(al, code_f<1>(w[i]), be), fmaf(al, code_f<2>(w[i]), be),
-                  fmaf(al, code_f<3>(w[i]), be)};
-    if (has_gain) {
+    out[2 * i] = pack_bf16x2(fmaf(al, code_f<0>(w[i]), be), fmaf(al, code_f<1>(w[i]), be));
+    out[2 * i + 1] = pack_bf16x2(fmaf(al, code_f<2>(w[i]), be), fmaf(al, code_f<3>(w[i]), be));
+  }
+  if (has_gain) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = bf16_round(v[j]) * g[4 * i + j];
-    }
-    out[2 * i] = pack_bf16x2(v[0], v[1]);
-    out[2 * i + 1] = pack_bf16x2(v[2], v[3]);
+    for (int j = 0; j < 8; ++j) out[j] = bf16x2_mul(out[j], g2[j]);
   }
 }
 
@@ -215,6 +223,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
     // can sync and arrive once per tile.
     const int t = threadIdx.x - 64;
     const int c = t & 3;  // items t + 128 j: every item of a thread has chunk c
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int m = m_blk * GEMM_BM + row;
+    const bool row_ok = m < args.M;
+    const int pre = nkb < STAGES ? nkb : STAGES;
+    float rscale = 1.f;
+    bool have_scale = false;
+    // after the stages whose codes were requested before the dependency wait:
+    // the epilogue's inputs come from earlier kernels, and their loads then
+    // overlap the rest of the main loop
+    auto epilogue_inputs = [&]() {
+      griddep_wait();
+      prefetch_epilogue_inputs<BN, EPI>(args, m, n0, row_ok);
+      rscale = norm_row_scale(args, m, row_ok);
+      misc_scale[row] = rscale;
+      have_scale = true;
+    };
     for (int i = 0; i < nkb; ++i) {
       if (__any_sync(0xffffffffu, misc[1] != 0)) break;
       const int s = i % STAGES, b = i % C::B_BUFS;
@@ -239,15 +264,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
       const uint8_t* qs = st + C::A_BYTES;
       const uint32_t* ps = reinterpret_cast<const uint32_t*>(st + C::A_BYTES + C::Q_BYTES);
       uint8_t* bs = bbuf(b);
-      float g[16];
-      {
-        const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          g[2 * j] = gain ? bf2f((uint16_t)(gw[j] & 0xFFFFu)) : 1.f;
-          g[2 * j + 1] = gain ? bf2f((uint16_t)(gw[j] >> 16)) : 1.f;
-        }
-      }
+      const uint32_t g2[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
       // item = (row r, 16-code chunk c): 16 operand values = logical 16-byte
       // chunks 2c, 2c + 1 of the row's 128 bytes, stored at chunk ^ (r % 8)
 #pragma unroll
@@ -257,7 +274,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
         const uint32_t ab = ps[r];
         const float al = bf2f((uint16_t)(ab & 0xFFFFu)), be = bf2f((uint16_t)(ab >> 16));
         uint32_t o[8];
-        dequant16(qv, al, be, g, gain != nullptr, o);
+        dequant16(qv, al, be, g2, gain != nullptr, o);
         uint8_t* row = bs + r * 128;
         const int sw = r & 7;
         *reinterpret_cast<uint4*>(row + (((2 * c) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -266,15 +283,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
       fence_proxy_async_cta();  // generic stores -> visible to the tensor cores' async proxy
       __syncwarp();
       if (lane == 0) mbar_arrive(b_full(b));
+      if (i == pre - 1) epilogue_inputs();
     }
-    griddep_wait();  // outputs, residuals, biases and positions come from earlier kernels
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const int m = m_blk * GEMM_BM + row;
-    const bool row_ok = m < args.M;
-    prefetch_epilogue_inputs<BN, EPI>(args, m, n0, row_ok);
-    const float rscale = norm_row_scale(args, m, row_ok);
-    misc_scale[row] = rscale;
+    if (!have_scale) epilogue_inputs();  // the loop stopped early (time-out)
     bool ok = mbar_wait(acc_bar, 0, lim);
     if (!ok) {
       misc[1] = 1;
@@ -327,22 +338,15 @@ __global__ void __launch_bounds__(256) dequant_affine8_kernel(const uint8_t* __r
     const int n = (int)(idx / cpr), k = (int)(idx % cpr) * 16;
     const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + (size_t)n * K + k));
     const uint32_t pr = __ldg(reinterpret_cast<const uint32_t*>(ab) + (size_t)(k / W8_GROUP) * N + n);
-    float g[16];
+    uint4 g0 = make_uint4(0u, 0u, 0u, 0u), g1 = g0;
     if (gain) {
       const uint4* gp = reinterpret_cast<const uint4*>(gain + k);
-      const uint4 g0 = __ldg(gp), g1 = __ldg(gp + 1);
-      const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        g[2 * j] = bf2f((uint16_t)(gw[j] & 0xFFFFu));
-        g[2 * j + 1] = bf2f((uint16_t)(gw[j] >> 16));
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) g[j] = 1.f;
+      g0 = __ldg(gp);
+      g1 = __ldg(gp + 1);
     }
+    const uint32_t g2[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
     uint32_t o[8];
-    dequant16(qv, bf2f((uint16_t)(pr & 0xFFFFu)), bf2f((uint16_t)(pr >> 16)), g, gain != nullptr, o);
+    dequant16(qv, bf2f((uint16_t)(pr & 0xFFFFu)), bf2f((uint16_t)(pr >> 16)), g2, gain != nullptr, o);
     uint4* dst = reinterpret_cast<uint4*>(out + (size_t)n * K + k);
     dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
     dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
