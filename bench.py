@@ -41,6 +41,9 @@ L2_BYTES = 126 * 1024 * 1024
 #  - the persistent denoise kernel: profiles/denoise_fused_kernel_smolvla_b1.md.
 NCU_TRAFFIC_GEMM_B1 = 3.698e6
 NCU_TRAFFIC_FUSED = 1.9916e9
+#  - the int8 prefill's gate/up GEMM (gemm_w8_kernel<64, SwiGLU, 4>, M=177, N=5120, K=960):
+#    profiles/gemm_w8_kernel_smolvla_b1.md.
+NCU_TRAFFIC_W8_GATE_UP_B1 = 5.6445e6
 
 
 def _peaks():
@@ -403,6 +406,11 @@ def int8_prefix(args, dev, barrier, hbm_peak, peak_kind):
         w8, w16 = prefix_projection_bytes(s, 8), prefix_projection_bytes(s, 16)
         pre_bytes = chunk_work(s, wl.B, wl.L, wl.H, 0)[0] - w16 + w8
         achieved = pre_bytes / (t8 * 1e-3) / 1e9
+        if wl.B == 1:
+            M, N, K = wl.L, 2 * s.p_ffn, s.p_width
+            out["gemm_w8_gate_up_b1"] = {"kernel": "gemm_w8_kernel<64, SwiGLU, 4>", "M": M, "N": N, "K": K,
+                                         "algorithmic_bytes_per_launch": int(N * K + N * (K // 64) * 4 + 2 * M * K),
+                                         "traffic": NCU_TRAFFIC_W8_GATE_UP_B1}
         out[name] = {"prefill_ms": round(t8, 4), "prefill_ms_dense_same_handle": round(t16, 4),
                      "chunk_ms": round(c8 / wl.B, 4) if wl.B == 1 else None,
                      "chunks_per_s": round(wl.B / (c8 * 1e-3), 2) if wl.B > 1 else None,
