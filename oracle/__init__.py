@@ -37,3 +37,4 @@ from .model import (  # noqa: F401
 from .philox import philox4x32_10, gaussian_noise  # noqa: F401
 from .assembly import pixel_shuffle, connector, state_token, assemble_prefix  # noqa: F401
 from .quant import quantize_affine8, dequantize_affine8, quantize_prefix  # noqa: F401
+from .train import train_step, trainable_names, loss_np  # noqa: F401
