@@ -104,6 +104,11 @@ SVLA_API svla_status svla_create(const svla_config* cfg, const void* blob, size_
  *     Needs p_width and p_ffn multiples of 64 (they are, by check_config).
  * flags = 0 is svla_create. Unknown flag bits: SVLA_ERR_ARG. */
 #define SVLA_CREATE_PREFIX_INT8 1u
+/*   SVLA_CREATE_TRAIN  also keep the expert and head weights as given (no
+ *     folding or interleaving) and allocate the workspace of svla_train_step
+ *     for max_batch x max_chunk rows (every expert layer's activations are
+ *     kept for the backward: about 0.55 MB per row at the SmolVLA shape). */
+#define SVLA_CREATE_TRAIN 2u
 SVLA_API svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob_bytes,
                            int device, unsigned flags, svla_handle** out);
 
@@ -113,6 +118,30 @@ SVLA_API svla_status svla_create_ex(const svla_config* cfg, const void* blob, si
 SVLA_API svla_status svla_set_prefix_weights(svla_handle* h, int bits);
 /* The prefix weight width svla_prefill uses (16 or 8); 0 for a NULL handle. */
 SVLA_API int svla_prefix_weights(const svla_handle* h);
+
+/* Training step of the action expert ("noeira docs, SmolVLA" §Architecture,
+ * the fine-tune's flow-matching objective; §Fine-tuning: the 16 expert layers
+ * and the action and time projections train, the language model is frozen).
+ * Readings: x_t = t_b eps + (1 - t_b) a per query, v = v(x_t, t_b | prefix),
+ * loss = mean over the B H A terms of (v - (eps - a))^2; the result is the loss
+ * and its gradient with respect to every expert and head tensor (no optimiser
+ * update).
+ *   kv_cache, pad_mask: the frozen prefix, as for svla_denoise (device).
+ *   actions: the target chunk a, noise: eps, device float32 [B, H, A];
+ *   t: device float32 [B], the flow time of each query.
+ *   loss: device float32 scalar (written).
+ *   grads: device float32, svla_train_grad_elems(h) elements, 16-byte aligned:
+ *     every tensor of the blob from the first expert layer's in_norm to b_out,
+ *     in manifest order and shape ([out, in] for matrices) (written in full).
+ * The forward uses the weights given to svla_create_ex; work is stream-ordered
+ * and bitwise reproducible (fixed-order reductions). Needs a handle created
+ * with SVLA_CREATE_TRAIN (else SVLA_ERR_UNSUPPORTED); B, L, H within the
+ * handle's limits (else SVLA_ERR_SHAPE). */
+SVLA_API svla_status svla_train_step(svla_handle* h, const void* kv_cache, const uint8_t* pad_mask, int B,
+                            int L, const float* actions, const float* noise, const float* t, int H,
+                            float* loss, float* grads, void* stream);
+/* Number of float32 gradient elements of svla_train_step (0 without a training workspace). */
+SVLA_API size_t svla_train_grad_elems(const svla_handle* h);
 
 /* Free everything the handle owns (synchronises its device first). NULL is ok. */
 SVLA_API svla_status svla_destroy(svla_handle* h);

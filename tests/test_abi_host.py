@@ -131,7 +131,7 @@ def test_int8_argument_checks_and_plan():
     blob = np.zeros(16, np.uint16)
     h = ctypes.c_void_p()
     cfg = config_from_shape(s, 1, 24, 8)
-    assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, 2,
+    assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, 4,
                               ctypes.byref(h)) == _abi.SVLA_ERR_ARG
     cfg = config_from_shape(s.replace(p_heads=3, p_kv_heads=1), 1, 24, 8)  # O projection K = 96
     assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0,
@@ -160,3 +160,19 @@ def test_int8_argument_checks_and_plan():
     assert lib.svla_op_gemm_w8_splits(5664, 5120, 960) == 1
     assert lib.svla_op_gemm_w8_tile_n(5664, 5120, 960) == 128
     assert lib.svla_op_gemm_w8_splits(177, 1600, 100) == 0
+
+
+def test_train_argument_checks():
+    lib = _abi.load()
+    assert lib.svla_train_grad_elems(None) == 0
+    p = ctypes.c_void_p(16)
+    assert lib.svla_train_step(None, p, p, 1, 1, p, p, p, 1, p, p, None) == _abi.SVLA_ERR_ARG
+    s = synth.SHAPES["tiny"]
+    blob = np.zeros(16, np.uint16)
+    h = ctypes.c_void_p()
+    cfg = config_from_shape(s, 1, 24, 8)
+    # unknown flag bits are rejected before the blob size
+    assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, 4,
+                              ctypes.byref(h)) == _abi.SVLA_ERR_ARG
+    assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, _abi.CREATE_TRAIN,
+                              ctypes.byref(h)) == _abi.SVLA_ERR_BLOB_SIZE

@@ -1,0 +1,111 @@
+"""The training step of the expert (the flow-matching fine-tune; readings 25-27
+in ``oracle/train.py``) through the C ABI against the oracle: the loss and the
+gradient of every trainable tensor, on the tiny shape and on the SmolVLA shape
+(two queries with padded prefixes, chunk 50, prefix 177), plus bitwise
+reproducibility and the handle flag.
+
+Gates, derived from the arithmetic of the step: the forward keeps bf16
+activations and the backward rounds every GEMM operand (the residual's
+gradient, dgu, dq/dk/dv, the transposed activations) to bf16 once per layer,
+each rounding a relative 2^-9; sixteen layers of such roundings stay well
+inside 3e-2 relative L2 per gradient tensor. The loss is dominated by the
+target eps - a and is held to 1e-3 relative.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+import synth  # noqa: E402
+from oracle import train as ot  # noqa: E402
+from tests import helpers as H  # noqa: E402
+from vision_language_action_b200 import _abi  # noqa: E402
+from vision_language_action_b200.runtime import SmolVLA  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+DEV = "cuda:0"
+GRAD_REL_L2 = 3e-2
+LOSS_REL = 1e-3
+
+
+def make_case(shape, B, L, Hc, seed):
+    s = synth.SHAPES[shape]
+    wb = synth.gen_weights(s, seed, random_affine=True)
+    rng = np.random.default_rng([seed, 31])
+    kv_bits = synth.f32_to_bf16_bits(rng.standard_normal((2, s.p_layers, B, L, s.p_kv_width)).astype(np.float32))
+    valid = np.ones((B, L), np.uint8)
+    valid[0, 1] = 0
+    if B > 1:
+        valid[1, L - 3:] = 0
+    a = (0.5 * rng.standard_normal((B, Hc, s.action_dim))).astype(np.float32)
+    eps = rng.standard_normal((B, Hc, s.action_dim)).astype(np.float32)
+    t = rng.uniform(0.05, 0.95, B).astype(np.float32)
+    return s, wb, kv_bits, valid, a, eps, t
+
+
+def oracle_step(s, wb, kv_bits, valid, a, eps, t):
+    W = oracle.load_weights(wb)
+    B, L = valid.shape
+    kv = synth.bf16_bits_to_f32(kv_bits).astype(np.float64)          # [2, layers, B, L, kv*hd]
+    K = kv[0].transpose(1, 0, 2, 3).reshape(B, s.p_layers, L, s.p_kv_heads, s.head_dim)
+    V = kv[1].transpose(1, 0, 2, 3).reshape(B, s.p_layers, L, s.p_kv_heads, s.head_dim)
+    return ot.train_step(W, s, K, V, valid, a.astype(np.float64), eps.astype(np.float64), t.astype(np.float64))
+
+
+def gpu_step(m, kv_bits, valid, a, eps, t):
+    kv = torch.from_numpy(kv_bits.view(np.int16)).to(DEV).view(torch.bfloat16)
+    loss, grads = m.train_step(kv, torch.from_numpy(valid).to(DEV), torch.from_numpy(a).to(DEV),
+                               torch.from_numpy(eps).to(DEV), torch.from_numpy(t).to(DEV))
+    assert m.device_status() == _abi.SVLA_OK
+    torch.cuda.synchronize()
+    return float(loss.item()), grads.cpu().numpy()
+
+
+def split_grads(s, g):
+    out, off = {}, 0
+    for name, shp in synth.manifest(s):
+        if name.startswith("p"):
+            continue
+        n = int(np.prod(shp))
+        out[name] = g[off:off + n].reshape(shp)
+        off += n
+    assert off == g.size
+    return out
+
+
+@pytest.mark.parametrize("shape,B,L,Hc", [("tiny", 2, 24, 8), ("smolvla", 2, 177, 50)])
+def test_train_step_matches_oracle(shape, B, L, Hc):
+    s, wb, kv_bits, valid, a, eps, t = make_case(shape, B, L, Hc, 7)
+    m = SmolVLA(s, synth.pack_blob(s, wb), max_batch=B, max_prefix=L, max_chunk=Hc, train=True)
+    try:
+        assert int(m.lib.svla_train_grad_elems(m.h)) == synth.param_count(s, "expert")
+        loss, g = gpu_step(m, kv_bits, valid, a, eps, t)
+        loss2, g2 = gpu_step(m, kv_bits, valid, a, eps, t)
+    finally:
+        m.close()
+    assert loss == loss2 and np.array_equal(g, g2), "training step is not bitwise reproducible"
+    ref_loss, ref = oracle_step(s, wb, kv_bits, valid, a, eps, t)
+    got = split_grads(s, g)
+    errs = {n: H.rel_l2(got[n], ref[n]) for n in ot.trainable_names(s)}
+    worst = sorted(errs.items(), key=lambda kv: -kv[1])
+    print(f"\n{shape}: loss {loss:.6f} oracle {ref_loss:.6f}; worst gradient rel L2:",
+          ", ".join(f"{n} {e:.2e}" for n, e in worst[:8]))
+    assert abs(loss - ref_loss) <= LOSS_REL * ref_loss, (loss, ref_loss)
+    bad = [(n, e) for n, e in worst if not e <= GRAD_REL_L2]
+    assert not bad, bad
+
+
+def test_train_step_needs_the_flag():
+    s, wb, kv_bits, valid, a, eps, t = make_case("tiny", 1, 24, 8, 3)
+    m = SmolVLA(s, synth.pack_blob(s, wb), max_batch=1, max_prefix=24, max_chunk=8)
+    try:
+        assert int(m.lib.svla_train_grad_elems(m.h)) == 0
+        with pytest.raises(_abi.SvlaError):
+            gpu_step(m, kv_bits, valid, a, eps, t)
+    finally:
+        m.close()

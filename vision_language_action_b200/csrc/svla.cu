@@ -24,6 +24,7 @@
 #include "denoise_fused.cuh"
 #include "gemm_host.cuh"
 #include "small_kernels.cuh"
+#include "train.cuh"
 
 using namespace svla;
 
@@ -227,6 +228,26 @@ struct Q8Mat {
   int N = 0, K = 0;
 };
 
+// Training workspace (svla_create_ex with SVLA_CREATE_TRAIN), sized by
+// max_batch, max_chunk and max_prefix. Per expert layer the forward keeps the
+// residual entering the layer and after attention (fp32), both normalised
+// operands, q / k / v / attention output, the gate/up pre-activations (fp32)
+// and the SwiGLU output.
+struct TrainWs {
+  uint16_t* tw = nullptr;  // expert + head weights as given (manifest order, no folding or interleaving)
+  size_t base = 0;         // manifest offset of the first expert tensor (= offset 0 of tw and of the gradients)
+  int Me = 0;              // rows max_batch * max_chunk
+  float *r = nullptr, *rm = nullptr, *gu = nullptr;
+  uint16_t *y = nullptr, *y2 = nullptr, *q = nullptr, *k = nullptr, *v = nullptr, *o = nullptr, *hs = nullptr;
+  float *xt = nullptr, *aemb = nullptr, *z1 = nullptr, *yf = nullptr, *dv = nullptr, *loss_row = nullptr;
+  float *dyf = nullptr, *b_t1f = nullptr;
+  uint16_t *cat = nullptr, *h1 = nullptr;
+  // backward
+  float *dr = nullptr, *dx = nullptr, *dz = nullptr, *rs = nullptr, *P = nullptr, *dS = nullptr;
+  uint16_t *drb = nullptr, *dgu = nullptr, *dqkv = nullptr, *dkx = nullptr, *dvx = nullptr, *dob = nullptr;
+  uint16_t *wt = nullptr, *ta = nullptr, *tb = nullptr;
+};
+
 struct GraphEntry {
   std::vector<uint64_t> key;
   cudaGraphExec_t exec = nullptr;
@@ -269,6 +290,7 @@ struct svla_handle {
   uint16_t* q8_deq = nullptr;  // one dequantised projection (bf16), for many-tile GEMMs
   std::vector<Q8Mat> q8m;    // per prefix layer: QKV, O, gate/up (interleaved rows), down
   int prefix_bits = 16;      // weights svla_prefill uses
+  TrainWs* tr = nullptr;     // training workspace (SVLA_CREATE_TRAIN)
   // prefix assembly (svla_set_assembly): connector and state-projection weights, workspaces
   uint16_t* asm_w = nullptr;   // W_c [p_width, r*r*C] | W_s [p_width, S] | b_s [p_width]
   uint16_t* asm_a = nullptr;   // gathered connector operand [max_batch * max_images * tpi, r*r*C]
@@ -316,6 +338,8 @@ cudaError_t halloc(svla_handle* h, T** p, size_t count) {
 }
 
 void free_all(svla_handle* h) {
+  delete h->tr;
+  h->tr = nullptr;
   for (auto& g : h->graphs)
     if (g.exec) cudaGraphExecDestroy(g.exec);
   h->graphs.clear();
@@ -456,6 +480,285 @@ void norm_consumer(GemmArgs& a, const float* ss, int tiles, int M, int D, float 
   a.ss_ld = M;
   a.norm_inv_dim = 1.f / (float)D;
   a.norm_eps = eps;
+}
+
+// ---- training step of the expert (flow-matching fine-tune) ------------------
+// Forward over the B H rows at the flow times t_b, keeping every layer's
+// activations (weights as given: RMSNorm gains applied by the norm kernel, not
+// folded), the loss and the head's backward, then the backward of the 16
+// layers and of the time MLP / action_in. Products run on the tcgen05 GEMM as
+// C = A B^T: dX = dY W uses a transposed copy of W, dW = dY^T X uses
+// transposed copies of dY and X (rows zero-padded to a multiple of 64). Those
+// GEMMs launch after everything before them (pdl = false): their B operand is
+// written by the kernel before, and the GEMM streams B before its dependency
+// wait. Gradients are fp32, in manifest order from the first expert tensor.
+cudaError_t record_train(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* act,
+                         const float* eps, const float* t, int H, float* loss, float* grads, cudaStream_t s) {
+  const svla_config& c = h->cfg;
+  TrainWs& T = *h->tr;
+  const Layout& Ly = h->lay;
+  const int M = B * H, E = c.e_width, hd = c.head_dim, A = c.action_dim, F = c.e_ffn;
+  const int nq = c.e_heads, nkv = c.e_kv_heads;
+  const int qw = nq * hd, kvw = nkv * hd, pkvw = c.p_kv_heads * hd, qkvw = qw + 2 * kvw;
+  const int Lb = B * L;
+  const int Mp = (M + 63) / 64 * 64, Lp = (Lb + 63) / 64 * 64;
+  const uint16_t* cache = reinterpret_cast<const uint16_t*>(kv);
+  const size_t layer_elems = (size_t)Lb * pkvw;
+  const size_t Me = (size_t)T.Me;
+  const float inv_n = 1.f / (float)((size_t)M * A);
+  const float scale = (float)(1.0 / std::sqrt((double)hd));
+  auto TW = [&](size_t off) { return T.tw + (off - T.base); };
+  auto G = [&](size_t off) { return grads + (off - T.base); };
+  auto R = [&](int l) { return T.r + (size_t)l * Me * E; };
+  auto RM = [&](int l) { return T.rm + (size_t)l * Me * E; };
+  auto Y = [&](int l) { return T.y + (size_t)l * Me * E; };
+  auto Y2 = [&](int l) { return T.y2 + (size_t)l * Me * E; };
+  auto Q = [&](int l) { return T.q + (size_t)l * Me * qw; };
+  auto O = [&](int l) { return T.o + (size_t)l * Me * qw; };
+  auto Kl = [&](int l) { return T.k + (size_t)l * Me * kvw; };
+  auto Vl = [&](int l) { return T.v + (size_t)l * Me * kvw; };
+  auto GU = [&](int l) { return T.gu + (size_t)l * Me * 2 * F; };
+  auto HS = [&](int l) { return T.hs + (size_t)l * Me * F; };
+  auto KX = [&](int l) { return reinterpret_cast<uint16_t*>(h->kvx) + (size_t)(l / 2) * 2 * Lb * kvw; };
+  auto bf = [](const uint16_t* p) { return reinterpret_cast<const bf16*>(p); };
+  auto ew = [](size_t n) { return dim3((unsigned)std::min<size_t>((n + 255) / 256, 8 * NUM_SMS_B200)); };
+  // C[Mr, N] = A[Mr, K] B[N, K]^T, after all earlier work
+  auto mm = [&](int epi, const uint16_t* Am, int lda, const uint16_t* Bm, int ldb, int Mr, int N, int K,
+                GemmArgs ga) {
+    return gemm(h, epi, bf(Am), lda, bf(Bm), ldb, Mr, N, K, ga, h->e_part, h->e_cnt, s, /*pdl=*/false);
+  };
+  auto tr16 = [&](const uint16_t* in, int Rr, int C, size_t ld, uint16_t* out, int Rp) {
+    return launch_pdl(transpose_kernel<uint16_t>, dim3((C + 31) / 32, (Rp + 31) / 32), dim3(32, 8), 0, s, in, Rr, C,
+                      ld, out, Rp);
+  };
+  auto norm_bwd = [&](const float* r, const uint16_t* g, const float* dy, float* dg) {
+    SVLA_TRY(launch_pdl(norm_bwd_kernel, dim3((M + 7) / 8), dim3(256), 0, s, r, g, dy, M, E, c.rms_eps, T.dr, T.drb,
+                        T.rs));
+    return launch_pdl(norm_gain_grad_kernel, dim3((E + 255) / 256), dim3(256), 0, s, r, (const float*)T.rs, dy, M, E,
+                      dg);
+  };
+  auto colsum = [&](const float* x, int C, int ld, float* out) {
+    return launch_pdl(colsum_kernel, dim3((C + 255) / 256), dim3(256), 0, s, x, M, C, ld, out);
+  };
+
+  // ---- forward ----
+  SVLA_TRY(launch_pdl(train_begin_kernel, dim3(M), dim3(256), 0, s, act, eps, t, H, A, E, TW(Ly.w_in.off),
+                      TW(Ly.b_in.off), (const double*)h->inv_period, T.xt, T.aemb, T.cat));
+  SVLA_TRY(mm(GE_F32, T.cat, 2 * E, TW(Ly.w_t1.off), 2 * E, M, E, 2 * E, out_args(T.z1, E, T.b_t1f)));
+  SVLA_TRY(launch_pdl(silu_fwd_kernel, ew((size_t)M * E), dim3(256), 0, s, (const float*)T.z1, (size_t)M * E, T.h1));
+  SVLA_TRY(mm(GE_F32, T.h1, E, TW(Ly.w_t2.off), E, M, E, E, out_args(R(0), E, h->b_t2_f32)));
+  for (int l = 0; l < c.e_layers; ++l) {
+    const Entry* e = &Ly.e[9 * l];
+    SVLA_TRY(rmsnorm(R(l), false, nullptr, bf(TW(e[0].off)), M, E, c.rms_eps, reinterpret_cast<bf16*>(Y(l)), s));
+    if (l % 2 == 0) {
+      GemmArgs qa = out_args(nullptr, 0);
+      qa.q_out = reinterpret_cast<bf16*>(Q(l));
+      qa.ldq = qw;
+      qa.k_out = reinterpret_cast<bf16*>(Kl(l));
+      qa.v_out = reinterpret_cast<bf16*>(Vl(l));
+      qa.ldkv = kvw;
+      qa.q_cols = qw;
+      qa.kv_cols = kvw;
+      qa.pos = nullptr;
+      qa.pos_mod = H;  // chunk positions 0..H-1 (reading 4)
+      qa.rope_cs = h->rope_cs;
+      SVLA_TRY(mm(hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32, Y(l), E, TW(e[1].off), E, M, qkvw, E, qa));
+      SVLA_TRY(attention(bf(Q(l)), qw, bf(Kl(l)), bf(Vl(l)), kvw, nullptr, B, nq, nkv, hd, H, H, 1,
+                         reinterpret_cast<bf16*>(O(l)), qw, s));
+    } else {
+      SVLA_TRY(mm(GE_BF16, Y(l), E, TW(e[1].off), E, M, qw, E, out_args(Q(l), qw)));
+      uint16_t* kx = KX(l);
+      uint16_t* vx = kx + (size_t)Lb * kvw;
+      SVLA_TRY(mm(GE_BF16, cache + (size_t)l * layer_elems, pkvw, TW(e[2].off), pkvw, Lb, kvw, pkvw, out_args(kx, kvw)));
+      SVLA_TRY(mm(GE_BF16, cache + (size_t)(c.p_layers + l) * layer_elems, pkvw, TW(e[3].off), pkvw, Lb, kvw, pkvw,
+                  out_args(vx, kvw)));
+      SVLA_TRY(attention(bf(Q(l)), qw, bf(kx), bf(vx), kvw, pad, B, nq, nkv, hd, H, L, 0,
+                         reinterpret_cast<bf16*>(O(l)), qw, s));
+    }
+    SVLA_TRY(cudaMemcpyAsync(RM(l), R(l), (size_t)M * E * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    SVLA_TRY(mm(GE_ADD_F32, O(l), qw, TW(e[4].off), qw, M, E, qw, out_args(RM(l), E)));
+    SVLA_TRY(rmsnorm(RM(l), false, nullptr, bf(TW(e[5].off)), M, E, c.rms_eps, reinterpret_cast<bf16*>(Y2(l)), s));
+    SVLA_TRY(mm(GE_F32, Y2(l), E, TW(e[6].off), E, M, 2 * F, E, out_args(GU(l), 2 * F)));  // [gate | up] rows
+    SVLA_TRY(launch_pdl(swiglu_fwd_kernel, ew((size_t)M * F), dim3(256), 0, s, (const float*)GU(l), M, F, HS(l)));
+    SVLA_TRY(cudaMemcpyAsync(R(l + 1), RM(l), (size_t)M * E * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    SVLA_TRY(mm(GE_ADD_F32, HS(l), F, TW(e[8].off), F, M, E, F, out_args(R(l + 1), E)));
+  }
+  // ---- loss and the head ----
+  const float* Rf = R(c.e_layers);
+  SVLA_TRY(launch_pdl(train_head_kernel, dim3(M), dim3(256), (size_t)(E + 2 * A + 32) * sizeof(float), s, Rf,
+                      TW(Ly.final_norm.off), TW(Ly.w_out.off), TW(Ly.b_out.off), act, eps, E, A, inv_n, c.rms_eps,
+                      T.yf, T.dv, T.loss_row, T.dyf));
+  SVLA_TRY(launch_pdl(loss_reduce_kernel, dim3(1), dim3(1024), 0, s, (const float*)T.loss_row, M, inv_n, loss));
+  SVLA_TRY(colsum(T.dv, A, A, G(Ly.b_out.off)));
+  SVLA_TRY(launch_pdl(outer_kernel, dim3((unsigned)(((size_t)A * E + 255) / 256)), dim3(256), 0, s,
+                      (const float*)T.dv, A, (const float*)T.yf, E, M, A, E, G(Ly.w_out.off)));
+  SVLA_TRY(cudaMemsetAsync(T.dr, 0, (size_t)M * E * sizeof(float), s));
+  SVLA_TRY(norm_bwd(Rf, TW(Ly.final_norm.off), T.dyf, G(Ly.final_norm.off)));
+  // ---- the layers, last first; T.dr holds dL/d(residual) ----
+  for (int l = c.e_layers - 1; l >= 0; --l) {
+    const Entry* e = &Ly.e[9 * l];
+    // down: R(l+1) = RM(l) + HS W_d^T
+    SVLA_TRY(tr16(T.drb, M, E, E, T.ta, Mp));
+    SVLA_TRY(tr16(HS(l), M, F, F, T.tb, Mp));
+    SVLA_TRY(mm(GE_F32, T.ta, Mp, T.tb, Mp, E, F, Mp, out_args(G(e[8].off), F)));
+    SVLA_TRY(tr16(TW(e[8].off), E, F, F, T.wt, E));
+    SVLA_TRY(mm(GE_F32, T.drb, E, T.wt, E, M, F, E, out_args(T.dx, F)));
+    SVLA_TRY(launch_pdl(swiglu_bwd_kernel, ew((size_t)M * F), dim3(256), 0, s, (const float*)GU(l), (const float*)T.dx,
+                        M, F, T.dgu));
+    // gate/up: GU = Y2 [W_g; W_u]^T
+    SVLA_TRY(tr16(T.dgu, M, 2 * F, 2 * F, T.ta, Mp));
+    SVLA_TRY(tr16(Y2(l), M, E, E, T.tb, Mp));
+    SVLA_TRY(mm(GE_F32, T.ta, Mp, T.tb, Mp, 2 * F, E, Mp, out_args(G(e[6].off), E)));
+    SVLA_TRY(tr16(TW(e[6].off), 2 * F, E, E, T.wt, 2 * F));
+    SVLA_TRY(mm(GE_F32, T.dgu, 2 * F, T.wt, 2 * F, M, E, 2 * F, out_args(T.dx, E)));
+    SVLA_TRY(norm_bwd(RM(l), TW(e[5].off), T.dx, G(e[5].off)));  // T.dr = dL/dRM(l)
+    // O: RM(l) = R(l) + O W_o^T
+    SVLA_TRY(tr16(T.drb, M, E, E, T.ta, Mp));
+    SVLA_TRY(tr16(O(l), M, qw, qw, T.tb, Mp));
+    SVLA_TRY(mm(GE_F32, T.ta, Mp, T.tb, Mp, E, qw, Mp, out_args(G(e[4].off), qw)));
+    SVLA_TRY(tr16(TW(e[4].off), E, qw, qw, T.wt, E));
+    SVLA_TRY(mm(GE_BF16, T.drb, E, T.wt, E, M, qw, E, out_args(T.dob, qw)));
+    // attention
+    AttnBwdArgs ab;
+    ab.q = Q(l);
+    ab.ldq = qw;
+    ab.dout = T.dob;
+    ab.ldo = qw;
+    ab.B = B;
+    ab.nq = nq;
+    ab.nkv = nkv;
+    ab.hd = hd;
+    ab.Tq = H;
+    ab.scale = scale;
+    ab.P = T.P;
+    ab.dS = T.dS;
+    ab.dq = T.dqkv;
+    if (l % 2 == 0) {
+      ab.k = Kl(l);
+      ab.v = Vl(l);
+      ab.ldkv = kvw;
+      ab.key_valid = nullptr;
+      ab.Tk = H;
+      ab.causal = 1;
+      ab.lddq = qkvw;
+      ab.dk = T.dqkv + qw;
+      ab.dv = T.dqkv + qw + kvw;
+      ab.lddkv = qkvw;
+      ab.rope_cs = h->rope_cs;
+    } else {
+      ab.k = KX(l);
+      ab.v = KX(l) + (size_t)Lb * kvw;
+      ab.ldkv = kvw;
+      ab.key_valid = pad;
+      ab.Tk = L;
+      ab.causal = 0;
+      ab.lddq = qw;
+      ab.dk = T.dkx;
+      ab.dv = T.dvx;
+      ab.lddkv = kvw;
+      ab.rope_cs = nullptr;
+    }
+    SVLA_TRY(launch_pdl(attn_bwd_rows_kernel, dim3((unsigned)(((size_t)B * nq * H + 7) / 8)), dim3(256),
+                        (size_t)8 * 3 * hd * sizeof(float), s, ab));
+    SVLA_TRY(launch_pdl(attn_bwd_keys_kernel, dim3((unsigned)(((size_t)B * nkv * ab.Tk + 7) / 8)), dim3(256),
+                        (size_t)8 * 2 * hd * sizeof(float), s, ab));
+    const int wq_rows = l % 2 == 0 ? qkvw : qw;  // even: [W_q; W_k; W_v] share the input y
+    SVLA_TRY(tr16(T.dqkv, M, wq_rows, wq_rows, T.ta, Mp));
+    SVLA_TRY(tr16(Y(l), M, E, E, T.tb, Mp));
+    SVLA_TRY(mm(GE_F32, T.ta, Mp, T.tb, Mp, wq_rows, E, Mp, out_args(G(e[1].off), E)));
+    SVLA_TRY(tr16(TW(e[1].off), wq_rows, E, E, T.wt, wq_rows));
+    SVLA_TRY(mm(GE_F32, T.dqkv, wq_rows, T.wt, wq_rows, M, E, wq_rows, out_args(T.dx, E)));
+    if (l % 2 == 1) {
+      // the cross projections of the frozen cache: K' = K_c W_k^T, V' = V_c W_v^T
+      SVLA_TRY(tr16(T.dkx, Lb, kvw, kvw, T.ta, Lp));
+      SVLA_TRY(tr16(cache + (size_t)l * layer_elems, Lb, pkvw, pkvw, T.tb, Lp));
+      SVLA_TRY(mm(GE_F32, T.ta, Lp, T.tb, Lp, kvw, pkvw, Lp, out_args(G(e[2].off), pkvw)));
+      SVLA_TRY(tr16(T.dvx, Lb, kvw, kvw, T.ta, Lp));
+      SVLA_TRY(tr16(cache + (size_t)(c.p_layers + l) * layer_elems, Lb, pkvw, pkvw, T.tb, Lp));
+      SVLA_TRY(mm(GE_F32, T.ta, Lp, T.tb, Lp, kvw, pkvw, Lp, out_args(G(e[3].off), pkvw)));
+    }
+    SVLA_TRY(norm_bwd(R(l), TW(e[0].off), T.dx, G(e[0].off)));  // T.dr = dL/dR(l)
+  }
+  // ---- time MLP and action_in: R(0) = silu(Z1) W_t2^T + b_t2, Z1 = [a_emb | e(t)] W_t1^T + b_t1 ----
+  SVLA_TRY(colsum(T.dr, E, E, G(Ly.b_t2.off)));
+  SVLA_TRY(tr16(T.drb, M, E, E, T.ta, Mp));
+  SVLA_TRY(tr16(T.h1, M, E, E, T.tb, Mp));
+  SVLA_TRY(mm(GE_F32, T.ta, Mp, T.tb, Mp, E, E, Mp, out_args(G(Ly.w_t2.off), E)));
+  SVLA_TRY(tr16(TW(Ly.w_t2.off), E, E, E, T.wt, E));
+  SVLA_TRY(mm(GE_F32, T.drb, E, T.wt, E, M, E, E, out_args(T.dx, E)));
+  uint16_t* dzb = T.dgu;  // bf16 dZ1 [M, E]
+  SVLA_TRY(launch_pdl(silu_bwd_kernel, ew((size_t)M * E), dim3(256), 0, s, (const float*)T.z1, (const float*)T.dx,
+                      (size_t)M * E, T.dz, dzb));
+  SVLA_TRY(colsum(T.dz, E, E, G(Ly.b_t1.off)));
+  SVLA_TRY(tr16(dzb, M, E, E, T.ta, Mp));
+  SVLA_TRY(tr16(T.cat, M, 2 * E, 2 * E, T.tb, Mp));
+  SVLA_TRY(mm(GE_F32, T.ta, Mp, T.tb, Mp, E, 2 * E, Mp, out_args(G(Ly.w_t1.off), 2 * E)));
+  SVLA_TRY(tr16(TW(Ly.w_t1.off), E, E, 2 * E, T.wt, E));  // W_t1[:, :E]^T
+  SVLA_TRY(mm(GE_F32, dzb, E, T.wt, E, M, E, E, out_args(T.dx, E)));  // dL/d a_emb
+  SVLA_TRY(colsum(T.dx, E, E, G(Ly.b_in.off)));
+  SVLA_TRY(launch_pdl(outer_kernel, dim3((unsigned)(((size_t)E * A + 255) / 256)), dim3(256), 0, s,
+                      (const float*)T.dx, E, (const float*)T.xt, A, M, E, A, G(Ly.w_in.off)));
+  return cudaSuccess;
+}
+
+// Allocate the training workspace (after the weights and tw are in place).
+cudaError_t alloc_train(svla_handle* h) {
+  const svla_config& c = h->cfg;
+  TrainWs& T = *h->tr;
+  const size_t Me = (size_t)c.max_batch * c.max_chunk, Lb = (size_t)c.max_batch * c.max_prefix;
+  const size_t E = c.e_width, F = c.e_ffn, A = c.action_dim, hd = c.head_dim;
+  const size_t qw = c.e_heads * hd, kvw = c.e_kv_heads * hd, pkvw = c.p_kv_heads * hd, qkvw = qw + 2 * kvw;
+  const size_t NL = c.e_layers;
+  const size_t Mp = (Me + 63) / 64 * 64, Lp = (Lb + 63) / 64 * 64;
+  T.Me = (int)Me;
+  cudaError_t e = cudaSuccess;
+  auto al = [&](auto** p, size_t n) {
+    if (e == cudaSuccess) e = halloc(h, p, n);
+  };
+  al(&T.r, (NL + 1) * Me * E);
+  al(&T.rm, NL * Me * E);
+  al(&T.y, NL * Me * E);
+  al(&T.y2, NL * Me * E);
+  al(&T.q, NL * Me * qw);
+  al(&T.o, NL * Me * qw);
+  al(&T.k, NL * Me * kvw);
+  al(&T.v, NL * Me * kvw);
+  al(&T.gu, NL * Me * 2 * F);
+  al(&T.hs, NL * Me * F);
+  al(&T.xt, Me * A);
+  al(&T.aemb, Me * E);
+  al(&T.z1, Me * E);
+  al(&T.yf, Me * E);
+  al(&T.dv, Me * A);
+  al(&T.loss_row, Me);
+  al(&T.dyf, Me * E);
+  al(&T.b_t1f, E);
+  al(&T.cat, Me * 2 * E);
+  al(&T.h1, Me * E);
+  const size_t maxw = std::max({2 * F, qkvw, 2 * E});
+  al(&T.dr, Me * E);
+  al(&T.dx, Me * maxw);
+  al(&T.dz, Me * E);
+  al(&T.rs, Me);
+  const size_t pn = (size_t)c.max_batch * c.e_heads * c.max_chunk * std::max(c.max_chunk, c.max_prefix);
+  al(&T.P, pn);
+  al(&T.dS, pn);
+  al(&T.drb, Me * E);
+  al(&T.dgu, Me * 2 * F);
+  al(&T.dqkv, Me * qkvw);
+  al(&T.dkx, Lb * kvw);
+  al(&T.dvx, Lb * kvw);
+  al(&T.dob, Me * qw);
+  const size_t maxnk = std::max({2 * F * E, qkvw * E, E * qw, E * F, 2 * E * E, kvw * pkvw});
+  al(&T.wt, maxnk);
+  const size_t maxc = std::max({2 * F, qkvw, 2 * E, F, qw, pkvw, kvw, E});
+  al(&T.ta, maxc * std::max(Mp, Lp));
+  al(&T.tb, maxc * std::max(Mp, Lp));
+  if (e == cudaSuccess) {
+    bf16_to_f32_kernel<<<(unsigned)((E + 255) / 256), 256>>>(T.tw + (h->lay.b_t1.off - T.base), T.b_t1f, (int)E);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 // ---- prefill schedule -------------------------------------------------------
@@ -850,7 +1153,7 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
                            svla_handle** out) {
   if (out) *out = nullptr;
   if (!cfg || !blob || !out) return fail(nullptr, SVLA_ERR_ARG, "null argument");
-  if (flags & ~SVLA_CREATE_PREFIX_INT8) return fail(nullptr, SVLA_ERR_ARG, "unknown flag bits");
+  if (flags & ~(SVLA_CREATE_PREFIX_INT8 | SVLA_CREATE_TRAIN)) return fail(nullptr, SVLA_ERR_ARG, "unknown flag bits");
   if ((flags & SVLA_CREATE_PREFIX_INT8) && (cfg->p_heads * cfg->head_dim) % 64)
     return fail(nullptr, SVLA_ERR_SHAPE, "int8 prefix weights need p_heads * head_dim to be a multiple of 64");
   if (const char* why = check_config(*cfg)) return fail(nullptr, SVLA_ERR_SHAPE, why);
@@ -880,6 +1183,15 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
   cudaError_t e;
   if ((e = halloc(h, &h->w, lay.total)) != cudaSuccess) return bail(e, "weights");
   if ((e = cudaMemcpy(h->w, blob, blob_bytes, cudaMemcpyDefault)) != cudaSuccess) return bail(e, "weight copy");
+  if (flags & SVLA_CREATE_TRAIN) {
+    // the expert and head weights as given, before the layout changes below
+    h->tr = new TrainWs();
+    h->tr->base = lay.e[0].off;
+    const size_t n = lay.total - h->tr->base;
+    if ((e = halloc(h, &h->tr->tw, n)) != cudaSuccess) return bail(e, "training weights");
+    if ((e = cudaMemcpy(h->tr->tw, h->w + h->tr->base, n * 2, cudaMemcpyDeviceToDevice)) != cudaSuccess)
+      return bail(e, "training weights");
+  }
   // gate/up rows -> interleaved 32-row groups [gate | up], in place via a scratch copy
   {
     size_t max_gu = std::max((size_t)2 * c.p_ffn * c.p_width, (size_t)2 * c.e_ffn * c.e_width);
@@ -1049,6 +1361,7 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
   }
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming);
   if (e != cudaSuccess) return bail(e, "streams");
+  if (h->tr && (e = alloc_train(h)) != cudaSuccess) return bail(e, "training workspace");
   if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(e, "create");
   *out = h;
   return SVLA_OK;
@@ -1166,6 +1479,27 @@ svla_status svla_set_prefix_weights(svla_handle* h, int bits) {
 }
 
 int svla_prefix_weights(const svla_handle* h) { return h ? h->prefix_bits : 0; }
+
+size_t svla_train_grad_elems(const svla_handle* h) { return h && h->tr ? h->lay.total - h->tr->base : 0; }
+
+svla_status svla_train_step(svla_handle* h, const void* kv_cache, const uint8_t* pad_mask, int B, int L,
+                            const float* actions, const float* noise, const float* t, int H, float* loss,
+                            float* grads, void* stream) {
+  if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
+  if (!kv_cache || !pad_mask || !actions || !noise || !t || !loss || !grads)
+    return fail(h, SVLA_ERR_ARG, "null pointer");
+  if (!h->tr) return fail(h, SVLA_ERR_UNSUPPORTED, "the handle has no training workspace (create it with SVLA_CREATE_TRAIN)");
+  if (B < 1 || L < 1 || B > h->cfg.max_batch || L > h->cfg.max_prefix)
+    return fail(h, SVLA_ERR_SHAPE, "B or L outside [1, max_batch] x [1, max_prefix]");
+  if (H < 1 || H > h->cfg.max_chunk) return fail(h, SVLA_ERR_SHAPE, "H outside [1, max_chunk]");
+  if (((uintptr_t)grads & 15) || ((uintptr_t)kv_cache & 15))
+    return fail(h, SVLA_ERR_ARG, "grads and kv_cache must be 16-byte aligned");
+  DeviceGuard dg(h->device);
+  const cudaError_t e = record_train(h, kv_cache, pad_mask, B, L, actions, noise, t, H, loss, grads,
+                                     reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, e, "train step");
+  return SVLA_OK;
+}
 
 int svla_denoise_fused_supported(const svla_handle* h, int B, int H) {
   return h && fused_ok(h, B, H, h->cfg.max_prefix) ? 1 : 0;

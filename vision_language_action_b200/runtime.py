@@ -45,11 +45,12 @@ class SmolVLA:
     ``blob`` is the flat bf16 weight blob in manifest order, as a numpy uint16
     array, a torch uint16/bfloat16 tensor (host or CUDA), or raw bytes.
     ``prefix_int8`` builds the weight-only int8 copy of the prefix LM's
-    projections (the vlm-8bit preset) and selects it for the prefill.
+    projections (the vlm-8bit preset) and selects it for the prefill;
+    ``train`` allocates the workspace of ``train_step``.
     """
 
     def __init__(self, shape, blob, max_batch: int, max_prefix: int, max_chunk: int,
-                 device: int = 0, prefix_int8: bool = False):
+                 device: int = 0, prefix_int8: bool = False, train: bool = False):
         self.lib = _abi.load()
         self.cfg = config_from_shape(shape, max_batch, max_prefix, max_chunk)
         self.action_dim = shape.action_dim
@@ -64,7 +65,7 @@ class SmolVLA:
             ptr, nbytes = arr.ctypes.data, arr.nbytes
             self._blob_keep = arr
         h = ctypes.c_void_p()
-        flags = _abi.CREATE_PREFIX_INT8 if prefix_int8 else 0
+        flags = (_abi.CREATE_PREFIX_INT8 if prefix_int8 else 0) | (_abi.CREATE_TRAIN if train else 0)
         st = self.lib.svla_create_ex(ctypes.byref(self.cfg), ctypes.c_void_p(ptr), nbytes, device, flags,
                                      ctypes.byref(h))
         self._blob_keep = None
@@ -180,6 +181,21 @@ class SmolVLA:
     def set_denoise_path(self, path: int) -> None:
         """_abi.DENOISE_AUTO (default), DENOISE_GRAPH or DENOISE_FUSED."""
         _abi.check(self.lib.svla_set_denoise_path(self.h, path), self.h)
+
+    def train_step(self, kv_cache: torch.Tensor, pad_mask: torch.Tensor, actions: torch.Tensor,
+                   noise: torch.Tensor, t: torch.Tensor, grads: Optional[torch.Tensor] = None, stream=None):
+        """One training step of the expert: (loss [1] float32, gradients float32 in
+        manifest order from the first expert tensor), both on the device."""
+        B, H, _ = actions.shape
+        L = pad_mask.shape[1]
+        n = int(self.lib.svla_train_grad_elems(self.h))
+        if grads is None:
+            grads = torch.empty(n, dtype=torch.float32, device=actions.device)
+        loss = torch.empty(1, dtype=torch.float32, device=actions.device)
+        st = self.lib.svla_train_step(self.h, _ptr(kv_cache), _ptr(pad_mask), B, L, _ptr(actions), _ptr(noise),
+                                      _ptr(t), H, _ptr(loss), _ptr(grads), _stream(stream))
+        _abi.check(st, self.h)
+        return loss, grads
 
     def set_prefix_weights(self, bits: int) -> None:
         """16 = dense bf16 prefix weights, 8 = the int8 copy (needs prefix_int8=True)."""
