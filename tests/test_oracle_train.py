@@ -189,3 +189,32 @@ def test_pins_catch_planted_train_mistake(name):
         except AssertionError:
             failed += 1
     assert failed >= 1, f"no pin caught the planted mistake {name}"
+
+
+def test_inputs_are_well_conditioned_for_bf16():
+    """The GPU parity test of the training step draws W_in 10x wider so that a
+    chunk's rows differ: then rounding the attention's q, k, v and output to
+    bf16 (the GPU's storage points) moves no gradient by more than 1e-2, while
+    with the narrow W_in it moves the self-attention W_q / W_k gradients by
+    several percent (cancellation in the softmax gradient)."""
+    def rb(x):
+        return x + (x.to(torch.bfloat16).to(torch.float64) - x).detach()
+
+    def grads(w_in_scale, emulate):
+        W, K, V, valid, a, eps, t = _case(4)
+        W["w_in"] = W["w_in"] * w_in_scale
+        orig_split, orig_att = ot._split, ot._attention
+        if emulate:
+            ot._split = lambda x, n: rb(orig_split(x, n))
+            ot._attention = lambda q, k, v, al: rb(orig_att(rb(q), rb(k), rb(v), al))
+        try:
+            return ot.train_step(W, S, K, V, valid, a, eps, t)[1]
+        finally:
+            ot._split, ot._attention = orig_split, orig_att
+
+    def worst(scale):
+        g0, g1 = grads(scale, False), grads(scale, True)
+        return max(np.linalg.norm(g1[n] - g0[n]) / np.linalg.norm(g0[n]) for n in g0)
+
+    assert worst(10.0) <= 1e-2
+    assert worst(1.0) > 2e-2
