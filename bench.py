@@ -123,6 +123,30 @@ def prefix_projection_bytes(s, bits):
     return tot
 
 
+def train_flops(s, B, L, H):
+    """Algorithmic FLOPs of one training step of the expert (svla_train_step):
+    every forward GEMM, its weight gradient, and its input gradient except
+    where the input is frozen (the prefix cache of the cross projections) or
+    not needed (the time half of the time MLP's input); attention forward 2
+    products per score block, backward 5 (scores again, dP, dQ, dK, dV)."""
+    hd = s.head_dim
+    M, Lb, E, F = B * H, B * L, s.e_width, s.e_ffn
+    qw, kvw, pkvw = s.e_heads * hd, s.e_kv_heads * hd, s.p_kv_width
+    g = 2 * M * 2 * E * E * 2 + 2 * M * E * E        # W_t1: forward + weight grad, input grad of the action half
+    g += 2 * M * E * E * 3                            # W_t2
+    att = 0
+    for l in range(s.e_layers):
+        if l % 2 == 0:
+            g += 2 * M * E * (qw + 2 * kvw) * 3
+            tk = H
+        else:
+            g += 2 * M * E * qw * 3 + 2 * (2 * Lb * pkvw * kvw) * 2
+            tk = L
+        g += 2 * M * qw * E * 3 + 2 * M * E * 2 * F * 3 + 2 * M * F * E * 3
+        att += (2 + 5) * 2 * B * s.e_heads * H * tk * hd
+    return g + att
+
+
 def launches_per_chunk(s, n_steps, fused):
     """Kernels libsvla launches for one prefill + denoise (the CUDA graphs' kernel nodes)."""
     pre = 2 + s.p_layers + 4 * (s.p_layers - 1)   # positions, residual init, QKV per layer, attn/O/GU/D
@@ -423,6 +447,40 @@ def int8_prefix(args, dev, barrier, hbm_peak, peak_kind):
     return out
 
 
+def train_block(args, dev, barrier, tf_peak, peak_kind):
+    """The expert's training step (svla_train_step: loss and every gradient) on
+    the SmolVLA shape with two queries, the shape its GPU parity test covers."""
+    import torch
+    from vision_language_action_b200.runtime import SmolVLA
+    s = synth.SHAPES["smolvla"]
+    B, L, H = 2, 177, 50
+    d = f"cuda:{dev}"
+    m = SmolVLA(s, synth.pack_blob(s, synth.gen_weights(s, 7, random_affine=True)), max_batch=B, max_prefix=L,
+                max_chunk=H, device=dev, train=True)
+    try:
+        rng = np.random.default_rng(7)
+        kv = torch.from_numpy(synth.f32_to_bf16_bits(rng.standard_normal((2, s.p_layers, B, L, s.p_kv_width))
+                                                     .astype(np.float32)).view(np.int16)).to(d).view(torch.bfloat16)
+        valid = torch.ones((B, L), dtype=torch.uint8, device=d)
+        a = torch.from_numpy((0.5 * rng.standard_normal((B, H, s.action_dim))).astype(np.float32)).to(d)
+        eps = torch.from_numpy(rng.standard_normal((B, H, s.action_dim)).astype(np.float32)).to(d)
+        t = torch.from_numpy(rng.uniform(0.05, 0.95, B).astype(np.float32)).to(d)
+        grads = torch.empty(int(m.lib.svla_train_grad_elems(m.h)), dtype=torch.float32, device=d)
+        steps = max(3, args.steps // 4)
+        ms = time_steps(lambda: m.train_step(kv, valid, a, eps, t, grads=grads), steps, args.warmup, barrier) / steps
+        if m.device_status() != 0:
+            raise RuntimeError("device status after the training step timing")
+    finally:
+        m.close()
+    fl = train_flops(s, B, L, H)
+    tf = fl / (ms * 1e-3) / 1e12
+    return {"workload": "smolvla expert, 2 queries, prefix 177, chunk 50 (frozen prefix cache)",
+            "ms_per_step": round(ms, 4), "steps": steps, "samples_per_s": round(B / (ms * 1e-3), 2),
+            "algorithmic_flops": int(fl),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": tf_peak, "unit": "TFLOP/s",
+                         "frac": round(tf / tf_peak, 5), "peak_kind": f"{peak_kind} bf16"}}
+
+
 def ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -546,6 +604,13 @@ def ours(args, rank, world, local_rank):
                                 "euler_steps": wl3.n_steps}}
         m3.close()
 
+    train = None
+    if not args.no_train:
+        try:
+            train = train_block(args, dev, barrier, tf_peak, peak_kind)
+        except Exception as exc:  # the headline line must not depend on this block
+            train = {"error": f"{type(exc).__name__}: {exc}"}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         run = oracle_chunk_timer("smolvla_b1")
@@ -575,6 +640,7 @@ def ours(args, rank, world, local_rank):
                           "note": "each call timed alone on rank 0, same steps and warm-up"},
             "prefix_assembly": asm,
             "int8_prefix": q8,
+            "train_step": train,
             "gpu_launches": launches_per_chunk(s, wl.n_steps, fused) * args.steps,
             "graph_gemm_roofline": graph_gemm if fused else None,
             "clocks": clk,
@@ -592,6 +658,8 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-int8", action="store_true")
+    ap.add_argument("--no-train", action="store_true")
+    ap.add_argument("--train-only", action="store_true", help="time only the expert's training step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -600,6 +668,12 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         reference_arm(args, rank)
+        return
+    if args.train_only:
+        import torch
+        torch.cuda.set_device(local_rank)
+        _, tf_peak, _, peak_kind = _peaks()
+        print(json.dumps({"train_step": train_block(args, local_rank, lambda: None, tf_peak, peak_kind)}), flush=True)
         return
     if world > 1:
         import datetime
