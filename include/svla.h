@@ -12,6 +12,12 @@
  *      K/V; a sinusoidal time embedding enters through the action-time MLP;
  *      each step applies x <- x + dt * v, dt = -1/n_steps, from Gaussian
  *      noise at t = 1 toward t = 0 (flow matching: x_t = t*eps + (1-t)*a).
+ * Around that path: the prefix overwrite at a chunk junction
+ * (svla_denoise_prefix), the prefix assembly from vision features
+ * (svla_set_assembly / svla_assemble_prefix), the weight-only int8 prefix
+ * (svla_create_ex with SVLA_CREATE_PREFIX_INT8), the expert's training step
+ * (svla_train_step), and single kernels for callers that compose their own
+ * schedule (svla_op_*).
  *
  * Conventions for every function below.
  *   - Pointers named "device" must point to memory of the handle's device

@@ -27,8 +27,12 @@ Parity pins (checked by ``tests/test_oracle_pins.py`` against things other
 than the oracle itself): block mask / joint pass, constant velocity, GQA =
 MHA with repeated heads, brute-force loops on the tiny shape, RoPE closed
 form, L = 1 attention, padding and batch invariance, parameter counts, and
-the Philox4x32-10 known-answer vectors. Parity against the real SmolVLA
-checkpoint is unpinned: no weights or activation dumps exist here.
+the Philox4x32-10 known-answer vectors. ``assembly.py`` (prefix assembly),
+``quant.py`` (the weight-only int8 preset) and ``train.py`` (the expert's
+training step) carry their own pins in ``tests/test_oracle_assembly.py``,
+``tests/test_oracle_quant.py`` and ``tests/test_oracle_train.py``. Parity
+against the real SmolVLA checkpoint is unpinned: no weights or activation
+dumps exist here.
 """
 from .model import (  # noqa: F401
     load_weights, rms_norm, rope, attention, silu, prefix_positions, prefill,
