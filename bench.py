@@ -701,6 +701,12 @@ def ours(args, rank, world, local_rank):
         times = [run() for _ in range(3)]
         cpu = {"value": round(float(np.mean(times)), 2), "unit": "ms", "cores": _blas_threads(), "kind": "oracle",
                "sample": "3 full chunks of smolvla_b1 (prefill + 10 Euler steps, query 0), float64 numpy"}
+        try:  # the same oracle on one core
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                cpu["one_core"] = {"value": round(run(), 2), "unit": "ms", "cores": 1, "sample": "1 chunk"}
+        except Exception as exc:
+            cpu["one_core"] = {"error": f"{type(exc).__name__}: {exc}"}
 
     if rank == 0:
         achieved_chunk = hbm_bytes / chunk_s / 1e9
