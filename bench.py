@@ -250,9 +250,20 @@ def oracle_chunk_timer(wl_name):
 
     def run():
         t0 = time.perf_counter()
-        oracle.sample(W, s, emb, valid, noise, wl.n_steps)
+        run.chunk = oracle.sample(W, s, emb, valid, noise, wl.n_steps)[-1]
         return (time.perf_counter() - t0) * 1e3
+    run.chunk = None
     return run
+
+
+def chunk_delta(gpu: np.ndarray, ref: np.ndarray, gate: float = 2e-2) -> dict:
+    """|GPU chunk - oracle chunk| over [H, A]: median, p95 and max overall and per
+    action dimension, beside the parity gate on the max."""
+    d = np.abs(np.asarray(gpu, np.float64) - np.asarray(ref, np.float64))
+    return {"median": float(np.median(d)), "p95": float(np.percentile(d, 95)), "max": float(d.max()),
+            "per_dim_p95": [round(float(x), 7) for x in np.percentile(d, 95, axis=0)],
+            "per_dim_max": [round(float(x), 7) for x in d.max(axis=0)],
+            "gate_max": gate, "pass": bool(d.max() <= gate)}
 
 
 def reference_arm(args, rank):
@@ -629,6 +640,7 @@ def ours(args, rank, world, local_rank):
                "algorithmic_bytes": int(asm_bytes),
                "note": "pixel-shuffle gather + connector GEMM (12288 -> 960) + state token and layout, 3 kernels"}
 
+    gpu_chunk = d["actions"][0].cpu().numpy()  # query 0 of the last timed step (same inputs every step)
     hbm_bytes, gflops, aflops = chunk_work(s, wl.B, wl.L, wl.H, wl.n_steps)
     chunk_s = value * 1e-3 * world  # per-rank chunk latency in s
     fused = m.fused_supported(wl.B, wl.H)
@@ -701,6 +713,10 @@ def ours(args, rank, world, local_rank):
         times = [run() for _ in range(3)]
         cpu = {"value": round(float(np.mean(times)), 2), "unit": "ms", "cores": _blas_threads(), "kind": "oracle",
                "sample": "3 full chunks of smolvla_b1 (prefill + 10 Euler steps, query 0), float64 numpy"}
+        try:  # the headline chunk against the oracle's, same weights, embeddings and noise
+            cpu["delta_vs_gpu"] = chunk_delta(gpu_chunk, run.chunk)
+        except Exception as exc:
+            cpu["delta_vs_gpu"] = {"error": f"{type(exc).__name__}: {exc}"}
         try:  # the same oracle on one core
             from threadpoolctl import threadpool_limits
             with threadpool_limits(limits=1):
