@@ -1,0 +1,46 @@
+"""Host-side checks of the figures bench.py reports: the algorithmic work of the
+int8 prefill and of the training step counted independently from the
+manifest, and the chunk delta summary on a constructed difference."""
+import numpy as np
+
+import bench
+import synth
+
+S = synth.SHAPES["smolvla"]
+
+
+def test_prefix_projection_bytes_from_the_manifest():
+    man = dict(synth.manifest(S))
+    dense = 0
+    for l in range(S.p_layers):
+        names = ("wq", "wk", "wv") if l == S.p_layers - 1 else ("wq", "wk", "wv", "wo", "wg", "wu", "wd")
+        dense += sum(2 * int(np.prod(man[f"p{l}.{n}"])) for n in names)
+    assert bench.prefix_projection_bytes(S, 16) == dense
+    # int8: one byte per weight plus a bf16 (alpha, beta) pair per 64 weights
+    assert bench.prefix_projection_bytes(S, 8) == dense // 2 + dense // 2 // 64 * 4
+
+
+def test_train_flops_counts_three_products_per_weight_gemm():
+    B, L, H = 2, 177, 50
+    M, E = B * H, S.e_width
+    expert_mats = 0
+    for l in range(S.e_layers):
+        for n in ("wq", "wo", "wg", "wu", "wd") + (("wk", "wv") if l % 2 == 0 else ()):
+            expert_mats += int(np.prod(dict(synth.manifest(S))[f"e{l}.{n}"]))
+    gemm = 3 * 2 * M * expert_mats                                   # forward, dX, dW
+    gemm += 2 * 2 * (2 * B * L * S.p_kv_width * S.e_kv_width) * (S.e_layers // 2)  # cross K/V: forward, dW
+    gemm += 2 * 2 * M * E * 2 * E + 2 * M * E * E + 3 * 2 * M * E * E  # time MLP
+    att = sum(7 * 2 * B * S.e_heads * H * (H if l % 2 == 0 else L) * S.head_dim for l in range(S.e_layers))
+    assert bench.train_flops(S, B, L, H) == gemm + att
+
+
+def test_chunk_delta_summary():
+    ref = np.zeros((50, 32))
+    gpu = ref.copy()
+    gpu[:, 3] = np.linspace(0, 1e-2, 50)
+    gpu[7, 5] = 3e-2
+    d = bench.chunk_delta(gpu, ref)
+    assert d["max"] == 3e-2 and not d["pass"]
+    assert d["per_dim_max"][5] == 3e-2 and abs(d["per_dim_max"][3] - 1e-2) < 1e-12
+    assert d["median"] == 0.0
+    assert bench.chunk_delta(ref, ref)["pass"]
