@@ -17,6 +17,7 @@ Prints ONE JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -291,7 +292,7 @@ def reference_arm(args, rank):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
-def gpu_setup(wl_name, dev, B=None, prefix_int8=False):
+def gpu_setup(wl_name, dev, B=None, prefix_int8=False, hash_blob=False):
     import torch
     from vision_language_action_b200.runtime import SmolVLA
     wl = synth.WORKLOADS[wl_name]
@@ -299,6 +300,7 @@ def gpu_setup(wl_name, dev, B=None, prefix_int8=False):
     B = wl.B if B is None else B
     blob = synth.pack_blob(s, synth.gen_weights(s, wl.seed))
     m = SmolVLA(s, blob, max_batch=B, max_prefix=wl.L, max_chunk=wl.H, device=dev, prefix_int8=prefix_int8)
+    m.blob_sha256 = hashlib.sha256(blob.tobytes()).hexdigest() if hash_blob else None
     del blob
     inp = synth.gen_inputs(wl, B=B)
     host = {
@@ -342,6 +344,22 @@ def time_steps(fn, steps, warmup, barrier):
     torch.cuda.synchronize()
     barrier()
     return e0.elapsed_time(e1)
+
+
+def step_spread(fn, steps):
+    """Per-step device times (an event after every step, after the timed region):
+    median, p10 and p90 in ms."""
+    import torch
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    torch.cuda.synchronize()
+    ev[0].record()
+    for i in range(steps):
+        fn()
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    t = np.array([ev[i].elapsed_time(ev[i + 1]) for i in range(steps)])
+    return {"median": round(float(np.median(t)), 4), "p10": round(float(np.percentile(t, 10)), 4),
+            "p90": round(float(np.percentile(t, 90)), 4), "steps": steps}
 
 
 def gemm_roofline(s, B, L, H, n_steps, dev, hbm_peak):
@@ -576,7 +594,7 @@ def ours(args, rank, world, local_rank):
     barrier = (lambda: dist.barrier()) if world > 1 else (lambda: None)
     hbm_peak, tf_peak, tf_sus, peak_kind = _peaks()
 
-    m, wl, host, d = gpu_setup("smolvla_b1", dev)
+    m, wl, host, d = gpu_setup("smolvla_b1", dev, hash_blob=True)
     s = wl.model
 
     def step():
@@ -613,6 +631,10 @@ def ours(args, rank, world, local_rank):
         torch.cuda.current_stream().synchronize()
 
     ms_e2e = max_over_ranks(time_steps(e2e_step, args.steps, args.warmup, barrier), world, f"cuda:{dev}")
+    try:  # per-step distribution, outside the timed region
+        spread = step_spread(step, args.steps)
+    except Exception as exc:
+        spread = {"error": f"{type(exc).__name__}: {exc}"}
 
     # the two calls of a step timed on their own (same warm-up and step count)
     ms_pre = time_steps(lambda: m.prefill(d["embeds"], d["valid"], d["kv"]), args.steps, args.warmup, barrier)
@@ -641,6 +663,7 @@ def ours(args, rank, world, local_rank):
                "note": "pixel-shuffle gather + connector GEMM (12288 -> 960) + state token and layout, 3 kernels"}
 
     gpu_chunk = d["actions"][0].cpu().numpy()  # query 0 of the last timed step (same inputs every step)
+    blob_sha = m.blob_sha256[:16]
     hbm_bytes, gflops, aflops = chunk_work(s, wl.B, wl.L, wl.H, wl.n_steps)
     chunk_s = value * 1e-3 * world  # per-rank chunk latency in s
     fused = m.fused_supported(wl.B, wl.H)
@@ -732,7 +755,7 @@ def ours(args, rank, world, local_rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.B, "prefix_len": wl.L, "chunk": wl.H,
                        "euler_steps": wl.n_steps, "global_batch": wl.B * world,
-                       "parallelism": f"replicas x{world}",
+                       "parallelism": f"replicas x{world}", "weights_sha256": blob_sha,
                        "l2_policy": "no flush: every step streams 514 MB of weights (> 126 MB L2)"},
             "roofline": roof,
             "chunk_roofline": {"bound": "hbm", "achieved": round(achieved_chunk, 1), "peak": hbm_peak,
@@ -741,6 +764,7 @@ def ours(args, rank, world, local_rank):
             "cpu_baseline": cpu,
             "e2e": {"value": round(ms_e2e / (args.steps * chunks_per_step), 4), "unit": "ms",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "step_spread_ms": spread,
             "breakdown": {"prefill_ms": round(ms_pre / args.steps, 4), "denoise_ms": round(ms_den / args.steps, 4),
                           "note": "each call timed alone on rank 0, same steps and warm-up"},
             "prefix_assembly": asm,
