@@ -12,6 +12,16 @@ secondary line-item measures chunks/s at b = 32 (smolvla_b32). For N > 1 (one
 process per GPU under torchrun) every rank runs its own replica of the same
 workload (independent queries, no collective on the path): weak scaling.
 
+Further objects of the line, each measured after the headline's timed region:
+the per-step spread, the prefill / denoise breakdown, the prefix assembly, the
+int8 (vlm-8bit) prefix at batch 1 and 32, the batch-8 / prefix-321 / chunk-100
+step and the batch-256 denoise ("batched"), and the expert's training step.
+The CPU leg times the oracle on the host's cores and on one core and reports
+the headline chunk's difference from the oracle's.
+    --no-secondary  skip batch 32 and the batched workloads
+    --no-int8 / --no-train / --no-cpu   skip those blocks
+    --train-only    time only the training step
+
 Prints ONE JSON line on rank 0.
 """
 from __future__ import annotations
