@@ -176,3 +176,19 @@ def test_train_argument_checks():
                               ctypes.byref(h)) == _abi.SVLA_ERR_ARG
     assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, _abi.CREATE_TRAIN,
                               ctypes.byref(h)) == _abi.SVLA_ERR_BLOB_SIZE
+
+
+def test_op_wrappers_refuse_host_tensors():
+    """The kernel-level wrappers marshal device tensors only: host tensors fail loudly
+    (there is no CPU fallback)."""
+    import torch
+    from vision_language_action_b200 import runtime as rt
+    A = torch.zeros(4, 64, dtype=torch.bfloat16)
+    W = torch.zeros(8, 64, dtype=torch.bfloat16)
+    C = torch.zeros(4, 8)
+    with pytest.raises(ValueError):
+        rt.op_gemm("f32", A, W, C)
+    with pytest.raises(ValueError):
+        rt.op_quantize_affine8(W)
+    with pytest.raises(ValueError):
+        rt.op_rmsnorm(C, torch.zeros(8, dtype=torch.bfloat16), torch.zeros(4, 8, dtype=torch.bfloat16))

@@ -211,3 +211,68 @@ class SmolVLA:
     def device_status(self, stream=None) -> int:
         """Synchronise the stream; return (and clear) the device-side status."""
         return int(self.lib.svla_device_status(self.h, _stream(stream)))
+
+
+# ----------------------------------------------------------------------
+# single kernels (svla_op_*), for callers that compose their own schedule
+# ----------------------------------------------------------------------
+_EPI = {"f32": 0, "bf16": 1, "add_f32": 2, "silu_bf16": 3}
+
+
+def op_gemm(epilogue: str, A: torch.Tensor, W: torch.Tensor, C: torch.Tensor, bias: Optional[torch.Tensor] = None,
+            splits: int = 0, status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """svla_op_gemm: C = A W^T (+ bias) with the epilogue 'f32', 'bf16', 'add_f32' or 'silu_bf16'."""
+    lib = _abi.load()
+    M, K = A.shape
+    N = W.shape[0]
+    ws_bytes = int(lib.svla_op_gemm_workspace_bytes(M, N, K, splits))
+    ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=A.device) if ws_bytes else None
+    st = lib.svla_op_gemm(_EPI[epilogue], _ptr(A), A.stride(0), _ptr(W), W.stride(0), M, N, K, _ptr(C), C.stride(0),
+                          _ptr(bias), splits, _ptr(ws), ws_bytes, _ptr(status), _stream(stream))
+    _abi.check(st)
+    return C
+
+
+def op_quantize_affine8(W: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """svla_op_quantize_affine8: bf16 W [N, K] -> (codes uint8 [N, K], (alpha, beta) bf16 [K/64, N, 2])."""
+    lib = _abi.load()
+    N, K = W.shape
+    q = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    ab = torch.empty((K // 64, N, 2), dtype=torch.bfloat16, device=W.device)
+    _abi.check(lib.svla_op_quantize_affine8(_ptr(W), W.stride(0), N, K, _ptr(q), q.stride(0), _ptr(ab),
+                                            _stream(stream)))
+    return q, ab
+
+
+def op_gemm_w8(epilogue: str, A: torch.Tensor, q: torch.Tensor, ab: torch.Tensor, C: torch.Tensor,
+               gain: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None, splits: int = 0,
+               status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """svla_op_gemm_w8: C = A W^T with W = bf16(bf16(alpha q + beta) * gain) from op_quantize_affine8's output."""
+    lib = _abi.load()
+    M, K = A.shape
+    N = q.shape[0]
+    st = lib.svla_op_gemm_w8(_EPI[epilogue], _ptr(A), A.stride(0), _ptr(q), q.stride(0), _ptr(ab), _ptr(gain), M, N,
+                             K, _ptr(C), C.stride(0), _ptr(bias), splits, _ptr(status), _stream(stream))
+    _abi.check(st)
+    return C
+
+
+def op_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, n_q: int, n_kv: int,
+                 head_dim: int, key_valid: Optional[torch.Tensor] = None, causal: bool = False,
+                 stream=None) -> torch.Tensor:
+    """svla_op_attention on [B, Lq, n_q * hd] queries and [B, Lk, n_kv * hd] keys / values."""
+    lib = _abi.load()
+    B, Lq, _ = q.shape
+    Lk = k.shape[1]
+    st = lib.svla_op_attention(_ptr(q), q.stride(1), _ptr(k), _ptr(v), k.stride(1), _ptr(key_valid), B, n_q, n_kv,
+                               head_dim, Lq, Lk, int(causal), _ptr(out), out.stride(1), _stream(stream))
+    _abi.check(st)
+    return out
+
+
+def op_rmsnorm(x: torch.Tensor, g: torch.Tensor, y: torch.Tensor, eps: float = 1e-5, stream=None) -> torch.Tensor:
+    """svla_op_rmsnorm: y (bf16) = x (f32) / sqrt(mean(x^2) + eps) * g."""
+    lib = _abi.load()
+    M, D = x.shape
+    _abi.check(lib.svla_op_rmsnorm(_ptr(x), _ptr(g), M, D, eps, _ptr(y), _stream(stream)))
+    return y
