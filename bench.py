@@ -21,6 +21,7 @@ the headline chunk's difference from the oracle's.
     --no-secondary  skip batch 32 and the batched workloads
     --no-int8 / --no-train / --no-cpu   skip those blocks
     --train-only    time only the training step
+    --batched-only  time only the batch-8 and batch-256 workloads
 
 Prints ONE JSON line on rank 0.
 """
@@ -800,6 +801,7 @@ def main():
     ap.add_argument("--no-int8", action="store_true")
     ap.add_argument("--no-train", action="store_true")
     ap.add_argument("--train-only", action="store_true", help="time only the expert's training step")
+    ap.add_argument("--batched-only", action="store_true", help="time only the batch-8 and batch-256 workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -808,6 +810,13 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         reference_arm(args, rank)
+        return
+    if args.batched_only:
+        import torch
+        torch.cuda.set_device(local_rank)
+        hbm_peak, tf_peak, tf_sus, peak_kind = _peaks()
+        print(json.dumps({"batched": batched_configs(args, local_rank, lambda: None, hbm_peak, tf_peak, tf_sus,
+                                                     peak_kind)}), flush=True)
         return
     if args.train_only:
         import torch
