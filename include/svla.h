@@ -361,10 +361,13 @@ SVLA_API svla_status svla_op_rmsnorm(const float* x, const void* g, int M, int D
  *   (svla_op_gemm_workspace_bytes(M, N, K, splits) > 8 MiB) is rejected with
  *   SVLA_ERR_SHAPE and a message naming both sizes; nothing is launched.
  *   The first call on a device resolves the array's device address and zeroes
- *   it synchronously, so make that first call before any stream capture. Each
- *   later call clears the counter part of the scratch on `stream` before its
- *   launch. The function never calls cudaMalloc, cudaFree or any allocating
- *   library routine.
+ *   its 4 KiB counter area synchronously, so make that first call before any
+ *   stream capture. The address is kept for the life of the process: do not
+ *   call this entry point after cudaDeviceReset. Each call that splits K
+ *   clears the counter area on `stream` before its launch; a plan whose
+ *   counters would not fit in it is rejected with SVLA_ERR_SHAPE. The
+ *   function never calls cudaMalloc, cudaFree or any allocating library
+ *   routine.
  *   All calls on a device share the one scratch array: calls whose kernels
  *   overlap on the GPU (different streams, or several host threads) race and
  *   may give wrong results; issue them in one stream order. */

@@ -131,6 +131,45 @@ def test_gemm_timeout_path_reports_and_recovers(M, splits):
     assert torch.allclose(C.double(), ref, rtol=1e-4, atol=1e-4)
 
 
+@pytest.mark.parametrize("splits", [12, 16])
+def test_gemm_timeout_leaves_the_global_counters_zeroed(splits):
+    """More than 8 splits reduce through the caller's workspace with one arrival
+    counter per tile. A CTA aborted by a wait that ran out still takes its turn
+    on that counter, so after the failed launch every counter is back at zero
+    and the next launch on the same workspace is correct."""
+    lib = _abi.load()
+    g = torch.Generator(device="cpu").manual_seed(9)
+    M, N, K = 50, 720, 2048
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16).to(DEV)
+    W = (0.05 * torch.randn(N, K, generator=g)).to(torch.bfloat16).to(DEV)
+    ws_bytes = lib.svla_op_gemm_workspace_bytes(M, N, K, splits)
+    assert ws_bytes > 0
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=DEV)
+    # the workspace starts with one int counter per output tile, padded to 256
+    # bytes: M = 50 and N = 720 give fewer than 64 tiles at any tile width
+
+    def run(C, status):
+        _abi.check(lib.svla_op_gemm(_abi.EPI_F32, P(A), K, P(W), K, M, N, K, P(C), N, None, splits, P(ws),
+                                    ws_bytes, P(status), S()))
+
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    C = torch.zeros(M, N, device=DEV)
+    try:
+        lib.svla_set_wait_limit_ns(0)
+        run(C, status)
+        torch.cuda.synchronize()
+    finally:
+        lib.svla_set_wait_limit_ns(1_000_000_000)
+    assert status.item() == _abi.SVLA_ERR_TIMEOUT
+    assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0
+    status.zero_()
+    run(C, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = A.double() @ W.double().T
+    assert ((C.double() - ref).abs() <= 1e-5 * (A.double().abs() @ W.double().abs().T) + 1e-6).all()
+
+
 # ---------------------------------------------------------------------------
 # attention
 # ---------------------------------------------------------------------------

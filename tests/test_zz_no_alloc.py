@@ -69,12 +69,20 @@ def test_noalloc_matches_workspace_entry_point_twice(M, N, K, splits, epi):
     with_workspace(epi, A, W, ref, bias, splits)
     scale = (A.double().abs() @ W.double().abs().T) + bias.double().abs() + R0.double().abs()
     tol = 1e-5 * scale + 1e-6 if epi != _abi.EPI_BF16 else 2 ** -8 * scale + 1e-4
+    # float64 reference of the same contraction (fp32 accumulation of K products)
+    exact = A.double() @ W.double().T + bias.double()
+    if epi == _abi.EPI_ADD_F32:
+        exact = exact + R0.double()
+    assert ((ref.double() - exact).abs() <= tol).all()
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     for _ in range(2):   # two calls in a row share (and must re-arm) the static scratch
         out = R0.clone()
         without_workspace(epi, A, W, out, bias, splits, status)
         assert status.item() == 0
-        assert ((out.double() - ref.double()).abs() <= tol).all()
+        # same plan, same split order: the partial sums are added in the same
+        # order as with a caller-owned workspace, so the result is bit for bit equal
+        assert torch.equal(out, ref)
+        assert ((out.double() - exact).abs() <= tol).all()
 
 
 def test_noalloc_rejects_plans_larger_than_its_scratch():

@@ -416,6 +416,35 @@ SVLA_DEV void gemm_accumulator_out(const GemmArgs& args, uint32_t tmem_base, uin
   }
 }
 
+// Epilogue warps, after their wait for the accumulator (`ok` = this thread's
+// wait succeeded): the four warps first agree on the abort flag (named
+// barrier), so they all take the same branch below. Then the epilogue runs,
+// or, when the CTA was aborted by a bounded wait that ran out, the CTA still
+// takes its turn on the global split-K counter of its tile without writing a
+// result: every CTA of a tile arrives exactly once, so the last one re-arms the
+// counter to zero and the next launch on the same workspace starts clean.
+template <int BN, int EPI, bool CLUSTER_OK>
+SVLA_DEV void gemm_epilogue_after_wait(bool ok, const GemmArgs& args, uint32_t tmem_base, uint8_t* ring,
+                                       volatile uint32_t* misc, int quad, int row, int m, int n0, bool row_ok,
+                                       float rscale, int m_blk, int n_blk, int split, int splits) {
+  if (!ok) {
+    misc[1] = 1;
+    set_status(args.status, SVLA_ERR_TIMEOUT);
+  }
+  epi_bar();
+  tc_fence_after();
+  if (misc[1] == 0) {
+    gemm_accumulator_out<BN, EPI, CLUSTER_OK>(args, tmem_base, ring, misc, quad, row, m, n0, row_ok, rscale, m_blk,
+                                              n_blk, split, splits);
+  } else if (splits > 1 && !(CLUSTER_OK && args.red_mode == GEMM_RED_CLUSTER)) {
+    if (threadIdx.x == 64) {
+      const int tile = m_blk * gridDim.x + n_blk;
+      const int old = atomicAdd(args.counters + tile, 1);
+      if (old == splits - 1) args.counters[tile] = 0;
+    }
+  }
+}
+
 // Cluster split-K tail, run by every thread of every CTA of the cluster after
 // the main loop: CTA r sums rows r, r + S, .. of the peers' staged partial
 // tiles in split order and runs their epilogue.
@@ -591,17 +620,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES, A_ROWS>::MIN
     prefetch_epilogue_inputs<BN, EPI>(args, m, n0, row_ok);
     const float rscale = norm_row_scale(args, m, row_ok);  // overlaps the main loop
     misc_scale[row] = rscale;
-    bool ok = mbar_wait(acc_bar, 0, lim);
-    if (!ok) {
-      misc[1] = 1;
-      set_status(args.status, SVLA_ERR_TIMEOUT);
-    }
-    ok = __all_sync(0xffffffffu, ok);
-    tc_fence_after();
-    const bool aborted = misc[1] != 0;
-    if (ok && !aborted)
-      gemm_accumulator_out<BN, EPI, C::CLUSTER_OK>(args, tmem_base, ring, misc, quad, row, m, n0, row_ok, rscale,
-                                                   m_blk, n_blk, split, splits);
+    const bool ok = mbar_wait(acc_bar, 0, lim);
+    gemm_epilogue_after_wait<BN, EPI, C::CLUSTER_OK>(ok, args, tmem_base, ring, misc, quad, row, m, n0, row_ok,
+                                                     rscale, m_blk, n_blk, split, splits);
     tc_fence_before();
   }
 

@@ -286,17 +286,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
       if (i == pre - 1) epilogue_inputs();
     }
     if (!have_scale) epilogue_inputs();  // the loop stopped early (time-out)
-    bool ok = mbar_wait(acc_bar, 0, lim);
-    if (!ok) {
-      misc[1] = 1;
-      set_status(args.status, SVLA_ERR_TIMEOUT);
-    }
-    ok = __all_sync(0xffffffffu, ok);
-    tc_fence_after();
-    const bool aborted = misc[1] != 0;
-    if (ok && !aborted)
-      gemm_accumulator_out<BN, EPI, C::CLUSTER_OK>(args, tmem_base, ring, misc, quad, row, m, n0, row_ok, rscale,
-                                                   m_blk, n_blk, split, splits);
+    const bool ok = mbar_wait(acc_bar, 0, lim);
+    gemm_epilogue_after_wait<BN, EPI, C::CLUSTER_OK>(ok, args, tmem_base, ring, misc, quad, row, m, n0, row_ok,
+                                                     rscale, m_blk, n_blk, split, splits);
     tc_fence_before();
   }
 

@@ -1608,6 +1608,15 @@ int svla_op_gemm_splits(int M, int N, int K) {
 
 static size_t cnt_bytes(const GemmPlan& p) { return (((size_t)p.m_tiles * p.n_tiles * sizeof(int)) + 255) / 256 * 256; }
 
+// Bytes of the counter area at the start of svla_op_gemm's workspace for this
+// plan (0 when the plan needs no workspace); used by svla_op_gemm_noalloc,
+// which clears a fixed counter area on every call.
+size_t svla_internal_gemm_counter_bytes(int M, int N, int K, int splits) {
+  if (M < 1 || N < 1 || K < 1 || splits < 0) return 0;
+  GemmPlan p = plan_gemm(M, N, K, splits);
+  return p.red == GEMM_RED_GLOBAL ? cnt_bytes(p) : 0;
+}
+
 size_t svla_op_gemm_workspace_bytes(int M, int N, int K, int splits) {
   if (M < 1 || N < 1 || K < 1 || splits < 0) return 0;
   GemmPlan p = plan_gemm(M, N, K, splits);

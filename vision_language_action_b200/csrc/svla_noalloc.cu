@@ -16,6 +16,7 @@
 #include "../../include/svla.h"
 
 svla_status svla_internal_fail(svla_status s, const char* msg);
+extern "C" size_t svla_internal_gemm_counter_bytes(int M, int N, int K, int splits);
 
 namespace {
 
@@ -28,7 +29,9 @@ std::mutex g_mu;
 void* g_scratch_addr[64] = {};
 
 // Device address of the scratch on the current device; the first call on a
-// device resolves it and zeroes the counter area (synchronously).
+// device resolves it and zeroes the 4 KiB counter area (synchronously). The
+// address is kept for the life of the process (cudaDeviceReset would move the
+// array: the header tells callers not to use this entry point after one).
 svla_status scratch_for_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -63,6 +66,10 @@ extern "C" svla_status svla_op_gemm_noalloc(int epilogue, const void* A, int lda
                             " (use fewer splits or svla_op_gemm with a workspace)";
     return svla_internal_fail(SVLA_ERR_SHAPE, msg.c_str());
   }
+  // the plan's counters must lie inside the area that every call clears
+  if (svla_internal_gemm_counter_bytes(M, N, K, splits) > kCounterBytes)
+    return svla_internal_fail(SVLA_ERR_SHAPE, "this GEMM's split-K counters do not fit in the 4 KiB counter area of "
+                                              "the static scratch (use fewer splits or svla_op_gemm)");
   void* scratch = nullptr;
   if (svla_status st = scratch_for_current_device(&scratch); st != SVLA_OK) return st;
   if (need > 0) {
