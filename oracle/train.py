@@ -23,6 +23,23 @@ Readings (numbered after those of ``quant.py``):
 27. A step's result is the loss and its gradient with respect to every
     trainable tensor; the optimiser update is not part of it.
 
+28. Storage rounding (optional, ``bf16_storage=True``; off by default). The
+    CSDN precision post (§3-§7, §9) shows that where a bf16 pipeline rounds
+    decides how far it lands from an fp32 one, and its §11 asks to keep that
+    precision-change error apart from the error of the port itself. To tell
+    the two apart, the forward can round to bfloat16
+    (nearest, ties to even, from the float32 value) at the points where the
+    GPU stores bf16: the action embedding and the time features entering the
+    time MLP, the time MLP's hidden layer, both RMSNorm outputs of every
+    layer, q and k after RoPE and v (the cross layers' projected prefix keys
+    and values too), the unnormalised probabilities in P V (the softmax sum
+    stays unrounded) and the attention output, and the SwiGLU output. Each
+    rounding passes its gradient straight through, so the backward is the
+    derivative of the rounded forward taken at the rounded values, except
+    that the attention's derivative is that of the unrounded softmax: a
+    backward that recomputes P from the stored q and k (as the GPU's does)
+    never sees the rounded P. The default path is unchanged.
+
 The forward is the velocity of ``model.py`` restated in float64 torch, so
 that autograd returns the exact derivative of the written forward; the tests
 pin this forward to ``model.velocity`` and the gradients to central
@@ -116,45 +133,87 @@ def _silu(x):
     return x / (1.0 + (-x).exp())
 
 
-def velocity_torch(P, s, x, t: float, K, V, valid):
-    """model.velocity restated on torch tensors (P: name -> float64 tensor)."""
+def bf16_round(x):
+    """Reading 28: the value of x rounded to bfloat16 (nearest, ties to even,
+    from its float32 value), with the gradient passed straight through."""
     torch = _torch()
+    r = x.detach().to(torch.float32).to(torch.bfloat16).to(torch.float64)
+    return x + (r - x).detach()
+
+
+def _identity(x):
+    return x
+
+
+def _attention_rounded(q, k, v, allowed, rnd):
+    """Attention whose value has the unnormalised probabilities rounded where
+    they enter P V (the softmax sum over the unrounded values), and whose
+    derivative is that of the unrounded softmax attention: the backward
+    recomputes P from the stored q and k, it never sees the rounded P
+    (reading 28)."""
+    torch = _torch()
+    n_q, hd = q.shape[0], q.shape[-1]
+    group = n_q // k.shape[0]
+    outs = []
+    for h in range(n_q):
+        g = h // group
+        sc = (q[h] @ k[g].T) / math.sqrt(hd)
+        sc = sc.masked_fill(~allowed, float("-inf"))
+        exact = torch.softmax(sc, dim=-1) @ v[g]
+        pt = (sc - sc.max(dim=-1, keepdim=True).values).exp().detach()
+        stored = (rnd(pt) @ v[g].detach()) / pt.sum(dim=-1, keepdim=True)
+        outs.append(exact + (stored - exact).detach())
+    return torch.stack(outs)
+
+
+def velocity_torch(P, s, x, t: float, K, V, valid, bf16_storage: bool = False):
+    """model.velocity restated on torch tensors (P: name -> float64 tensor);
+    ``bf16_storage`` rounds at the GPU's storage points (reading 28)."""
+    torch = _torch()
+    rnd = bf16_round if bf16_storage else _identity
     H, L = x.shape[0], K.shape[1]
     De = s.e_width
     a = x @ P["w_in"].T + P["b_in"]
     e = torch.as_tensor(om.time_embedding(t, De, s.t_min_period, s.t_max_period)).expand(H, De)
-    h = _silu(torch.cat([a, e], dim=1) @ P["w_t1"].T + P["b_t1"])
+    h = rnd(_silu(torch.cat([rnd(a), rnd(e)], dim=1) @ P["w_t1"].T + P["b_t1"]))
     r = h @ P["w_t2"].T + P["b_t2"]
     pos = np.arange(H)
     causal = torch.tril(torch.ones(H, H, dtype=torch.bool))
     cross = torch.as_tensor(np.asarray(valid, bool))[None, :].expand(H, L)
+
+    def attend(q, k, v, allowed):
+        if not bf16_storage:
+            return _attention(q, k, v, allowed)
+        return rnd(_attention_rounded(q, k, v, allowed, rnd))
+
     for l in range(s.e_layers):
         p = f"e{l}."
-        y = _rms_norm(r, P[p + "in_norm"], s.rms_eps)
+        y = rnd(_rms_norm(r, P[p + "in_norm"], s.rms_eps))
         q = _split(y @ P[p + "wq"].T, s.e_heads)
         if l % 2 == 0:
-            k = _rope(_split(y @ P[p + "wk"].T, s.e_kv_heads), pos, s.rope_base)
-            v = _split(y @ P[p + "wv"].T, s.e_kv_heads)
-            o = _attention(_rope(q, pos, s.rope_base), k, v, causal)
+            k = rnd(_rope(_split(y @ P[p + "wk"].T, s.e_kv_heads), pos, s.rope_base))
+            v = rnd(_split(y @ P[p + "wv"].T, s.e_kv_heads))
+            o = attend(rnd(_rope(q, pos, s.rope_base)), k, v, causal)
         else:
             kc = K[l].reshape(L, s.p_kv_width)
             vc = V[l].reshape(L, s.p_kv_width)
-            k = _split(kc @ P[p + "wk"].T, s.e_kv_heads)
-            v = _split(vc @ P[p + "wv"].T, s.e_kv_heads)
-            o = _attention(q, k, v, cross)
+            k = rnd(_split(kc @ P[p + "wk"].T, s.e_kv_heads))
+            v = rnd(_split(vc @ P[p + "wv"].T, s.e_kv_heads))
+            o = attend(rnd(q), k, v, cross)
         r = r + _merge(o) @ P[p + "wo"].T
-        y = _rms_norm(r, P[p + "post_norm"], s.rms_eps)
-        r = r + (_silu(y @ P[p + "wg"].T) * (y @ P[p + "wu"].T)) @ P[p + "wd"].T
+        y = rnd(_rms_norm(r, P[p + "post_norm"], s.rms_eps))
+        r = r + rnd(_silu(y @ P[p + "wg"].T) * (y @ P[p + "wu"].T)) @ P[p + "wd"].T
     yf = _rms_norm(r, P["final_norm"], s.rms_eps)
     return yf @ P["w_out"].T + P["b_out"]
 
 
 def train_step(W: Dict[str, np.ndarray], s, K: np.ndarray, V: np.ndarray, valid: np.ndarray, a: np.ndarray,
-               eps: np.ndarray, t: np.ndarray) -> Tuple[float, Dict[str, np.ndarray]]:
+               eps: np.ndarray, t: np.ndarray, bf16_storage: bool = False) -> Tuple[float, Dict[str, np.ndarray]]:
     """Readings 25-27: (loss, {trainable name: dL/dW}) for one batch.
 
     K/V [B, p_layers, L, p_kv_heads, hd] (frozen prefix cache), valid [B, L],
     a (the target chunk) and eps (the noise) [B, H, A], t [B].
+    ``bf16_storage``: round the forward at the GPU's storage points (reading 28).
     """
     torch = _torch()
     names = trainable_names(s)
@@ -164,7 +223,7 @@ def train_step(W: Dict[str, np.ndarray], s, K: np.ndarray, V: np.ndarray, valid:
     for b in range(a.shape[0]):
         x = torch.as_tensor(flow_input(a[b], eps[b], float(t[b])))
         v = velocity_torch(P, s, x, float(t[b]), torch.as_tensor(np.asarray(K[b], np.float64)),
-                           torch.as_tensor(np.asarray(V[b], np.float64)), valid[b])
+                           torch.as_tensor(np.asarray(V[b], np.float64)), valid[b], bf16_storage)
         target = torch.as_tensor(np.asarray(eps[b], np.float64) - np.asarray(a[b], np.float64))
         term = (v - target).pow(2).sum()
         tot = term if tot is None else tot + term
