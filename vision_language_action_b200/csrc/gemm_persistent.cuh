@@ -171,8 +171,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int mb, nb;
       tile_mn((int)blockIdx.x + tc * (int)gridDim.x, mb, nb);
       const int m = mb * GEMM_BM + row;
-      prefetch_epilogue_inputs<BN, EPI>(args, m, nb * BN, m < args.M);
-      const float rscale = norm_row_scale(args, m, m < args.M);  // before the accumulator is ready
+      EpiPre<BN, EPI> pre;
+      epi_prefetch<BN, EPI>(args, m, nb * BN, m < args.M, pre);  // before the accumulator is ready
       bool ok = mbar_wait(accf_bar(buf), aph, lim);
       if (!ok) {
         misc[1] = 1;
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       AccSource<BN> src;
       src.taddr_row = tmem_base + (uint32_t)(buf * C::TMEM_COLS) + ((uint32_t)(quad * 32) << 16);
       src.smem_row = nullptr;
-      run_epilogue<BN, EPI>(args, src, m, nb * BN, m < args.M, rscale);
+      run_epilogue<BN, EPI>(args, src, m, nb * BN, m < args.M, pre);
       tc_fence_before();
       mbar_arrive(acce_bar(buf));  // this thread's reads of the buffer are complete
     }

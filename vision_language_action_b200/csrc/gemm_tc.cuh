@@ -169,20 +169,30 @@ SVLA_DEV void add_bias16(float (&v)[16], const float* bias, int col, int N) {
   }
 }
 
-// Fetches 16 accumulator columns [c, c+16) of this thread's row: from TMEM,
-// or (split-K reducer) from the reduced tile staged in shared memory.
+// Fetches N accumulator columns [c, c+N) of this thread's row (N a multiple
+// of 16): from TMEM, all N / 16 loads in flight before one wait, or (split-K
+// reducer) from the reduced tile staged in shared memory.
 template <int BN>
 struct AccSource {
   uint32_t taddr_row;
   const float* smem_row;  // null: read TMEM
   float scale = 1.f;      // fused RMSNorm row factor
-  SVLA_DEV void get(int c, float (&v)[16]) const {
+  template <int N>
+  SVLA_DEV void get(int c, float (&v)[N]) const {
+    static_assert(N % 16 == 0, "whole 16-column loads");
     if (smem_row == nullptr) {
-      tmem_ld16(taddr_row + (uint32_t)c, v);
+      uint32_t r[N / 16][16];
+#pragma unroll
+      for (int j = 0; j < N / 16; ++j) tmem_ld16_nowait(taddr_row + (uint32_t)(c + 16 * j), r[j]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < N / 16; ++j)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[16 * j + i] = __uint_as_float(r[j][i]);
     } else {
       const float4* p = reinterpret_cast<const float4*>(smem_row + c);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < N / 4; ++i) {
         const float4 t = p[i];
         v[4 * i] = t.x;
         v[4 * i + 1] = t.y;
@@ -191,23 +201,9 @@ struct AccSource {
       }
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] *= scale;
+    for (int i = 0; i < N; ++i) v[i] *= scale;
   }
 };
-
-// The residual-add epilogue reads its row segment of the output: start that
-// read (into L1) as soon as the earlier kernels are complete, long before the
-// accumulator is ready.
-template <int BN, int EPI>
-SVLA_DEV void prefetch_epilogue_inputs(const GemmArgs& a, int m, int n0, bool row_ok) {
-  if constexpr (EPI == GE_ADD_F32) {
-    if (row_ok && n0 < a.N) {
-      const float* p = reinterpret_cast<const float*>(a.out) + (size_t)m * a.ldo + n0;
-#pragma unroll
-      for (int c = 0; c < BN; c += 32) prefetch_l1(p + c);
-    }
-  }
-}
 
 // Fused RMSNorm row factor of row m (1 when the GEMM consumes no norm).
 SVLA_DEV float norm_row_scale(const GemmArgs& a, int m, bool row_ok) {
@@ -215,6 +211,62 @@ SVLA_DEV float norm_row_scale(const GemmArgs& a, int m, bool row_ok) {
   float s = 0.f;
   for (int t = 0; t < a.ss_tiles; ++t) s += __ldg(a.ss_in + (size_t)t * a.ss_ld + m);
   return rsqrtf(s * a.norm_inv_dim + a.norm_eps);
+}
+
+// Epilogue inputs of one row that do not depend on the accumulator, loaded into
+// registers by the epilogue warps before they wait for it (the wait overlaps
+// their latency): the norm row factor, the row's residual segment (residual
+// add: its first RES columns; the rest, for wide tiles, is loaded chunk by
+// chunk) and the row's RoPE (cos, sin) pairs (one position per row, the same
+// for every head of the tile).
+template <int BN, int EPI>
+struct EpiPre {
+  static constexpr int RES = EPI == GE_ADD_F32 && BN <= 96 ? BN : 0;
+  static constexpr int CS = EPI == GE_QKV_ROPE64 ? 32 : (EPI == GE_QKV_ROPE32 ? 16 : 0);
+  float scale = 1.f;
+  float4 res[RES > 0 ? RES / 4 : 1];
+  float2 cs[CS > 0 ? CS : 1];
+};
+
+// float4 j of a row segment of an f32 output [.., ldo] starting at column col
+// (zeros outside the N columns)
+SVLA_DEV float4 load_res4(const GemmArgs& a, int m, int col) {
+  const float* p = reinterpret_cast<const float*>(a.out) + (size_t)m * a.ldo + col;
+  if (col + 4 <= a.N) return __ldcg(reinterpret_cast<const float4*>(p));
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (col < a.N) v.x = p[0];
+  if (col + 1 < a.N) v.y = p[1];
+  if (col + 2 < a.N) v.z = p[2];
+  return v;
+}
+
+template <int BN, int EPI>
+SVLA_DEV void epi_prefetch(const GemmArgs& a, int m, int n0, bool row_ok, EpiPre<BN, EPI>& pre) {
+  pre.scale = norm_row_scale(a, m, row_ok);
+  if constexpr (EpiPre<BN, EPI>::RES > 0) {
+#pragma unroll
+    for (int j = 0; j < EpiPre<BN, EPI>::RES / 4; ++j)
+      pre.res[j] = row_ok ? load_res4(a, m, n0 + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  if constexpr (EPI == GE_ADD_F32) {
+    // wider tiles: the row segment is read chunk by chunk through L1; start
+    // bringing its lines there now
+    if (row_ok) {
+      const float* p = reinterpret_cast<const float*>(a.out) + (size_t)m * a.ldo + n0;
+#pragma unroll
+      for (int c = EpiPre<BN, EPI>::RES; c < BN; c += 32)
+        if (n0 + c < a.N) prefetch_l1(p + c);
+    }
+  }
+  if constexpr (EpiPre<BN, EPI>::CS > 0) {
+    int p = 0;
+    if (row_ok) {
+      p = a.pos ? __ldg(a.pos + m) : (m % a.pos_mod);
+      if (p < 0) p = 0;  // leading pad slots (unspecified output)
+    }
+#pragma unroll
+    for (int i = 0; i < EpiPre<BN, EPI>::CS; ++i) pre.cs[i] = __ldg(a.rope_cs + (size_t)p * EpiPre<BN, EPI>::CS + i);
+  }
 }
 
 // Split-K reduction by the last CTA of a tile: the 128 epilogue threads sum
@@ -248,8 +300,9 @@ SVLA_DEV void reduce_partials(const float* tile_part, int splits, int rows, floa
 }
 
 template <int BN, int EPI>
-SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, bool row_ok, float row_scale) {
-  src.scale = row_scale;
+SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, bool row_ok,
+                           const EpiPre<BN, EPI>& pre) {
+  src.scale = pre.scale;
   // tcgen05.ld is warp-collective: every lane walks the same columns; only
   // rows inside M store.
   if constexpr (EPI == GE_SWIGLU) {
@@ -258,34 +311,27 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, 
     const int F = a.N / 2;
 #pragma unroll 1
     for (int j = 0; j < BN / 64; ++j) {
-#pragma unroll 1
-      for (int c = 0; c < 32; c += 16) {
-        float g[16], u[16];
-        src.get(64 * j + c, g);
-        src.get(64 * j + 32 + c, u);
-        const int f = n0 / 2 + 32 * j + c;
-        if (row_ok && f < F) {
+      float gu[64];
+      src.get(64 * j, gu);
+      const int f = n0 / 2 + 32 * j;
+      if (row_ok && f < F) {
+#pragma unroll
+        for (int c = 0; c < 32; c += 16) {
           float h[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) h[i] = silu_f(g[i]) * u[i];
-          store16_bf16(out + (size_t)m * a.ldo + f, h, F - f);
+          for (int i = 0; i < 16; ++i) h[i] = silu_f(gu[c + i]) * gu[32 + c + i];
+          if (f + c < F) store16_bf16(out + (size_t)m * a.ldo + f + c, h, F - f - c);
         }
       }
     }
   } else if constexpr (EPI == GE_QKV_ROPE64 || EPI == GE_QKV_ROPE32) {
     constexpr int HD = EPI == GE_QKV_ROPE64 ? 64 : 32;
     constexpr int HALF = HD / 2;
-    int p = 0;
-    if (row_ok) {
-      p = a.pos ? __ldg(a.pos + m) : (m % a.pos_mod);
-      if (p < 0) p = 0;  // leading pad slots (unspecified output)
-    }
 #pragma unroll 1
     for (int hb = 0; hb < BN; hb += HD) {
       const int col = n0 + hb;
       float x[HD];
-#pragma unroll
-      for (int c = 0; c < HD; c += 16) src.get(hb + c, *reinterpret_cast<float(*)[16]>(x + c));
+      src.get(hb, x);
       if (!row_ok || col >= a.N) continue;
       bf16* dst;
       bool rot = true;
@@ -299,10 +345,9 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, 
       }
       if (rot) {
         // rotate-half RoPE: pairs (i, i + HD/2), angle pos * base^(-2i/HD)
-        const float2* cs = a.rope_cs + (size_t)p * HALF;
 #pragma unroll
         for (int i = 0; i < HALF; ++i) {
-          const float2 t = __ldg(cs + i);
+          const float2 t = pre.cs[i];
           const float x1 = x[i], x2 = x[i + HALF];
           x[i] = x1 * t.x - x2 * t.y;
           x[i + HALF] = x2 * t.x + x1 * t.y;
@@ -312,46 +357,69 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, 
       for (int c = 0; c < HD; c += 16) store16_bf16(dst + c, *reinterpret_cast<float(*)[16]>(x + c), 16);
     }
   } else {
+    constexpr int RES = EpiPre<BN, EPI>::RES;
+    // residual add with the row segment in registers: 32 columns per TMEM wait,
+    // unrolled so the residual registers are indexed by constants; otherwise
+    // 16 columns per wait, the residual (if any) read through L1, where
+    // epi_prefetch brought its lines
+    constexpr int CW = RES > 0 ? 32 : 16;
     float ss = 0.f;  // sum of squares of this row's outputs in this tile (fused RMSNorm)
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
-      float v[16];
+    auto chunk = [&](int c) {
+      float v[CW];
       src.get(c, v);
-      const int col = n0 + c;
-      if (!row_ok || col >= a.N) continue;
-      const int ncols = a.N - col;
-      add_bias16(v, a.bias, col, a.N);
-      if constexpr (EPI == GE_F32 || EPI == GE_ADD_F32) {
-        float* dst = reinterpret_cast<float*>(a.out) + (size_t)m * a.ldo + col;
-        if constexpr (EPI == GE_ADD_F32) {
-          if (ncols >= 16) {
-            const float4* d4 = reinterpret_cast<const float4*>(dst);
+      if (!row_ok || n0 + c >= a.N) return;
+#pragma unroll
+      for (int h = 0; h < CW; h += 16) {
+        const int col = n0 + c + h;
+        if (col >= a.N) break;
+        const int ncols = a.N - col;
+        float (&w)[16] = *reinterpret_cast<float(*)[16]>(v + h);
+        add_bias16(w, a.bias, col, a.N);
+        if constexpr (EPI == GE_F32 || EPI == GE_ADD_F32) {
+          float* dst = reinterpret_cast<float*>(a.out) + (size_t)m * a.ldo + col;
+          if constexpr (EPI == GE_ADD_F32) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const float4 o = d4[i];
-              v[4 * i] += o.x;
-              v[4 * i + 1] += o.y;
-              v[4 * i + 2] += o.z;
-              v[4 * i + 3] += o.w;
+              float4 o;
+              if constexpr (RES > 0) {
+                o = pre.res[(c + h) / 4 + i];  // c + h < BN = RES: a constant once unrolled
+              } else if (ncols >= 16) {
+                o = reinterpret_cast<const float4*>(dst)[i];
+              } else {
+                o = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (4 * i < ncols) o.x = dst[4 * i];
+                if (4 * i + 1 < ncols) o.y = dst[4 * i + 1];
+                if (4 * i + 2 < ncols) o.z = dst[4 * i + 2];
+                if (4 * i + 3 < ncols) o.w = dst[4 * i + 3];
+              }
+              w[4 * i] += o.x;
+              w[4 * i + 1] += o.y;
+              w[4 * i + 2] += o.z;
+              w[4 * i + 3] += o.w;
             }
-          } else {
-            for (int i = 0; i < ncols; ++i) v[i] += dst[i];
           }
-        }
-        store16_f32(dst, v, ncols);
-        if (a.rb_out) {
-          store16_bf16(a.rb_out + (size_t)m * a.ld_rb + col, v, ncols);
+          store16_f32(dst, w, ncols);
+          if (a.rb_out) {
+            store16_bf16(a.rb_out + (size_t)m * a.ld_rb + col, w, ncols);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (i < ncols) ss = fmaf(v[i], v[i], ss);
-        }
-      } else if constexpr (EPI == GE_BF16) {
-        store16_bf16(reinterpret_cast<bf16*>(a.out) + (size_t)m * a.ldo + col, v, ncols);
-      } else if constexpr (EPI == GE_SILU_BF16) {
+            for (int i = 0; i < 16; ++i)
+              if (i < ncols) ss = fmaf(w[i], w[i], ss);
+          }
+        } else if constexpr (EPI == GE_BF16) {
+          store16_bf16(reinterpret_cast<bf16*>(a.out) + (size_t)m * a.ldo + col, w, ncols);
+        } else if constexpr (EPI == GE_SILU_BF16) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = silu_f(v[i]);
-        store16_bf16(reinterpret_cast<bf16*>(a.out) + (size_t)m * a.ldo + col, v, ncols);
+          for (int i = 0; i < 16; ++i) w[i] = silu_f(w[i]);
+          store16_bf16(reinterpret_cast<bf16*>(a.out) + (size_t)m * a.ldo + col, w, ncols);
+        }
       }
+    };
+    if constexpr (RES > 0) {
+#pragma unroll
+      for (int c = 0; c < BN; c += CW) chunk(c);
+    } else {
+#pragma unroll 1
+      for (int c = 0; c < BN; c += CW) chunk(c);
     }
     if constexpr (EPI == GE_F32 || EPI == GE_ADD_F32) {
       if (a.ss_out && row_ok) a.ss_out[(size_t)(n0 / BN) * a.ss_ld + m] = ss;
@@ -366,13 +434,14 @@ SVLA_DEV void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 // this split's partial tile to the cluster or global-workspace reduction.
 template <int BN, int EPI, bool CLUSTER_OK>
 SVLA_DEV void gemm_accumulator_out(const GemmArgs& args, uint32_t tmem_base, uint8_t* ring, volatile uint32_t* misc,
-                                   int quad, int row, int m, int n0, bool row_ok, float rscale, int m_blk, int n_blk,
+                                   int quad, int row, int m, int n0, bool row_ok, const EpiPre<BN, EPI>& pre,
+                                   int m_blk, int n_blk,
                                    int split, int splits) {
   AccSource<BN> src;
   src.taddr_row = tmem_base + ((uint32_t)(quad * 32) << 16);
   src.smem_row = nullptr;
   if (splits == 1) {
-    run_epilogue<BN, EPI>(args, src, m, n0, row_ok, rscale);
+    run_epilogue<BN, EPI>(args, src, m, n0, row_ok, pre);
   } else if (CLUSTER_OK && args.red_mode == GEMM_RED_CLUSTER) {
     // stage this split's partial tile in shared memory (the operand ring is idle)
     float* red = reinterpret_cast<float*>(ring);
@@ -410,7 +479,7 @@ SVLA_DEV void gemm_accumulator_out(const GemmArgs& args, uint32_t tmem_base, uin
       reduce_partials<BN>(tile_part, splits, rows, red, threadIdx.x - 64);
       epi_bar();
       src.smem_row = red + row * (BN + 4);
-      run_epilogue<BN, EPI>(args, src, m, n0, row_ok, rscale);
+      run_epilogue<BN, EPI>(args, src, m, n0, row_ok, pre);
       if (threadIdx.x == 64) args.counters[tile] = 0;  // re-arm for the next launch
     }
   }
@@ -426,7 +495,8 @@ SVLA_DEV void gemm_accumulator_out(const GemmArgs& args, uint32_t tmem_base, uin
 template <int BN, int EPI, bool CLUSTER_OK>
 SVLA_DEV void gemm_epilogue_after_wait(bool ok, const GemmArgs& args, uint32_t tmem_base, uint8_t* ring,
                                        volatile uint32_t* misc, int quad, int row, int m, int n0, bool row_ok,
-                                       float rscale, int m_blk, int n_blk, int split, int splits) {
+                                       const EpiPre<BN, EPI>& pre, int m_blk, int n_blk, int split,
+                                       int splits) {
   if (!ok) {
     misc[1] = 1;
     set_status(args.status, SVLA_ERR_TIMEOUT);
@@ -434,7 +504,7 @@ SVLA_DEV void gemm_epilogue_after_wait(bool ok, const GemmArgs& args, uint32_t t
   epi_bar();
   tc_fence_after();
   if (misc[1] == 0) {
-    gemm_accumulator_out<BN, EPI, CLUSTER_OK>(args, tmem_base, ring, misc, quad, row, m, n0, row_ok, rscale, m_blk,
+    gemm_accumulator_out<BN, EPI, CLUSTER_OK>(args, tmem_base, ring, misc, quad, row, m, n0, row_ok, pre, m_blk,
                                               n_blk, split, splits);
   } else if (splits > 1 && !(CLUSTER_OK && args.red_mode == GEMM_RED_CLUSTER)) {
     if (threadIdx.x == 64) {
@@ -450,7 +520,7 @@ SVLA_DEV void gemm_epilogue_after_wait(bool ok, const GemmArgs& args, uint32_t t
 // tiles in split order and runs their epilogue.
 template <int BN, int EPI, bool CLUSTER_OK>
 SVLA_DEV void gemm_cluster_reduce(const GemmArgs& args, uint8_t* ring, volatile uint32_t* misc,
-                                  const float* misc_scale, int m_blk, int n_blk, int splits) {
+                                  const EpiPre<BN, EPI>& pre, int m_blk, int n_blk, int splits) {
   if constexpr (CLUSTER_OK) {
     if (args.red_mode == GEMM_RED_CLUSTER && splits > 1) {
       // Every thread of every CTA of the cluster reaches both barriers exactly
@@ -492,7 +562,7 @@ SVLA_DEV void gemm_cluster_reduce(const GemmArgs& args, uint8_t* ring, volatile 
           AccSource<BN> src;
           src.taddr_row = 0;
           src.smem_row = fin + row * (BN + 4);
-          run_epilogue<BN, EPI>(args, src, m, n_blk * BN, true, misc_scale[row]);
+          run_epilogue<BN, EPI>(args, src, m, n_blk * BN, true, pre);  // this thread's own row: its prefetch
         }
       }
       cluster_sync();  // peers have finished reading this CTA's partial tile
@@ -513,7 +583,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES, A_ROWS>::MIN
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(bars + 2 * STAGES + 1);
   // misc[0] tmem base, misc[1] abort flag, misc[2] k-blocks issued, misc[3] k-blocks consumed,
   // misc[4] "this CTA reduces"
-  float* misc_scale = reinterpret_cast<float*>(smem + C::RING_BYTES + 512);  // [128] row factors
+  EpiPre<BN, EPI> pre;  // the epilogue warps' inputs of their row, loaded before the accumulator is ready
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -617,12 +687,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES, A_ROWS>::MIN
     const int m = m_blk * GEMM_BM + row;
     const bool row_ok = m < args.M;
     const int n0 = n_blk * BN;
-    prefetch_epilogue_inputs<BN, EPI>(args, m, n0, row_ok);
-    const float rscale = norm_row_scale(args, m, row_ok);  // overlaps the main loop
-    misc_scale[row] = rscale;
+    epi_prefetch<BN, EPI>(args, m, n0, row_ok, pre);  // overlaps the main loop
     const bool ok = mbar_wait(acc_bar, 0, lim);
     gemm_epilogue_after_wait<BN, EPI, C::CLUSTER_OK>(ok, args, tmem_base, ring, misc, quad, row, m, n0, row_ok,
-                                                     rscale, m_blk, n_blk, split, splits);
+                                                     pre, m_blk, n_blk, split, splits);
     tc_fence_before();
   }
 
@@ -637,7 +705,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES, A_ROWS>::MIN
     if (threadIdx.x == 32) mbar_wait(acc_bar, 0, GEMM_DRAIN_NS);
     __syncthreads();
   }
-  gemm_cluster_reduce<BN, EPI, C::CLUSTER_OK>(args, ring, misc, misc_scale, m_blk, n_blk, splits);
+  gemm_cluster_reduce<BN, EPI, C::CLUSTER_OK>(args, ring, misc, pre, m_blk, n_blk, splits);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);

@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(bars + 3 * STAGES + 2 * C::B_BUFS + 1);
   // misc[0] tmem base, misc[1] abort flag, misc[2] stages issued, misc[3] stages consumed,
   // misc[4] "this CTA reduces"
-  float* misc_scale = reinterpret_cast<float*>(smem + C::RING_BYTES + 512);
+  EpiPre<BN, EPI> epre;  // the epilogue warps' inputs of their row, loaded before the accumulator is ready
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -228,16 +228,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
     const int m = m_blk * GEMM_BM + row;
     const bool row_ok = m < args.M;
     const int pre = nkb < STAGES ? nkb : STAGES;
-    float rscale = 1.f;
     bool have_scale = false;
     // after the stages whose codes were requested before the dependency wait:
     // the epilogue's inputs come from earlier kernels, and their loads then
     // overlap the rest of the main loop
     auto epilogue_inputs = [&]() {
       griddep_wait();
-      prefetch_epilogue_inputs<BN, EPI>(args, m, n0, row_ok);
-      rscale = norm_row_scale(args, m, row_ok);
-      misc_scale[row] = rscale;
+      epi_prefetch<BN, EPI>(args, m, n0, row_ok, epre);
       have_scale = true;
     };
     for (int i = 0; i < nkb; ++i) {
@@ -288,7 +285,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
     if (!have_scale) epilogue_inputs();  // the loop stopped early (time-out)
     const bool ok = mbar_wait(acc_bar, 0, lim);
     gemm_epilogue_after_wait<BN, EPI, C::CLUSTER_OK>(ok, args, tmem_base, ring, misc, quad, row, m, n0, row_ok,
-                                                     rscale, m_blk, n_blk, split, splits);
+                                                     epre, m_blk, n_blk, split, splits);
     tc_fence_before();
   }
 
@@ -306,7 +303,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
     if (threadIdx.x == 32) mbar_wait(acc_bar, 0, GEMM_DRAIN_NS);
     __syncthreads();
   }
-  gemm_cluster_reduce<BN, EPI, C::CLUSTER_OK>(args, ring, misc, misc_scale, m_blk, n_blk, splits);
+  gemm_cluster_reduce<BN, EPI, C::CLUSTER_OK>(args, ring, misc, epre, m_blk, n_blk, splits);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
