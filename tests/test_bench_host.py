@@ -44,3 +44,11 @@ def test_chunk_delta_summary():
     assert d["per_dim_max"][5] == 3e-2 and abs(d["per_dim_max"][3] - 1e-2) < 1e-12
     assert d["median"] == 0.0
     assert bench.chunk_delta(ref, ref)["pass"]
+
+
+def test_oracle_subsets_are_the_batched_workloads_query_subsets():
+    """The CPU baseline times the oracle on 4 of 32, 2 of 8 and 4 of 256 queries
+    of the batched workloads; each subset is a proper prefix of the batch."""
+    assert bench.ORACLE_SUBSETS == {"smolvla_b32": 4, "long_prefix_b8": 2, "denoise_b256": 4}
+    for name, n in bench.ORACLE_SUBSETS.items():
+        assert 0 < n < synth.WORKLOADS[name].B
