@@ -140,7 +140,10 @@ SVLA_API int svla_prefix_weights(const svla_handle* h);
  *     every tensor of the blob from the first expert layer's in_norm to b_out,
  *     in manifest order and shape ([out, in] for matrices) (written in full).
  * The forward uses the weights given to svla_create_ex; work is stream-ordered
- * and bitwise reproducible (fixed-order reductions). Needs a handle created
+ * and bitwise reproducible (fixed-order reductions). The step runs as one CUDA
+ * graph, captured on the first call with a given (B, L, H, buffers) and
+ * replayed afterwards (like svla_denoise), so make that first call before
+ * any stream capture of your own. Needs a handle created
  * with SVLA_CREATE_TRAIN (else SVLA_ERR_UNSUPPORTED); B, L, H within the
  * handle's limits (else SVLA_ERR_SHAPE). */
 SVLA_API svla_status svla_train_step(svla_handle* h, const void* kv_cache, const uint8_t* pad_mask, int B,

@@ -1495,10 +1495,17 @@ svla_status svla_train_step(svla_handle* h, const void* kv_cache, const uint8_t*
   if (((uintptr_t)grads & 15) || ((uintptr_t)kv_cache & 15))
     return fail(h, SVLA_ERR_ARG, "grads and kv_cache must be 16-byte aligned");
   DeviceGuard dg(h->device);
-  const cudaError_t e = record_train(h, kv_cache, pad_mask, B, L, actions, noise, t, H, loss, grads,
-                                     reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(h, e, "train step");
-  return SVLA_OK;
+  // the whole step (~600 launches) as one CUDA graph per (shape, buffers)
+  const std::vector<uint64_t> key = {4u, (uint64_t)B, (uint64_t)L, (uint64_t)H, (uint64_t)(uintptr_t)kv_cache,
+                                     (uint64_t)(uintptr_t)pad_mask, (uint64_t)(uintptr_t)actions,
+                                     (uint64_t)(uintptr_t)noise, (uint64_t)(uintptr_t)t, (uint64_t)(uintptr_t)loss,
+                                     (uint64_t)(uintptr_t)grads, g_wait_ns.load()};
+  return run_graph(
+      h, key,
+      [&](cudaStream_t cs) {
+        return record_train(h, kv_cache, pad_mask, B, L, actions, noise, t, H, loss, grads, cs);
+      },
+      reinterpret_cast<cudaStream_t>(stream), "train step");
 }
 
 int svla_denoise_fused_supported(const svla_handle* h, int B, int H) {
