@@ -46,16 +46,35 @@ import synth  # noqa: E402
 METRIC = "ms per 50-action chunk (b=1)"
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM bytes (read + write) per launch from ncu captures, None whenever the
-# kernel has changed since its capture:
-#  - the batch-1 GEMM kernel (gemm_tc_kernel): mean of the three launches of
-#    the capture summarised in profiles/gemm_tc_kernel_smolvla_b1.md;
-#  - the persistent denoise kernel: profiles/denoise_fused_kernel_smolvla_b1.md.
-NCU_TRAFFIC_GEMM_B1 = 3.698e6
-NCU_TRAFFIC_FUSED = 1.9916e9
-#  - the int8 prefill's gate/up GEMM (gemm_w8_kernel<64, SwiGLU, 4>, M=177, N=5120, K=960):
-#    profiles/gemm_w8_kernel_smolvla_b1.md.
-NCU_TRAFFIC_W8_GATE_UP_B1 = 5.6445e6
+# DRAM bytes (read + write) per launch of the dominant kernels, from the ncu
+# captures summarised in profiles/ncu_traffic.json. Each entry records a hash
+# of the CUDA sources it was taken on; when the sources have changed since,
+# the figure no longer describes the kernel and is reported as None.
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+
+
+def sources_sha16() -> str:
+    """First 16 hex digits of the SHA-256 over the CUDA sources and the header."""
+    import glob
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "vision_language_action_b200", "csrc", "*")))
+    for f in files + [os.path.join(ROOT, "include", "svla.h")]:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from its capture, or None (no capture,
+    or the sources changed since it was taken)."""
+    try:
+        rec = json.load(open(TRAFFIC_FILE))["kernels"].get(kernel)
+    except (OSError, ValueError, KeyError):
+        return None
+    if not rec or rec.get("sources_sha16") != sources_sha16():
+        return None
+    return float(rec["dram_bytes_per_launch"])
 
 
 def _peaks():
@@ -469,7 +488,7 @@ def gemm_roofline(s, B, L, H, n_steps, dev, hbm_peak):
     achieved = bytes_chunk / (t_chunk * 1e-3) / 1e9
     return {"bound": "hbm", "kernel": "gemm_tc_kernel", "achieved": round(achieved, 1), "peak": hbm_peak,
             "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-            "traffic": NCU_TRAFFIC_GEMM_B1,
+            "traffic": ncu_traffic("gemm_tc_kernel_b1"),
             "launches_per_chunk": n_launch, "avg_launch_us": round(1e3 * t_chunk / n_launch, 2),
             "algorithmic_bytes_per_launch": int(bytes_chunk / n_launch),
             "gemm_ms_per_chunk": round(float(t_chunk), 4)}
@@ -508,7 +527,7 @@ def int8_prefix(args, dev, barrier, hbm_peak, peak_kind):
             M, N, K = wl.L, 2 * s.p_ffn, s.p_width
             out["gemm_w8_gate_up_b1"] = {"kernel": "gemm_w8_kernel<64, SwiGLU, 4>", "M": M, "N": N, "K": K,
                                          "algorithmic_bytes_per_launch": int(N * K + N * (K // 64) * 4 + 2 * M * K),
-                                         "traffic": NCU_TRAFFIC_W8_GATE_UP_B1}
+                                         "traffic": ncu_traffic("gemm_w8_kernel_gate_up_b1")}
         out[name] = {"prefill_ms": round(t8, 4), "prefill_ms_dense_same_handle": round(t16, 4),
                      "chunk_ms": round(c8 / wl.B, 4) if wl.B == 1 else None,
                      "chunks_per_s": round(wl.B / (c8 * 1e-3), 2) if wl.B > 1 else None,
@@ -721,7 +740,7 @@ def ours(args, rank, world, local_rank):
         t_den = ms_den / args.steps * 1e-3
         achieved = dbytes / t_den / 1e9
         roof = {"bound": "hbm", "kernel": "denoise_fused_kernel", "achieved": round(achieved, 1), "peak": hbm_peak,
-                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": NCU_TRAFFIC_FUSED,
+                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": ncu_traffic("denoise_fused_kernel_b1"),
                 "algorithmic_bytes_per_launch": int(dbytes), "launch_ms": round(t_den * 1e3, 4),
                 "timed_as": "svla_denoise call (16 hoisted K'/V' projection GEMMs + denoise_fused_kernel), CUDA events",
                 "peak_kind": f"{peak_kind} HBM copy"}

@@ -52,3 +52,17 @@ def test_oracle_subsets_are_the_batched_workloads_query_subsets():
     assert bench.ORACLE_SUBSETS == {"smolvla_b32": 4, "long_prefix_b8": 2, "denoise_b256": 4}
     for name, n in bench.ORACLE_SUBSETS.items():
         assert 0 < n < synth.WORKLOADS[name].B
+
+
+def test_traffic_figures_follow_the_sources_they_were_captured_on(tmp_path, monkeypatch):
+    """A recorded ncu traffic figure is reported only while the CUDA sources
+    hash to the value recorded with it."""
+    import json
+    f = tmp_path / "t.json"
+    f.write_text(json.dumps({"kernels": {"k": {"dram_bytes_per_launch": 123.0,
+                                               "sources_sha16": bench.sources_sha16()}}}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.ncu_traffic("k") == 123.0
+    assert bench.ncu_traffic("absent") is None
+    f.write_text(json.dumps({"kernels": {"k": {"dram_bytes_per_launch": 123.0, "sources_sha16": "0" * 16}}}))
+    assert bench.ncu_traffic("k") is None
