@@ -224,6 +224,7 @@ struct EpiPre {
   static constexpr int RES = EPI == GE_ADD_F32 && BN <= 96 ? BN : 0;
   static constexpr int CS = EPI == GE_QKV_ROPE64 ? 32 : (EPI == GE_QKV_ROPE32 ? 16 : 0);
   float scale = 1.f;
+  bool have_res = false;  // res holds the row segment (else the epilogue reads it)
   float4 res[RES > 0 ? RES / 4 : 1];
   float2 cs[CS > 0 ? CS : 1];
 };
@@ -240,13 +241,19 @@ SVLA_DEV float4 load_res4(const GemmArgs& a, int m, int col) {
   return v;
 }
 
+// want_res: this CTA runs the epilogue of this row (split-K: only one CTA of
+// a tile does, so the others leave the residual to it)
 template <int BN, int EPI>
-SVLA_DEV void epi_prefetch(const GemmArgs& a, int m, int n0, bool row_ok, EpiPre<BN, EPI>& pre) {
+SVLA_DEV void epi_prefetch(const GemmArgs& a, int m, int n0, bool row_ok, EpiPre<BN, EPI>& pre,
+                           bool want_res = true) {
   pre.scale = norm_row_scale(a, m, row_ok);
   if constexpr (EpiPre<BN, EPI>::RES > 0) {
+    if (want_res) {
 #pragma unroll
-    for (int j = 0; j < EpiPre<BN, EPI>::RES / 4; ++j)
-      pre.res[j] = row_ok ? load_res4(a, m, n0 + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < EpiPre<BN, EPI>::RES / 4; ++j)
+        pre.res[j] = row_ok ? load_res4(a, m, n0 + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      pre.have_res = true;
+    }
   }
   if constexpr (EPI == GE_ADD_F32) {
     // wider tiles: the row segment is read chunk by chunk through L1; start
@@ -382,7 +389,8 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, 
             for (int i = 0; i < 4; ++i) {
               float4 o;
               if constexpr (RES > 0) {
-                o = pre.res[(c + h) / 4 + i];  // c + h < BN = RES: a constant once unrolled
+                // c + h < BN = RES: a constant once unrolled
+                o = pre.have_res ? pre.res[(c + h) / 4 + i] : load_res4(a, m, col + 4 * i);
               } else if (ncols >= 16) {
                 o = reinterpret_cast<const float4*>(dst)[i];
               } else {
@@ -687,7 +695,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<BN, STAGES, A_ROWS>::MIN
     const int m = m_blk * GEMM_BM + row;
     const bool row_ok = m < args.M;
     const int n0 = n_blk * BN;
-    epi_prefetch<BN, EPI>(args, m, n0, row_ok, pre);  // overlaps the main loop
+    // the residual in registers only where this CTA finishes the row: one
+    // split, or the cluster rank that reduces it
+    bool want_res = splits == 1;
+    if constexpr (C::CLUSTER_OK)
+      if (splits > 1 && args.red_mode == GEMM_RED_CLUSTER) want_res = row % splits == (int)cluster_ctarank();
+    epi_prefetch<BN, EPI>(args, m, n0, row_ok, pre, want_res);  // overlaps the main loop
     const bool ok = mbar_wait(acc_bar, 0, lim);
     gemm_epilogue_after_wait<BN, EPI, C::CLUSTER_OK>(ok, args, tmem_base, ring, misc, quad, row, m, n0, row_ok,
                                                      pre, m_blk, n_blk, split, splits);

@@ -234,7 +234,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
     // overlap the rest of the main loop
     auto epilogue_inputs = [&]() {
       griddep_wait();
-      epi_prefetch<BN, EPI>(args, m, n0, row_ok, epre);
+      bool want_res = splits == 1;  // as in gemm_tc_kernel
+      if constexpr (C::CLUSTER_OK)
+        if (splits > 1 && args.red_mode == GEMM_RED_CLUSTER) want_res = row % splits == (int)cluster_ctarank();
+      epi_prefetch<BN, EPI>(args, m, n0, row_ok, epre, want_res);
       have_scale = true;
     };
     for (int i = 0; i < nkb; ++i) {
