@@ -28,7 +28,7 @@ than the oracle itself): block mask / joint pass, constant velocity, GQA =
 MHA with repeated heads, brute-force loops on the tiny shape, RoPE closed
 form, L = 1 attention, padding and batch invariance, parameter counts, and
 the Philox4x32-10 known-answer vectors. ``assembly.py`` (prefix assembly),
-``quant.py`` (the weight-only int8 preset) and ``train.py`` (the expert's
+``quant.py`` (the weight-only int8 presets of the prefix and of the expert) and ``train.py`` (the expert's
 training step) carry their own pins in ``tests/test_oracle_assembly.py``,
 ``tests/test_oracle_quant.py`` and ``tests/test_oracle_train.py``. Parity
 against the real SmolVLA checkpoint is unpinned: no weights or activation
@@ -40,5 +40,5 @@ from .model import (  # noqa: F401
 )
 from .philox import philox4x32_10, gaussian_noise  # noqa: F401
 from .assembly import pixel_shuffle, connector, state_token, assemble_prefix  # noqa: F401
-from .quant import quantize_affine8, dequantize_affine8, quantize_prefix  # noqa: F401
+from .quant import quantize_affine8, dequantize_affine8, quantize_prefix, quantize_expert  # noqa: F401
 from .train import train_step, trainable_names, loss_np  # noqa: F401

@@ -1,4 +1,5 @@
-"""Weight-only int8 quantisation of the prefix LM ("vlm-8bit"), plain definition.
+"""Weight-only int8 quantisation of the prefix LM ("vlm-8bit") and of the action
+expert, plain definition.
 
 TEST INFRASTRUCTURE ONLY (see the package docstring): the CUDA library must
 never import this module.
@@ -28,6 +29,14 @@ Readings (numbered after those of ``assembly.py``):
     The quantised model is the dense bf16 model with every quantised matrix
     replaced by w^; where a norm gain is folded into a projection, it is
     applied to w^ as it is to the dense weight.
+29. The expert preset (the scope "prefix/expert" of the int8 row): the same
+    scheme applied to the weight matrices of every action-expert layer —
+    W_q, W_k, W_v (the odd layers' W_k, W_v act on the prefix cache), W_o,
+    W_g, W_u, W_d; the expert's heads (action_in, the time MLP, action_out)
+    and its norm gains stay bf16. The expert's 720-wide inputs are not a
+    multiple of 64: where K mod 64 is not zero, the last group of each row
+    holds the K mod 64 remaining inputs (columns 64 (G - 1) .. K - 1,
+    G = ceil(K / 64)), with its own scale and offset by the same rules.
 """
 from __future__ import annotations
 
@@ -38,6 +47,7 @@ import numpy as np
 GROUP = 64
 QMAX = 255
 PREFIX_LINEARS = ("wq", "wk", "wv", "wo", "wg", "wu", "wd")
+EXPERT_LINEARS = PREFIX_LINEARS
 
 
 def _bf16_rne(x: np.ndarray) -> np.ndarray:
@@ -47,31 +57,47 @@ def _bf16_rne(x: np.ndarray) -> np.ndarray:
     return u.astype(np.uint32).view(np.float32)
 
 
+def group_bounds(K: int) -> List[Tuple[int, int]]:
+    """Column ranges of the groups of a K-wide row: runs of 64, the last one
+    holding the K mod 64 remaining inputs when that is not zero (reading 29)."""
+    return [(k0, min(k0 + GROUP, K)) for k0 in range(0, K, GROUP)]
+
+
 def quantize_affine8(w: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
-    """[N, K] weights (bf16 values, K a multiple of 64) -> codes uint8 [N, K],
-    alpha and beta float32 [N, K/64] holding bf16 values (reading 23)."""
+    """[N, K] weights (bf16 values) -> codes uint8 [N, K], alpha and beta
+    float32 [N, G] holding bf16 values, G = ceil(K / 64) (readings 23, 29)."""
     w = np.asarray(w, np.float32)
     N, K = w.shape
-    if K % GROUP:
-        raise ValueError("the input width must be a multiple of 64")
-    g = w.reshape(N, K // GROUP, GROUP)
-    lo = g.min(axis=-1)
-    hi = g.max(axis=-1)
-    alpha = _bf16_rne((hi - lo) / np.float32(QMAX))
-    beta = lo
-    safe = np.where(alpha > 0, alpha, np.float32(1)).astype(np.float32)
-    t = np.rint((g - beta[..., None]) / safe[..., None])
-    q = np.clip(t, 0, QMAX)
-    q = np.where(alpha[..., None] > 0, q, 0).astype(np.uint8)
-    return q.reshape(N, K), alpha.astype(np.float32), beta.astype(np.float32)
+    if K < 1:
+        raise ValueError("empty input width")
+    bounds = group_bounds(K)
+    q = np.zeros((N, K), np.uint8)
+    alpha = np.zeros((N, len(bounds)), np.float32)
+    beta = np.zeros((N, len(bounds)), np.float32)
+    for g, (k0, k1) in enumerate(bounds):
+        grp = w[:, k0:k1]
+        lo = grp.min(axis=1)
+        hi = grp.max(axis=1)
+        a = _bf16_rne((hi - lo) / np.float32(QMAX))
+        safe = np.where(a > 0, a, np.float32(1)).astype(np.float32)
+        t = np.rint((grp - lo[:, None]) / safe[:, None])
+        codes = np.clip(t, 0, QMAX)
+        q[:, k0:k1] = np.where(a[:, None] > 0, codes, 0).astype(np.uint8)
+        alpha[:, g] = a
+        beta[:, g] = lo
+    return q, alpha, beta
 
 
 def dequantize_affine8(q: np.ndarray, alpha: np.ndarray, beta: np.ndarray) -> np.ndarray:
-    """w^ = bf16(fp32(alpha q + beta)) as float64 values (reading 24)."""
+    """w^ = bf16(fp32(alpha q + beta)) as float64 values (reading 24), group by group."""
     N, K = q.shape
-    qf = np.asarray(q, np.float32).reshape(N, K // GROUP, GROUP)
-    v = np.asarray(alpha, np.float32)[..., None] * qf + np.asarray(beta, np.float32)[..., None]
-    return _bf16_rne(v.astype(np.float32)).astype(np.float64).reshape(N, K)
+    out = np.zeros((N, K), np.float64)
+    for g, (k0, k1) in enumerate(group_bounds(K)):
+        a = np.asarray(alpha, np.float32)[:, g:g + 1]
+        b = np.asarray(beta, np.float32)[:, g:g + 1]
+        v = a * np.asarray(q[:, k0:k1], np.float32) + b
+        out[:, k0:k1] = _bf16_rne(v.astype(np.float32)).astype(np.float64)
+    return out
 
 
 def prefix_matrix_names(p_layers: int) -> List[str]:
@@ -84,5 +110,19 @@ def quantize_prefix(W: Dict[str, np.ndarray], p_layers: int) -> Dict[str, np.nda
     replaced by their dequantised values, every other tensor unchanged."""
     out = dict(W)
     for name in prefix_matrix_names(p_layers):
+        out[name] = dequantize_affine8(*quantize_affine8(W[name]))
+    return out
+
+
+def expert_matrix_names(e_layers: int) -> List[str]:
+    """The matrices the expert preset quantises (reading 29)."""
+    return [f"e{l}.{m}" for l in range(e_layers) for m in EXPERT_LINEARS]
+
+
+def quantize_expert(W: Dict[str, np.ndarray], e_layers: int) -> Dict[str, np.ndarray]:
+    """The weights of the int8-expert model: the expert layers' linear matrices
+    replaced by their dequantised values, every other tensor unchanged."""
+    out = dict(W)
+    for name in expert_matrix_names(e_layers):
         out[name] = dequantize_affine8(*quantize_affine8(W[name]))
     return out

@@ -111,7 +111,88 @@ def pin_constant_group(quantize, dequantize):
     assert np.array_equal(dequantize(q, a, b), w.astype(np.float64))
 
 
-PINS = [pin_grid_round_trip, pin_nearest_code, pin_error_bound, pin_group_min_exact, pin_constant_group]
+def _ragged_grid_matrix(rng, N, n_full, tail):
+    """Rows of n_full 64-groups and one `tail`-wide group, each on its own grid
+    w = alpha (j - c0) with codes 0 and the top code present. The tail's offset
+    c0 is -1, so its values alpha (j + 1) are all positive (and j + 1 <= 256 keeps
+    them bf16 values): a tail that is padded with zeros, or merged with the group
+    before it, gets another minimum."""
+    K = 64 * n_full + tail
+    w = np.zeros((N, K), np.float32)
+    codes = np.zeros((N, K), np.int64)
+    alpha = np.zeros((N, n_full + 1), np.float32)
+    beta = np.zeros((N, n_full + 1), np.float32)
+    for n in range(N):
+        for g in range(n_full + 1):
+            width = 64 if g < n_full else tail
+            j = rng.integers(0, 256, size=width)
+            j[0], j[1] = 0, 255
+            rng.shuffle(j)
+            e = float(rng.choice((-13, -11, -9)))
+            al = np.float32(2.0 ** e)
+            c0 = int(rng.integers(0, 256)) if g < n_full else -1
+            k0 = 64 * g
+            w[n, k0:k0 + width] = al * (j - c0).astype(np.float32)
+            codes[n, k0:k0 + width] = j
+            alpha[n, g] = al
+            beta[n, g] = -al * c0
+    assert np.array_equal(_bf16(w), w)  # |j - c0| <= 256: 8 significant bits
+    return w, codes, alpha, beta
+
+
+def pin_ragged_grid_round_trip(quantize, dequantize):
+    """K = 64 G + 16 (the expert's 720 = 11 * 64 + 16): every group, the 16-wide
+    last one included, recovers its grid exactly (reading 29)."""
+    rng = np.random.default_rng(21)
+    for n_full, tail in ((3, 16), (11, 16), (0, 48)):
+        w, j, alpha, beta = _ragged_grid_matrix(rng, 5, n_full, tail)
+        q, a, b = quantize(w)
+        assert q.shape == w.shape and a.shape == (5, n_full + 1)
+        assert np.array_equal(q.astype(np.int64), j)
+        assert np.array_equal(a, alpha) and np.array_equal(b, beta)
+        assert np.array_equal(dequantize(q, a, b), w.astype(np.float64))
+
+
+def pin_ragged_nearest_code(quantize, dequantize):
+    """With a ragged last group every code is still the nearest of its own group's
+    256 grid points (exact float64 search, the group found by column index)."""
+    rng = np.random.default_rng(22)
+    w = _random_matrix(rng, 4, 80)
+    w[1, 64:] = 0.3 + 1e-3 * rng.standard_normal(16).astype(np.float32)  # a tail far from the row
+    w = _bf16(w)
+    q, a, b = quantize(w)
+    codes = np.arange(256, dtype=np.float64)
+    for n in range(4):
+        for k in range(80):
+            g = k // 64
+            al, be = float(a[n, g]), float(b[n, g])
+            err = np.abs(be + al * codes - float(w[n, k]))
+            assert err[int(q[n, k])] <= err.min() + 1e-6 * max(al, 1e-30)
+        tail = w[n, 64:].astype(np.float64)
+        assert float(b[n, 1]) == tail.min()
+
+
+def pin_ragged_groups_are_independent(quantize, dequantize):
+    """Changing the inputs of one group changes nothing of the others (the 16-wide
+    last group is not padded, merged or shared)."""
+    rng = np.random.default_rng(23)
+    w = _random_matrix(rng, 3, 208)
+    q0, a0, b0 = quantize(w)
+    w2 = w.copy()
+    w2[:, 128:192] *= np.float32(4.0)
+    q1, a1, b1 = quantize(w2)
+    assert np.array_equal(q0[:, 192:], q1[:, 192:]) and np.array_equal(a0[:, 3], a1[:, 3])
+    assert np.array_equal(b0[:, 3], b1[:, 3])
+    w3 = w.copy()
+    w3[:, 192:] = np.float32(-1.5)
+    q2, a2, b2 = quantize(w3)
+    assert np.array_equal(q0[:, :192], q2[:, :192]) and np.array_equal(a0[:, :3], a2[:, :3])
+    assert np.all(a2[:, 3] == 0) and np.all(b2[:, 3] == np.float32(-1.5))
+    assert np.array_equal(dequantize(q2, a2, b2)[:, 192:], np.full((3, 16), -1.5))
+
+
+PINS = [pin_grid_round_trip, pin_nearest_code, pin_error_bound, pin_group_min_exact, pin_constant_group,
+        pin_ragged_grid_round_trip, pin_ragged_nearest_code, pin_ragged_groups_are_independent]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -125,9 +206,9 @@ def test_scale_and_offset_are_bf16_values():
     assert np.array_equal(_bf16(a), a) and np.array_equal(_bf16(b), b)
 
 
-def test_rejects_ragged_input_width():
+def test_rejects_empty_input_width():
     with pytest.raises(ValueError):
-        oq.quantize_affine8(np.zeros((2, 96), np.float32))
+        oq.quantize_affine8(np.zeros((2, 0), np.float32))
 
 
 def test_preset_scope_and_identity_on_grid_weights():
@@ -159,6 +240,46 @@ def test_preset_scope_and_identity_on_grid_weights():
     K0, V0 = oracle.prefill(Wg, s, emb, valid)
     K1, V1 = oracle.prefill(Wgq, s, emb, valid)
     assert np.array_equal(K0, K1) and np.array_equal(V0, V1)
+
+
+def test_expert_preset_scope_and_identity_on_grid_weights():
+    """The expert preset (reading 29) touches exactly the expert layers' seven
+    matrices; on weights already on their groups' grids (the tiny expert's
+    96-wide inputs have a 32-wide last group) it is the identity, so the
+    quantised model's denoise equals the dense one."""
+    import oracle
+
+    s = synth.SHAPES["tiny"]
+    W = oracle.load_weights(synth.gen_weights(s, 4, random_affine=True))
+    names = set(oq.expert_matrix_names(s.e_layers))
+    assert len(names) == 7 * s.e_layers
+    assert any(W[k].shape[1] % 64 for k in names)  # ragged groups are exercised
+    Wq = oq.quantize_expert(W, s.e_layers)
+    for k in W:
+        if k in names:
+            assert not np.array_equal(Wq[k], W[k])
+        else:
+            assert Wq[k] is W[k]
+    rng = np.random.default_rng(24)
+    Wg = dict(W)
+    for k in names:
+        N, K = W[k].shape
+        if K % 64:
+            Wg[k] = _ragged_grid_matrix(rng, N, K // 64, K % 64)[0].astype(np.float64)
+        else:
+            Wg[k] = _grid_matrix(rng, N, K)[0].astype(np.float64)
+        Wg[k] *= 8.0  # same grids, scales nearer the workloads' weights
+    Wgq = oq.quantize_expert(Wg, s.e_layers)
+    for k in names:
+        assert np.array_equal(Wgq[k], Wg[k])
+    L, H = 6, 5
+    valid = np.array([1, 1, 0, 1, 1, 1], bool)
+    Kc = 0.5 * rng.standard_normal((s.p_layers, L, s.p_kv_width))
+    Vc = 0.5 * rng.standard_normal((s.p_layers, L, s.p_kv_width))
+    noise = rng.standard_normal((H, s.action_dim))
+    x0 = oracle.denoise(Wg, s, Kc, Vc, valid, noise, 3)[2]
+    x1 = oracle.denoise(Wgq, s, Kc, Vc, valid, noise, 3)[2]
+    assert np.array_equal(x0, x1)
 
 
 # ----------------------------------------------------------------------------
@@ -217,7 +338,54 @@ def _dq_f32_scale_code(q, a, b):
     return oq._bf16_rne(v.astype(np.float32)).astype(np.float64).reshape(N, K)
 
 
+def _q_tail_zero_padded(w):
+    """mistake: the ragged last group is padded with zeros to 64 inputs"""
+    w = np.asarray(w, np.float32)
+    N, K = w.shape
+    pad = (-K) % 64
+    q, a, b = oq.quantize_affine8(np.concatenate([w, np.zeros((N, pad), np.float32)], axis=1))
+    return q[:, :K], a, b
+
+
+def _q_tail_merged(w):
+    """mistake: the ragged tail joins the group before it (one (64 + r)-wide group)"""
+    w = np.asarray(w, np.float32)
+    N, K = w.shape
+    q, a, b = oq.quantize_affine8(w)
+    r = K % 64
+    if r == 0 or K < 64 + r:
+        return q, a, b
+    k0 = K - 64 - r
+    qm, am, bm = oq.quantize_affine8(w[:, k0:])  # 64 + r wide: groups [0, 64) and the tail
+    lo, hi = w[:, k0:].min(1), w[:, k0:].max(1)
+    al = oq._bf16_rne((hi - lo) / np.float32(255))
+    safe = np.where(al > 0, al, np.float32(1)).astype(np.float32)
+    qq = np.clip(np.rint((w[:, k0:] - lo[:, None]) / safe[:, None]), 0, 255).astype(np.uint8)
+    q[:, k0:] = qq
+    a[:, -2:] = al[:, None]
+    b[:, -2:] = lo[:, None]
+    return q, a, b
+
+
+def _q_tail_previous_scale(w):
+    """mistake: the tail is coded on the previous group's scale and offset"""
+    w = np.asarray(w, np.float32)
+    N, K = w.shape
+    q, a, b = oq.quantize_affine8(w)
+    if K % 64 == 0 or K < 64:
+        return q, a, b
+    k0 = K - K % 64
+    al, be = a[:, -2], b[:, -2]
+    safe = np.where(al > 0, al, np.float32(1)).astype(np.float32)
+    q[:, k0:] = np.clip(np.rint((w[:, k0:] - be[:, None]) / safe[:, None]), 0, 255).astype(np.uint8)
+    a[:, -1], b[:, -1] = al, be
+    return q, a, b
+
+
 MUTANTS = {
+    "tail_zero_padded": (_q_tail_zero_padded, oq.dequantize_affine8),
+    "tail_merged_with_previous": (_q_tail_merged, oq.dequantize_affine8),
+    "tail_on_previous_scale": (_q_tail_previous_scale, oq.dequantize_affine8),
     "floor_rounding": (_q_floor, oq.dequantize_affine8),
     "256_levels": (_q_256, oq.dequantize_affine8),
     "groups_along_outputs": (_q_columns, oq.dequantize_affine8),
@@ -234,6 +402,6 @@ def test_pins_catch_planted_quant_mistake(name):
     for pin in PINS:
         try:
             pin(qf, dqf)
-        except AssertionError:
+        except Exception:  # a wrong value, or a mutant that cannot take a ragged row
             failed += 1
     assert failed >= 1, f"no pin caught the planted mistake {name}"
