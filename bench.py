@@ -356,14 +356,15 @@ def reference_arm(args, rank):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
-def gpu_setup(wl_name, dev, B=None, prefix_int8=False, hash_blob=False):
+def gpu_setup(wl_name, dev, B=None, prefix_int8=False, hash_blob=False, expert_int8=False):
     import torch
     from vision_language_action_b200.runtime import SmolVLA
     wl = synth.WORKLOADS[wl_name]
     s = wl.model
     B = wl.B if B is None else B
     blob = synth.pack_blob(s, synth.gen_weights(s, wl.seed))
-    m = SmolVLA(s, blob, max_batch=B, max_prefix=wl.L, max_chunk=wl.H, device=dev, prefix_int8=prefix_int8)
+    m = SmolVLA(s, blob, max_batch=B, max_prefix=wl.L, max_chunk=wl.H, device=dev, prefix_int8=prefix_int8,
+                expert_int8=expert_int8)
     m.blob_sha256 = hashlib.sha256(blob.tobytes()).hexdigest() if hash_blob else None
     del blob
     inp = synth.gen_inputs(wl, B=B)

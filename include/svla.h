@@ -115,6 +115,18 @@ SVLA_API svla_status svla_create(const svla_config* cfg, const void* blob, size_
  *     for max_batch x max_chunk rows (every expert layer's activations are
  *     kept for the backward: about 0.55 MB per row at the SmolVLA shape). */
 #define SVLA_CREATE_TRAIN 2u
+/*   SVLA_CREATE_EXPERT_INT8  also build the weight-only int8 copy of the action
+ *     expert's projections and select it for svla_denoise / svla_sample (the
+ *     same scheme as SVLA_CREATE_PREFIX_INT8, on W_q, W_k, W_v, W_o, W_g, W_u,
+ *     W_d of every expert layer, the odd layers' cross W_k / W_v included; the
+ *     expert's 720-wide inputs are not a multiple of 64, so the last group of a
+ *     row holds its K mod 64 remaining inputs). The heads (action_in, the time
+ *     MLP, action_out) and the norm gains stay bf16; the dense weights stay
+ *     resident, so svla_set_expert_weights can switch back. Both denoise paths
+ *     read the codes: the persistent kernel dequantises each weight slice in
+ *     shared memory, the multi-kernel path uses the int8 GEMM (few tiles) or a
+ *     per-matrix dequantisation before the dense GEMM (many tiles). */
+#define SVLA_CREATE_EXPERT_INT8 4u
 SVLA_API svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob_bytes,
                            int device, unsigned flags, svla_handle** out);
 
@@ -124,6 +136,14 @@ SVLA_API svla_status svla_create_ex(const svla_config* cfg, const void* blob, si
 SVLA_API svla_status svla_set_prefix_weights(svla_handle* h, int bits);
 /* The prefix weight width svla_prefill uses (16 or 8); 0 for a NULL handle. */
 SVLA_API int svla_prefix_weights(const svla_handle* h);
+
+/* Expert weights svla_denoise, svla_denoise_prefix and svla_sample use from
+ * the next call on: 16 = dense bf16 (default), 8 = the int8 copy
+ * (SVLA_ERR_UNSUPPORTED unless the handle was created with
+ * SVLA_CREATE_EXPERT_INT8). Other values: SVLA_ERR_ARG. */
+SVLA_API svla_status svla_set_expert_weights(svla_handle* h, int bits);
+/* The expert weight width the denoise uses (16 or 8); 0 for a NULL handle. */
+SVLA_API int svla_expert_weights(const svla_handle* h);
 
 /* Training step of the action expert ("noeira docs, SmolVLA" §Architecture,
  * the fine-tune's flow-matching objective; §Fine-tuning: the 16 expert layers
@@ -324,11 +344,15 @@ SVLA_API svla_status svla_op_attention(const void* q, int ldq, const void* k, co
                               const uint8_t* key_valid, int B, int n_q, int n_kv, int hd,
                               int Lq, int Lk, int causal, void* out, int ldo, void* stream);
 
-/* The vlm-8bit quantiser (svla_create_ex, SVLA_CREATE_PREFIX_INT8) on one matrix.
+/* The int8 quantiser of the vlm-8bit and expert presets (svla_create_ex,
+ * SVLA_CREATE_PREFIX_INT8 / SVLA_CREATE_EXPERT_INT8) on one matrix: groups of
+ * 64 consecutive inputs of a row, the last group holding the K mod 64
+ * remaining inputs where K % 64 != 0 (mlx-smolvla PyPI page, §Run a checkpoint,
+ * for the scheme's name; the group rules are this library's readings).
  *   W:  device bf16 [N, K], row stride ldw >= K elements (even), 4-byte aligned.
  *   q:  device uint8 [N, K] codes, row stride ldq >= K bytes (even).
- *   ab: device bf16 [K/64][N][2]: (alpha, beta) of row n, group g at (g, n).
- *   K % 64 == 0, N >= 1; weights must be finite. Asynchronous on `stream`. */
+ *   ab: device bf16 [G][N][2], G = ceil(K/64): (alpha, beta) of row n, group g at (g, n).
+ *   K % 16 == 0, N >= 1; weights must be finite. Asynchronous on `stream`. */
 SVLA_API svla_status svla_op_quantize_affine8(const void* W, int ldw, int N, int K, void* q, int ldq,
                                      void* ab, void* stream);
 
@@ -338,7 +362,7 @@ SVLA_API svla_status svla_op_quantize_affine8(const void* W, int ldw, int N, int
  *   A: device bf16, row stride lda >= K (multiple of 8), 16-byte aligned.
  *   q, ab: as written by svla_op_quantize_affine8 (ldq a multiple of 16).
  *   gain: NULL (g = 1) or device bf16 [K], 16-byte aligned.
- *   K % 64 == 0, N % 8 == 0. splits: 0 = choose, else 1..8 (cluster split-K;
+ *   K % 16 == 0, N % 8 == 0. splits: 0 = choose, else 1..8 (cluster split-K;
  *   no workspace). status: as svla_op_gemm. */
 SVLA_API svla_status svla_op_gemm_w8(int epilogue, const void* A, int lda, const void* q, int ldq,
                             const void* ab, const void* gain, int M, int N, int K, void* C, int ldc,

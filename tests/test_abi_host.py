@@ -131,24 +131,27 @@ def test_int8_argument_checks_and_plan():
     blob = np.zeros(16, np.uint16)
     h = ctypes.c_void_p()
     cfg = config_from_shape(s, 1, 24, 8)
-    assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, 4,
+    assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, 8,
                               ctypes.byref(h)) == _abi.SVLA_ERR_ARG
     cfg = config_from_shape(s.replace(p_heads=3, p_kv_heads=1), 1, 24, 8)  # O projection K = 96
     assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0,
                               _abi.CREATE_PREFIX_INT8, ctypes.byref(h)) == _abi.SVLA_ERR_SHAPE
     assert lib.svla_set_prefix_weights(None, 8) == _abi.SVLA_ERR_ARG
     assert lib.svla_prefix_weights(None) == 0
-    # quantiser: K a multiple of 64, aligned pointers
-    assert lib.svla_op_quantize_affine8(p, 96, 4, 96, p, 96, p, None) == _abi.SVLA_ERR_SHAPE
+    assert lib.svla_set_expert_weights(None, 8) == _abi.SVLA_ERR_ARG
+    assert lib.svla_expert_weights(None) == 0
+    # quantiser: K a multiple of 16 (a ragged last group of K mod 64 inputs), aligned pointers
+    assert lib.svla_op_quantize_affine8(p, 88, 4, 88, p, 88, p, None) == _abi.SVLA_ERR_SHAPE
+    assert lib.svla_op_quantize_affine8(p, 8, 4, 8, p, 8, p, None) == _abi.SVLA_ERR_SHAPE
     assert lib.svla_op_quantize_affine8(None, 64, 4, 64, p, 64, p, None) == _abi.SVLA_ERR_ARG
     assert lib.svla_op_quantize_affine8(ctypes.c_void_p(18), 64, 4, 64, p, 64, p, None) == _abi.SVLA_ERR_ARG
-    # int8 GEMM: epilogue, K % 64, N % 8, splits <= 8, 16-byte alignment
+    # int8 GEMM: epilogue, K % 16, N % 8, splits <= 8, 16-byte alignment
     args = lambda **kw: dict(dict(epi=0, lda=64, ldq=64, g=None, M=4, N=8, K=64, ldc=8, sp=0), **kw)
     def call(a):
         return lib.svla_op_gemm_w8(a["epi"], p, a["lda"], p, a["ldq"], p, a["g"], a["M"], a["N"], a["K"], p,
                                    a["ldc"], None, a["sp"], None, None)
     assert call(args(epi=9)) == _abi.SVLA_ERR_ARG
-    assert call(args(K=96, lda=96, ldq=96)) == _abi.SVLA_ERR_SHAPE
+    assert call(args(K=40, lda=40, ldq=48)) == _abi.SVLA_ERR_SHAPE
     assert call(args(N=12, ldc=12)) == _abi.SVLA_ERR_SHAPE
     assert call(args(sp=9)) == _abi.SVLA_ERR_SHAPE
     assert call(args(ldq=72)) == _abi.SVLA_ERR_SHAPE
@@ -158,6 +161,10 @@ def test_int8_argument_checks_and_plan():
     for (M, N, K) in [(177, 1600, 960), (177, 960, 960), (177, 5120, 960), (177, 960, 2560), (354, 960, 2560)]:
         assert lib.svla_op_gemm_w8_splits(M, N, K) == lib.svla_op_gemm_splits(M, N, K), (M, N, K)
     assert lib.svla_op_gemm_w8_splits(5664, 5120, 960) == 1
+    # ragged K (the expert's 720 = 11 x 64 + 16) plans like any other width
+    assert lib.svla_op_gemm_w8_splits(1600, 4096, 720) == 1
+    assert lib.svla_op_gemm_w8_splits(50, 1600, 720) >= 1
+    assert lib.svla_op_gemm_w8_splits(50, 1600, 40) == 0
     assert lib.svla_op_gemm_w8_tile_n(5664, 5120, 960) == 128
     assert lib.svla_op_gemm_w8_splits(177, 1600, 100) == 0
 
@@ -172,7 +179,7 @@ def test_train_argument_checks():
     h = ctypes.c_void_p()
     cfg = config_from_shape(s, 1, 24, 8)
     # unknown flag bits are rejected before the blob size
-    assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, 4,
+    assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, 8,
                               ctypes.byref(h)) == _abi.SVLA_ERR_ARG
     assert lib.svla_create_ex(ctypes.byref(cfg), ctypes.c_void_p(blob.ctypes.data), 32, 0, _abi.CREATE_TRAIN,
                               ctypes.byref(h)) == _abi.SVLA_ERR_BLOB_SIZE

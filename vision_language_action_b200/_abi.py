@@ -40,6 +40,8 @@ SIGNATURES = {
     "svla_create_ex": (_I, [ctypes.POINTER(SvlaConfig), _P, _S, _I, ctypes.c_uint, ctypes.POINTER(_P)]),
     "svla_set_prefix_weights": (_I, [_P, _I]),
     "svla_prefix_weights": (_I, [_P]),
+    "svla_set_expert_weights": (_I, [_P, _I]),
+    "svla_expert_weights": (_I, [_P]),
     "svla_train_step": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _I, _P, _P, _P]),
     "svla_train_grad_elems": (_S, [_P]),
     "svla_destroy": (_I, [_P]),
@@ -73,6 +75,7 @@ SIGNATURES = {
 DENOISE_AUTO, DENOISE_GRAPH, DENOISE_FUSED = 0, 1, 2
 CREATE_PREFIX_INT8 = 1
 CREATE_TRAIN = 2
+CREATE_EXPERT_INT8 = 4
 
 _lib = None
 

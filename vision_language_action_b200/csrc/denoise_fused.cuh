@@ -45,9 +45,17 @@
 // time-out the CTA records SVLA_ERR_TIMEOUT, raises the abort word, drains its
 // bulk copies and returns; the other CTAs see the abort word at their next
 // barrier.
+//
+// Weight-only int8 expert (the vlm-8bit scheme applied to the expert): a job's
+// weight rows arrive as int8 codes with their (alpha, beta) pairs, half the
+// bytes, and the CTA dequantises them in shared memory into the bf16 rows the
+// products read, w = bf16(bf16(alpha q + beta) * g) with the RMSNorm gain g
+// (the operand the dense path folds); this runs while the activation operand
+// is still in flight after the barrier.
 #pragma once
 
 #include "attention.cuh"
+#include "gemm_w8.cuh"
 
 namespace svla {
 
@@ -85,7 +93,14 @@ struct FdLayer {
   const bf16* w_d;    // [E, ffn + 8]
   const bf16* kx;     // odd: hoisted K' [B * L, nkv * hd]
   const bf16* vx;     // odd: hoisted V'
+  // int8 expert (null: the bf16 weights above): the same rows as K codes
+  // followed by ceil(K/64) (alpha, beta) bf16 pairs, row pitch fd_q8_pitch(K)
+  const uint8_t *q_qkv, *q_o, *q_gu, *q_d;
+  const bf16 *g_in, *g_post;  // RMSNorm gains applied to the dequantised QKV / gate-up rows
 };
+
+// row pitch (bytes) of an int8 weight row: K codes, ceil(K/64) pairs, 16-byte multiple
+__host__ __device__ inline int fd_q8_pitch(int K) { return (K + 4 * w8_groups(K) + 15) / 16 * 16; }
 
 struct FdArgs {
   int B, H, L, M, E, A, hd, nq, nkv, ffn, n_steps, n_layers;
@@ -112,6 +127,7 @@ struct FdArgs {
   int* status;
   unsigned long long wait_ns;
   int slot_bytes;             // bytes of one weight slot
+  int stage_bytes;            // int8 expert: bytes of the dequantised (bf16) job weights; else 0
   int a_bytes;                // bytes of the activation / attention region
 };
 
@@ -122,8 +138,10 @@ struct FdGemm {
   int epi;
   FdAct A;
   int K;
-  const bf16* W;   // row pitch K + 8
-  int w;           // W rows per job (two runs of w / 2)
+  const bf16* W;       // row pitch K + 8
+  const uint8_t* Q;    // int8 rows (row pitch fd_q8_pitch(K)) instead of W, or null
+  const bf16* gain;    // with Q: the gain applied at dequantisation, or null
+  int w;               // W rows per job (two runs of w / 2)
   int n_jobs;
   bool norm;
   int layer;
@@ -141,6 +159,8 @@ SVLA_DEV FdGemm fd_gemm(const FdArgs& p, int g) {
   FdGemm s;
   s.norm = false;
   s.layer = -1;
+  s.Q = nullptr;
+  s.gain = nullptr;
   s.K = p.E;
   s.w = 8;
   s.n_jobs = p.E / 8;
@@ -156,19 +176,21 @@ SVLA_DEV FdGemm fd_gemm(const FdArgs& p, int g) {
   const FdLayer& L = fd_layers[l];
   s.layer = l;
   if (sub == 0) {
-    s.A = p.rb; s.W = L.w_qkv; s.norm = true;
+    s.A = p.rb; s.W = L.w_qkv; s.Q = L.q_qkv; s.gain = L.g_in; s.norm = true;
     if (l % 2 == 0) {
       s.epi = FD_QKV_ROPE; s.w = 16; s.n_jobs = (p.nq + 2 * p.nkv) * (p.hd / 16);
     } else {
       s.epi = FD_Q; s.n_jobs = p.nq * p.hd / 8;
     }
   } else if (sub == 1) {
-    s.epi = FD_RES_ADD; s.A = p.o; s.K = p.nq * p.hd; s.W = L.w_o;
+    s.epi = FD_RES_ADD; s.A = p.o; s.K = p.nq * p.hd; s.W = L.w_o; s.Q = L.q_o;
   } else if (sub == 2) {
-    s.epi = FD_SWIGLU; s.A = p.rb; s.W = L.w_gu; s.w = 32; s.n_jobs = p.ffn / 16; s.norm = true;
+    s.epi = FD_SWIGLU; s.A = p.rb; s.W = L.w_gu; s.Q = L.q_gu; s.gain = L.g_post; s.w = 32; s.n_jobs = p.ffn / 16;
+    s.norm = true;
   } else {
-    s.epi = FD_RES_ADD; s.A = p.hh; s.K = p.ffn; s.W = L.w_d;
+    s.epi = FD_RES_ADD; s.A = p.hh; s.K = p.ffn; s.W = L.w_d; s.Q = L.q_d;
   }
+  if (!s.Q) s.gain = nullptr;  // dense weights carry their gains folded in
   return s;
 }
 
@@ -222,13 +244,18 @@ SVLA_DEV void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
 // abandoned (abort word raised, or this wait ran out of time). Every thread
 // first orders its global stores before the bulk copies that other CTAs issue
 // after the barrier.
-SVLA_DEV bool fd_grid_sync(const FdArgs& p, unsigned idx, int* flag) {
+// `during` runs on every thread between this CTA's arrival and its wait (work
+// that touches only this CTA's shared memory, hidden behind the barrier's
+// latency).
+template <typename During>
+SVLA_DEV bool fd_grid_sync(const FdArgs& p, unsigned idx, int* flag, During&& during) {
   fence_proxy_async_global();
   __syncthreads();
+  // release: this CTA's writes (ordered before this thread by the barrier above)
+  if (threadIdx.x == 0) red_release_add(p.sync, 1u);
+  during();
   if (threadIdx.x == 0) {
     int ok = 1;
-    // release: this CTA's writes (ordered before this thread by the barrier above)
-    red_release_add(p.sync, 1u);
     const unsigned target = (idx + 1) * gridDim.x;
     uint64_t t0 = 0;
     for (uint32_t i = 1;; ++i) {
@@ -261,6 +288,8 @@ struct FdPipe {
   int issued, consumed;    // weight slices issued / consumed so far (slot = count % 2)
   int total_g;
   int a_iss[2], a_use[2];  // activation-buffer copies issued / waited for (mbarrier parity)
+  int slot_g[2];           // GEMM stage of the slice issued into each slot
+  int pre;                 // int8: the stage buffer already holds the next job's dequantised weights
 };
 
 // advance (g, j) to this CTA's next job at or after it
@@ -282,12 +311,21 @@ SVLA_DEV void fd_issue(const FdArgs& p, FdPipe& pp, uint8_t* slots, uint32_t bar
   fd_job_rows(p, s, pp.next_j, r0, r1);
   const int slot = pp.issued & 1;
   const uint32_t bar = bar_base + 8 * slot;
-  const uint32_t pitch = (uint32_t)(s.K + 8), run_bytes = (uint32_t)(s.w / 2) * pitch * 2;
   const uint32_t dst = smem_u32(slots + (size_t)slot * p.slot_bytes);
+  pp.slot_g[slot] = pp.next_g;
   fence_proxy_async_smem();  // generic-proxy reads of this slot are ordered before the async writes
-  mbar_arrive_expect_tx(bar, 2 * run_bytes);
-  bulk_load(dst, s.W + (size_t)r0 * pitch, run_bytes, bar);
-  bulk_load(dst + run_bytes, s.W + (size_t)r1 * pitch, run_bytes, bar);
+  if (s.Q) {
+    // int8 rows: pitch fd_q8_pitch(K) bytes (a 16-byte multiple)
+    const uint32_t pitch = (uint32_t)fd_q8_pitch(s.K), run_bytes = (uint32_t)(s.w / 2) * pitch;
+    mbar_arrive_expect_tx(bar, 2 * run_bytes);
+    bulk_load(dst, s.Q + (size_t)r0 * pitch, run_bytes, bar);
+    bulk_load(dst + run_bytes, s.Q + (size_t)r1 * pitch, run_bytes, bar);
+  } else {
+    const uint32_t pitch = (uint32_t)(s.K + 8), run_bytes = (uint32_t)(s.w / 2) * pitch * 2;
+    mbar_arrive_expect_tx(bar, 2 * run_bytes);
+    bulk_load(dst, s.W + (size_t)r0 * pitch, run_bytes, bar);
+    bulk_load(dst + run_bytes, s.W + (size_t)r1 * pitch, run_bytes, bar);
+  }
   ++pp.issued;
   pp.next_j += gridDim.x;
   fd_next_job(p, pp.next_g, pp.next_j, pp.total_g);
@@ -350,18 +388,78 @@ SVLA_DEV void fd_mma_plane(const bf16* ab, int apitch, const uint8_t* wsl, int w
 }
 
 // ---------------------------------------------------------------------------
+// int8 job weights: `rows` staged rows of K codes + ceil(K/64) (alpha, beta)
+// pairs (pitch fd_q8_pitch(K)) -> bf16 rows with pitch K + 8, the layout the
+// products read: w = bf16(bf16(alpha q + beta) * g[k]) (g = 1 without a gain).
+// One item = 16 codes of one row (K % 16 == 0); all FD_THREADS threads.
+// ---------------------------------------------------------------------------
+SVLA_DEV void fd_dequant(const uint8_t* src, int K, int rows, const bf16* gain, bf16* dst) {
+  const int pitch = fd_q8_pitch(K), cpr = K / 16;
+  for (int i = threadIdx.x; i < rows * cpr; i += FD_THREADS) {
+    const int r = i / cpr, k = (i - r * cpr) * 16;
+    const uint8_t* row = src + (size_t)r * pitch;
+    const uint4 qv = *reinterpret_cast<const uint4*>(row + k);
+    const uint32_t pr = *reinterpret_cast<const uint32_t*>(row + K + 4 * (k / W8_GROUP));
+    uint4 g0 = make_uint4(0u, 0u, 0u, 0u), g1 = g0;
+    if (gain) {
+      const uint4* gp = reinterpret_cast<const uint4*>(gain + k);
+      g0 = __ldg(gp);
+      g1 = __ldg(gp + 1);
+    }
+    const uint32_t g2[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    uint32_t o[8];
+    dequant16(qv, bf2f((uint16_t)(pr & 0xFFFFu)), bf2f((uint16_t)(pr >> 16)), g2, gain != nullptr, o);
+    uint4* d = reinterpret_cast<uint4*>(dst + (size_t)r * (K + 8) + k);
+    d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// Inside a grid barrier: if the next job this CTA consumes has int8 weights
+// that are not staged yet, wait (bounded) for its slot, dequantise it into the
+// stage buffer and hand the slot back to the weight stream, so the job starts
+// with its operand ready. All threads; a time-out raises the abort word (the
+// barrier's own wait then gives up).
+SVLA_DEV void fd_prestage(const FdArgs& p, FdPipe& pp, uint8_t* slots, bf16* stage, uint32_t bar_base, int* flag) {
+  if (pp.pre || pp.consumed >= pp.issued) return;
+  const int slot = pp.consumed & 1;
+  const FdGemm s = fd_gemm(p, pp.slot_g[slot]);
+  if (!s.Q) return;
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(bar_base + 8 * slot, (uint32_t)((pp.consumed >> 1) & 1), p.wait_ns);
+    if (!ok) {
+      set_status(p.status, SVLA_ERR_TIMEOUT);
+      atomicExch(p.sync + 1, 1u);
+    }
+    *flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  if (*flag == 0) return;
+  fd_dequant(slots + (size_t)slot * p.slot_bytes, s.K, s.w, s.gain, stage);
+  fence_proxy_async_smem();  // this thread's generic reads of the slot before its async re-fill
+  __syncthreads();
+  if (threadIdx.x == FD_PIPE_TID) {
+    pp.pre = 1;
+    ++pp.consumed;
+    fd_issue(p, pp, slots, bar_base);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // GEMM job: the M rows of A times the w staged W rows over the full K, fp32
 // accumulate, fused epilogue. A arrives plane by plane (one bulk copy each,
-// two buffers); all FD_THREADS threads take part.
+// two buffers); all FD_THREADS threads take part. With int8 weights the slot
+// is dequantised into `stage` first and handed back to the weight stream.
 // ---------------------------------------------------------------------------
 template <int HD>
 SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, uint8_t* slots, uint32_t bar_base,
-                          bf16* abuf, float* red, float* rscale, int* flag) {
+                          bf16* abuf, bf16* stage, float* red, float* rscale, int* flag) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int M = p.M, K = s.K, P = s.A.P, Kp = K / P, apitch = Kp + 8;
   const uint32_t plane_bytes = (uint32_t)M * apitch * 2;
   const uint32_t abar = bar_base + 16;  // activation buffers' mbarriers: abar, abar + 8
   const int slot = pp.consumed & 1;
+  const bool q8 = s.Q != nullptr;
   const uint8_t* wsl = slots + (size_t)slot * p.slot_bytes;
   const int wld = K + 8;  // staged W row (elements)
 
@@ -403,6 +501,35 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, u
     }
   }
 
+  if (q8) {
+    const bool staged = pp.pre != 0;  // dequantised during the last grid barrier
+    if (!staged) {
+      // the int8 slot (issued two jobs ago, normally landed): dequantise it
+      // while the activation planes are in flight, then hand the slot back
+      if (tid == 0) {
+        const bool ok = mbar_wait(bar_base + 8 * slot, (uint32_t)((pp.consumed >> 1) & 1), p.wait_ns);
+        if (!ok) {
+          set_status(p.status, SVLA_ERR_TIMEOUT);
+          atomicExch(p.sync + 1, 1u);
+        }
+        *flag = ok ? 1 : 0;
+      }
+      __syncthreads();
+      if (*flag == 0) return false;
+      fd_dequant(wsl, K, s.w, s.gain, stage);
+      fence_proxy_async_smem();  // this thread's generic reads of the slot before its async re-fill
+      __syncthreads();
+      if (tid == FD_PIPE_TID) {
+        ++pp.consumed;
+        fd_issue(p, pp, slots, bar_base);
+      }
+    } else {
+      __syncthreads();  // every thread has read pp.pre
+      if (tid == FD_PIPE_TID) pp.pre = 0;
+    }
+    wsl = reinterpret_cast<const uint8_t*>(stage);
+  }
+
   const int nt_n = s.w / 8;
   float acc2[2][4][4];
 #pragma unroll
@@ -415,7 +542,7 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, u
     const int buf = q & 1;
     if (tid == 0) {
       bool ok = true;
-      if (q == 0) ok = mbar_wait(bar_base + 8 * slot, (uint32_t)((pp.consumed >> 1) & 1), p.wait_ns);
+      if (q == 0 && !q8) ok = mbar_wait(bar_base + 8 * slot, (uint32_t)((pp.consumed >> 1) & 1), p.wait_ns);
       ok = ok && mbar_wait(abar + 8 * buf, (uint32_t)(pp.a_use[buf] & 1), p.wait_ns);
       if (ok) ++pp.a_use[buf];
       if (!ok) {
@@ -465,7 +592,7 @@ SVLA_DEV bool fd_gemm_job(const FdArgs& p, const FdGemm& s, int j, FdPipe& pp, u
     }
   }
   __syncthreads();
-  if (tid == FD_PIPE_TID) {
+  if (tid == FD_PIPE_TID && !q8) {
     // the weight slot is free: a thread of warp 4 (idle in the epilogue)
     // hands it the job after next
     ++pp.consumed;
@@ -950,7 +1077,8 @@ template <int HD>
 __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __grid_constant__ FdArgs p) {
   extern __shared__ __align__(1024) uint8_t fd_smem[];
   uint8_t* slots = fd_smem;                                         // 2 weight slots
-  uint8_t* ubuf = slots + 2 * (size_t)p.slot_bytes;                 // activation planes / attention
+  bf16* stage = reinterpret_cast<bf16*>(slots + 2 * (size_t)p.slot_bytes);  // int8: dequantised job weights
+  uint8_t* ubuf = slots + 2 * (size_t)p.slot_bytes + p.stage_bytes;  // activation planes / attention
   float* red = reinterpret_cast<float*>(ubuf + p.a_bytes);          // [4 m-tiles][4 n-tiles][4][32]
   float* rscale = red + 4 * 4 * 4 * 32;                             // [64]
   float* fbuf = rscale + FD_MAX_M;                                  // [E + 64 + 8] row stage
@@ -969,6 +1097,8 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
     pp.next_g = 0;
     pp.next_j = blockIdx.x;
     pp.issued = pp.consumed = 0;
+    pp.slot_g[0] = pp.slot_g[1] = 0;
+    pp.pre = 0;
     fd_next_job(p, pp.next_g, pp.next_j, pp.total_g);
     fd_issue(p, pp, slots, bar_base);
     fd_issue(p, pp, slots, bar_base);
@@ -977,9 +1107,10 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
 
   unsigned nbar = 0;
   bool alive = true;
+  auto prestage = [&] { fd_prestage(p, pp, slots, stage, bar_base, &flag); };
   alive = fd_row_stage(p, -1, 0, fbuf, ubuf, pp, bar_base, &flag);
   fd_time_c(p, 0, blockIdx.x, gridDim.x, fbuf);
-  if (alive) alive = fd_grid_sync(p, nbar++, &flag);
+  if (alive) alive = fd_grid_sync(p, nbar++, &flag, prestage);
   const int gps = fd_gemms_per_step(p);
   for (int k = 0; k < p.n_steps && alive; ++k) {
     for (int gi = 0; gi < gps && alive; ++gi) {
@@ -1004,9 +1135,10 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
         prefetch_l2_bulk(p.w_in, (uint32_t)p.A * p.E * 2);
       }
       for (int j = blockIdx.x; j < s.n_jobs && alive; j += gridDim.x)
-        alive = fd_gemm_job<HD>(p, s, j, pp, slots, bar_base, reinterpret_cast<bf16*>(ubuf), red, rscale, &flag);
+        alive = fd_gemm_job<HD>(p, s, j, pp, slots, bar_base, reinterpret_cast<bf16*>(ubuf), stage, red, rscale,
+                                &flag);
       if (!alive) break;
-      alive = fd_grid_sync(p, nbar++, &flag);
+      alive = fd_grid_sync(p, nbar++, &flag, prestage);
       if (!alive) break;
       if (s.layer >= 0 && (gi - 2) % 4 == 0) {
         // attention of this layer (after its QKV stage)
@@ -1043,12 +1175,12 @@ __global__ void __launch_bounds__(FD_THREADS, 1) denoise_fused_kernel(const __gr
           else
             fd_time_c(p, k + 1, (int)blockIdx.x, G, fbuf);
         }
-        alive = fd_grid_sync(p, nbar++, &flag);
+        alive = fd_grid_sync(p, nbar++, &flag, prestage);
       }
     }
     if (!alive) break;
     alive = fd_row_stage(p, k, k + 1, fbuf, ubuf, pp, bar_base, &flag);
-    if (alive && k + 1 < p.n_steps) alive = fd_grid_sync(p, nbar++, &flag);
+    if (alive && k + 1 < p.n_steps) alive = fd_grid_sync(p, nbar++, &flag, prestage);
   }
   // drain: wait (bounded) for this CTA's bulk copies still in flight
   if (threadIdx.x == 0) {

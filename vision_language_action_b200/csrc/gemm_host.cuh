@@ -405,7 +405,7 @@ inline bool w8_many_tiles(int M, int N) {
 
 inline GemmPlan plan_gemm_w8(int M, int N, int K, int forced_splits, int min_bn = 32) {
   GemmPlan p;
-  const int KB = K / GEMM_BK;
+  const int KB = (K + GEMM_BK - 1) / GEMM_BK;
   p.m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
   auto tiles = [&](int bn) { return p.m_tiles * ((N + bn - 1) / bn); };
   auto clamp_splits = [&](int sp) {
@@ -500,15 +500,15 @@ inline cudaError_t set_attrs_w8() {
 }
 
 // Full launch of the int8 GEMM. Q: codes [N, K] (row stride ldq bytes); ab:
-// (alpha, beta) pairs [K/64][N][2]; gain: bf16 [K] or null. K % 64 == 0 and
-// N % 4 == 0 (TMA strides), checked by the callers.
+// (alpha, beta) pairs [ceil(K/64)][N][2]; gain: bf16 [K] or null. K % 16 == 0
+// and N % 4 == 0 (TMA strides), checked by the callers.
 inline cudaError_t run_gemm_w8(int epi, const void* A, int lda, const uint8_t* Q, size_t ldq, const uint16_t* ab,
                                const uint16_t* gain, int M, int N, int K, GemmArgs args, const GemmPlan& p,
                                cudaStream_t s) {
   CUtensorMap ta, tq, ts;
   if (!make_tmap_bf16(&ta, A, M, K, lda, GEMM_BM)) return cudaErrorInvalidValue;
   if (!make_tmap_u8(&tq, Q, N, K, ldq, p.bn)) return cudaErrorInvalidValue;
-  if (!make_tmap_pairs(&ts, ab, N, K / W8_GROUP, p.bn)) return cudaErrorInvalidValue;
+  if (!make_tmap_pairs(&ts, ab, N, (K + W8_GROUP - 1) / W8_GROUP, p.bn)) return cudaErrorInvalidValue;
   args.M = M;
   args.N = N;
   args.K = K;

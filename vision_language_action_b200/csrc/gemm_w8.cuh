@@ -1,19 +1,21 @@
 // Weight-only int8 GEMM on the tcgen05 tensor cores, and the quantiser that
 // produces its weights (the vlm-8bit preset of the mlx-smolvla PyPI page,
-// §Run a checkpoint: the prefix LM's projections in 8 bits, activations bf16).
+// §Run a checkpoint: the prefix LM's projections in 8 bits, activations bf16;
+// the same scheme serves the action expert's projections).
 //
 //   C[M, N] = A[M, K] · W^[N, K]^T,   W^[n, k] = bf16(bf16(alpha q + beta) * g[k])
 //
 // Quantisation: affine groups of 64 consecutive input weights of one output
-// row; per group lo = min, hi = max, alpha = bf16((hi - lo) / 255), beta = lo,
+// row (where K % 64 != 0, the row's last group holds its K mod 64 remaining
+// inputs; that group is the kernel's last, partly zero-filled, k-block); per group lo = min, hi = max, alpha = bf16((hi - lo) / 255), beta = lo,
 // code q = clamp(rint((w - beta) / alpha), 0, 255), every step an IEEE fp32
 // operation rounded to nearest even. g is the RMSNorm gain folded into a
 // projection that consumes normalised activations (1 where there is none), so
 // the operand equals the dense path's folded weight computed from W^.
 //
 // Storage: codes uint8 [N, K] row-major; (alpha, beta) as bf16 pairs in a
-// group-major array [K/64][N][2], so the pairs of one k-block of a tile are
-// one contiguous TMA box.
+// group-major array [ceil(K/64)][N][2], so the pairs of one k-block of a tile
+// are one contiguous TMA box.
 //
 // CTA (same roles as the dense kernel, one more stage of work):
 //   warp 0      : TMA producer: A (bf16, 128-byte swizzle), the int8 code tile
@@ -35,6 +37,8 @@
 namespace svla {
 
 constexpr int W8_GROUP = 64;  // = GEMM_BK: one (alpha, beta) pair per row and k-block
+// groups of a K-wide row (the last one narrower where K % 64 != 0)
+__host__ __device__ inline int w8_groups(int K) { return (K + W8_GROUP - 1) / W8_GROUP; }
 
 template <int BN, int STAGES_>
 struct W8Cfg {
@@ -110,7 +114,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_blk = blockIdx.x, m_blk = blockIdx.y, split = blockIdx.z, splits = gridDim.z;
-  const int KB = args.K / GEMM_BK;
+  const int KB = (args.K + GEMM_BK - 1) / GEMM_BK;  // a ragged last k-block is the row's last (narrower) group
   const int kb0 = (int)(((long long)split * KB) / splits);
   const int kb1 = (int)(((long long)(split + 1) * KB) / splits);
   const int nkb = kb1 - kb0;
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, W8Cfg<BN, STAGES>::MIN_BLOCKS)
       const int k0 = (kb0 + i) * GEMM_BK;
       // the gain does not depend on the stage's data: load it before waiting
       uint4 g0 = make_uint4(0u, 0u, 0u, 0u), g1 = g0;
-      if (gain) {
+      if (gain && k0 + 16 * c < args.K) {  // K % 16 == 0: a chunk is wholly inside or past K
         const uint4* gp = reinterpret_cast<const uint4*>(gain + k0 + 16 * c);
         g0 = __ldg(gp);
         g1 = __ldg(gp + 1);
@@ -347,18 +351,27 @@ __global__ void __launch_bounds__(256) dequant_affine8_kernel(const uint8_t* __r
 
 // One warp per (row n, group g): lanes hold inputs 2 lane, 2 lane + 1 of the group.
 //   W: bf16 [N, K] (row stride ldw, even); q: uint8 [N, K] (row stride ldq);
-//   ab: bf16 pairs [K/64][N][2].
+//   ab: bf16 pairs [G][N][2], G = ceil(K / 64). K % 16 == 0; where K % 64 != 0
+//   the last group of a row is its K mod 64 remaining inputs (lanes past them
+//   take no part in the minimum and maximum and store nothing).
 __global__ void __launch_bounds__(256) quantize_affine8_kernel(const uint16_t* __restrict__ W, size_t ldw, int N,
                                                                int K, uint8_t* __restrict__ q, size_t ldq,
                                                                uint16_t* __restrict__ ab) {
-  const int G = K / W8_GROUP;
+  const int G = (K + W8_GROUP - 1) / W8_GROUP;
   const long long wid = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (wid >= (long long)N * G) return;  // whole warps exit together
   const int n = (int)(wid / G), g = (int)(wid % G);
-  const uint32_t v = *reinterpret_cast<const uint32_t*>(W + (size_t)n * ldw + (size_t)g * W8_GROUP + 2 * lane);
-  const float w0 = bf2f((uint16_t)(v & 0xFFFFu)), w1 = bf2f((uint16_t)(v >> 16));
-  float lo = fminf(w0, w1), hi = fmaxf(w0, w1);
+  const int width = min(W8_GROUP, K - g * W8_GROUP);
+  const bool mine = 2 * lane < width;  // width is even: a lane holds both inputs or none
+  float w0 = 0.f, w1 = 0.f, lo = INFINITY, hi = -INFINITY;
+  if (mine) {
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(W + (size_t)n * ldw + (size_t)g * W8_GROUP + 2 * lane);
+    w0 = bf2f((uint16_t)(v & 0xFFFFu));
+    w1 = bf2f((uint16_t)(v >> 16));
+    lo = fminf(w0, w1);
+    hi = fmaxf(w0, w1);
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
@@ -370,8 +383,10 @@ __global__ void __launch_bounds__(256) quantize_affine8_kernel(const uint16_t* _
     const float c = rintf(__fdiv_rn(__fsub_rn(w, lo), al));
     return (uint32_t)fminf(fmaxf(c, 0.f), 255.f);
   };
-  const uint32_t c0 = code(w0), c1 = code(w1);
-  *reinterpret_cast<uint16_t*>(q + (size_t)n * ldq + (size_t)g * W8_GROUP + 2 * lane) = (uint16_t)(c0 | (c1 << 8));
+  if (mine) {
+    const uint32_t c0 = code(w0), c1 = code(w1);
+    *reinterpret_cast<uint16_t*>(q + (size_t)n * ldq + (size_t)g * W8_GROUP + 2 * lane) = (uint16_t)(c0 | (c1 << 8));
+  }
   if (lane == 0) {
     const __nv_bfloat16 a = __float2bfloat16_rn(al), b = __float2bfloat16_rn(lo);
     ab[((size_t)g * N + n) * 2] = *reinterpret_cast<const uint16_t*>(&a);

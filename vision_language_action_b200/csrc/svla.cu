@@ -221,12 +221,43 @@ __global__ void pad_rows_kernel(const uint16_t* __restrict__ src, size_t src_ld,
   }
 }
 
-// One int8 prefix projection: codes [N, K] at q_off, (alpha, beta) pairs
-// [K/64][N][2] bf16 at ab_off (byte offsets into the handle's int8 buffer).
+// One int8 projection: codes [N, K] at q_off, (alpha, beta) pairs
+// [ceil(K/64)][N][2] bf16 at ab_off (byte offsets into the handle's int8
+// buffer of the prefix or of the expert).
 struct Q8Mat {
   size_t q_off = 0, ab_off = 0;
   int N = 0, K = 0;
 };
+
+// Row pitch (bytes) of the persistent denoise kernel's int8 weight copy: a row
+// is its K codes followed by its ceil(K/64) (alpha, beta) pairs (bf16 x 2), so
+// a job's rows arrive with one bulk copy per run of rows.
+inline size_t fq_pitch(int K) { return ((size_t)K + 4 * (size_t)w8_groups(K) + 15) / 16 * 16; }
+
+// Byte offsets of that copy (per expert layer: QKV or Q, O, gate/up, down).
+struct FusedQ8 {
+  std::vector<size_t> qkv, o, gu, d;
+  size_t total = 0;
+};
+
+// dst row n = [q[n, 0..K) | (alpha, beta) of row n for g = 0..G)], pitch fq_pitch(K)
+__global__ void pack_fused_q8_kernel(const uint8_t* __restrict__ q, const uint32_t* __restrict__ ab, int N, int K,
+                                     uint8_t* __restrict__ dst, size_t pitch) {
+  const int G = w8_groups(K);
+  const size_t row_words = pitch / 4;
+  const size_t n_words = (size_t)N * row_words;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_words; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t n = i / row_words, w = i % row_words;
+    uint32_t v = 0;
+    if (4 * w < (size_t)K) {
+      v = *reinterpret_cast<const uint32_t*>(q + n * K + 4 * w);
+    } else {
+      const size_t g = w - (size_t)K / 4;
+      if (g < (size_t)G) v = ab[g * N + n];
+    }
+    reinterpret_cast<uint32_t*>(dst + n * pitch)[w] = v;
+  }
+}
 
 // Training workspace (svla_create_ex with SVLA_CREATE_TRAIN), sized by
 // max_batch, max_chunk and max_prefix. Per expert layer the forward keeps the
@@ -290,6 +321,12 @@ struct svla_handle {
   uint16_t* q8_deq = nullptr;  // one dequantised projection (bf16), for many-tile GEMMs
   std::vector<Q8Mat> q8m;    // per prefix layer: QKV, O, gate/up (interleaved rows), down
   int prefix_bits = 16;      // weights svla_prefill uses
+  // weight-only int8 expert (svla_create_ex with SVLA_CREATE_EXPERT_INT8)
+  uint8_t* e8 = nullptr;     // codes and (alpha, beta) pairs of the expert projections
+  std::vector<Q8Mat> e8m;    // per expert layer: QKV (odd: Q), O, gate/up, down, cross K, cross V (odd only)
+  uint8_t* fq = nullptr;     // the persistent kernel's int8 copy (rows of codes and pairs)
+  FusedQ8 fql;
+  int expert_bits = 16;      // weights the denoise uses
   TrainWs* tr = nullptr;     // training workspace (SVLA_CREATE_TRAIN)
   // prefix assembly (svla_set_assembly): connector and state-projection weights, workspaces
   uint16_t* asm_w = nullptr;   // W_c [p_width, r*r*C] | W_s [p_width, S] | b_s [p_width]
@@ -389,12 +426,12 @@ cudaError_t gemm(svla_handle* h, int epi, const bf16* A, int lda, const bf16* W,
 // the matrix is dequantised once into the handle's bf16 buffer and the dense
 // GEMM (its plan, so its partial-sum order) runs on it, launched after the
 // dequantisation completes.
-cudaError_t gemm8(svla_handle* h, int epi, const bf16* A, int lda, const Q8Mat& w, const uint16_t* gain, int M,
-                  GemmArgs args, float* part, int* cnt, cudaStream_t s) {
-  const uint8_t* q = h->q8 + w.q_off;
-  const uint16_t* ab = reinterpret_cast<const uint16_t*>(h->q8 + w.ab_off);
+cudaError_t gemm8(svla_handle* h, int epi, const bf16* A, int lda, const uint8_t* base, const Q8Mat& w,
+                  const uint16_t* gain, int M, GemmArgs args, float* part, int* cnt, cudaStream_t s) {
+  const uint8_t* q = base + w.q_off;
+  const uint16_t* ab = reinterpret_cast<const uint16_t*>(base + w.ab_off);
   if (w8_many_tiles(M, w.N)) {
-    const long long chunks = (long long)w.N * (w.K / 16);
+    const long long chunks = (long long)w.N * (w.K / 16);  // K % 16 == 0
     const unsigned blocks = (unsigned)std::min<long long>((chunks + 255) / 256, 8LL * NUM_SMS_B200);
     const cudaError_t e = launch_pdl(dequant_affine8_kernel, dim3(blocks), dim3(256), 0, s, q, ab, gain, w.N, w.K,
                                      h->q8_deq);
@@ -802,21 +839,21 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
     norm_consumer(qa, h->p_ss, l == 0 ? 1 : d_tiles, M, D, c.rms_eps);
     const bf16* xin = l == 0 ? reinterpret_cast<const bf16*>(embeds) : rb;
     const int qkv_epi = hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32;
-    SVLA_TRY(q8 ? gemm8(h, qkv_epi, xin, D, qm[0], in_gain, M, qa, h->p_part, h->p_cnt, s)
+    SVLA_TRY(q8 ? gemm8(h, qkv_epi, xin, D, h->q8, qm[0], in_gain, M, qa, h->p_part, h->p_cnt, s)
                 : gemm(h, qkv_epi, xin, D, h->W(e[1].off), D, M, qw + 2 * kvw, D, qa, h->p_part, h->p_cnt, s));
     if (l == c.p_layers - 1) break;  // nothing reads the last layer's attention / MLP output
     SVLA_TRY(attention(h->p_q, qw, Kl, Vl, kvw, pad, B, c.p_heads, c.p_kv_heads, hd, L, L, 0, h->p_o, qw, s));
     GemmArgs oa = out_args(h->p_x, D);
     norm_producer(oa, rb, D, h->p_ss, M);
-    SVLA_TRY(q8 ? gemm8(h, GE_ADD_F32, h->p_o, qw, qm[1], nullptr, M, oa, h->p_part, h->p_cnt, s)
+    SVLA_TRY(q8 ? gemm8(h, GE_ADD_F32, h->p_o, qw, h->q8, qm[1], nullptr, M, oa, h->p_part, h->p_cnt, s)
                 : gemm(h, GE_ADD_F32, h->p_o, qw, h->W(e[4].off), qw, M, D, qw, oa, h->p_part, h->p_cnt, s));
     GemmArgs ga = out_args(h->p_h, c.p_ffn);
     norm_consumer(ga, h->p_ss, o_tiles, M, D, c.rms_eps);
-    SVLA_TRY(q8 ? gemm8(h, GE_SWIGLU, rb, D, qm[2], post_gain, M, ga, h->p_part, h->p_cnt, s)
+    SVLA_TRY(q8 ? gemm8(h, GE_SWIGLU, rb, D, h->q8, qm[2], post_gain, M, ga, h->p_part, h->p_cnt, s)
                 : gemm(h, GE_SWIGLU, rb, D, h->W(e[6].off), D, M, 2 * c.p_ffn, D, ga, h->p_part, h->p_cnt, s));
     GemmArgs da = out_args(h->p_x, D);
     norm_producer(da, rb, D, h->p_ss, M);
-    SVLA_TRY(q8 ? gemm8(h, GE_ADD_F32, h->p_h, c.p_ffn, qm[3], nullptr, M, da, h->p_part, h->p_cnt, s)
+    SVLA_TRY(q8 ? gemm8(h, GE_ADD_F32, h->p_h, c.p_ffn, h->q8, qm[3], nullptr, M, da, h->p_part, h->p_cnt, s)
                 : gemm(h, GE_ADD_F32, h->p_h, c.p_ffn, h->W(e[8].off), c.p_ffn, M, D, c.p_ffn, da, h->p_part,
                        h->p_cnt, s));
   }
@@ -830,7 +867,7 @@ cudaError_t record_prefill(svla_handle* h, const void* embeds, const uint8_t* pa
 // fits), the k-half reduction buffer, the row scales, the row-stage vectors
 // and four mbarriers.
 struct FusedPlan {
-  int slot_bytes = 0, a_bytes = 0;
+  int slot_bytes = 0, stage_bytes = 0, a_bytes = 0;
   int p_e = 1, p_o = 1, p_h = 1;  // column planes of the E-, q- and ffn-wide operands
   size_t smem = 0;
 };
@@ -839,14 +876,20 @@ size_t fused_misc_bytes(const svla_config& c) {
   return 4 * 4 * 4 * 32 * sizeof(float) + FD_MAX_M * sizeof(float) + ((size_t)c.e_width + 128) * sizeof(float) + 32;
 }
 
-bool fused_plan(const svla_config& c, int M, int L, FusedPlan* fp) {
+bool fused_plan(const svla_config& c, int M, int L, bool q8, FusedPlan* fp) {
   const int E = c.e_width, qw = c.e_heads * c.head_dim;
   auto sl = [](int w, int K) { return (size_t)w * (K + 8) * 2; };
-  size_t slot = std::max({sl(8, E), sl(16, E), sl(8, qw), sl(32, E), sl(8, c.e_ffn)});
+  auto sl8 = [](int w, int K) { return (size_t)w * fd_q8_pitch(K); };
+  // a job's weight rows: bf16 (time MLP: 8 rows of E; dense layers) or int8
+  // (layers of the int8 expert, dequantised into the stage buffer)
+  const size_t layers_bf16 = std::max({sl(16, E), sl(8, E), sl(8, qw), sl(32, E), sl(8, c.e_ffn)});
+  size_t slot = q8 ? std::max({sl(8, E), sl8(16, E), sl8(8, E), sl8(8, qw), sl8(32, E), sl8(8, c.e_ffn)})
+                   : layers_bf16;
   slot = (slot + 127) / 128 * 128;
+  const size_t stage = q8 ? (layers_bf16 + 127) / 128 * 128 : 0;
   const size_t misc = fused_misc_bytes(c);
-  if (2 * slot + misc > (size_t)FD_SMEM_MAX) return false;
-  const size_t budget = (size_t)FD_SMEM_MAX - 2 * slot - misc;
+  if (2 * slot + stage + misc > (size_t)FD_SMEM_MAX) return false;
+  const size_t budget = (size_t)FD_SMEM_MAX - 2 * slot - stage - misc;
   // the attention jobs (all keys staged) and the row stage's W_out, W_in share the region
   const size_t att = std::max(c.head_dim == 64 ? fd_att_smem<64>(L) : fd_att_smem<32>(L),
                               c.head_dim == 64 ? fd_att_smem<64>(c.max_chunk) : fd_att_smem<32>(c.max_chunk));
@@ -868,8 +911,9 @@ bool fused_plan(const svla_config& c, int M, int L, FusedPlan* fp) {
   FusedPlan f;
   if (!planes(E, &f.p_e) || !planes(qw, &f.p_o) || !planes(c.e_ffn, &f.p_h)) return false;
   f.slot_bytes = (int)slot;
+  f.stage_bytes = (int)stage;
   f.a_bytes = (int)((need + 127) / 128 * 128);
-  f.smem = 2 * slot + f.a_bytes + misc;
+  f.smem = 2 * slot + stage + f.a_bytes + misc;
   if (f.smem > (size_t)FD_SMEM_MAX) return false;
   if (fp) *fp = f;
   return true;
@@ -881,7 +925,9 @@ bool fused_ok(const svla_handle* h, int B, int H, int L) {
   if ((long long)B * H > FD_MAX_M || H > ATT_BQ || H > ATT_BK) return false;
   if (c.e_layers > FD_MAX_LAYERS || c.e_ffn % 32 || c.e_width % 16) return false;
   if (h->num_sms < 1 || !h->fw) return false;
-  return fused_plan(c, B * H, L, nullptr);
+  const bool q8 = h->expert_bits == 8;
+  if (q8 && !h->fq) return false;
+  return fused_plan(c, B * H, L, q8, nullptr);
 }
 
 cudaError_t launch_fused(svla_handle* h, const void* kv, const uint8_t* pad, int B, int L, const float* noise, int H,
@@ -898,7 +944,8 @@ cudaError_t launch_fused(svla_handle* h, const void* kv, const uint8_t* pad, int
   a.dt = -1.0f / (float)n_steps;
   a.noise = noise; a.x = actions; a.trace = trace; a.prefix = d > 0 ? prefix : nullptr; a.d = d; a.pad = pad;
   FusedPlan fp;
-  if (!fused_plan(c, B * H, L, &fp)) return cudaErrorInvalidValue;
+  const bool q8 = h->expert_bits == 8;
+  if (!fused_plan(c, B * H, L, q8, &fp)) return cudaErrorInvalidValue;
   const FusedWeights& F = h->fwl;
   a.w_in = h->W(Lh.w_in.off); a.b_in = h->W(Lh.b_in.off); a.w_t1 = h->W(Lh.w_t1.off);
   a.b_t1 = h->W(Lh.b_t1.off); a.b_t2 = h->b_t2_f32;
@@ -912,6 +959,15 @@ cudaError_t launch_fused(svla_handle* h, const void* kv, const uint8_t* pad, int
     fl.w_o = h->FW(F.o[l]);
     fl.w_gu = h->FW(F.gu[l]);
     fl.w_d = h->FW(F.d[l]);
+    if (q8) {
+      const FusedQ8& Q = h->fql;
+      fl.q_qkv = h->fq + Q.qkv[l];
+      fl.q_o = h->fq + Q.o[l];
+      fl.q_gu = h->fq + Q.gu[l];
+      fl.q_d = h->fq + Q.d[l];
+      fl.g_in = h->W(e[0].off);
+      fl.g_post = h->W(e[5].off);
+    }
     if (l % 2 == 1) {
       fl.kx = h->kvx + (size_t)(l / 2) * 2 * Mp * kvw;
       fl.vx = fl.kx + (size_t)Mp * kvw;
@@ -928,6 +984,7 @@ cudaError_t launch_fused(svla_handle* h, const void* kv, const uint8_t* pad, int
   a.q = h->e_q; a.k = h->e_k; a.v = h->e_v; a.c = h->e_c;
   a.sync = h->fd_sync; a.status = h->status; a.wait_ns = g_wait_ns.load();
   a.slot_bytes = fp.slot_bytes;
+  a.stage_bytes = fp.stage_bytes;
   a.a_bytes = fp.a_bytes;
   const size_t smem = fp.smem;
   SVLA_TRY(cudaMemsetAsync(h->fd_sync, 0, 2 * sizeof(unsigned), s));
@@ -960,7 +1017,18 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
   // GEMMs are independent and each fills only part of the GPU at batch 1: they run as
   // 4 parallel branches of the graph (fork / join events), unless their plan needs the
   // shared split-K workspace (then one after another).
-  const bool par = plan_gemm(Mp, kvw, pkvw, 0, gemm_min_bn(GE_BF16)).red != GEMM_RED_GLOBAL;
+  const bool e8 = h->expert_bits == 8;
+  // one expert projection of layer l (which: 0 QKV / Q, 1 O, 2 gate/up, 3 down,
+  // 4 cross K, 5 cross V): the dense weights (gains folded at create) or the
+  // int8 copy (the gain applied to the dequantised weights)
+  auto eg = [&](int epi, const bf16* A, int lda, int l, int which, size_t dense_off, const uint16_t* gain, int Mg,
+                int N, int K, GemmArgs args, cudaStream_t st) {
+    if (e8) return gemm8(h, epi, A, lda, h->e8, h->e8m[6 * l + which], gain, Mg, args, h->e_part, h->e_cnt, st);
+    return gemm(h, epi, A, lda, h->W(dense_off), K, Mg, N, K, args, h->e_part, h->e_cnt, st);
+  };
+  // (the int8 GEMMs with many tiles share the handle's dequantisation buffer)
+  const bool par = e8 ? !w8_many_tiles(Mp, kvw)
+                      : plan_gemm(Mp, kvw, pkvw, 0, gemm_min_bn(GE_BF16)).red != GEMM_RED_GLOBAL;
   if (par) {
     SVLA_TRY(cudaEventRecord(h->fork, s));
     for (int i = 0; i < 4; ++i) SVLA_TRY(cudaStreamWaitEvent(h->side[i], h->fork, 0));
@@ -971,10 +1039,10 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
     bf16* kx = h->kvx + (size_t)(l / 2) * 2 * Mp * kvw;
     bf16* vx = kx + (size_t)Mp * kvw;
     cudaStream_t sk = par ? h->side[branch++ % 4] : s, sv = par ? h->side[branch++ % 4] : s;
-    SVLA_TRY(gemm(h, GE_BF16, cache + (size_t)l * layer_elems, pkvw, h->W(e[2].off), pkvw, Mp, kvw, pkvw,
-                  out_args(kx, kvw), h->e_part, h->e_cnt, sk));
-    SVLA_TRY(gemm(h, GE_BF16, cache + (size_t)(c.p_layers + l) * layer_elems, pkvw, h->W(e[3].off), pkvw, Mp, kvw,
-                  pkvw, out_args(vx, kvw), h->e_part, h->e_cnt, sv));
+    SVLA_TRY(eg(GE_BF16, cache + (size_t)l * layer_elems, pkvw, l, 4, e[2].off, nullptr, Mp, kvw, pkvw,
+                out_args(kx, kvw), sk));
+    SVLA_TRY(eg(GE_BF16, cache + (size_t)(c.p_layers + l) * layer_elems, pkvw, l, 5, e[3].off, nullptr, Mp, kvw,
+                pkvw, out_args(vx, kvw), sv));
   }
   if (par) {
     for (int i = 0; i < 4; ++i) {
@@ -1027,28 +1095,27 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
         qa.pos_mod = H;  // chunk positions 0..H-1 (reading 4)
         qa.rope_cs = h->rope_cs;
         norm_consumer(qa, h->e_ss, in_tiles, M, E, c.rms_eps);
-        SVLA_TRY(gemm(h, hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32, rb, E, h->W(e[1].off), E, M, qw + 2 * kvw, E, qa,
-                      h->e_part, h->e_cnt, s));
+        SVLA_TRY(eg(hd == 64 ? GE_QKV_ROPE64 : GE_QKV_ROPE32, rb, E, l, 0, e[1].off, h->w + e[0].off, M,
+                    qw + 2 * kvw, E, qa, s));
         SVLA_TRY(attention(h->e_q, qw, h->e_k, h->e_v, kvw, nullptr, B, c.e_heads, c.e_kv_heads, hd, H, H, 1, h->e_o,
                            qw, s));
       } else {
         GemmArgs qa = out_args(h->e_q, qw);
         norm_consumer(qa, h->e_ss, in_tiles, M, E, c.rms_eps);
-        SVLA_TRY(gemm(h, GE_BF16, rb, E, h->W(e[1].off), E, M, qw, E, qa, h->e_part, h->e_cnt, s));
+        SVLA_TRY(eg(GE_BF16, rb, E, l, 0, e[1].off, h->w + e[0].off, M, qw, E, qa, s));
         const bf16* kx = h->kvx + (size_t)(l / 2) * 2 * Mp * kvw;
         SVLA_TRY(attention(h->e_q, qw, kx, kx + (size_t)Mp * kvw, kvw, pad, B, c.e_heads, c.e_kv_heads, hd, H, L, 0,
                            h->e_o, qw, s));
       }
       GemmArgs oa = out_args(h->e_r, E);
       norm_producer(oa, rb, E, h->e_ss, M);
-      SVLA_TRY(gemm(h, GE_ADD_F32, h->e_o, qw, h->W(e[4].off), qw, M, E, qw, oa, h->e_part, h->e_cnt, s));
+      SVLA_TRY(eg(GE_ADD_F32, h->e_o, qw, l, 1, e[4].off, nullptr, M, E, qw, oa, s));
       GemmArgs ga = out_args(h->e_h, c.e_ffn);
       norm_consumer(ga, h->e_ss, o_tiles, M, E, c.rms_eps);
-      SVLA_TRY(gemm(h, GE_SWIGLU, rb, E, h->W(e[6].off), E, M, 2 * c.e_ffn, E, ga, h->e_part, h->e_cnt, s));
+      SVLA_TRY(eg(GE_SWIGLU, rb, E, l, 2, e[6].off, h->w + e[5].off, M, 2 * c.e_ffn, E, ga, s));
       GemmArgs da = out_args(h->e_r, E);
       norm_producer(da, rb, E, h->e_ss, M);
-      SVLA_TRY(gemm(h, GE_ADD_F32, h->e_h, c.e_ffn, h->W(e[8].off), c.e_ffn, M, E, c.e_ffn, da, h->e_part, h->e_cnt,
-                    s));
+      SVLA_TRY(eg(GE_ADD_F32, h->e_h, c.e_ffn, l, 3, e[8].off, nullptr, M, E, c.e_ffn, da, s));
     }
     StepEndArgs se;
     se.r = h->e_r;
@@ -1153,7 +1220,8 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
                            svla_handle** out) {
   if (out) *out = nullptr;
   if (!cfg || !blob || !out) return fail(nullptr, SVLA_ERR_ARG, "null argument");
-  if (flags & ~(SVLA_CREATE_PREFIX_INT8 | SVLA_CREATE_TRAIN)) return fail(nullptr, SVLA_ERR_ARG, "unknown flag bits");
+  if (flags & ~(SVLA_CREATE_PREFIX_INT8 | SVLA_CREATE_TRAIN | SVLA_CREATE_EXPERT_INT8))
+    return fail(nullptr, SVLA_ERR_ARG, "unknown flag bits");
   if ((flags & SVLA_CREATE_PREFIX_INT8) && (cfg->p_heads * cfg->head_dim) % 64)
     return fail(nullptr, SVLA_ERR_SHAPE, "int8 prefix weights need p_heads * head_dim to be a multiple of 64");
   if (const char* why = check_config(*cfg)) return fail(nullptr, SVLA_ERR_SHAPE, why);
@@ -1222,7 +1290,7 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
       m.q_off = off;
       off += ((size_t)N * K + 255) / 256 * 256;
       m.ab_off = off;
-      off += ((size_t)N * (K / W8_GROUP) * 4 + 255) / 256 * 256;
+      off += ((size_t)N * w8_groups(K) * 4 + 255) / 256 * 256;
       return m;
     };
     const int D = c.p_width, qw = c.p_heads * c.head_dim, kvw = c.p_kv_heads * c.head_dim;
@@ -1233,15 +1301,12 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
       h->q8m.push_back(add(D, c.p_ffn));
     }
     if ((e = halloc(h, &h->q8, off)) != cudaSuccess) return bail(e, "int8 weights");
-    size_t max_nk = 0;
-    for (const Q8Mat& m : h->q8m) max_nk = std::max(max_nk, (size_t)m.N * m.K);
-    if ((e = halloc(h, &h->q8_deq, max_nk)) != cudaSuccess) return bail(e, "int8 dequantisation buffer");
     for (int l = 0; l < c.p_layers && e == cudaSuccess; ++l) {
       const Entry* en = &lay.p[9 * l];
       const size_t src[4] = {en[1].off, en[4].off, en[6].off, en[8].off};
       for (int i = 0; i < 4 && e == cudaSuccess; ++i) {
         const Q8Mat& m = h->q8m[4 * l + i];
-        const long long warps = (long long)m.N * (m.K / W8_GROUP);
+        const long long warps = (long long)m.N * w8_groups(m.K);
         quantize_affine8_kernel<<<(unsigned)((warps + 7) / 8), 256>>>(
             h->w + src[i], (size_t)m.K, m.N, m.K, h->q8 + m.q_off, (size_t)m.K,
             reinterpret_cast<uint16_t*>(h->q8 + m.ab_off));
@@ -1251,6 +1316,55 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return bail(e, "int8 quantisation");
     h->prefix_bits = 8;
+  }
+  // int8 expert: the same quantiser on the expert's projections (gate/up
+  // interleaved, gains not yet folded); the odd layers' cross K / V act on the
+  // prefix cache (K = p_kv_heads * head_dim)
+  if (flags & SVLA_CREATE_EXPERT_INT8) {
+    size_t off = 0;
+    auto add = [&](int N, int K) {
+      Q8Mat m;
+      m.N = N;
+      m.K = K;
+      m.q_off = off;
+      off += ((size_t)N * K + 255) / 256 * 256;
+      m.ab_off = off;
+      off += ((size_t)N * w8_groups(K) * 4 + 255) / 256 * 256;
+      return m;
+    };
+    const int E = c.e_width, qw = c.e_heads * c.head_dim, kvw = c.e_kv_heads * c.head_dim;
+    const int pkvw = c.p_kv_heads * c.head_dim;
+    for (int l = 0; l < c.e_layers; ++l) {
+      h->e8m.push_back(add(l % 2 == 0 ? qw + 2 * kvw : qw, E));
+      h->e8m.push_back(add(E, qw));
+      h->e8m.push_back(add(2 * c.e_ffn, E));
+      h->e8m.push_back(add(E, c.e_ffn));
+      h->e8m.push_back(l % 2 == 1 ? add(kvw, pkvw) : Q8Mat());
+      h->e8m.push_back(l % 2 == 1 ? add(kvw, pkvw) : Q8Mat());
+    }
+    if ((e = halloc(h, &h->e8, off)) != cudaSuccess) return bail(e, "int8 expert weights");
+    for (int l = 0; l < c.e_layers && e == cudaSuccess; ++l) {
+      const Entry* en = &lay.e[9 * l];
+      const size_t src[6] = {en[1].off, en[4].off, en[6].off, en[8].off, en[2].off, en[3].off};
+      for (int i = 0; i < 6 && e == cudaSuccess; ++i) {
+        const Q8Mat& m = h->e8m[6 * l + i];
+        if (m.N == 0) continue;
+        const long long warps = (long long)m.N * w8_groups(m.K);
+        quantize_affine8_kernel<<<(unsigned)((warps + 7) / 8), 256>>>(
+            h->w + src[i], (size_t)m.K, m.N, m.K, h->e8 + m.q_off, (size_t)m.K,
+            reinterpret_cast<uint16_t*>(h->e8 + m.ab_off));
+        e = cudaGetLastError();
+      }
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return bail(e, "int8 expert quantisation");
+    h->expert_bits = 8;
+  }
+  if (h->q8 || h->e8) {
+    size_t max_nk = 0;
+    for (const Q8Mat& m : h->q8m) max_nk = std::max(max_nk, (size_t)m.N * m.K);
+    for (const Q8Mat& m : h->e8m) max_nk = std::max(max_nk, (size_t)m.N * m.K);
+    if ((e = halloc(h, &h->q8_deq, max_nk)) != cudaSuccess) return bail(e, "int8 dequantisation buffer");
   }
   // fold the RMSNorm gains into the projections that consume the normalised
   // activations: QKV (in_norm) and gate/up (post_norm) of every layer, and the
@@ -1291,6 +1405,36 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
     }
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return bail(e, "fused weights");
+  }
+  // the persistent kernel's int8 copy: the expert int8 codes re-packed row by row
+  if (h->e8) {
+    FusedQ8& Q = h->fql;
+    size_t off = 0;
+    auto addq = [&](int N, int K) {
+      const size_t o = off;
+      off += ((size_t)N * fq_pitch(K) + 255) / 256 * 256;
+      return o;
+    };
+    const int E = c.e_width, qw = c.e_heads * c.head_dim, kvw = c.e_kv_heads * c.head_dim;
+    for (int l = 0; l < c.e_layers; ++l) {
+      Q.qkv.push_back(addq(l % 2 == 0 ? qw + 2 * kvw : qw, E));
+      Q.o.push_back(addq(E, qw));
+      Q.gu.push_back(addq(2 * c.e_ffn, E));
+      Q.d.push_back(addq(E, c.e_ffn));
+    }
+    Q.total = off;
+    if ((e = halloc(h, &h->fq, off)) != cudaSuccess) return bail(e, "fused int8 weights");
+    for (int l = 0; l < c.e_layers && e == cudaSuccess; ++l) {
+      const size_t dst[4] = {Q.qkv[l], Q.o[l], Q.gu[l], Q.d[l]};
+      for (int i = 0; i < 4 && e == cudaSuccess; ++i) {
+        const Q8Mat& m = h->e8m[6 * l + i];
+        pack_fused_q8_kernel<<<512, 256>>>(h->e8 + m.q_off, reinterpret_cast<const uint32_t*>(h->e8 + m.ab_off), m.N,
+                                           m.K, h->fq + dst[i], fq_pitch(m.K));
+        e = cudaGetLastError();
+      }
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return bail(e, "fused int8 weights");
   }
   if ((e = halloc(h, &h->b_t2_f32, c.e_width)) != cudaSuccess) return bail(e, "bias");
   bf16_to_f32_kernel<<<(c.e_width + 255) / 256, 256>>>(h->w + lay.b_t2.off, h->b_t2_f32, c.e_width);
@@ -1418,7 +1562,8 @@ static svla_status denoise_impl(svla_handle* h, const void* kv, const uint8_t* p
   std::vector<uint64_t> key = {fused ? 3u : 2u, (uint64_t)B, (uint64_t)L, (uint64_t)H, (uint64_t)n_steps,
                                (uint64_t)(uintptr_t)kv, (uint64_t)(uintptr_t)pad, (uint64_t)(uintptr_t)noise,
                                (uint64_t)(uintptr_t)actions, (uint64_t)(uintptr_t)trace, g_wait_ns.load(),
-                               (uint64_t)(uintptr_t)(d > 0 ? prefix : nullptr), (uint64_t)d};
+                               (uint64_t)(uintptr_t)(d > 0 ? prefix : nullptr), (uint64_t)d,
+                               (uint64_t)h->expert_bits};
   return run_graph(
       h, key,
       [&](cudaStream_t cs) {
@@ -1479,6 +1624,17 @@ svla_status svla_set_prefix_weights(svla_handle* h, int bits) {
 }
 
 int svla_prefix_weights(const svla_handle* h) { return h ? h->prefix_bits : 0; }
+
+svla_status svla_set_expert_weights(svla_handle* h, int bits) {
+  if (!h) return fail(nullptr, SVLA_ERR_ARG, "null handle");
+  if (bits != 16 && bits != 8) return fail(h, SVLA_ERR_ARG, "bits must be 16 or 8");
+  if (bits == 8 && !h->e8)
+    return fail(h, SVLA_ERR_UNSUPPORTED, "the handle has no int8 expert weights (create it with SVLA_CREATE_EXPERT_INT8)");
+  h->expert_bits = bits;
+  return SVLA_OK;
+}
+
+int svla_expert_weights(const svla_handle* h) { return h ? h->expert_bits : 0; }
 
 size_t svla_train_grad_elems(const svla_handle* h) { return h && h->tr ? h->lay.total - h->tr->base : 0; }
 
@@ -1664,11 +1820,11 @@ svla_status svla_op_gemm(int epilogue, const void* A, int lda, const void* W, in
 
 svla_status svla_op_quantize_affine8(const void* W, int ldw, int N, int K, void* q, int ldq, void* ab, void* stream) {
   if (!W || !q || !ab) return fail(nullptr, SVLA_ERR_ARG, "null pointer");
-  if (N < 1 || K < W8_GROUP || K % W8_GROUP || ldw < K || ldq < K || ldw % 2 || ldq % 2)
-    return fail(nullptr, SVLA_ERR_SHAPE, "bad sizes or strides (K a multiple of 64, even strides)");
+  if (N < 1 || K < 16 || K % 16 || ldw < K || ldq < K || ldw % 2 || ldq % 2)
+    return fail(nullptr, SVLA_ERR_SHAPE, "bad sizes or strides (K a multiple of 16, even strides)");
   if ((uintptr_t)W & 3 || (uintptr_t)q & 1 || (uintptr_t)ab & 3)
     return fail(nullptr, SVLA_ERR_ARG, "W and ab must be 4-byte aligned, q 2-byte aligned");
-  const long long warps = (long long)N * (K / W8_GROUP);
+  const long long warps = (long long)N * w8_groups(K);
   quantize_affine8_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const uint16_t*>(W), (size_t)ldw, N, K, reinterpret_cast<uint8_t*>(q), (size_t)ldq,
       reinterpret_cast<uint16_t*>(ab));
@@ -1677,12 +1833,12 @@ svla_status svla_op_quantize_affine8(const void* W, int ldw, int N, int K, void*
 }
 
 int svla_op_gemm_w8_splits(int M, int N, int K) {
-  if (M < 1 || N < 1 || K < W8_GROUP || K % W8_GROUP) return 0;
+  if (M < 1 || N < 1 || K < 16 || K % 16) return 0;
   return plan_gemm_w8(M, N, K, 0).splits;
 }
 
 int svla_op_gemm_w8_tile_n(int M, int N, int K) {
-  if (M < 1 || N < 1 || K < W8_GROUP || K % W8_GROUP) return 0;
+  if (M < 1 || N < 1 || K < 16 || K % 16) return 0;
   return plan_gemm_w8(M, N, K, 0).bn;
 }
 
@@ -1692,7 +1848,7 @@ svla_status svla_op_gemm_w8(int epilogue, const void* A, int lda, const void* q,
   const int epi = epi_code(epilogue);
   if (epi < 0) return fail(nullptr, SVLA_ERR_ARG, "unknown epilogue");
   if (!A || !q || !ab || !C) return fail(nullptr, SVLA_ERR_ARG, "null pointer");
-  if (M < 1 || N < 8 || N % 8 || K < W8_GROUP || K % W8_GROUP || splits < 0 || splits > GEMM_MAX_CLUSTER ||
+  if (M < 1 || N < 8 || N % 8 || K < 16 || K % 16 || splits < 0 || splits > GEMM_MAX_CLUSTER ||
       lda < K || lda % 8 || ldq < K || ldq % 16 || ldc < N || (epi != GE_F32 && epi != GE_ADD_F32 ? ldc % 8 : ldc % 4))
     return fail(nullptr, SVLA_ERR_SHAPE, "bad sizes or strides");
   if (((uintptr_t)A | (uintptr_t)q | (uintptr_t)ab | (uintptr_t)C | (uintptr_t)gain) & 15)

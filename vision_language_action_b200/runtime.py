@@ -46,11 +46,13 @@ class SmolVLA:
     array, a torch uint16/bfloat16 tensor (host or CUDA), or raw bytes.
     ``prefix_int8`` builds the weight-only int8 copy of the prefix LM's
     projections (the vlm-8bit preset) and selects it for the prefill;
-    ``train`` allocates the workspace of ``train_step``.
+    ``expert_int8`` builds the int8 copy of the expert's projections and
+    selects it for the denoise; ``train`` allocates the workspace of
+    ``train_step``.
     """
 
     def __init__(self, shape, blob, max_batch: int, max_prefix: int, max_chunk: int,
-                 device: int = 0, prefix_int8: bool = False, train: bool = False):
+                 device: int = 0, prefix_int8: bool = False, train: bool = False, expert_int8: bool = False):
         self.lib = _abi.load()
         self.cfg = config_from_shape(shape, max_batch, max_prefix, max_chunk)
         self.action_dim = shape.action_dim
@@ -65,7 +67,8 @@ class SmolVLA:
             ptr, nbytes = arr.ctypes.data, arr.nbytes
             self._blob_keep = arr
         h = ctypes.c_void_p()
-        flags = (_abi.CREATE_PREFIX_INT8 if prefix_int8 else 0) | (_abi.CREATE_TRAIN if train else 0)
+        flags = (_abi.CREATE_PREFIX_INT8 if prefix_int8 else 0) | (_abi.CREATE_TRAIN if train else 0) | \
+            (_abi.CREATE_EXPERT_INT8 if expert_int8 else 0)
         st = self.lib.svla_create_ex(ctypes.byref(self.cfg), ctypes.c_void_p(ptr), nbytes, device, flags,
                                      ctypes.byref(h))
         self._blob_keep = None
@@ -204,6 +207,14 @@ class SmolVLA:
     @property
     def prefix_weights(self) -> int:
         return int(self.lib.svla_prefix_weights(self.h))
+
+    def set_expert_weights(self, bits: int) -> None:
+        """16 = dense bf16 expert weights, 8 = the int8 copy (needs expert_int8=True)."""
+        _abi.check(self.lib.svla_set_expert_weights(self.h, bits), self.h)
+
+    @property
+    def expert_weights(self) -> int:
+        return int(self.lib.svla_expert_weights(self.h))
 
     def fused_supported(self, B: int, H: int) -> bool:
         return bool(self.lib.svla_denoise_fused_supported(self.h, B, H))
