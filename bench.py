@@ -154,6 +154,19 @@ def prefix_projection_bytes(s, bits):
     return tot
 
 
+def expert_projection_bytes(s, bits):
+    """Bytes of the expert layers' projections one Euler step reads (the odd
+    layers' cross K / V projections included): bf16 weights, or int8 codes plus
+    a bf16 (alpha, beta) pair per group of 64 inputs, the last group of a row
+    holding the K mod 64 remaining inputs (the int8 expert)."""
+    tot = 0
+    for name, shp in synth.manifest(s):
+        if name.startswith("e") and name.split(".")[-1] in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+            N, K = shp
+            tot += 2 * N * K if bits == 16 else N * K + N * ((K + 63) // 64) * 4
+    return tot
+
+
 def train_flops(s, B, L, H):
     """Algorithmic FLOPs of one training step of the expert (svla_train_step):
     every forward GEMM, its weight gradient, and its input gradient except
@@ -541,6 +554,67 @@ def int8_prefix(args, dev, barrier, hbm_peak, peak_kind):
     return out
 
 
+def int8_expert(args, dev, barrier, hbm_peak, peak_kind):
+    """The int8 expert (the vlm-8bit scheme on the expert's projections) at
+    batch 1 (persistent kernel) and batch 32 (multi-kernel path): denoise and
+    chunk times on one handle, switched between its int8 and dense expert
+    weights, the denoise's bytes against HBM, and at batch 1 the chunk with
+    both the prefix and the expert in int8."""
+    out = {"preset": "expert int8: the expert layers' projections (cross K/V included) in int8, affine groups "
+                     "of 64 (a 720-wide row's last group holds 16 inputs), bf16 (alpha, beta); prefix and heads bf16"}
+    for name in ("smolvla_b1", "smolvla_b32"):
+        m, wl, _, d = gpu_setup(name, dev, expert_int8=True)
+        s = wl.model
+        steps = args.steps if wl.B == 1 else max(3, args.steps // 2)
+
+        def den():
+            m.denoise(d["kv"], d["valid"], d["noise"], wl.n_steps, actions=d["actions"])
+
+        def chunk():
+            m.prefill(d["embeds"], d["valid"], d["kv"])
+            den()
+
+        chunk()
+        t8 = time_steps(den, steps, args.warmup, barrier) / steps
+        c8 = time_steps(chunk, steps, args.warmup, barrier) / steps
+        m.set_expert_weights(16)
+        t16 = time_steps(den, steps, args.warmup, barrier) / steps
+        m.set_expert_weights(8)
+        if m.device_status() != 0:
+            raise RuntimeError("device status after the int8 expert timing")
+        m.close()
+        del d
+        e8, e16 = expert_projection_bytes(s, 8), expert_projection_bytes(s, 16)
+        den_bytes = chunk_work(s, wl.B, wl.L, wl.H, wl.n_steps)[0] - chunk_work(s, wl.B, wl.L, wl.H, 0)[0]
+        den_bytes8 = den_bytes - wl.n_steps * (e16 - e8)
+        achieved = den_bytes8 / (t8 * 1e-3) / 1e9
+        row = {"denoise_ms": round(t8, 4), "denoise_ms_dense_same_handle": round(t16, 4),
+               "chunk_ms": round(c8 / wl.B, 4) if wl.B == 1 else None,
+               "chunks_per_s": round(wl.B / (c8 * 1e-3), 2) if wl.B > 1 else None,
+               "projection_bytes_per_step_int8": int(e8), "projection_bytes_per_step_bf16": int(e16),
+               "denoise_roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                                    "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                                    "algorithmic_bytes": int(den_bytes8), "peak_kind": peak_kind}}
+        if wl.B == 1:
+            m, wl, _, d = gpu_setup(name, dev, prefix_int8=True, expert_int8=True)
+
+            def chunk_all():
+                m.prefill(d["embeds"], d["valid"], d["kv"])
+                m.denoise(d["kv"], d["valid"], d["noise"], wl.n_steps, actions=d["actions"])
+
+            chunk_all()
+            ca = time_steps(chunk_all, steps, args.warmup, barrier) / steps
+            if m.device_status() != 0:
+                raise RuntimeError("device status after the int8 prefix + expert timing")
+            m.close()
+            del d
+            row["chunk_ms_prefix_and_expert_int8"] = round(ca, 4)
+        out[name] = row
+    import torch
+    torch.cuda.empty_cache()
+    return out
+
+
 def batched_configs(args, dev, barrier, hbm_peak, tf_peak, tf_sus, peak_kind):
     """The two batched workloads beside the headline and batch 32: batch 8 with
     prefix 321 and chunk 100 (prefill + denoise, tensor and HBM fractions), and
@@ -752,6 +826,7 @@ def ours(args, rank, world, local_rank):
     torch.cuda.empty_cache()
 
     q8 = None if args.no_int8 else int8_prefix(args, dev, barrier, hbm_peak, peak_kind)
+    e8 = None if args.no_int8 else int8_expert(args, dev, barrier, hbm_peak, peak_kind)
 
     secondary = None
     if not args.no_secondary:
@@ -849,6 +924,7 @@ def ours(args, rank, world, local_rank):
                           "note": "each call timed alone on rank 0, same steps and warm-up"},
             "prefix_assembly": asm,
             "int8_prefix": q8,
+            "int8_expert": e8,
             "train_step": train,
             "gpu_launches": launches_per_chunk(s, wl.n_steps, fused) * args.steps,
             "graph_gemm_roofline": graph_gemm if fused else None,

@@ -20,6 +20,22 @@ def test_prefix_projection_bytes_from_the_manifest():
     assert bench.prefix_projection_bytes(S, 8) == dense // 2 + dense // 2 // 64 * 4
 
 
+def test_expert_projection_bytes_from_the_manifest():
+    """Every expert layer's seven projections (the odd layers' cross K / V act on
+    the 320-wide cache); int8: one byte per weight plus a bf16 (alpha, beta) pair
+    per group, 720-wide rows having 12 groups (11 of 64 and one of 16)."""
+    man = dict(synth.manifest(S))
+    dense = int8 = 0
+    for l in range(S.e_layers):
+        for n in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+            N, K = man[f"e{l}.{n}"]
+            dense += 2 * N * K
+            int8 += N * K + N * {720: 12, 960: 15, 2048: 32, 320: 5}[K] * 4
+    assert bench.expert_projection_bytes(S, 16) == dense
+    assert bench.expert_projection_bytes(S, 8) == int8
+    assert 0.5 < int8 / dense < 0.54
+
+
 def test_train_flops_counts_three_products_per_weight_gemm():
     B, L, H = 2, 177, 50
     M, E = B * H, S.e_width
