@@ -22,6 +22,7 @@ the headline chunk's difference from the oracle's.
     --no-int8 / --no-train / --no-cpu   skip those blocks
     --train-only    time only the training step
     --batched-only  time only the batch-8 and batch-256 workloads
+    --profile CASE  run a workload untimed for ncu (the commands in profiles/)
 
 Prints ONE JSON line on rank 0.
 """
@@ -935,6 +936,53 @@ def ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def profile_case(spec, dev, reps):
+    """A workload run for a profiler to attach to (untimed): 'NAME' runs the
+    prefill and the denoise of workload NAME `reps` times after one warm-up
+    call; options ':graph' / ':fused' pick the denoise path, ':int8p' /
+    ':int8e' the int8 prefix / expert; 'denoise_b256' runs the batch-256
+    denoise from its given K/V cache."""
+    import torch
+    from vision_language_action_b200 import _abi
+    from vision_language_action_b200.runtime import SmolVLA
+    name, *opts = spec.split(":")
+    if name == "denoise_b256":
+        wl = synth.WORKLOADS[name]
+        s = wl.model
+        m = SmolVLA(s, synth.pack_blob(s, synth.gen_weights(s, wl.seed)), max_batch=wl.B, max_prefix=wl.L,
+                    max_chunk=wl.H, device=dev)
+        inp = synth.gen_inputs(wl)
+        kv = np.stack([inp["k"], inp["v"]]).reshape(2, s.p_layers, wl.B, wl.L, -1)
+        d = {"kv": torch.from_numpy(kv.view(np.int16)).to(f"cuda:{dev}").view(torch.bfloat16),
+             "valid": torch.from_numpy(inp["valid"]).to(f"cuda:{dev}"),
+             "noise": torch.from_numpy(inp["noise"]).to(f"cuda:{dev}")}
+        d["actions"] = torch.empty_like(d["noise"])
+        pre = None
+    else:
+        m, wl, _, d = gpu_setup(name, dev, prefix_int8="int8p" in opts, expert_int8="int8e" in opts)
+
+        def pre():
+            m.prefill(d["embeds"], d["valid"], d["kv"])
+    path = {"graph": _abi.DENOISE_GRAPH, "fused": _abi.DENOISE_FUSED}
+    for o in opts:
+        if o in path:
+            m.set_denoise_path(path[o])
+
+    def call():
+        if pre:
+            pre()
+        m.denoise(d["kv"], d["valid"], d["noise"], wl.n_steps, actions=d["actions"])
+
+    for _ in range(1 + reps):
+        call()
+    torch.cuda.synchronize()
+    st = m.device_status()
+    m.close()
+    print(json.dumps({"profile_case": spec, "calls": 1 + reps, "status": st}), flush=True)
+    if st != 0:
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -947,6 +995,7 @@ def main():
     ap.add_argument("--no-train", action="store_true")
     ap.add_argument("--train-only", action="store_true", help="time only the expert's training step")
     ap.add_argument("--batched-only", action="store_true", help="time only the batch-8 and batch-256 workloads")
+    ap.add_argument("--profile", metavar="CASE", help="run CASE untimed for a profiler (see profile_case)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -955,6 +1004,11 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         reference_arm(args, rank)
+        return
+    if args.profile:
+        import torch
+        torch.cuda.set_device(local_rank)
+        profile_case(args.profile, local_rank, max(1, args.steps))
         return
     if args.batched_only:
         import torch
