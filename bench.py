@@ -155,16 +155,22 @@ def prefix_projection_bytes(s, bits):
     return tot
 
 
-def expert_projection_bytes(s, bits):
-    """Bytes of the expert layers' projections one Euler step reads (the odd
-    layers' cross K / V projections included): bf16 weights, or int8 codes plus
-    a bf16 (alpha, beta) pair per group of 64 inputs, the last group of a row
-    holding the K mod 64 remaining inputs (the int8 expert)."""
+def expert_projection_bytes(s, bits, cross=None):
+    """Bytes of the expert layers' projections: bf16 weights, or int8 codes
+    plus a bf16 (alpha, beta) pair per group of 64 inputs, the last group of a
+    row holding the K mod 64 remaining inputs (the int8 expert). cross=None:
+    all of them; True: only the odd layers' cross K / V projections (read once
+    per denoise call, by the hoist); False: the others (read every step)."""
     tot = 0
     for name, shp in synth.manifest(s):
-        if name.startswith("e") and name.split(".")[-1] in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
-            N, K = shp
-            tot += 2 * N * K if bits == 16 else N * K + N * ((K + 63) // 64) * 4
+        layer, _, mat = name.partition(".")
+        if not layer.startswith("e") or mat not in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+            continue
+        is_cross = int(layer[1:]) % 2 == 1 and mat in ("wk", "wv")
+        if cross is not None and is_cross != cross:
+            continue
+        N, K = shp
+        tot += 2 * N * K if bits == 16 else N * K + N * ((K + 63) // 64) * 4
     return tot
 
 
@@ -585,9 +591,9 @@ def int8_expert(args, dev, barrier, hbm_peak, peak_kind):
             raise RuntimeError("device status after the int8 expert timing")
         m.close()
         del d
-        e8, e16 = expert_projection_bytes(s, 8), expert_projection_bytes(s, 16)
-        den_bytes = chunk_work(s, wl.B, wl.L, wl.H, wl.n_steps)[0] - chunk_work(s, wl.B, wl.L, wl.H, 0)[0]
-        den_bytes8 = den_bytes - wl.n_steps * (e16 - e8)
+        e8, e16 = expert_projection_bytes(s, 8, False), expert_projection_bytes(s, 16, False)
+        c8, c16 = expert_projection_bytes(s, 8, True), expert_projection_bytes(s, 16, True)
+        den_bytes8 = denoise_bytes(s, wl.B, wl.L, wl.H, wl.n_steps) - wl.n_steps * (e16 - e8) - (c16 - c8)
         achieved = den_bytes8 / (t8 * 1e-3) / 1e9
         row = {"denoise_ms": round(t8, 4), "denoise_ms_dense_same_handle": round(t16, 4),
                "chunk_ms": round(c8 / wl.B, 4) if wl.B == 1 else None,

@@ -34,6 +34,11 @@ def test_expert_projection_bytes_from_the_manifest():
     assert bench.expert_projection_bytes(S, 16) == dense
     assert bench.expert_projection_bytes(S, 8) == int8
     assert 0.5 < int8 / dense < 0.54
+    for bits in (8, 16):  # per-step projections + the hoisted cross K / V ones
+        assert bench.expert_projection_bytes(S, bits, False) + bench.expert_projection_bytes(S, bits, True) == \
+            bench.expert_projection_bytes(S, bits)
+    cross = sum(2 * int(np.prod(man[f"e{l}.{n}"])) for l in range(1, S.e_layers, 2) for n in ("wk", "wv"))
+    assert bench.expert_projection_bytes(S, 16, True) == cross
 
 
 def test_train_flops_counts_three_products_per_weight_gemm():

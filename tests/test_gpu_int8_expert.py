@@ -227,3 +227,32 @@ def test_int8_expert_trace_and_prefix_overwrite_on_both_paths():
             assert torch.equal(ap[:, :d], prev)
     finally:
         m.close()
+
+
+def test_int8_expert_persistent_timeout_reports_and_recovers():
+    """Wait limit 0 on the int8 persistent kernel: the first unsatisfied wait
+    (a grid barrier, a weight slot awaited for its dequantisation) gives up, the
+    kernel records SVLA_ERR_TIMEOUT and drains; the next launch is exact."""
+    wl_name = "tiny"
+    wl = synth.WORKLOADS[wl_name]
+    s, _, blob = H.weights(wl_name)
+    m = SmolVLA(s, blob, max_batch=wl.B, max_prefix=wl.L, max_chunk=wl.H, expert_int8=True)
+    lib = _abi.load()
+    try:
+        m.set_denoise_path(_abi.DENOISE_FUSED)
+        embeds, valid, noise = inputs(wl_name)
+        kv = m.prefill(embeds, valid)
+        ref, _ = m.denoise(kv, valid, noise, wl.n_steps)
+        assert m.device_status() == _abi.SVLA_OK
+        lib.svla_set_wait_limit_ns(0)
+        try:
+            m.denoise(kv, valid, noise, wl.n_steps)
+            st = m.device_status()
+        finally:
+            lib.svla_set_wait_limit_ns(1_000_000_000)
+        assert st == _abi.SVLA_ERR_TIMEOUT
+        again, _ = m.denoise(kv, valid, noise, wl.n_steps)
+        assert m.device_status() == _abi.SVLA_OK
+        assert torch.equal(again, ref)
+    finally:
+        m.close()
