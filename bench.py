@@ -592,8 +592,8 @@ def int8_expert(args, dev, barrier, hbm_peak, peak_kind):
         m.close()
         del d
         e8, e16 = expert_projection_bytes(s, 8, False), expert_projection_bytes(s, 16, False)
-        c8, c16 = expert_projection_bytes(s, 8, True), expert_projection_bytes(s, 16, True)
-        den_bytes8 = denoise_bytes(s, wl.B, wl.L, wl.H, wl.n_steps) - wl.n_steps * (e16 - e8) - (c16 - c8)
+        x8, x16 = expert_projection_bytes(s, 8, True), expert_projection_bytes(s, 16, True)
+        den_bytes8 = denoise_bytes(s, wl.B, wl.L, wl.H, wl.n_steps) - wl.n_steps * (e16 - e8) - (x16 - x8)
         achieved = den_bytes8 / (t8 * 1e-3) / 1e9
         row = {"denoise_ms": round(t8, 4), "denoise_ms_dense_same_handle": round(t16, 4),
                "chunk_ms": round(c8 / wl.B, 4) if wl.B == 1 else None,
