@@ -9,7 +9,7 @@ the C ABI.
   weights.
 * The chunk of an int8-expert handle (dense prefix) against the oracle run on
   the dequantised expert, on the persistent kernel (batch 1) and on the
-  multi-kernel path (batch 1 and batch 32).
+  multi-kernel path (batch 1, batch 32, batch 8 with prefix 321 and chunk 100).
 * Bit for bit against a dense handle given the dequantised blob where both
   take the same partial-sum order: the persistent kernel's in-shared-memory
   dequantisation and the many-tile path's dequantise-then-dense GEMM produce
@@ -123,7 +123,7 @@ def inputs(wl_name):
 
 CASES = [("tiny", _abi.DENOISE_FUSED, [0]), ("tiny", _abi.DENOISE_GRAPH, [0]),
          ("smolvla_b1", _abi.DENOISE_FUSED, [0]), ("smolvla_b1", _abi.DENOISE_GRAPH, [0]),
-         ("smolvla_b32", _abi.DENOISE_AUTO, [5, 31])]
+         ("smolvla_b32", _abi.DENOISE_AUTO, [5, 31]), ("long_prefix_b8", _abi.DENOISE_AUTO, [0, 7])]
 
 
 @pytest.mark.parametrize("wl_name,path,queries", CASES, ids=[f"{c[0]}-{c[1]}" for c in CASES])
