@@ -229,18 +229,16 @@ struct Q8Mat {
   int N = 0, K = 0;
 };
 
-// Row pitch (bytes) of the persistent denoise kernel's int8 weight copy: a row
-// is its K codes followed by its ceil(K/64) (alpha, beta) pairs (bf16 x 2), so
-// a job's rows arrive with one bulk copy per run of rows.
-inline size_t fq_pitch(int K) { return ((size_t)K + 4 * (size_t)w8_groups(K) + 15) / 16 * 16; }
-
-// Byte offsets of that copy (per expert layer: QKV or Q, O, gate/up, down).
+// Byte offsets of the persistent denoise kernel's int8 weight copy (per expert
+// layer: QKV or Q, O, gate/up, down). A row is its K codes followed by its
+// ceil(K/64) (alpha, beta) pairs (bf16 x 2), pitch fd_q8_pitch(K), so a job's
+// rows arrive with one bulk copy per run of rows.
 struct FusedQ8 {
   std::vector<size_t> qkv, o, gu, d;
   size_t total = 0;
 };
 
-// dst row n = [q[n, 0..K) | (alpha, beta) of row n for g = 0..G)], pitch fq_pitch(K)
+// dst row n = [q[n, 0..K) | (alpha, beta) of row n for g = 0..G)], pitch fd_q8_pitch(K)
 __global__ void pack_fused_q8_kernel(const uint8_t* __restrict__ q, const uint32_t* __restrict__ ab, int N, int K,
                                      uint8_t* __restrict__ dst, size_t pitch) {
   const int G = w8_groups(K);
@@ -1412,7 +1410,7 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
     size_t off = 0;
     auto addq = [&](int N, int K) {
       const size_t o = off;
-      off += ((size_t)N * fq_pitch(K) + 255) / 256 * 256;
+      off += ((size_t)N * fd_q8_pitch(K) + 255) / 256 * 256;
       return o;
     };
     const int E = c.e_width, qw = c.e_heads * c.head_dim, kvw = c.e_kv_heads * c.head_dim;
@@ -1429,7 +1427,7 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
       for (int i = 0; i < 4 && e == cudaSuccess; ++i) {
         const Q8Mat& m = h->e8m[6 * l + i];
         pack_fused_q8_kernel<<<512, 256>>>(h->e8 + m.q_off, reinterpret_cast<const uint32_t*>(h->e8 + m.ab_off), m.N,
-                                           m.K, h->fq + dst[i], fq_pitch(m.K));
+                                           m.K, h->fq + dst[i], fd_q8_pitch(m.K));
         e = cudaGetLastError();
       }
     }
