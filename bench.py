@@ -231,28 +231,91 @@ def denoise_bytes(s, B, L, H, n_steps):
 # ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
-class Clocks:
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+CLOCK_REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+                 ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_index):
-        self.idx = gpu_index
+
+def summarize_clocks(samples):
+    """[(sm_mhz, max_sm_mhz, reasons_bitmask)] sampled during a timed region ->
+    {"sm_mhz": median, "sm_max_mhz", "reasons": the clock-event reasons seen
+    active among hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown,
+    sw_power_cap, "samples"}; None without samples."""
+    if not samples:
+        return None
+    reasons = sorted({name for _, _, m in samples for name, bit in CLOCK_REASONS if m & bit})
+    return {"sm_mhz": statistics.median(s[0] for s in samples), "sm_max_mhz": max(s[1] for s in samples),
+            "reasons": reasons, "samples": len(samples)}
+
+
+class Clocks:
+    """SM clocks and clock-event reasons of the bench's GPU, sampled during the
+    timed region: NVML polled from a thread every 10 ms (the device found by the
+    UUID torch reports, so a CUDA_VISIBLE_DEVICES remapping cannot point it at
+    another GPU), else nvidia-smi every 50 ms. Read-only: no setting changes."""
+    Q = ("uuid,clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, cuda_dev):
+        self.dev = cuda_dev
+        self.samples = []
+        self.thread = None
+        self.stop_flag = False
         self.proc = None
         self.path = None
+        self.uuid = None
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(cuda_dev).uuid)
+            self.uuid = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            self.uuid = None
+
+    def _poll(self, nv, handle):
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.samples.append((float(sm), float(mx), int(rs)))
+            except Exception:
+                return
+            time.sleep(0.01)
 
     def start(self):
+        self.samples = []
+        self.stop_flag = False
+        try:
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            handle = nv.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.thread = threading.Thread(target=self._poll, args=(nv, handle), daemon=True)
+            self.thread.start()
+            while not self.samples and self.thread.is_alive():  # sampling runs before the region starts
+                time.sleep(0.001)
+            return
+        except Exception:
+            self.thread = None
         try:
             import tempfile
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+            target = self.uuid if self.uuid else str(self.dev)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", target, f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while os.path.getsize(self.path) == 0 and time.time() - t0 < 5:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=2)
+            return summarize_clocks(self.samples)
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -263,17 +326,11 @@ class Clocks:
         rows = []
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
-            if len(f) >= 9:
-                rows.append(f)
+            if len(f) >= 7 and f[1].replace(".", "").isdigit() and f[2].replace(".", "").isdigit():
+                bits = sum(bit for (name, bit), v in zip(CLOCK_REASONS, f[3:7]) if v.lower() == "active")
+                rows.append((float(f[1]), float(f[2]), bits))
         os.unlink(self.path)
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        return summarize_clocks(rows)
 
 
 # ---------------------------------------------------------------------------

@@ -87,3 +87,19 @@ def test_traffic_figures_follow_the_sources_they_were_captured_on(tmp_path, monk
     assert bench.ncu_traffic("absent") is None
     f.write_text(json.dumps({"kernels": {"k": {"dram_bytes_per_launch": 123.0, "sources_sha16": "0" * 16}}}))
     assert bench.ncu_traffic("k") is None
+
+
+def test_clock_summary_decodes_the_event_reasons():
+    """The sampler keeps (SM MHz, max SM MHz, NVML clock-event reason bits); the
+    summary reports the median, the maximum and the throttle reasons seen."""
+    assert bench.summarize_clocks([]) is None
+    s = bench.summarize_clocks([(1965.0, 1965.0, 0x0), (1950.0, 1965.0, 0x4), (1965.0, 1965.0, 0x1)])
+    assert s == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    s = bench.summarize_clocks([(1200.0, 1965.0, 0x8 | 0x40), (1100.0, 1965.0, 0x20)])
+    assert s["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+    assert s["sm_mhz"] == 1150.0
+    # without a GPU the sampler reports nothing rather than failing
+    c = bench.Clocks(0)
+    c.start()
+    r = c.stop()
+    assert r is None or isinstance(r, dict)
