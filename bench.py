@@ -151,7 +151,7 @@ def prefix_projection_bytes(s, bits):
         for i, (N, K) in enumerate(mats):
             if l == s.p_layers - 1 and i > 0:
                 break
-            tot += 2 * N * K if bits == 16 else N * K + N * (K // 64) * 4
+            tot += 2 * N * K if bits == 16 else N * K + N * ((K + 63) // 64) * 4
     return tot
 
 
@@ -604,7 +604,7 @@ def int8_prefix(args, dev, barrier, hbm_peak, peak_kind):
         if wl.B == 1:
             M, N, K = wl.L, 2 * s.p_ffn, s.p_width
             out["gemm_w8_gate_up_b1"] = {"kernel": "gemm_w8_kernel<64, SwiGLU, 4>", "M": M, "N": N, "K": K,
-                                         "algorithmic_bytes_per_launch": int(N * K + N * (K // 64) * 4 + 2 * M * K),
+                                         "algorithmic_bytes_per_launch": int(N * K + N * ((K + 63) // 64) * 4 + 2 * M * K),
                                          "traffic": ncu_traffic("gemm_w8_kernel_gate_up_b1")}
         out[name] = {"prefill_ms": round(t8, 4), "prefill_ms_dense_same_handle": round(t16, 4),
                      "chunk_ms": round(c8 / wl.B, 4) if wl.B == 1 else None,

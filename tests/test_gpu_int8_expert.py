@@ -69,6 +69,23 @@ def test_quantizer_ragged_groups_match_oracle_bit_for_bit(N, K):
     assert np.array_equal(synth.bf16_bits_to_f32(abn[..., 1].T), b_ref)
 
 
+@pytest.mark.parametrize("N,K", [(960, 720), (7, 80), (64, 960)])
+def test_python_binding_sizes_the_scale_pairs_for_ragged_k(N, K):
+    """runtime.op_quantize_affine8 allocates ceil(K/64) (alpha, beta) groups,
+    the number the kernel writes, and returns the oracle's codes and pairs."""
+    from vision_language_action_b200 import runtime
+
+    w = ragged_matrix(N + K, N, K)
+    q_ref, a_ref, b_ref = oq.quantize_affine8(w)
+    q, ab = runtime.op_quantize_affine8(bf16_dev(w))
+    torch.cuda.synchronize()
+    assert tuple(ab.shape) == (groups(K), N, 2)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    abn = ab.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(abn[..., 0].T, synth.f32_to_bf16_bits(a_ref))
+    assert np.array_equal(synth.bf16_bits_to_f32(abn[..., 1].T), b_ref)
+
+
 @pytest.mark.parametrize("M,N,K", [(50, 1600, 720), (50, 4096, 720), (177, 960, 720), (1600, 4096, 720),
                                    (3, 64, 80)])
 @pytest.mark.parametrize("with_gain", [False, True])

@@ -245,11 +245,12 @@ def op_gemm(epilogue: str, A: torch.Tensor, W: torch.Tensor, C: torch.Tensor, bi
 
 
 def op_quantize_affine8(W: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """svla_op_quantize_affine8: bf16 W [N, K] -> (codes uint8 [N, K], (alpha, beta) bf16 [K/64, N, 2])."""
+    """svla_op_quantize_affine8: bf16 W [N, K] -> (codes uint8 [N, K], (alpha, beta) bf16 [G, N, 2]) with
+    G = ceil(K / 64) groups (the last one holds the K mod 64 remaining inputs when K % 64 != 0)."""
     lib = _abi.load()
     N, K = W.shape
     q = torch.empty((N, K), dtype=torch.uint8, device=W.device)
-    ab = torch.empty((K // 64, N, 2), dtype=torch.bfloat16, device=W.device)
+    ab = torch.empty(((K + 63) // 64, N, 2), dtype=torch.bfloat16, device=W.device)
     _abi.check(lib.svla_op_quantize_affine8(_ptr(W), W.stride(0), N, K, _ptr(q), q.stride(0), _ptr(ab),
                                             _stream(stream)))
     return q, ab
