@@ -113,15 +113,29 @@ struct GemmCfg {
 };
 
 // ---------------------------------------------------------------------------
-// epilogue helpers (one thread = one output row, 16 consecutive columns)
+// epilogue helpers (one thread = one output row, 16 consecutive columns). The
+// ragged tails are unrolled with predicates: a loop bounded by ncols would
+// index the value array at run time and move it to local memory.
 // ---------------------------------------------------------------------------
 SVLA_DEV void store16_f32(float* dst, const float (&v)[16], int ncols) {
   if (ncols >= 16) {
-    float4* d4 = reinterpret_cast<float4*>(dst);
+    if (aligned32(dst)) {  // whole 32-byte sectors (measured: 10.7 against 11.2 ms per batch-32 denoise)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      for (int h = 0; h < 16; h += 8) {
+        uint32_t u[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) u[i] = __float_as_uint(v[h + i]);
+        st_global_v8(dst + h, u);
+      }
+    } else {
+      float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
   } else {
-    for (int i = 0; i < ncols; ++i) dst[i] = v[i];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < ncols) dst[i] = v[i];
   }
 }
 
@@ -138,7 +152,9 @@ SVLA_DEV void add16_f32(float* dst, const float (&v)[16], int ncols) {
       d4[i] = o;
     }
   } else {
-    for (int i = 0; i < ncols; ++i) dst[i] += v[i];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < ncols) dst[i] += v[i];
   }
 }
 
@@ -153,11 +169,18 @@ SVLA_DEV void store16_bf16(bf16* dst, const float (&v)[16], int ncols) {
     b.y = pack_bf16x2(v[10], v[11]);
     b.z = pack_bf16x2(v[12], v[13]);
     b.w = pack_bf16x2(v[14], v[15]);
-    uint4* d = reinterpret_cast<uint4*>(dst);
-    d[0] = a;
-    d[1] = b;
+    if (aligned32(dst)) {
+      const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      st_global_v8(dst, u);
+    } else {
+      uint4* d = reinterpret_cast<uint4*>(dst);
+      d[0] = a;
+      d[1] = b;
+    }
   } else {
-    for (int i = 0; i < ncols; ++i) dst[i] = __float2bfloat16_rn(v[i]);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < ncols) dst[i] = __float2bfloat16_rn(v[i]);
   }
 }
 
@@ -216,12 +239,13 @@ SVLA_DEV float norm_row_scale(const GemmArgs& a, int m, bool row_ok) {
 // Epilogue inputs of one row that do not depend on the accumulator, loaded into
 // registers by the epilogue warps before they wait for it (the wait overlaps
 // their latency): the norm row factor, the row's residual segment (residual
-// add: its first RES columns; the rest, for wide tiles, is loaded chunk by
-// chunk) and the row's RoPE (cos, sin) pairs (one position per row, the same
-// for every head of the tile).
+// add: the whole segment up to 96 columns; for wider tiles its first 32
+// columns, the rest loaded one 32-column chunk ahead of the chunk being added)
+// and the row's RoPE (cos, sin) pairs (one position per row, the same for
+// every head of the tile).
 template <int BN, int EPI>
 struct EpiPre {
-  static constexpr int RES = EPI == GE_ADD_F32 && BN <= 96 ? BN : 0;
+  static constexpr int RES = EPI == GE_ADD_F32 ? (BN <= 96 ? BN : 32) : 0;
   static constexpr int CS = EPI == GE_QKV_ROPE64 ? 32 : (EPI == GE_QKV_ROPE32 ? 16 : 0);
   float scale = 1.f;
   bool have_res = false;  // res holds the row segment (else the epilogue reads it)
@@ -230,15 +254,33 @@ struct EpiPre {
 };
 
 // float4 j of a row segment of an f32 output [.., ldo] starting at column col
-// (zeros outside the N columns)
+// (zeros outside the N columns). A plain (L1-allocating) load: a thread reads
+// the 8 float4 of one 128-byte line of its row, and L1 turns them into one line
+// fill where L2-only loads send 8 requests (measured on B200, residual add at
+// M = 12800, N = 720: 38 against 51 us at K = 960, 59 against 82 us at K = 2048).
+// Each residual element is read and then written by the one thread that owns
+// it, after the producing kernel's writes are visible (griddepcontrol.wait).
 SVLA_DEV float4 load_res4(const GemmArgs& a, int m, int col) {
   const float* p = reinterpret_cast<const float*>(a.out) + (size_t)m * a.ldo + col;
-  if (col + 4 <= a.N) return __ldcg(reinterpret_cast<const float4*>(p));
+  if (col + 4 <= a.N) return *reinterpret_cast<const float4*>(p);
   float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
   if (col < a.N) v.x = p[0];
   if (col + 1 < a.N) v.y = p[1];
   if (col + 2 < a.N) v.z = p[2];
   return v;
+}
+// float4 pair (lo, hi) from column col: one 256-bit load where it is whole and aligned
+SVLA_DEV void load_res8(const GemmArgs& a, int m, int col, float4& lo, float4& hi) {
+  const float* p = reinterpret_cast<const float*>(a.out) + (size_t)m * a.ldo + col;
+  if (col + 8 <= a.N && aligned32(p)) {
+    uint32_t u[8];
+    ld_global_v8(p, u);
+    lo = make_float4(__uint_as_float(u[0]), __uint_as_float(u[1]), __uint_as_float(u[2]), __uint_as_float(u[3]));
+    hi = make_float4(__uint_as_float(u[4]), __uint_as_float(u[5]), __uint_as_float(u[6]), __uint_as_float(u[7]));
+  } else {
+    lo = load_res4(a, m, col);
+    hi = load_res4(a, m, col + 4);
+  }
 }
 
 // want_res: this CTA runs the epilogue of this row (split-K: only one CTA of
@@ -250,19 +292,15 @@ SVLA_DEV void epi_prefetch(const GemmArgs& a, int m, int n0, bool row_ok, EpiPre
   if constexpr (EpiPre<BN, EPI>::RES > 0) {
     if (want_res) {
 #pragma unroll
-      for (int j = 0; j < EpiPre<BN, EPI>::RES / 4; ++j)
-        pre.res[j] = row_ok ? load_res4(a, m, n0 + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < EpiPre<BN, EPI>::RES / 4; j += 2) {
+        if (row_ok) {
+          load_res8(a, m, n0 + 4 * j, pre.res[j], pre.res[j + 1]);
+        } else {
+          pre.res[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          pre.res[j + 1] = pre.res[j];
+        }
+      }
       pre.have_res = true;
-    }
-  }
-  if constexpr (EPI == GE_ADD_F32) {
-    // wider tiles: the row segment is read chunk by chunk through L1; start
-    // bringing its lines there now
-    if (row_ok) {
-      const float* p = reinterpret_cast<const float*>(a.out) + (size_t)m * a.ldo + n0;
-#pragma unroll
-      for (int c = EpiPre<BN, EPI>::RES; c < BN; c += 32)
-        if (n0 + c < a.N) prefetch_l1(p + c);
     }
   }
   if constexpr (EpiPre<BN, EPI>::CS > 0) {
@@ -365,13 +403,16 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, 
     }
   } else {
     constexpr int RES = EpiPre<BN, EPI>::RES;
-    // residual add with the row segment in registers: 32 columns per TMEM wait,
-    // unrolled so the residual registers are indexed by constants; otherwise
-    // 16 columns per wait, the residual (if any) read through L1, where
-    // epi_prefetch brought its lines
+    // residual add: 32 columns per TMEM wait, the residual of the chunk in
+    // registers (r, indexed by constants once unrolled): from the prefetched
+    // segment up to 96 columns; for wider tiles the next chunk's residual is
+    // loaded before this chunk is added, so its latency overlaps the work
+    // (the shared-memory ring leaves L1 too small to hold the tile's rows).
+    // Other epilogues: 16 columns per wait.
     constexpr int CW = RES > 0 ? 32 : 16;
+    constexpr bool PIPE = RES > 0 && RES < BN;
     float ss = 0.f;  // sum of squares of this row's outputs in this tile (fused RMSNorm)
-    auto chunk = [&](int c) {
+    auto chunk = [&](int c, const float4 (&r)[8]) {
       float v[CW];
       src.get(c, v);
       if (!row_ok || n0 + c >= a.N) return;
@@ -380,7 +421,9 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, 
         const int col = n0 + c + h;
         if (col >= a.N) break;
         const int ncols = a.N - col;
-        float (&w)[16] = *reinterpret_cast<float(*)[16]>(v + h);
+        float w[16];  // a copy, not a reference into v: v stays in registers
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = v[h + i];
         add_bias16(w, a.bias, col, a.N);
         if constexpr (EPI == GE_F32 || EPI == GE_ADD_F32) {
           float* dst = reinterpret_cast<float*>(a.out) + (size_t)m * a.ldo + col;
@@ -388,18 +431,7 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, 
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               float4 o;
-              if constexpr (RES > 0) {
-                // c + h < BN = RES: a constant once unrolled
-                o = pre.have_res ? pre.res[(c + h) / 4 + i] : load_res4(a, m, col + 4 * i);
-              } else if (ncols >= 16) {
-                o = reinterpret_cast<const float4*>(dst)[i];
-              } else {
-                o = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (4 * i < ncols) o.x = dst[4 * i];
-                if (4 * i + 1 < ncols) o.y = dst[4 * i + 1];
-                if (4 * i + 2 < ncols) o.z = dst[4 * i + 2];
-                if (4 * i + 3 < ncols) o.w = dst[4 * i + 3];
-              }
+              o = r[h / 4 + i];  // h / 4 + i: a constant once unrolled
               w[4 * i] += o.x;
               w[4 * i + 1] += o.y;
               w[4 * i + 2] += o.z;
@@ -422,12 +454,48 @@ SVLA_DEV void run_epilogue(const GemmArgs& a, AccSource<BN> src, int m, int n0, 
         }
       }
     };
-    if constexpr (RES > 0) {
+    // the residual of columns c .. c + 31 of this row: prefetched, or loaded now
+    auto load_chunk = [&](int c, float4 (&r)[8]) {
 #pragma unroll
-      for (int c = 0; c < BN; c += CW) chunk(c);
-    } else {
+      for (int i = 0; i < 8; i += 2) {
+        if (row_ok) {
+          load_res8(a, m, n0 + c + 4 * i, r[i], r[i + 1]);
+        } else {
+          r[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          r[i + 1] = r[i];
+        }
+      }
+    };
+    auto res_chunk = [&](int c, float4 (&r)[8]) {
+      if (c < RES && pre.have_res) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r[i] = pre.res[(c + 4 * i) % (RES > 0 ? RES : 1) / 4];
+      } else {
+        load_chunk(c, r);
+      }
+    };
+    if constexpr (PIPE) {
+      float4 cur[8];
+      res_chunk(0, cur);
 #pragma unroll 1
-      for (int c = 0; c < BN; c += CW) chunk(c);
+      for (int c = 0; c < BN; c += CW) {
+        float4 nxt[8];
+        if (c + CW < BN) load_chunk(c + CW, nxt);
+        chunk(c, cur);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
+      }
+    } else if constexpr (RES > 0) {
+#pragma unroll
+      for (int c = 0; c < BN; c += CW) {
+        float4 r[8];
+        res_chunk(c, r);
+        chunk(c, r);
+      }
+    } else {
+      const float4 none[8] = {};
+#pragma unroll 1
+      for (int c = 0; c < BN; c += CW) chunk(c, none);
     }
     if constexpr (EPI == GE_F32 || EPI == GE_ADD_F32) {
       if (a.ss_out && row_ok) a.ss_out[(size_t)(n0 / BN) * a.ss_ld + m] = ss;
