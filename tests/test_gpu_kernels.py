@@ -87,6 +87,42 @@ def test_gemm_epilogues(M, N, K):
     assert ((Cs.double() - silu).abs() <= 2 ** -7 * silu.abs() + 1e-3).all()
 
 
+def _offset(shape, dtype, elems, fill):
+    """A contiguous [M, N] view whose first element sits `elems` elements past a fresh allocation."""
+    M, N = shape
+    store = torch.full((M * N + elems,), fill, dtype=dtype, device=DEV)
+    return store[elems:].view(M, N)
+
+
+@pytest.mark.parametrize("M,N,K", [(50, 720, 2048), (177, 960, 720), (1600, 720, 960), (4096, 720, 2048),
+                                   (1600, 4096, 720), (300, 96, 128)])
+def test_gemm_outputs_at_16_byte_offsets_match_aligned(M, N, K):
+    """The epilogue moves 32 bytes per access where the address allows it and 16 otherwise: outputs
+    (and residuals) that start 16 bytes past a 32-byte boundary give the same bits."""
+    g = torch.Generator(device="cpu").manual_seed(M + N + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16).to(DEV)
+    W = (0.05 * torch.randn(N, K, generator=g)).to(torch.bfloat16).to(DEV)
+    bias = torch.randn(N, generator=g).to(DEV)
+    R0 = torch.randn(M, N, generator=g).to(DEV)
+    out = {}
+    for off in (0, 1):
+        Cf = _offset((M, N), torch.float32, 4 * off, float("nan"))
+        Cb = _offset((M, N), torch.bfloat16, 8 * off, float("nan"))
+        R = _offset((M, N), torch.float32, 4 * off, 0.0)
+        R.copy_(R0)
+        assert Cf.data_ptr() % 32 == 16 * off and Cb.data_ptr() % 32 == 16 * off and R.data_ptr() % 32 == 16 * off
+        gemm(_abi.EPI_F32, A, W, Cf, bias)
+        gemm(_abi.EPI_BF16, A, W, Cb, bias)
+        gemm(_abi.EPI_ADD_F32, A, W, R, bias)
+        torch.cuda.synchronize()
+        out[off] = (Cf.clone(), Cb.clone(), R.clone())
+    for a, b in zip(out[0], out[1]):
+        assert torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a.view(torch.int32),
+                           b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32))
+    ref = A.double() @ W.double().T + bias.double()
+    np.testing.assert_allclose(out[1][2].double().cpu(), (R0.double() + ref).cpu(), rtol=1e-5, atol=1e-4)
+
+
 @pytest.mark.parametrize("splits", [2, 5, 8, 16])
 def test_gemm_split_k_is_deterministic(splits):
     """<= 8 splits reduce across a thread-block cluster, more through the global
