@@ -322,6 +322,10 @@ struct svla_handle {
   // weight-only int8 expert (svla_create_ex with SVLA_CREATE_EXPERT_INT8)
   uint8_t* e8 = nullptr;     // codes and (alpha, beta) pairs of the expert projections
   std::vector<Q8Mat> e8m;    // per expert layer: QKV (odd: Q), O, gate/up, down, cross K, cross V (odd only)
+  // the multi-kernel denoise's in-loop projections (QKV or Q, O, gate/up, down of every
+  // layer) dequantised once per call: element offsets in e8_loop of (layer, which)
+  uint16_t* e8_loop = nullptr;
+  std::vector<size_t> e8_loop_off;
   uint8_t* fq = nullptr;     // the persistent kernel's int8 copy (rows of codes and pairs)
   FusedQ8 fql;
   int expert_bits = 16;      // weights the denoise uses
@@ -1019,8 +1023,14 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
   // one expert projection of layer l (which: 0 QKV / Q, 1 O, 2 gate/up, 3 down,
   // 4 cross K, 5 cross V): the dense weights (gains folded at create) or the
   // int8 copy (the gain applied to the dequantised weights)
+  auto loop_deq = [&](int l, int which, int Mg) {
+    return e8 && !fused && which < 4 && h->e8_loop != nullptr && w8_many_tiles(Mg, h->e8m[6 * l + which].N);
+  };
   auto eg = [&](int epi, const bf16* A, int lda, int l, int which, size_t dense_off, const uint16_t* gain, int Mg,
                 int N, int K, GemmArgs args, cudaStream_t st) {
+    if (loop_deq(l, which, Mg))  // dequantised before the step loop (below)
+      return gemm(h, epi, A, lda, reinterpret_cast<const bf16*>(h->e8_loop + h->e8_loop_off[4 * l + which]), K, Mg,
+                  N, K, args, h->e_part, h->e_cnt, st);
     if (e8) return gemm8(h, epi, A, lda, h->e8, h->e8m[6 * l + which], gain, Mg, args, h->e_part, h->e_cnt, st);
     return gemm(h, epi, A, lda, h->W(dense_off), K, Mg, N, K, args, h->e_part, h->e_cnt, st);
   };
@@ -1050,6 +1060,24 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
   }
   if (fused) return launch_fused(h, kv, pad, B, L, noise, H, n_steps, actions, trace, prefix, d, s);
   const Layout& Lh = h->lay;
+  // int8 expert, many tiles: the weights do not change between Euler steps, so
+  // each in-loop projection is dequantised once per call (the kernel gemm8 runs
+  // per GEMM: same codes, gain and bits), and the steps run the dense GEMMs on it
+  bool loop_dequantised = false;
+  for (int l = 0; l < c.e_layers; ++l) {
+    const Entry* e = &h->lay.e[9 * l];
+    for (int which = 0; which < 4; ++which) {
+      if (!loop_deq(l, which, M)) continue;
+      const Q8Mat& w = h->e8m[6 * l + which];
+      const uint16_t* gain = which == 0 ? h->w + e[0].off : (which == 2 ? h->w + e[5].off : nullptr);
+      const long long chunks = (long long)w.N * (w.K / 16);  // K % 16 == 0
+      const unsigned blocks = (unsigned)std::min<long long>((chunks + 255) / 256, 8LL * NUM_SMS_B200);
+      SVLA_TRY(launch_pdl(dequant_affine8_kernel, dim3(blocks), dim3(256), 0, s, h->e8 + w.q_off,
+                          reinterpret_cast<const uint16_t*>(h->e8 + w.ab_off), gain, w.N, w.K,
+                          h->e8_loop + h->e8_loop_off[4 * l + which]));
+      loop_dequantised = true;
+    }
+  }
   int se_blocks = (M + SE_WARPS - 1) / SE_WARPS;
   if (se_blocks > 2 * NUM_SMS_B200) se_blocks = 2 * NUM_SMS_B200;
   const int t2_tiles = residual_tiles(M, E, E), o_tiles = residual_tiles(M, E, qw);
@@ -1070,7 +1098,15 @@ cudaError_t record_denoise(svla_handle* h, const void* kv, const uint8_t* pad, i
     sb.a_out = h->e_a;
     sb.c_out = h->e_c;
     sb.nA = (M + 7) / 8;
-    SVLA_TRY(launch_pdl(step_begin_kernel, dim3(sb.nA + (E + 7) / 8), dim3(256), 0, s, sb));
+    if (k == 0 && loop_dequantised) {
+      // a plain launch: it starts after the dequantisation kernels have finished, so
+      // no GEMM after it streams a dequantised matrix early (their weight loads come
+      // before the dependency wait)
+      step_begin_kernel<<<dim3(sb.nA + (E + 7) / 8), dim3(256), 0, s>>>(sb);
+      SVLA_TRY(cudaGetLastError());
+    } else {
+      SVLA_TRY(launch_pdl(step_begin_kernel, dim3(sb.nA + (E + 7) / 8), dim3(256), 0, s, sb));
+    }
     // time MLP: h1 = silu(W_t1[:, :E] a + c), r = W_t2 h1 + b_t2 (the residual stream starts here)
     SVLA_TRY(gemm(h, GE_SILU_BF16, h->e_a, E, h->W(Lh.w_t1.off), 2 * E, M, E, E, out_args(h->e_h1, E, h->e_c),
                   h->e_part, h->e_cnt, s));
@@ -1341,6 +1377,17 @@ svla_status svla_create_ex(const svla_config* cfg, const void* blob, size_t blob
       h->e8m.push_back(l % 2 == 1 ? add(kvw, pkvw) : Q8Mat());
     }
     if ((e = halloc(h, &h->e8, off)) != cudaSuccess) return bail(e, "int8 expert weights");
+    // the loop buffer only where some denoise of this handle takes the many-tile path
+    bool many = false;
+    size_t loop_elems = 0;
+    for (int l = 0; l < c.e_layers; ++l)
+      for (int i = 0; i < 4; ++i) {
+        h->e8_loop_off.push_back(loop_elems);
+        const Q8Mat& m = h->e8m[6 * l + i];
+        loop_elems += ((size_t)m.N * m.K + 127) / 128 * 128;  // 256-byte aligned matrices
+        many = many || w8_many_tiles(c.max_batch * c.max_chunk, m.N);
+      }
+    if (many && (e = halloc(h, &h->e8_loop, loop_elems)) != cudaSuccess) return bail(e, "int8 expert loop buffer");
     for (int l = 0; l < c.e_layers && e == cudaSuccess; ++l) {
       const Entry* en = &lay.e[9 * l];
       const size_t src[6] = {en[1].off, en[4].off, en[6].off, en[8].off, en[2].off, en[3].off};
