@@ -1004,11 +1004,35 @@ def profile_case(spec, dev, reps):
     prefill and the denoise of workload NAME `reps` times after one warm-up
     call; options ':graph' / ':fused' pick the denoise path, ':int8p' /
     ':int8e' the int8 prefix / expert; 'denoise_b256' runs the batch-256
-    denoise from its given K/V cache."""
+    denoise from its given K/V cache; 'train' the expert's training step on
+    the inputs train_block times."""
     import torch
     from vision_language_action_b200 import _abi
     from vision_language_action_b200.runtime import SmolVLA
     name, *opts = spec.split(":")
+    if name == "train":
+        s = synth.SHAPES["smolvla"]
+        B, L, H = 2, 177, 50
+        d = f"cuda:{dev}"
+        m = SmolVLA(s, synth.pack_blob(s, synth.gen_weights(s, 7, random_affine=True)), max_batch=B, max_prefix=L,
+                    max_chunk=H, device=dev, train=True)
+        rng = np.random.default_rng(7)
+        kv = torch.from_numpy(synth.f32_to_bf16_bits(rng.standard_normal((2, s.p_layers, B, L, s.p_kv_width))
+                                                     .astype(np.float32)).view(np.int16)).to(d).view(torch.bfloat16)
+        valid = torch.ones((B, L), dtype=torch.uint8, device=d)
+        a = torch.from_numpy((0.5 * rng.standard_normal((B, H, s.action_dim))).astype(np.float32)).to(d)
+        eps = torch.from_numpy(rng.standard_normal((B, H, s.action_dim)).astype(np.float32)).to(d)
+        t = torch.from_numpy(rng.uniform(0.05, 0.95, B).astype(np.float32)).to(d)
+        grads = torch.empty(int(m.lib.svla_train_grad_elems(m.h)), dtype=torch.float32, device=d)
+        for _ in range(1 + reps):
+            m.train_step(kv, valid, a, eps, t, grads=grads)
+        torch.cuda.synchronize()
+        st = m.device_status()
+        m.close()
+        print(json.dumps({"profile_case": spec, "calls": 1 + reps, "status": st}), flush=True)
+        if st != 0:
+            raise SystemExit(1)
+        return
     if name == "denoise_b256":
         wl = synth.WORKLOADS[name]
         s = wl.model

@@ -72,6 +72,12 @@ cudaError_t ensure_attrs(int dev) {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(attention_rows_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_ROWS_SMEM_MAX);
   if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_bwd_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)attn_bwd_rows_smem(64));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_bwd_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)attn_bwd_keys_smem(64));
+  if (e == cudaSuccess)
     e = cudaFuncSetAttribute(denoise_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, FD_SMEM_MAX);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(denoise_fused_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, FD_SMEM_MAX);
@@ -573,7 +579,7 @@ cudaError_t record_train(svla_handle* h, const void* kv, const uint8_t* pad, int
   auto norm_bwd = [&](const float* r, const uint16_t* g, const float* dy, float* dg) {
     SVLA_TRY(launch_pdl(norm_bwd_kernel, dim3((M + 7) / 8), dim3(256), 0, s, r, g, dy, M, E, c.rms_eps, T.dr, T.drb,
                         T.rs));
-    return launch_pdl(norm_gain_grad_kernel, dim3((E + 255) / 256), dim3(256), 0, s, r, (const float*)T.rs, dy, M, E,
+    return launch_pdl(norm_gain_grad_kernel, dim3((E + 63) / 64), dim3(64), 0, s, r, (const float*)T.rs, dy, M, E,
                       dg);
   };
   auto colsum = [&](const float* x, int C, int ld, float* out) {
@@ -697,10 +703,11 @@ cudaError_t record_train(svla_handle* h, const void* kv, const uint8_t* pad, int
       ab.lddkv = kvw;
       ab.rope_cs = nullptr;
     }
-    SVLA_TRY(launch_pdl(attn_bwd_rows_kernel, dim3((unsigned)(((size_t)B * nq * H + 7) / 8)), dim3(256),
-                        (size_t)8 * 3 * hd * sizeof(float), s, ab));
-    SVLA_TRY(launch_pdl(attn_bwd_keys_kernel, dim3((unsigned)(((size_t)B * nkv * ab.Tk + 7) / 8)), dim3(256),
-                        (size_t)8 * 2 * hd * sizeof(float), s, ab));
+    SVLA_TRY(launch_pdl(attn_bwd_rows_kernel, dim3((unsigned)((size_t)B * nq * ((H + ATB_WARPS - 1) / ATB_WARPS))),
+                        dim3(32 * ATB_WARPS), attn_bwd_rows_smem(hd), s, ab));
+    SVLA_TRY(launch_pdl(attn_bwd_keys_kernel,
+                        dim3((unsigned)((size_t)B * nkv * ((ab.Tk + ATB_KEYS - 1) / ATB_KEYS))),
+                        dim3(32 * ATB_WARPS), attn_bwd_keys_smem(hd), s, ab));
     const int wq_rows = l % 2 == 0 ? qkvw : qw;  // even: [W_q; W_k; W_v] share the input y
     SVLA_TRY(tr16(T.dqkv, M, wq_rows, wq_rows, T.ta, Mp));
     SVLA_TRY(tr16(Y(l), M, E, E, T.tb, Mp));

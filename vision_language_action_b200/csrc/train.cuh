@@ -172,7 +172,10 @@ __global__ void __launch_bounds__(1024) loss_reduce_kernel(const float* __restri
 // RMSNorm backward (reading 8, y = r rs g with rs = rsqrt(mean(r^2) + eps)):
 // with n = r rs and dn = dy g,  dr += rs (dn - n mean(dn n)). One warp per row;
 // dr is updated in place (it carries the residual's gradient), its bf16 copy
-// and the row's rs are written too.
+// and the row's rs are written too. Rows up to NORM_BWD_CACHE * 32 wide are
+// read once into registers (all loads in flight together) and the three passes
+// run from there; each lane sums its columns in increasing order either way.
+constexpr int NORM_BWD_CACHE = 32;
 __global__ void __launch_bounds__(256) norm_bwd_kernel(const float* __restrict__ r, const uint16_t* __restrict__ g,
                                                        const float* __restrict__ dy, int M, int E, float rms_eps,
                                                        float* __restrict__ dr, uint16_t* __restrict__ dr_bf,
@@ -183,6 +186,42 @@ __global__ void __launch_bounds__(256) norm_bwd_kernel(const float* __restrict__
   if (m >= M) return;
   const float* rr = r + (size_t)m * E;
   const float* dd = dy + (size_t)m * E;
+  float* drr = dr + (size_t)m * E;
+  if (E <= 32 * NORM_BWD_CACHE) {
+    float rv[NORM_BWD_CACHE], dn[NORM_BWD_CACHE];
+#pragma unroll
+    for (int t = 0; t < NORM_BWD_CACHE; ++t) {
+      const int e = lane + 32 * t;
+      rv[t] = e < E ? rr[e] : 0.f;
+      dn[t] = e < E ? dd[e] * bf2f(g[e]) : 0.f;
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int t = 0; t < NORM_BWD_CACHE; ++t)
+      if (lane + 32 * t < E) ss = fmaf(rv[t], rv[t], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rs = rsqrtf(ss / (float)E + rms_eps);
+    float dot = 0.f;
+#pragma unroll
+    for (int t = 0; t < NORM_BWD_CACHE; ++t)
+      if (lane + 32 * t < E) dot = fmaf(dn[t], rv[t] * rs, dot);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    const float mean = dot / (float)E;
+#pragma unroll
+    for (int t = 0; t < NORM_BWD_CACHE; ++t) {
+      const int e = lane + 32 * t;
+      if (e < E) {
+        const float n = rv[t] * rs;
+        const float v = drr[e] + rs * (dn[t] - n * mean);
+        drr[e] = v;
+        if (dr_bf) dr_bf[(size_t)m * E + e] = bf16_bits(v);
+      }
+    }
+    if (lane == 0) rs_out[m] = rs;
+    return;
+  }
   float ss = 0.f;
   for (int e = lane; e < E; e += 32) ss = fmaf(rr[e], rr[e], ss);
 #pragma unroll
@@ -195,23 +234,35 @@ __global__ void __launch_bounds__(256) norm_bwd_kernel(const float* __restrict__
   const float mean = dot / (float)E;
   for (int e = lane; e < E; e += 32) {
     const float n = rr[e] * rs;
-    const float v = dr[(size_t)m * E + e] + rs * (dd[e] * bf2f(g[e]) - n * mean);
-    dr[(size_t)m * E + e] = v;
+    const float v = drr[e] + rs * (dd[e] * bf2f(g[e]) - n * mean);
+    drr[e] = v;
     if (dr_bf) dr_bf[(size_t)m * E + e] = bf16_bits(v);
   }
   if (lane == 0) rs_out[m] = rs;
 }
 
-// Gain gradient of an RMSNorm: dg[e] = sum_m dy[m, e] r[m, e] rs[m] (thread per column, rows in order).
-__global__ void __launch_bounds__(256) norm_gain_grad_kernel(const float* __restrict__ r, const float* __restrict__ rs,
-                                                             const float* __restrict__ dy, int M, int E,
-                                                             float* __restrict__ dg) {
+// Gain gradient of an RMSNorm: dg[e] = sum_m dy[m, e] r[m, e] rs[m] (thread per
+// column, rows in order; the loads of 16 rows are issued before their products).
+__global__ void __launch_bounds__(64) norm_gain_grad_kernel(const float* __restrict__ r, const float* __restrict__ rs,
+                                                            const float* __restrict__ dy, int M, int E,
+                                                            float* __restrict__ dg) {
   griddep_launch_dependents();
   griddep_wait();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= E) return;
   float acc = 0.f;
-  for (int m = 0; m < M; ++m) acc = fmaf(dy[(size_t)m * E + e], r[(size_t)m * E + e] * rs[m], acc);
+  for (int m0 = 0; m0 < M; m0 += 16) {
+    float dv[16], xv[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int m = m0 + u;
+      dv[u] = m < M ? dy[(size_t)m * E + e] : 0.f;
+      xv[u] = m < M ? r[(size_t)m * E + e] * rs[m] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      if (m0 + u < M) acc = fmaf(dv[u], xv[u], acc);
+  }
   dg[e] = acc;
 }
 
@@ -320,86 +371,159 @@ struct AttnBwdArgs {
   const float2* rope_cs; // non-null: undo the rotate-half RoPE on dq (position i) and dk (position j)
 };
 
-// Pass 1, one warp per (query b, head h, row i): recompute p over the visible
-// keys, then dp_j = do . v_j, ds_j = p_j (dp_j - sum_j p_j dp_j) (kept for
-// pass 2), dq = scale sum_j ds_j k_j. Shared memory: 8 warps x (2 hd + hd) floats.
+// Key and value tiles of the attention backward: ATB_KT keys of one kv head
+// in shared memory, rows padded to hd + 2 bf16 (an odd number of words, so a
+// warp reading one element of 32 different keys touches 32 banks).
+constexpr int ATB_KT = 64;
+constexpr int ATB_WARPS = 8;
+
+// rows [k0, k0 + ATB_KT) of the kv head's columns [col, col + hd) of a bf16
+// [rows, ld] matrix into dst (pitch hd + 2), zeros past `rows`; all threads
+SVLA_DEV void atb_stage_keys(const uint16_t* src, size_t row0, int ld, int col, int hd, int k0, int rows,
+                             uint16_t* dst) {
+  const int cpr = hd / 8;  // 16-byte chunks per row
+  const int pitch = hd + 2;
+  for (int idx = threadIdx.x; idx < ATB_KT * cpr; idx += blockDim.x) {
+    const int r = idx / cpr, c = (idx - r * cpr) * 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (k0 + r < rows) v = *reinterpret_cast<const uint4*>(src + (row0 + k0 + r) * ld + col + c);
+    uint32_t* d = reinterpret_cast<uint32_t*>(dst + r * pitch + c);  // 4-byte aligned (pitch even)
+    d[0] = v.x;
+    d[1] = v.y;
+    d[2] = v.z;
+    d[3] = v.w;
+  }
+}
+
+// Pass 1, one warp per (query b, head h, row i), a block per 8 rows of one (b,
+// h): recompute p over the visible keys, then dp_j = do . v_j, ds_j = p_j (dp_j
+// - sum_j p_j dp_j) (kept for pass 2), dq = scale sum_j ds_j k_j. The block
+// brings the keys and values of its kv head into shared memory ATB_KT at a
+// time; each lane takes keys lane, lane + 32, .. and every sum runs over d (or
+// over j for dq) in increasing order, the same arithmetic as one warp reading
+// the rows from global memory.
+// Shared memory: 2 tiles of ATB_KT x (hd + 2) bf16, then per warp 3 hd + ATB_KT floats.
 __global__ void __launch_bounds__(256) attn_bwd_rows_kernel(const AttnBwdArgs a) {
   extern __shared__ float sh[];
   griddep_launch_dependents();
   griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long wid = (long long)blockIdx.x * 8 + warp;
-  if (wid >= (long long)a.B * a.nq * a.Tq) return;
-  const int i = (int)(wid % a.Tq), h = (int)((wid / a.Tq) % a.nq), b = (int)(wid / ((long long)a.Tq * a.nq));
+  const int rblocks = (a.Tq + ATB_WARPS - 1) / ATB_WARPS;
+  const int rb = (int)(blockIdx.x % rblocks), h = (int)((blockIdx.x / rblocks) % a.nq);
+  const int b = (int)(blockIdx.x / ((unsigned)rblocks * a.nq));
+  const int i = rb * ATB_WARPS + warp;
+  const bool active = i < a.Tq;
   const int g = h / (a.nq / a.nkv);
-  float* qs = sh + warp * 3 * a.hd;
-  float* dos = qs + a.hd;
-  float* dqs = dos + a.hd;
-  const size_t qrow = (size_t)b * a.Tq + i;
-  for (int d = lane; d < a.hd; d += 32) {
-    qs[d] = bf2f(a.q[qrow * a.ldq + (size_t)h * a.hd + d]);
-    dos[d] = bf2f(a.dout[qrow * a.ldo + (size_t)h * a.hd + d]);
+  const int hd = a.hd, pitch = hd + 2;
+  uint16_t* sK = reinterpret_cast<uint16_t*>(sh);
+  uint16_t* sV = sK + ATB_KT * pitch;
+  float* qs = reinterpret_cast<float*>(sV + ATB_KT * pitch) + warp * (3 * hd + ATB_KT);
+  float* dos = qs + hd;
+  float* dqs = dos + hd;
+  float* sds = dqs + hd;  // this row's ds over the current key tile
+  const size_t qrow = (size_t)b * a.Tq + (active ? i : 0);
+  if (active) {
+    for (int d = lane; d < hd; d += 32) {
+      qs[d] = bf2f(a.q[qrow * a.ldq + (size_t)h * hd + d]);
+      dos[d] = bf2f(a.dout[qrow * a.ldo + (size_t)h * hd + d]);
+    }
   }
   __syncwarp();
-  float* Prow = a.P + (((size_t)b * a.nq + h) * a.Tq + i) * a.Tk;
-  float* Srow = a.dS + (((size_t)b * a.nq + h) * a.Tq + i) * a.Tk;
+  float* Prow = a.P + (((size_t)b * a.nq + h) * a.Tq + (active ? i : 0)) * a.Tk;
+  float* Srow = a.dS + (((size_t)b * a.nq + h) * a.Tq + (active ? i : 0)) * a.Tk;
   auto visible = [&](int j) {
     if (a.causal && j > i) return false;
     return a.key_valid == nullptr || a.key_valid[(size_t)b * a.Tk + j] != 0;
   };
+  const int nkt = (a.Tk + ATB_KT - 1) / ATB_KT;
+  const size_t krow0 = (size_t)b * a.Tk;
   // scores and their maximum
   float mx = -INFINITY;
-  for (int j = lane; j < a.Tk; j += 32) {
-    float s = -INFINITY;
-    if (visible(j)) {
-      const uint16_t* kr = a.k + ((size_t)b * a.Tk + j) * a.ldkv + (size_t)g * a.hd;
-      float acc = 0.f;
-      for (int d = 0; d < a.hd; ++d) acc = fmaf(qs[d], bf2f(kr[d]), acc);
-      s = acc * a.scale;
+  for (int kt = 0; kt < nkt; ++kt) {
+    const int k0 = kt * ATB_KT;
+    __syncthreads();
+    atb_stage_keys(a.k, krow0, a.ldkv, g * hd, hd, k0, a.Tk, sK);
+    __syncthreads();
+    if (!active) continue;
+    for (int jj = lane; jj < ATB_KT && k0 + jj < a.Tk; jj += 32) {
+      const int j = k0 + jj;
+      float s = -INFINITY;
+      if (visible(j)) {
+        const uint16_t* kr = sK + jj * pitch;
+        float acc = 0.f;
+        for (int d = 0; d < hd; ++d) acc = fmaf(qs[d], bf2f(kr[d]), acc);
+        s = acc * a.scale;
+      }
+      Prow[j] = s;
+      mx = fmaxf(mx, s);
     }
-    Prow[j] = s;
-    mx = fmaxf(mx, s);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float sum = 0.f;
-  for (int j = lane; j < a.Tk; j += 32) {
-    const float s = Prow[j];
-    const float p = s == -INFINITY ? 0.f : __expf(s - mx);
-    Prow[j] = p;
-    sum += p;
+  if (active) {
+    for (int j = lane; j < a.Tk; j += 32) {
+      const float s = Prow[j];
+      const float p = s == -INFINITY ? 0.f : __expf(s - mx);
+      Prow[j] = p;
+      sum += p;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   const float inv = 1.f / sum;
   float D = 0.f;
-  for (int j = lane; j < a.Tk; j += 32) {
-    const float p = Prow[j] * inv;
-    Prow[j] = p;
-    float dp = 0.f;
-    if (p != 0.f) {
-      const uint16_t* vr = a.v + ((size_t)b * a.Tk + j) * a.ldkv + (size_t)g * a.hd;
-      for (int d = 0; d < a.hd; ++d) dp = fmaf(dos[d], bf2f(vr[d]), dp);
+  for (int kt = 0; kt < nkt; ++kt) {
+    const int k0 = kt * ATB_KT;
+    __syncthreads();
+    atb_stage_keys(a.v, krow0, a.ldkv, g * hd, hd, k0, a.Tk, sV);
+    __syncthreads();
+    if (!active) continue;
+    for (int jj = lane; jj < ATB_KT && k0 + jj < a.Tk; jj += 32) {
+      const int j = k0 + jj;
+      const float p = Prow[j] * inv;
+      Prow[j] = p;
+      float dp = 0.f;
+      if (p != 0.f) {
+        const uint16_t* vr = sV + jj * pitch;
+        for (int d = 0; d < hd; ++d) dp = fmaf(dos[d], bf2f(vr[d]), dp);
+      }
+      Srow[j] = dp;
+      D = fmaf(p, dp, D);
     }
-    Srow[j] = dp;
-    D = fmaf(p, dp, D);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) D += __shfl_xor_sync(0xffffffffu, D, o);
-  for (int j = lane; j < a.Tk; j += 32) Srow[j] = Prow[j] * (Srow[j] - D);
+  if (active)
+    for (int j = lane; j < a.Tk; j += 32) Srow[j] = Prow[j] * (Srow[j] - D);
   __syncwarp();
   __threadfence_block();
-  for (int d = lane; d < a.hd; d += 32) {
-    float acc = 0.f;
-    for (int j = 0; j < a.Tk; ++j) {
-      const float ds = Srow[j];
-      if (ds != 0.f) acc = fmaf(ds, bf2f(a.k[((size_t)b * a.Tk + j) * a.ldkv + (size_t)g * a.hd + d]), acc);
+  // dq = scale sum_j ds_j k_j (j in increasing order; lanes over d)
+  float acc[2] = {0.f, 0.f};  // d = lane, lane + 32 (hd <= 64)
+  for (int kt = 0; kt < nkt; ++kt) {
+    const int k0 = kt * ATB_KT;
+    __syncthreads();
+    atb_stage_keys(a.k, krow0, a.ldkv, g * hd, hd, k0, a.Tk, sK);
+    if (active)
+      for (int jj = lane; jj < ATB_KT; jj += 32) sds[jj] = k0 + jj < a.Tk ? Srow[k0 + jj] : 0.f;
+    __syncthreads();
+    if (!active) continue;
+    const int jn = min(ATB_KT, a.Tk - k0);
+    for (int jj = 0; jj < jn; ++jj) {
+      const float ds = sds[jj];
+      if (ds != 0.f) {
+        const uint16_t* kr = sK + jj * pitch;
+        acc[0] = fmaf(ds, bf2f(kr[lane]), acc[0]);
+        if (lane + 32 < hd) acc[1] = fmaf(ds, bf2f(kr[lane + 32]), acc[1]);
+      }
     }
-    dqs[d] = acc * a.scale;
   }
+  if (!active) return;
+  dqs[lane] = acc[0] * a.scale;
+  if (lane + 32 < hd) dqs[lane + 32] = acc[1] * a.scale;
   __syncwarp();
-  const int half = a.hd / 2;
-  for (int d = lane; d < a.hd; d += 32) {
+  const int half = hd / 2;
+  for (int d = lane; d < hd; d += 32) {
     float val = dqs[d];
     if (a.rope_cs) {
       // y1 = x1 c - x2 s, y2 = x2 c + x1 s  ->  dx1 = dy1 c + dy2 s, dx2 = dy2 c - dy1 s
@@ -407,53 +531,118 @@ __global__ void __launch_bounds__(256) attn_bwd_rows_kernel(const AttnBwdArgs a)
       const float2 cs = a.rope_cs[(size_t)i * half + p];
       val = d < half ? dqs[d] * cs.x + dqs[d + half] * cs.y : dqs[d] * cs.x - dqs[d - half] * cs.y;
     }
-    a.dq[qrow * a.lddq + (size_t)h * a.hd + d] = bf16_bits(val);
+    a.dq[qrow * a.lddq + (size_t)h * hd + d] = bf16_bits(val);
   }
 }
 
-// Pass 2, one warp per (query b, kv head g, key j): over the query heads of
-// the group and every row, dk_j = scale sum ds q, dv_j = sum p do.
-// Shared memory: 8 warps x 2 hd floats.
+inline size_t attn_bwd_rows_smem(int hd) {
+  return (size_t)2 * ATB_KT * (hd + 2) * sizeof(uint16_t) + (size_t)ATB_WARPS * (3 * hd + ATB_KT) * sizeof(float);
+}
+
+// Pass 2, for (query b, kv head g, key j): over the query heads of the group
+// and every row, dk_j = scale sum ds q, dv_j = sum p do (heads, then rows, in
+// increasing order). A block takes ATB_KEYS keys of one (b, g), 4 per warp; it
+// brings the rows' q and do of one head and the matching P and dS columns into
+// shared memory ATB_QT rows at a time, and each lane sums over d = lane, lane + 32.
+// Shared memory: 2 tiles of ATB_QT x hd bf16, 2 of ATB_QT x ATB_KEYS floats, and
+// per warp 4 keys x 2 hd floats.
+constexpr int ATB_KEYS = 32;
+constexpr int ATB_QT = 64;
 __global__ void __launch_bounds__(256) attn_bwd_keys_kernel(const AttnBwdArgs a) {
   extern __shared__ float sh[];
   griddep_launch_dependents();
   griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long wid = (long long)blockIdx.x * 8 + warp;
-  if (wid >= (long long)a.B * a.nkv * a.Tk) return;
-  const int j = (int)(wid % a.Tk), g = (int)((wid / a.Tk) % a.nkv), b = (int)(wid / ((long long)a.Tk * a.nkv));
+  const int kblocks = (a.Tk + ATB_KEYS - 1) / ATB_KEYS;
+  const int kb = (int)(blockIdx.x % kblocks), g = (int)((blockIdx.x / kblocks) % a.nkv);
+  const int b = (int)(blockIdx.x / ((unsigned)kblocks * a.nkv));
   const int group = a.nq / a.nkv;
-  float* dks = sh + warp * 2 * a.hd;
-  float* dvs = dks + a.hd;
-  for (int d = lane; d < a.hd; d += 32) {
-    float ak = 0.f, av = 0.f;
-    for (int hh = 0; hh < group; ++hh) {
-      const int h = g * group + hh;
-      const float* Pc = a.P + (((size_t)b * a.nq + h) * a.Tq) * a.Tk + j;
-      const float* Sc = a.dS + (((size_t)b * a.nq + h) * a.Tq) * a.Tk + j;
-      for (int i = 0; i < a.Tq; ++i) {
-        const float p = Pc[(size_t)i * a.Tk], ds = Sc[(size_t)i * a.Tk];
-        const size_t row = (size_t)b * a.Tq + i;
-        if (ds != 0.f) ak = fmaf(ds, bf2f(a.q[row * a.ldq + (size_t)h * a.hd + d]), ak);
-        if (p != 0.f) av = fmaf(p, bf2f(a.dout[row * a.ldo + (size_t)h * a.hd + d]), av);
+  const int hd = a.hd;
+  const int j0 = kb * ATB_KEYS;
+  uint16_t* sQ = reinterpret_cast<uint16_t*>(sh);
+  uint16_t* sO = sQ + ATB_QT * hd;
+  float* sP = reinterpret_cast<float*>(sO + ATB_QT * hd);
+  float* sS = sP + ATB_QT * ATB_KEYS;
+  float* outw = sS + ATB_QT * ATB_KEYS + warp * 4 * 2 * hd;  // [4 keys][dk hd | dv hd]
+  float ak[4][2] = {}, av[4][2] = {};
+  const int cpr = hd / 8;
+  for (int hh = 0; hh < group; ++hh) {
+    const int h = g * group + hh;
+    for (int i0 = 0; i0 < a.Tq; i0 += ATB_QT) {
+      const int rows = min(ATB_QT, a.Tq - i0);
+      __syncthreads();
+      for (int idx = threadIdx.x; idx < rows * cpr; idx += blockDim.x) {
+        const int r = idx / cpr, c = (idx - r * cpr) * 8;
+        const size_t row = (size_t)b * a.Tq + i0 + r;
+        *reinterpret_cast<uint4*>(sQ + r * hd + c) =
+            *reinterpret_cast<const uint4*>(a.q + row * a.ldq + (size_t)h * hd + c);
+        *reinterpret_cast<uint4*>(sO + r * hd + c) =
+            *reinterpret_cast<const uint4*>(a.dout + row * a.ldo + (size_t)h * hd + c);
+      }
+      const size_t pbase = (((size_t)b * a.nq + h) * a.Tq + i0) * a.Tk;
+      for (int idx = threadIdx.x; idx < rows * ATB_KEYS; idx += blockDim.x) {
+        const int r = idx / ATB_KEYS, c = idx - r * ATB_KEYS;
+        const bool ok = j0 + c < a.Tk;
+        sP[r * ATB_KEYS + c] = ok ? a.P[pbase + (size_t)r * a.Tk + j0 + c] : 0.f;
+        sS[r * ATB_KEYS + c] = ok ? a.dS[pbase + (size_t)r * a.Tk + j0 + c] : 0.f;
+      }
+      __syncthreads();
+      for (int r = 0; r < rows; ++r) {
+        const float q0 = bf2f(sQ[r * hd + lane]), o0 = bf2f(sO[r * hd + lane]);
+        const float q1 = lane + 32 < hd ? bf2f(sQ[r * hd + lane + 32]) : 0.f;
+        const float o1 = lane + 32 < hd ? bf2f(sO[r * hd + lane + 32]) : 0.f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int c = warp * 4 + t;
+          const float p = sP[r * ATB_KEYS + c], ds = sS[r * ATB_KEYS + c];
+          if (ds != 0.f) {
+            ak[t][0] = fmaf(ds, q0, ak[t][0]);
+            ak[t][1] = fmaf(ds, q1, ak[t][1]);
+          }
+          if (p != 0.f) {
+            av[t][0] = fmaf(p, o0, av[t][0]);
+            av[t][1] = fmaf(p, o1, av[t][1]);
+          }
+        }
       }
     }
-    dks[d] = ak * a.scale;
-    dvs[d] = av;
+  }
+  const int half = hd / 2;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    float* dks = outw + t * 2 * hd;
+    float* dvs = dks + hd;
+    dks[lane] = ak[t][0] * a.scale;
+    dvs[lane] = av[t][0];
+    if (lane + 32 < hd) {
+      dks[lane + 32] = ak[t][1] * a.scale;
+      dvs[lane + 32] = av[t][1];
+    }
   }
   __syncwarp();
-  const size_t krow = (size_t)b * a.Tk + j;
-  const int half = a.hd / 2;
-  for (int d = lane; d < a.hd; d += 32) {
-    float val = dks[d];
-    if (a.rope_cs) {
-      const int p = d % half;
-      const float2 cs = a.rope_cs[(size_t)j * half + p];
-      val = d < half ? dks[d] * cs.x + dks[d + half] * cs.y : dks[d] * cs.x - dks[d - half] * cs.y;
+#pragma unroll 1
+  for (int t = 0; t < 4; ++t) {
+    const int j = j0 + warp * 4 + t;
+    if (j >= a.Tk) break;
+    const float* dks = outw + t * 2 * hd;
+    const float* dvs = dks + hd;
+    const size_t krow = (size_t)b * a.Tk + j;
+    for (int d = lane; d < hd; d += 32) {
+      float val = dks[d];
+      if (a.rope_cs) {
+        const int p = d % half;
+        const float2 cs = a.rope_cs[(size_t)j * half + p];
+        val = d < half ? dks[d] * cs.x + dks[d + half] * cs.y : dks[d] * cs.x - dks[d - half] * cs.y;
+      }
+      a.dk[krow * a.lddkv + (size_t)g * hd + d] = bf16_bits(val);
+      a.dv[krow * a.lddkv + (size_t)g * hd + d] = bf16_bits(dvs[d]);
     }
-    a.dk[krow * a.lddkv + (size_t)g * a.hd + d] = bf16_bits(val);
-    a.dv[krow * a.lddkv + (size_t)g * a.hd + d] = bf16_bits(dvs[d]);
   }
+}
+
+inline size_t attn_bwd_keys_smem(int hd) {
+  return (size_t)2 * ATB_QT * hd * sizeof(uint16_t) + (size_t)2 * ATB_QT * ATB_KEYS * sizeof(float) +
+         (size_t)ATB_WARPS * 4 * 2 * hd * sizeof(float);
 }
 
 }  // namespace svla
