@@ -94,7 +94,9 @@ def split_grads(s, g):
     return out
 
 
-@pytest.mark.parametrize("shape,B,L,Hc", [("tiny", 2, 24, 8), ("smolvla", 2, 177, 50)])
+# the last case spans several key tiles (prefix 321) and two row tiles of the
+# attention backward's key pass (chunk 100), the long-prefix workload's shape
+@pytest.mark.parametrize("shape,B,L,Hc", [("tiny", 2, 24, 8), ("smolvla", 2, 177, 50), ("smolvla", 1, 321, 100)])
 def test_train_step_matches_oracle(shape, B, L, Hc):
     s, wb, kv_bits, valid, a, eps, t = make_case(shape, B, L, Hc, 7)
     m = SmolVLA(s, synth.pack_blob(s, wb), max_batch=B, max_prefix=L, max_chunk=Hc, train=True)
